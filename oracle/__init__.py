@@ -1,0 +1,149 @@
+"""CPU oracle of the masked routed-expert MoE layer -- TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may use
+this package.  The product path (the CUDA library and its Python binding)
+never imports it.
+
+The arithmetic lives in ``moe_oracle.c`` (plain fp64 C, see its header for
+the definition and the passages it follows).  This module compiles it with
+gcc and marshals numpy arrays through ctypes; it adds no arithmetic of its
+own except the threshold calibration's choice of population (the scores of
+the pairs the router selected), which is stated in ``calibrate_tau``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import tempfile
+from dataclasses import dataclass
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "moe_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(src: str = SRC, out: str = LIB, openmp: bool = True) -> str:
+    """Compile the oracle C source into a shared library (gcc -O2, OpenMP)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-o", out, src, "-lm"]
+    if openmp:
+        cmd.insert(1, "-fopenmp")
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(src, out):
+    return not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src)
+
+
+_P = ctypes.c_void_p
+
+
+@dataclass
+class OracleResult:
+    y: np.ndarray            # [T][d] float64
+    topk_idx: np.ndarray     # [T][k] int32
+    topk_w: np.ndarray       # [T][k] float64
+    logits: np.ndarray       # [T][E] float64
+    score: np.ndarray | None   # [T][k][f] float64
+    active: np.ndarray | None  # [T][k][f] uint8
+
+
+class Oracle:
+    """ctypes wrapper around one compiled oracle library."""
+
+    def __init__(self, path: str | None = None):
+        if path is None:
+            path = LIB
+            if _needs_build(SRC, LIB):
+                build()
+        self.path = path
+        self._lib = ctypes.CDLL(path)
+        f = self._lib.oracle_moe_forward
+        f.restype = ctypes.c_int
+        f.argtypes = [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                      ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, ctypes.c_int,
+                      _P, _P, _P, _P, _P, _P]
+        c = self._lib.oracle_calibrate_tau
+        c.restype = ctypes.c_double
+        c.argtypes = [_P, ctypes.c_long, ctypes.c_double]
+
+    @staticmethod
+    def _ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    def forward(self, x, w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None,
+                ws_down=None, *, top_k: int, tau: float, want_scores: bool = True,
+                nthreads: int = 0) -> OracleResult:
+        """All weight/x arguments are uint16 numpy arrays of bf16 bits (x @ W layout)."""
+        arrs = [np.ascontiguousarray(a, dtype=np.uint16) if a is not None else None
+                for a in (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)]
+        x, wr, wg, wu, wd, wsg, wsu, wsd = arrs
+        T, d = x.shape
+        E = wr.shape[0]
+        f = wg.shape[2]
+        S = 0 if wsg is None else wsg.shape[0]
+        k = int(top_k)
+        y = np.zeros((T, d), np.float64)
+        idx = np.zeros((T, k), np.int32)
+        w = np.zeros((T, k), np.float64)
+        lg = np.zeros((T, E), np.float64)
+        sc = np.zeros((T, k, f), np.float64) if want_scores else None
+        ac = np.zeros((T, k, f), np.uint8) if want_scores else None
+        rc = self._lib.oracle_moe_forward(
+            self._ptr(x), T, d, f, E, k, S, self._ptr(wr), self._ptr(wg), self._ptr(wu),
+            self._ptr(wd), self._ptr(wsg), self._ptr(wsu), self._ptr(wsd),
+            ctypes.c_float(tau), int(nthreads), self._ptr(y), self._ptr(idx), self._ptr(w),
+            self._ptr(lg), self._ptr(sc), self._ptr(ac))
+        if rc != 0:
+            raise RuntimeError(f"oracle_moe_forward failed ({rc})")
+        return OracleResult(y, idx, w, lg, sc, ac)
+
+    def calibrate_tau(self, scores: np.ndarray, sparsity: float) -> float:
+        """tau = the floor(q*N)-th smallest of the routed pairs' scores s = |silu(g)|.
+
+        The population is the T*k*f scores of the (token, expert) pairs the
+        router selected; shared-expert scores are excluded (they are never
+        masked).  The result is returned as a float32-representable value,
+        which is how the layer receives it."""
+        s = np.ascontiguousarray(scores, dtype=np.float64).reshape(-1)
+        t = self._lib.oracle_calibrate_tau(self._ptr(s), s.size, float(sparsity))
+        return float(np.float32(t))
+
+
+_default = None
+
+
+def load() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def build_variant(src_text: str, workdir: str | None = None) -> Oracle:
+    """Compile a modified copy of the oracle source (used to plant mistakes in tests)."""
+    workdir = workdir or tempfile.mkdtemp(prefix="oracle_variant_")
+    src = os.path.join(workdir, "variant.c")
+    with open(src, "w") as fh:
+        fh.write(src_text)
+    out = os.path.join(workdir, "libvariant.so")
+    build(src, out, openmp=False)
+    return Oracle(out)
+
+
+def layer_inputs(weights, x):
+    """Convert moe_inputs tensors to the bf16-bit numpy arrays the oracle takes."""
+    import torch  # local: only used to view bf16 tensors as raw bits
+
+    def bits(t):
+        if t is None:
+            return None
+        return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    return dict(x=bits(x), w_router=bits(weights.w_router), w_gate=bits(weights.w_gate),
+                w_up=bits(weights.w_up), w_down=bits(weights.w_down),
+                ws_gate=bits(weights.ws_gate), ws_up=bits(weights.ws_up),
+                ws_down=bits(weights.ws_down))

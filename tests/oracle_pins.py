@@ -1,0 +1,277 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError when the oracle
+disagrees with:
+  * a hand-worked closed-form example (tests/golden/handworked_micro.json),
+  * library special cases (tau=0 is the unmasked dense MoE layer, computed
+    here with torch fp64 softmax/topk/silu/matmul; tau=+inf leaves only the
+    shared expert),
+  * brute-force per-neuron enumeration on tiny inputs,
+  * invariants of the definition (nested masks, exact decomposition of the
+    output difference between two thresholds, the calibrated keep fraction),
+  * a stable-sort ranking of the router probabilities with deliberate ties.
+
+The same pins run against deliberately broken copies of the oracle in
+test_oracle_mutants.py, which shows each plausible mistake fails one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bf16(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _bits(t):
+    return None if t is None else t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _rand_layer(seed, d, E, f, k, S, T, scale_x=1.0):
+    g = torch.Generator().manual_seed(seed)
+
+    def rn(*shape, std):
+        return (torch.randn(*shape, generator=g) * std).to(torch.bfloat16)
+
+    W = dict(w_router=rn(E, d, std=d ** -0.5), w_gate=rn(E, d, f, std=d ** -0.5),
+             w_up=rn(E, d, f, std=d ** -0.5), w_down=rn(E, f, d, std=f ** -0.5))
+    if S:
+        W.update(ws_gate=rn(S, d, f, std=d ** -0.5), ws_up=rn(S, d, f, std=d ** -0.5),
+                 ws_down=rn(S, f, d, std=f ** -0.5))
+    else:
+        W.update(ws_gate=None, ws_up=None, ws_down=None)
+    x = rn(T, d, std=scale_x)
+    return x, W
+
+
+def _call(o, x, W, k, tau):
+    args = {n: _bits(t) for n, t in W.items()}
+    return o.forward(_bits(x), **args, top_k=k, tau=tau)
+
+
+def _torch_dense(x, W, k, with_routed=True, with_shared=True):
+    """The unmasked dense MoE layer from torch fp64 library calls."""
+    xd = x.double()
+    logits = xd @ W["w_router"].double().T
+    p = torch.softmax(logits, dim=-1)
+    # stable descending sort = top-k with ties to the lower index
+    order = np.argsort(-p.numpy(), axis=1, kind="stable")[:, :k]
+    idx = torch.as_tensor(order)
+    y = torch.zeros_like(xd)
+    if with_routed:
+        for t in range(x.shape[0]):
+            for r in range(k):
+                e = int(idx[t, r])
+                g = xd[t] @ W["w_gate"][e].double()
+                u = xd[t] @ W["w_up"][e].double()
+                y[t] += p[t, e] * ((F.silu(g) * u) @ W["w_down"][e].double())
+    if with_shared and W["ws_gate"] is not None:
+        for s in range(W["ws_gate"].shape[0]):
+            g = xd @ W["ws_gate"][s].double()
+            u = xd @ W["ws_up"][s].double()
+            y += (F.silu(g) * u) @ W["ws_down"][s].double()
+    return y.numpy(), idx.numpy(), p.numpy(), logits.numpy()
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ---------------------------------------------------------------- pins
+
+def pin_handworked(o):
+    """Closed-form micro layer worked by hand (golden fixture)."""
+    with open(os.path.join(GOLDEN, "handworked_micro.json")) as fh:
+        G = json.load(fh)
+
+    def sig(z):
+        return 1.0 / (1.0 + math.exp(-z))
+
+    def ev(s):
+        return float(eval(s, {"__builtins__": {}}, {"sig": sig, "inf": math.inf}))
+
+    x = _bf16(G["x"])
+    W = {n: _bf16(G[n]) for n in ("w_router", "w_gate", "w_up", "w_down",
+                                    "ws_gate", "ws_up", "ws_down")}
+    for case in G["cases"]:
+        tau = ev(case["tau"])
+        r = _call(o, x, W, G["top_k"], tau)
+        assert np.array_equal(r.topk_idx, np.array(G["topk_idx"])), ("idx", r.topk_idx)
+        want_w = np.array([[ev(v) for v in row] for row in G["topk_w"]])
+        assert np.allclose(r.topk_w, want_w, rtol=1e-14, atol=0), ("w", r.topk_w, want_w)
+        assert np.array_equal(r.active, np.array(case["active"], dtype=np.uint8)), \
+            ("active", case["tau"], r.active)
+        want_y = np.array([[ev(v) for v in row] for row in case["y"]])
+        assert np.allclose(r.y, want_y, rtol=1e-13, atol=1e-14), ("y", case["tau"], r.y, want_y)
+
+
+def pin_tau0_is_dense(o):
+    """tau = 0 keeps every neuron: the layer is the unmasked dense MoE (torch fp64)."""
+    for seed, S in ((11, 1), (12, 0), (13, 2)):
+        x, W = _rand_layer(seed, d=64, E=6, f=48, k=3, S=S, T=5)
+        r = _call(o, x, W, 3, 0.0)
+        y, idx, p, logits = _torch_dense(x, W, 3)
+        assert np.array_equal(r.topk_idx, idx), ("idx", r.topk_idx, idx)
+        assert _rel(r.y, y) < 1e-12, ("y", _rel(r.y, y))
+        assert r.active.all()
+
+
+def pin_tauinf_is_shared_only(o):
+    """tau = +inf keeps no routed neuron: only the shared experts remain (0 without one)."""
+    for seed, S in ((21, 1), (22, 2), (23, 0)):
+        x, W = _rand_layer(seed, d=64, E=6, f=48, k=2, S=S, T=4)
+        r = _call(o, x, W, 2, math.inf)
+        y, *_ = _torch_dense(x, W, 2, with_routed=False)
+        if S == 0:
+            assert not r.y.any()
+        else:
+            assert _rel(r.y, y) < 1e-12, ("y", _rel(r.y, y))
+        assert not r.active.any()
+
+
+def pin_bruteforce(o):
+    """Per-neuron enumeration with scalar Python arithmetic on a tiny layer."""
+    d, E, f, k, S, T = 16, 4, 8, 2, 1, 3
+    x, W = _rand_layer(31, d, E, f, k, S, T, scale_x=1.0)
+    X = x.float().double().tolist()
+    Wr = W["w_router"].double().tolist()
+    Wg = W["w_gate"].double().tolist()
+    Wu = W["w_up"].double().tolist()
+    Wd = W["w_down"].double().tolist()
+    Sg, Su, Sd = (W["ws_gate"].double().tolist(), W["ws_up"].double().tolist(),
+                  W["ws_down"].double().tolist())
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    # every selected neuron's score, then a threshold that splits them
+    scores, plan = [], []
+    for t in range(T):
+        lg = [sum(X[t][i] * Wr[e][i] for i in range(d)) for e in range(E)]
+        m = max(lg)
+        ex = [math.exp(v - m) for v in lg]
+        p = [v / sum(ex) for v in ex]
+        chosen = sorted(range(E), key=lambda e: (-p[e], e))[:k]
+        for e in chosen:
+            for j in range(f):
+                g = sum(X[t][i] * Wg[e][i][j] for i in range(d))
+                u = sum(X[t][i] * Wu[e][i][j] for i in range(d))
+                scores.append(abs(silu(g)))
+                plan.append((t, e, j, p[e], silu(g) * u))
+    tau = float(np.float32(sorted(scores)[len(scores) // 2] * 1.0001))
+    y = [[0.0] * d for _ in range(T)]
+    act = {}
+    for (t, e, j, pe, h), s in zip(plan, scores):
+        on = np.float32(s) >= np.float32(tau)
+        act[(t, e, j)] = on
+        if on:
+            for i in range(d):
+                y[t][i] += pe * h * Wd[e][j][i]
+    for t in range(T):
+        for s_ in range(S):
+            for j in range(f):
+                g = sum(X[t][i] * Sg[s_][i][j] for i in range(d))
+                u = sum(X[t][i] * Su[s_][i][j] for i in range(d))
+                for i in range(d):
+                    y[t][i] += silu(g) * u * Sd[s_][j][i]
+    r = _call(o, x, W, k, tau)
+    for t in range(T):
+        for r_ in range(k):
+            e = int(r.topk_idx[t, r_])
+            for j in range(f):
+                assert bool(r.active[t, r_, j]) == bool(act[(t, e, j)]), ("active", t, e, j)
+    assert _rel(r.y, np.array(y)) < 1e-12, ("y", _rel(r.y, np.array(y)))
+
+
+def pin_nested_masks(o):
+    """tau1 < tau2  =>  A(tau2) is a subset of A(tau1), for every pair."""
+    x, W = _rand_layer(41, d=64, E=8, f=64, k=2, S=1, T=6)
+    prev = None
+    for tau in (0.0, 0.1, 0.5, 1.0, 2.0, math.inf):
+        r = _call(o, x, W, 2, tau)
+        if prev is not None:
+            assert np.array_equal(r.topk_idx, prev.topk_idx)
+            assert not np.any(r.active & ~prev.active), ("not nested at", tau)
+        prev = r
+
+
+def pin_threshold_decomposition(o):
+    """y(t1) - y(t2) equals the sum of the contributions of neurons with t1 <= s < t2."""
+    d, E, f, k, S, T = 48, 5, 40, 2, 1, 4
+    x, W = _rand_layer(51, d, E, f, k, S, T)
+    t1, t2 = 0.3, 0.9
+    r1, r2 = _call(o, x, W, k, t1), _call(o, x, W, k, t2)
+    xd = x.double()
+    p = torch.softmax(xd @ W["w_router"].double().T, dim=-1).numpy()
+    diff = np.zeros((T, d))
+    for t in range(T):
+        for r_ in range(k):
+            e = int(r1.topk_idx[t, r_])
+            g = (xd[t] @ W["w_gate"][e].double())
+            u = (xd[t] @ W["w_up"][e].double())
+            a = F.silu(g).numpy()
+            s32 = np.abs(a).astype(np.float32)
+            band = (s32 >= np.float32(t1)) & (s32 < np.float32(t2))
+            h = a * u.numpy() * band
+            diff[t] += p[t, e] * (h @ W["w_down"][e].double().numpy())
+    got = r1.y - r2.y
+    assert _rel(got, diff) < 1e-10, ("decomposition", _rel(got, diff))
+
+
+def pin_router_ranking(o):
+    """Router weights are softmax(x Wr^T)[top-k]; ties go to the lower expert index."""
+    d, E, f, k, T = 32, 8, 16, 3, 6
+    x, W = _rand_layer(61, d, E, f, k, 0, T)
+    wr = W["w_router"].clone()
+    wr[5] = wr[1]          # experts 1 and 5 always tie
+    wr[6] = wr[2]          # experts 2 and 6 always tie
+    W["w_router"] = wr
+    r = _call(o, x, W, k, 0.5)
+    logits = (x.double() @ wr.double().T).numpy()
+    assert np.allclose(r.logits, logits, rtol=1e-13, atol=1e-13), "logits"
+    p = torch.softmax(torch.as_tensor(logits), dim=-1).numpy()
+    assert np.allclose(p.sum(1), 1.0, atol=1e-12)
+    want = np.argsort(-p, axis=1, kind="stable")[:, :k]
+    assert np.array_equal(r.topk_idx, want), ("idx", r.topk_idx, want)
+    assert np.allclose(r.topk_w, np.take_along_axis(p, want, 1), rtol=1e-13, atol=0), "w"
+    # the routing weight is softmax over all E, not renormalised over the top-k
+    assert np.all(r.topk_w.sum(1) < 1.0 - 1e-6)
+
+
+def pin_calibration(o):
+    """tau(q) = floor(q N)-th order statistic; kept fraction within 1/N of 1 - q."""
+    rng = np.random.default_rng(71)
+    s = np.abs(rng.standard_normal(10007))
+    for q in (0.0, 0.5, 0.8, 0.9, 0.95, 0.98):
+        tau64 = o._lib.oracle_calibrate_tau(o._ptr(s), s.size, q)
+        if q == 0.0:
+            assert tau64 == 0.0
+            continue
+        assert tau64 == np.partition(s, int(math.floor(q * s.size)))[int(math.floor(q * s.size))]
+        keep = float(np.mean(s >= tau64))
+        assert abs(keep - (1 - q)) <= 1.0 / s.size + 1e-15, (q, keep)
+    assert math.isinf(o._lib.oracle_calibrate_tau(o._ptr(s), s.size, 1.0))
+
+
+ALL_PINS = [pin_handworked, pin_tau0_is_dense, pin_tauinf_is_shared_only, pin_bruteforce,
+            pin_nested_masks, pin_threshold_decomposition, pin_router_ranking, pin_calibration]
+
+
+def run_all(o):
+    """Run every pin; return {name: None (passed) | error text}."""
+    out = {}
+    for pin in ALL_PINS:
+        try:
+            pin(o)
+            out[pin.__name__] = None
+        except Exception as exc:  # noqa: BLE001 - a mutant may fail in any way
+            out[pin.__name__] = f"{type(exc).__name__}: {str(exc)[:200]}"
+    return out
