@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE layer with intra-expert activation sparsity.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload olmoe] [--T 16] [--sparsity 0.9] [--no-sweep]
+
+One step is one forward of the whole layer (router + bucketing, gate
+projection, threshold mask and compaction, gathered up/down projection,
+shared experts, combine) over one batch of T synthetic tokens already
+resident in HBM.  The default workload is the OLMoE-shaped decode layer
+(d_model 2048, 64 experts, d_ff 1024, top-8, no shared expert) at T = 16 with
+tau calibrated on the GPU for 90% sparsity.  L2 is flushed (a write of twice
+its size) before every timed step, outside the step's CUDA events.
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
+replica of the layer on its own GPU ("replicas only": the layer has no
+exchange step); the step time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the plain fp64 definition of the
+layer) on the host cores instead -- rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "routed-MoE layer tokens/s and HBM GB/s (% roofline) at 90% intra-expert sparsity"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD_TEXT = {
+    "olmoe": "OLMoE-shaped decode layer: d_model=2048, 64 routed SwiGLU experts, d_ff=1024, "
+             "top-8 softmax router, no shared expert, bf16 weights ~N(0,1/fan_in)",
+    "dsv2lite": "DeepSeek-V2-Lite-shaped decode layer: d_model=2048, 64 routed experts d_ff=1408, "
+                "top-6, 2 dense shared experts d_ff=1408",
+    "large": "large sparse-routed decode layer: d_model=4096, 256 routed experts d_ff=1024, top-8, "
+             "1 dense shared expert d_ff=1024 (6.44 GB of expert weights)",
+    "tiny": "tiny MoE layer: d_model=256, 8 experts d_ff=512, top-2, 1 shared expert",
+    "crossover": "OLMoE shapes for the sparse/dense crossover sweep",
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="olmoe")
+    p.add_argument("--T", type=int, default=16)
+    p.add_argument("--sparsity", type=float, default=0.9)
+    p.add_argument("--path", choices=["auto", "sparse", "dense"], default="auto")
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    return p.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as fh:
+            return json.load(fh), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def recorded_traffic(kernel, workload_key):
+    """DRAM bytes per launch from a committed ncu summary, if its source hash still matches."""
+    path = os.path.join(HERE, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    want_sha = kernel_source_sha()
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) == 4 and parts[0] == kernel and parts[1] == workload_key and parts[2] == want_sha:
+            return float(parts[3])
+    return None
+
+
+def kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(HERE, "intra_expert_activation_router_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:12]
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_id)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:  # noqa: BLE001
+        return str(dev)
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_time_sample(shape, W_host, x_host, T, target_s, nthreads):
+    """The CPU oracle on repeats of the batch for about target_s seconds (rank 0, N=1)."""
+    import oracle
+    o = oracle.Oracle()
+    inputs = oracle.layer_inputs(W_host, x_host)
+    t0 = time.perf_counter()
+    o.forward(**inputs, top_k=shape.top_k, tau=1.0, want_scores=False, nthreads=nthreads)
+    one = time.perf_counter() - t0
+    reps = max(1, min(500, int(math.ceil(target_s / max(one, 1e-6)))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        o.forward(**inputs, top_k=shape.top_k, tau=1.0, want_scores=False, nthreads=nthreads)
+    el = time.perf_counter() - t0
+    return reps * T / el, reps, el
+
+
+def run_reference(args):
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return
+    import torch
+    import moe_inputs as mi
+    import oracle
+    shape = mi.SHAPES[args.workload]
+    W = mi.make_weights(shape, device="cpu")
+    x = mi.make_x(shape, args.T, device="cpu")
+    o = oracle.Oracle()
+    inputs = oracle.layer_inputs(W, x)
+    cores = cpu_cores()
+    # tau of the batch, then size each step's token sample so the run stays short
+    r = o.forward(**inputs, top_k=shape.top_k, tau=math.inf, nthreads=cores)
+    tau = o.calibrate_tau(r.score, args.sparsity)
+    t0 = time.perf_counter()
+    o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+    full = time.perf_counter() - t0
+    budget = 150.0
+    n_tok = args.T
+    if (args.steps + args.warmup) * full > budget:
+        n_tok = max(1, int(args.T * budget / ((args.steps + args.warmup) * full)))
+    sub = dict(inputs)
+    sub["x"] = inputs["x"][:n_tok]
+    for _ in range(args.warmup):
+        o.forward(**sub, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        o.forward(**sub, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+        times.append(time.perf_counter() - t0)
+    ms = 1000 * statistics.mean(times)
+    value = n_tok / (ms / 1000)
+    sample = f"{n_tok} of the {args.T} tokens per step, {args.steps} steps"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": args.T,
+                   "sparsity": args.sparsity, "tau": tau},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def time_steps(layer, x, tau, out, flush, steps, events=True, dense=False):
+    """Per-step CUDA-event timing with an L2 flush before each step (outside the events)."""
+    import torch
+    from intra_expert_activation_router_b200 import moe_set_launch_events
+    st = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for trio in kev:   # create the CUDA events before the library records them
+        for e in trio:
+            e.record(st)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(st)
+        if events:
+            moe_set_launch_events(layer.h, kev[i])
+        if dense:
+            layer.dense_forward(x, out=out)
+        else:
+            layer.forward(x, tau, out=out)
+        ends[i].record(st)
+    moe_set_launch_events(layer.h, None)
+    torch.cuda.synchronize()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    router_ms = [t[0].elapsed_time(t[1]) for t in kev]
+    expert_ms = [t[1].elapsed_time(t[2]) for t in kev]
+    return step_ms, router_ms, expert_ms
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    dev = torch.device("cuda", local)
+    shape = mi.SHAPES[args.workload]
+    T = args.T
+    sweep_T = [] if args.no_sweep or world > 1 else [t for t in shape.t_values]
+    max_tokens = max([T] + sweep_T + [64])
+    W = mi.make_weights(shape, device=dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max_tokens)
+    if args.path != "auto":
+        layer.set_path({"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
+    x = mi.make_x(shape, T, device=dev)
+    out = torch.empty_like(x)
+    tau = layer.calibrate_tau(x, args.sparsity)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        layer.forward(x, tau, out=out)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        step_ms, router_ms, expert_ms = time_steps(layer, x, tau, out, flush, args.steps)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1000)
+    st = layer.stats()
+    path = "sparse" if st["path"] == m.MOE_PATH_SPARSE else "dense"
+    alg = st["alg_bytes"] if path == "sparse" else st["dense_bytes"]
+    router_bytes = shape.n_experts * shape.d_model * 2 + T * shape.d_model * 2
+    expert_bytes = alg - router_bytes
+    expert_ms_mean = statistics.mean(expert_ms)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = expert_bytes / (expert_ms_mean / 1000) / 1e9
+    kname = "k_expert_sparse" if path == "sparse" else "k_dense"
+    traffic = recorded_traffic(kname, f"{args.workload}:T={T}")
+
+    # end to end through the host-pointer entry: pinned x in, pinned out back, every step
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    e2e_steps = min(args.steps, 50)
+    e2e_t = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        m.moe_sparse_forward_host(layer.h, xh, T, tau, oh)
+        e2e_t.append(time.perf_counter() - t0)
+    e2e_total = sum(e2e_t)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = world * T * e2e_steps / e2e_total
+
+    sweep = []
+    if rank == 0 and sweep_T:
+        for Ts in sweep_T:
+            xs = mi.make_x(shape, Ts, device=dev)
+            outs = torch.empty_like(xs)
+            taus = layer.calibrate_tau(xs, args.sparsity)
+            row = {"T": Ts, "tau": taus}
+            for mode in ("sparse", "dense"):
+                try:
+                    layer.set_path(m.MOE_PATH_SPARSE if mode == "sparse" else m.MOE_PATH_DENSE)
+                except m.MoeError:
+                    row[f"{mode}_us"] = None
+                    continue
+                for _ in range(3):
+                    layer.forward(xs, taus, out=outs)
+                sm_, rm_, em_ = time_steps(layer, xs, taus, outs, flush, 30)
+                s2 = layer.stats()
+                b = s2["alg_bytes"] if mode == "sparse" else s2["dense_bytes"]
+                row[f"{mode}_us"] = 1000 * statistics.mean(sm_)
+                row[f"{mode}_expert_us"] = 1000 * statistics.mean(em_)
+                row[f"{mode}_alg_bytes"] = b
+                row[f"{mode}_gbs"] = b / (statistics.mean(sm_) / 1000) / 1e9
+            layer.set_path(m.MOE_PATH_AUTO if args.path == "auto" else
+                           {"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
+            sweep.append(row)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = cpu_cores()
+        W_host = W.to("cpu")
+        tps, reps, el = oracle_time_sample(shape, W_host, x.cpu(), T, args.cpu_seconds, cores)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{reps} repeats of the {T}-token batch ({el:.1f} s, fp64 oracle, "
+                         f"OpenMP over tokens)"}
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": T,
+                       "sparsity": args.sparsity, "tau": tau, "path": path,
+                       "parallelism": f"replicas{world}",
+                       "l2": "flushed before every timed step (2x L2 written outside the step events)"},
+            "hbm_gbs": alg / (ms / 1000) / 1e9,
+            "latency_us": 1000 * ms,
+            "alg_bytes_per_step": alg,
+            "kernels_us": {"router": 1000 * statistics.mean(router_ms), kname: 1000 * expert_ms_mean},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "alg_bytes_per_launch": expert_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * shape.d_model * 2,
+                    "d2h_bytes_per_step": T * shape.d_model * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"]},
+            "stats": {"n_touched": st["n_touched"], "n_active": st["n_active"], "n_union": st["n_union"]},
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

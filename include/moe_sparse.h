@@ -1,0 +1,176 @@
+/*
+ * moe_sparse.h -- C ABI of the routed-expert MoE layer with intra-expert
+ * activation sparsity, for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Uncovering Intra-expert Activation Sparsity for Efficient
+ * Mixture-of-Expert Model Execution", technical summary, Methodology item 3;
+ * Hindi summary of the same paper, "How they did it: the skip-list system"):
+ * per token x (d_model values),
+ *
+ *   router     p = softmax(x Wr^T) over all E experts; the top_k experts by p
+ *              are selected (ties go to the lower index); weight w_e = p_e
+ *              (the router is kept unchanged; no renormalisation).
+ *   gate       g = x Wg[e]                      dense, every neuron of e
+ *   mask       neuron j active iff |silu(g_j)| >= tau    one pass, no sort
+ *   up/down    y += w_e * sum_{j active} silu(g_j) (x Wu[e][:,j]) Wd[e][j][:]
+ *   shared     y += sum_j silu(x Ws_g[:,j]) (x Ws_u[:,j]) Ws_d[j][:]
+ *              for each shared expert, every neuron, unweighted.
+ *   out        bf16(y), round to nearest even.
+ *
+ * Conventions for every function:
+ *   - bf16 tensors are passed as raw 16-bit patterns (any bf16 type works).
+ *   - "device pointer" means memory of the current CUDA device, "host
+ *     pointer" ordinary (pageable or pinned) host memory.
+ *   - `stream` is a cudaStream_t cast to void* (NULL = the legacy default
+ *     stream).  All work is enqueued on it; calls return once it is enqueued
+ *     unless stated otherwise.
+ *   - Every function returns MOE_OK (0) or a negative MOE_E* code; argument
+ *     errors are detected on the host before anything is launched.  No C++
+ *     exception crosses this boundary.
+ *   - A handle must only be used from one host thread at a time and only on
+ *     the device that was current when it was created.
+ */
+#ifndef MOE_SPARSE_H
+#define MOE_SPARSE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_EINVAL (-1)   /* bad size, NULL pointer, NaN tau, ...            */
+#define MOE_ENOMEM (-2)   /* device or host allocation failed (create only)  */
+#define MOE_ECUDA (-3)    /* a CUDA runtime call or kernel launch failed     */
+#define MOE_EALIGN (-4)   /* a pointer is not 16-byte aligned                */
+#define MOE_EHANDLE (-5)  /* NULL or destroyed handle                        */
+#define MOE_EDEVICE (-6)  /* a kernel reported an error word (e.g. a bounded
+                             wait ran out); the handle stays usable           */
+#define MOE_ENOTSUP (-7)  /* shape or path not supported by this build       */
+
+/* Path selection (moe_set_path). */
+#define MOE_PATH_AUTO 0    /* sparse gather path for T <= T*, dense above   */
+#define MOE_PATH_SPARSE 1  /* always the sparse gather path                 */
+#define MOE_PATH_DENSE 2   /* always the tensor-core grouped GEMM, masked    */
+
+typedef struct moe_sparse_s *moe_handle;
+
+/* Layer weights, all DEVICE pointers to bf16, caller-owned, x @ W layout:
+ *   w_router [E][d_model]
+ *   w_gate   [E][d_model][d_ff]      w_up [E][d_model][d_ff]
+ *   w_down   [E][d_ff][d_model]
+ *   ws_gate, ws_up [n_shared][d_model][d_ff], ws_down [n_shared][d_ff][d_model]
+ *   (ws_* must be NULL when n_shared == 0; the shared d_ff equals d_ff).
+ * Every pointer must be 16-byte aligned. */
+typedef struct {
+    const void *w_router;
+    const void *w_gate;
+    const void *w_up;
+    const void *w_down;
+    const void *ws_gate;
+    const void *ws_up;
+    const void *ws_down;
+} moe_weights;
+
+/* Statistics of the last forward on a handle (moe_query_stats). */
+typedef struct {
+    int path;              /* MOE_PATH_SPARSE or MOE_PATH_DENSE                 */
+    int n_tokens;          /* T                                                  */
+    int n_touched;         /* distinct routed experts selected by the batch      */
+    int t_star;            /* current sparse/dense switch point                  */
+    long long n_active;    /* sum over (token, expert) pairs of active neurons   */
+    long long n_union;     /* sum over touched experts of the union of their
+                              tokens' active neurons (rows of Wu/Wd read)        */
+    double alg_bytes;      /* algorithmic HBM bytes of the sparse path:
+                              full Wg of touched experts + 2*d_model*2 bytes per
+                              union-active neuron + shared experts + router +
+                              x and out                                          */
+    double dense_bytes;    /* the same for the dense path (all neurons)          */
+    int device_error;      /* last error word read back from the device (0 ok)  */
+} moe_stats;
+
+/* Create a layer.  Copies and repacks the weights into library-owned device
+ * memory (the caller may free its tensors afterwards) and allocates all
+ * workspace for up to `max_tokens` tokens per call, so that forward calls
+ * never allocate.  Synchronises the device before returning.
+ * Requirements (else MOE_EINVAL): 1 <= top_k <= E <= 1024; d_model >= 8 and
+ * d_model % 8 == 0; d_ff >= 32 and d_ff % 32 == 0; d_ff <= 65535;
+ * 0 <= n_shared <= 8; 1 <= max_tokens <= 65536 (0 selects 4096).
+ * Pointers must be 16-byte aligned (else MOE_EALIGN).  On failure *out is
+ * set to NULL and nothing is leaked. */
+int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_model, int d_ff,
+                      int n_shared, int max_tokens, moe_handle *out);
+
+/* The masked layer.  x: DEVICE [T][d_model] bf16; out: DEVICE [T][d_model]
+ * bf16 (may not alias x).  1 <= T <= max_tokens.  tau <= 0 keeps every
+ * neuron, tau = +inf keeps none; NaN tau is MOE_EINVAL.  The path follows
+ * moe_set_path (AUTO by default: sparse for T <= T*, the dense masked GEMM
+ * above).  Both paths give the same layer up to rounding.  Asynchronous. */
+int moe_sparse_forward(moe_handle h, const void *x, int T, float tau, void *out, void *stream);
+
+/* The unmasked layer (every neuron active) on the dense tensor-core path:
+ * the baseline the sparse path is measured against.  Same arguments and
+ * rules as moe_sparse_forward without tau. */
+int moe_dense_forward(moe_handle h, const void *x, int T, void *out, void *stream);
+
+/* Same as moe_sparse_forward but x and out are HOST pointers: copies x in,
+ * runs the layer and copies out back on `stream`, then synchronises it. */
+int moe_sparse_forward_host(moe_handle h, const void *x_host, int T, float tau, void *out_host,
+                            void *stream);
+
+/* Free everything the handle owns (synchronises the device first).  NULL is
+ * ignored; the handle must not be used afterwards. */
+void moe_sparse_destroy(moe_handle h);
+
+/* Force a path (MOE_PATH_*) for subsequent forwards; MOE_EINVAL otherwise. */
+int moe_set_path(moe_handle h, int path);
+
+/* Set the switch point T* of MOE_PATH_AUTO (sparse iff T <= t_star). */
+int moe_set_t_star(moe_handle h, int t_star);
+
+/* Router only: idx_out [T][top_k] int32 and w_out [T][top_k] fp32, both
+ * DEVICE pointers, in rank order.  Asynchronous. */
+int moe_debug_router(moe_handle h, const void *x, int T, int *idx_out, float *w_out, void *stream);
+
+/* Runs the sparse path and writes each (token, rank) pair's active-neuron
+ * list: idx_out DEVICE [T][top_k][d_ff] uint16, ascending, the first
+ * cnt_out[t][r] entries valid; cnt_out DEVICE [T][top_k] int32.  out may be
+ * NULL (the layer output is then discarded).  Asynchronous. */
+int moe_debug_active(moe_handle h, const void *x, int T, float tau, uint16_t *idx_out,
+                     int *cnt_out, void *out, void *stream);
+
+/* Threshold for a target sparsity q in [0, 1]: runs the router and the gate
+ * projection for x (DEVICE [T][d_model] bf16) and stores in *tau_out (HOST
+ * pointer) the floor(q*N)-th smallest score |silu(g)| (0-based, exact
+ * selection) among the N = T*top_k*d_ff scores of the (token, expert) pairs the
+ * router selects; shared experts are excluded.  q <= 0 gives 0 and
+ * floor(q*N) >= N gives +inf.  About 1 - q of the routed neurons then have
+ * s >= tau ("Uncovering Intra-expert Activation Sparsity...", Results:
+ * per-model sparsity cutoffs are set as a fraction of neurons kept).
+ * The first call allocates a score buffer of max_tokens*top_k*d_ff floats
+ * that the handle keeps (MOE_ENOMEM if that fails).  Synchronises `stream`. */
+int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
+                      void *stream);
+
+/* Timing hook for benchmarks: on every later forward, record caller-owned CUDA
+ * events (cudaEvent_t cast to void*, created on the handle's device) on the
+ * forward's stream -- events[0] before the router kernel, events[1] between
+ * the router and the expert kernel(s), events[2] after them.  n must be 3;
+ * events == NULL or n == 0 stops recording.  The handle keeps the three
+ * handles, not the array. */
+int moe_set_launch_events(moe_handle h, void *const *events, int n);
+
+/* Statistics of the last forward.  Synchronises the stream of that forward
+ * and reads device counters back; not for timed loops.  A nonzero device
+ * error word is reported in st->device_error and as MOE_EDEVICE. */
+int moe_query_stats(moe_handle h, moe_stats *st);
+
+/* Static English text for an error code. */
+const char *moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_SPARSE_H */

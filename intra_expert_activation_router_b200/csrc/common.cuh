@@ -1,0 +1,117 @@
+// common.cuh -- small device helpers shared by the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// 16-byte streaming load of weights: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ld_stream(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte read-only load that may be cached (activations reused by many warps).
+__device__ __forceinline__ uint4 ld_cached(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// bf16 pair (low half = element 0) -> two floats.  Exact widening.
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
+{
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+    f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+__device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b, float acc)
+{
+    acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);
+    acc = fmaf(bf16_hi(a.x), bf16_hi(b.x), acc);
+    acc = fmaf(bf16_lo(a.y), bf16_lo(b.y), acc);
+    acc = fmaf(bf16_hi(a.y), bf16_hi(b.y), acc);
+    acc = fmaf(bf16_lo(a.z), bf16_lo(b.z), acc);
+    acc = fmaf(bf16_hi(a.z), bf16_hi(b.z), acc);
+    acc = fmaf(bf16_lo(a.w), bf16_lo(b.w), acc);
+    acc = fmaf(bf16_hi(a.w), bf16_hi(b.w), acc);
+    return acc;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+// Reduce N per-lane partial sums across the warp with N-1 + (5-log2 N)
+// shuffles instead of 5N: each step hands half of the remaining values to
+// the partner lane.  On return, lane l holds the full sum of value index
+// (l >> (5 - log2 N)).  N must be a power of two <= 32.  The recursion keeps
+// every array index a compile-time constant, so v stays in registers.
+template <int M, int N, int O>
+struct TransposeReduce {
+    static __device__ __forceinline__ void run(float (&v)[M], int lane)
+    {
+        if constexpr (O == 0) {
+            return;
+        } else if constexpr (N > 1) {
+            const bool upper = (lane & O) != 0;
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                const float send = upper ? v[i] : v[i + N / 2];
+                const float keep = upper ? v[i + N / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(kFull, send, O);
+            }
+            TransposeReduce<M, N / 2, O / 2>::run(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(kFull, v[0], O);
+            TransposeReduce<M, 1, O / 2>::run(v, lane);
+        }
+    }
+};
+
+template <int N>
+__device__ __forceinline__ float transpose_reduce(float (&v)[N], int lane)
+{
+    static_assert(N >= 1 && N <= 32 && (N & (N - 1)) == 0, "N must be a power of two <= 32");
+    TransposeReduce<N, N, 16>::run(v, lane);
+    return v[0];
+}
+
+template <int N>
+struct Log2 { static constexpr int value = 1 + Log2<N / 2>::value; };
+template <>
+struct Log2<1> { static constexpr int value = 0; };
+
+__device__ __forceinline__ float silu_f(float g)
+{
+    return g / (1.0f + expf(-g));
+}
+
+__device__ __forceinline__ uint16_t f2bf_bits(float v)
+{
+    __nv_bfloat16 b = __float2bfloat16_rn(v);
+    return *reinterpret_cast<uint16_t *>(&b);
+}
+
+}  // namespace moe

@@ -1,0 +1,133 @@
+// misc.cu -- weight repacking, active-list compaction and last-call statistics.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// dst[b][c][r] = src[b][r][c]   (bf16 bits), 32x32 tiles through shared memory.
+__global__ void k_transpose(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, int rows,
+                            int cols)
+{
+    __shared__ uint16_t tile[32][33];
+    const size_t base = (size_t)blockIdx.z * rows * cols;
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[i][threadIdx.x] = src[base + (size_t)r * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) dst[base + (size_t)c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+
+cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows,
+                                    int cols, cudaStream_t st)
+{
+    dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches);
+    k_transpose<<<grid, dim3(32, 8), 0, st>>>(src, dst, rows, cols);
+    return cudaGetLastError();
+}
+
+// Mask words -> ascending active-neuron lists, one warp per (token, rank) pair:
+// a warp-wide exclusive scan of the words' popcounts places each word's bits.
+__global__ void k_mask_compact(const uint32_t *__restrict__ mask, int n_pairs, int words,
+                               uint16_t *__restrict__ idx_out, int *__restrict__ cnt_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (p >= n_pairs) return;
+    const uint32_t *row = mask + (size_t)p * words;
+    uint16_t *out = idx_out + (size_t)p * words * 32;
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        const uint32_t wv = (w0 + lane < words) ? row[w0 + lane] : 0u;
+        const int c = __popc(wv);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pos = base + incl - c;
+        for (uint32_t b = wv; b; b &= b - 1) out[pos++] = (uint16_t)((w0 + lane) * 32 + __ffs(b) - 1);
+        base += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) cnt_out[p] = base;
+}
+
+cudaError_t launch_mask_compact(const Workspace &ws, int n_pairs, int f, uint16_t *idx_out,
+                                int *cnt_out, cudaStream_t st)
+{
+    const int per_block = 8;
+    k_mask_compact<<<(n_pairs + per_block - 1) / per_block, 32 * per_block, 0, st>>>(
+        ws.mask, n_pairs, f / 32, idx_out, cnt_out);
+    return cudaGetLastError();
+}
+
+// out[0] += active neurons over all pairs, out[1] += union-active neurons over
+// touched experts, out[2] = touched experts.  One CTA per expert slot.
+__global__ void k_stats(Plan *plan, const int *perm, const uint32_t *mask, int words,
+                        unsigned long long *out)
+{
+    const int slot = blockIdx.x;
+    if (slot >= plan->n_touched) return;
+    const int e = plan->touched[slot];
+    const int b = plan->offsets[e], n = plan->offsets[e + 1] - b;
+    unsigned long long act = 0, uni = 0;
+    for (int w = threadIdx.x; w < words; w += blockDim.x) {
+        uint32_t u = 0;
+        for (int i = 0; i < n; ++i) {
+            const uint32_t v = mask[(size_t)perm[b + i] * words + w];
+            act += __popc(v);
+            u |= v;
+        }
+        uni += __popc(u);
+    }
+    atomicAdd(&out[0], act);
+    atomicAdd(&out[1], uni);
+    if (slot == 0 && threadIdx.x == 0) out[2] = plan->n_touched;
+}
+
+cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned long long *out3,
+                         cudaStream_t st)
+{
+    (void)T;
+    cudaError_t e = cudaMemsetAsync(out3, 0, 3 * sizeof(unsigned long long), st);
+    if (e != cudaSuccess) return e;
+    k_stats<<<dm.E, 128, 0, st>>>(ws.plan, ws.perm, ws.mask, dm.f / 32, out3);
+    return cudaGetLastError();
+}
+
+// One pass of an exact radix select over non-negative float bit patterns
+// (their uint32 order is their numeric order): histogram of the 8-bit digit
+// at `shift` among the values whose higher digits equal `prefix`.
+__global__ void k_radix_hist(const uint32_t *__restrict__ v, size_t n, uint32_t prefix,
+                             uint32_t prefix_mask, int shift, unsigned *__restrict__ hist)
+{
+    __shared__ unsigned sh[256];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const uint32_t u = v[i];
+        if ((u & prefix_mask) == prefix) atomicAdd(&sh[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (sh[i]) atomicAdd(&hist[i], sh[i]);
+}
+
+cudaError_t launch_radix_hist(const uint32_t *v, size_t n, uint32_t prefix, uint32_t prefix_mask,
+                              int shift, unsigned *hist, int n_sm, cudaStream_t st)
+{
+    cudaError_t e = cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned), st);
+    if (e != cudaSuccess) return e;
+    size_t blocks = (n + 255) / 256;
+    if (blocks > (size_t)n_sm * 8) blocks = (size_t)n_sm * 8;
+    if (blocks < 1) blocks = 1;
+    k_radix_hist<<<(unsigned)blocks, 256, 0, st>>>(v, n, prefix, prefix_mask, shift, hist);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

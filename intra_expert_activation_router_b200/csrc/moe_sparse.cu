@@ -1,0 +1,428 @@
+// moe_sparse.cu -- the C ABI (include/moe_sparse.h): argument checking,
+// weight repacking, workspace ownership and path dispatch.
+#include <climits>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <set>
+
+#include "../../include/moe_sparse.h"
+#include "internal.h"
+
+namespace moe {
+int sparse_blocks_per_sm(int mt);
+bool dense_path_available();
+cudaError_t launch_dense(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
+                         const uint16_t *x, int T, float tau, bool use_mask, uint16_t *out,
+                         int n_sm, cudaStream_t st);
+}
+
+namespace {
+
+constexpr unsigned kMagic = 0x4d6f4553u;   // "MoES"
+
+struct Block {   // bump allocator over one cudaMalloc
+    char *base = nullptr;
+    size_t used = 0, cap = 0;
+    void *take(size_t bytes)
+    {
+        size_t off = (used + 255) & ~size_t(255);
+        if (off + bytes > cap) return nullptr;
+        used = off + bytes;
+        return base + off;
+    }
+};
+
+}  // namespace
+
+struct moe_sparse_s {
+    unsigned magic;
+    int device;
+    int n_sm;
+    moe::Dims dm;
+    moe::DeviceWeights w;
+    moe::Workspace ws;
+    unsigned long long *stats_dev;
+    void *weight_mem;
+    void *ws_mem;
+    int path;
+    int t_star;
+    int grid_cap[4];   // sparse kernel CTAs that fit at once, per token-tile size
+    // the last forward
+    int last_T, last_path, last_masked;
+    cudaStream_t last_stream;
+    cudaEvent_t ev[3];   // optional launch events (moe_set_launch_events)
+    int n_ev;
+    float *scores;       // calibration buffer, allocated by the first moe_calibrate_tau
+    unsigned *hist;      // 256 bins, inside the workspace
+};
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Live handles, so that a NULL, foreign or destroyed handle is an error code
+// rather than a dereference of freed memory.
+static std::mutex g_live_mu;
+static std::set<moe_handle> g_live;
+
+static bool is_live(moe_handle h)
+{
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    return h && g_live.count(h) && h->magic == kMagic;
+}
+
+static int check_handle(moe_handle h)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ECUDA;
+    if (dev != h->device) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+static void free_handle(moe_handle h)
+{
+    if (!h) return;
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        g_live.erase(h);
+    }
+    cudaDeviceSynchronize();
+    if (h->weight_mem) cudaFree(h->weight_mem);
+    if (h->ws_mem) cudaFree(h->ws_mem);
+    if (h->scores) cudaFree(h->scores);
+    h->magic = 0;
+    delete h;
+}
+
+static int mt_index(int mt) { return mt <= 1 ? 0 : mt <= 2 ? 1 : mt <= 4 ? 2 : 3; }
+
+extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_model, int d_ff,
+                                 int n_shared, int max_tokens, moe_handle *out)
+{
+    if (!out) return MOE_EINVAL;
+    *out = nullptr;
+    if (!w) return MOE_EINVAL;
+    if (max_tokens == 0) max_tokens = 4096;
+    if (E < 1 || E > moe::kMaxExperts || top_k < 1 || top_k > E) return MOE_EINVAL;
+    if (d_model < 8 || d_model % 8 != 0) return MOE_EINVAL;
+    if (d_ff < 32 || d_ff % 32 != 0 || d_ff > 65535) return MOE_EINVAL;
+    if (n_shared < 0 || n_shared > 8 || max_tokens < 1 || max_tokens > 65536) return MOE_EINVAL;
+    if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_EINVAL;
+    const bool any_shared = w->ws_gate || w->ws_up || w->ws_down;
+    const bool all_shared = w->ws_gate && w->ws_up && w->ws_down;
+    if (n_shared > 0 ? !all_shared : any_shared) return MOE_EINVAL;
+    const void *ptrs[7] = {w->w_router, w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return MOE_EALIGN;
+
+    moe_handle h = new (std::nothrow) moe_sparse_s();
+    if (!h) return MOE_ENOMEM;
+    h->magic = kMagic;
+    h->path = MOE_PATH_AUTO;
+    h->t_star = moe::dense_path_available() ? 128 : INT_MAX;
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+        delete h;
+        return MOE_ECUDA;
+    }
+    moe::Dims &dm = h->dm;
+    dm.E = E; dm.k = top_k; dm.d = d_model; dm.f = d_ff; dm.S = n_shared; dm.max_tokens = max_tokens;
+    for (int i = 0; i < 4; ++i) h->grid_cap[i] = h->n_sm * moe::sparse_blocks_per_sm(1 << i);
+
+    const size_t fd = (size_t)d_ff * d_model;
+    const size_t wbytes = 2 * ((size_t)E * d_model + 3 * E * fd + 3 * (size_t)n_shared * fd) + 16 * 256;
+    const size_t T = max_tokens, P = T * top_k;
+    const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
+                           4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * P * d_model +
+                           2 * P * d_ff + 2 * 2 * T * d_model + 64 + 1024 + 32 * 256;
+    if (cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
+    if (cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
+
+    Block wb{(char *)h->weight_mem, 0, wbytes};
+    uint16_t *wr = (uint16_t *)wb.take(2 * (size_t)E * d_model);
+    uint16_t *wg = (uint16_t *)wb.take(2 * E * fd), *wu = (uint16_t *)wb.take(2 * E * fd);
+    uint16_t *wd = (uint16_t *)wb.take(2 * E * fd);
+    uint16_t *wsg = nullptr, *wsu = nullptr, *wsd = nullptr;
+    if (n_shared) {
+        wsg = (uint16_t *)wb.take(2 * n_shared * fd);
+        wsu = (uint16_t *)wb.take(2 * n_shared * fd);
+        wsd = (uint16_t *)wb.take(2 * n_shared * fd);
+    }
+    h->w = {wr, wg, wu, wd, wsg, wsu, wsd};
+
+    Block sb{(char *)h->ws_mem, 0, wsbytes};
+    moe::Workspace &ws = h->ws;
+    ws.logits = (float *)sb.take(4 * T * E);
+    ws.topk_idx = (int *)sb.take(4 * P);
+    ws.topk_w = (float *)sb.take(4 * P);
+    ws.perm = (int *)sb.take(4 * P);
+    ws.mask = (uint32_t *)sb.take(4 * P * (d_ff / 32));
+    ws.y_acc = (float *)sb.take(4 * T * d_model);
+    ws.tok_cnt = (int *)sb.take(4 * T);
+    ws.tile_ticket = (int *)sb.take(4 * ((T + 7) / 8));
+    ws.done_ticket = (int *)sb.take(4);
+    ws.error_word = (int *)sb.take(4);
+    ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
+    ws.x_perm = (uint16_t *)sb.take(2 * P * d_model);
+    ws.h_perm = (uint16_t *)sb.take(2 * P * d_ff);
+    ws.x_stage = (uint16_t *)sb.take(2 * T * d_model);
+    ws.out_stage = (uint16_t *)sb.take(2 * T * d_model);
+    h->stats_dev = (unsigned long long *)sb.take(64);
+    h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
+    if (!h->stats_dev || !h->hist) { free_handle(h); return MOE_ENOMEM; }
+
+    cudaStream_t st = nullptr;
+    bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(wr, w->w_router, 2 * (size_t)E * d_model, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_gate, wg, E, d_model, d_ff, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wu, E, d_model, d_ff, st) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(wd, w->w_down, 2 * E * fd, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    if (n_shared) {
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_gate, wsg, n_shared, d_model, d_ff, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsu, n_shared, d_model, d_ff, st) == cudaSuccess;
+        ok = ok && cudaMemcpyAsync(wsd, w->ws_down, 2 * n_shared * fd, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    }
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        free_handle(h);
+        return MOE_ECUDA;
+    }
+    h->last_T = 0;
+    h->last_path = MOE_PATH_SPARSE;
+    h->last_masked = 1;
+    h->last_stream = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        g_live.insert(h);
+    }
+    *out = h;
+    return MOE_OK;
+}
+
+extern "C" void moe_sparse_destroy(moe_handle h)
+{
+    if (!is_live(h)) return;
+    free_handle(h);
+}
+
+static int run_forward(moe_handle h, const void *x, int T, float tau, bool masked, void *out,
+                       void *stream, int forced_path)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!x || !out) return MOE_EINVAL;
+    if (T < 1 || T > h->dm.max_tokens) return MOE_EINVAL;
+    if (std::isnan(tau)) return MOE_EINVAL;
+    if (!aligned16(x) || !aligned16(out)) return MOE_EALIGN;
+    if (x == out) return MOE_EINVAL;
+    int path = forced_path;
+    if (path == MOE_PATH_AUTO) path = h->path;
+    if (path == MOE_PATH_AUTO) path = (T <= h->t_star) ? MOE_PATH_SPARSE : MOE_PATH_DENSE;
+    if (path == MOE_PATH_DENSE && !moe::dense_path_available()) return MOE_ENOTSUP;
+    cudaStream_t st = (cudaStream_t)stream;
+    const uint16_t *xb = (const uint16_t *)x;
+    uint16_t *ob = (uint16_t *)out;
+    cudaError_t e = cudaSuccess;
+    if (h->n_ev) e = cudaEventRecord(h->ev[0], st);
+    if (path == MOE_PATH_SPARSE) {
+        const int mt = moe::sparse_tile_tokens(T);
+        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, mt, st);
+        if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
+        if (e == cudaSuccess)
+            e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, mt,
+                                          h->grid_cap[mt_index(mt)], st);
+    } else {
+        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
+        if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
+        if (e == cudaSuccess)
+            e = moe::launch_dense(h->dm, h->w, h->ws, xb, T, tau, masked, ob, h->n_sm, st);
+    }
+    if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[2], st);
+    h->last_T = T;
+    h->last_path = path;
+    h->last_masked = masked;
+    h->last_stream = st;
+    return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+extern "C" int moe_sparse_forward(moe_handle h, const void *x, int T, float tau, void *out, void *stream)
+{
+    return run_forward(h, x, T, tau, true, out, stream, MOE_PATH_AUTO);
+}
+
+extern "C" int moe_dense_forward(moe_handle h, const void *x, int T, void *out, void *stream)
+{
+    return run_forward(h, x, T, 0.0f, false, out, stream, MOE_PATH_DENSE);
+}
+
+extern "C" int moe_sparse_forward_host(moe_handle h, const void *x_host, int T, float tau,
+                                       void *out_host, void *stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!x_host || !out_host || T < 1 || T > h->dm.max_tokens) return MOE_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = (size_t)T * h->dm.d * 2;
+    if (cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ECUDA;
+    rc = moe_sparse_forward(h, h->ws.x_stage, T, tau, h->ws.out_stage, stream);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(out_host, h->ws.out_stage, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ECUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+extern "C" int moe_set_path(moe_handle h, int path)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_SPARSE && path != MOE_PATH_DENSE) return MOE_EINVAL;
+    if (path == MOE_PATH_DENSE && !moe::dense_path_available()) return MOE_ENOTSUP;
+    h->path = path;
+    return MOE_OK;
+}
+
+extern "C" int moe_set_t_star(moe_handle h, int t_star)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (t_star < 0) return MOE_EINVAL;
+    h->t_star = t_star;
+    return MOE_OK;
+}
+
+extern "C" int moe_debug_router(moe_handle h, const void *x, int T, int *idx_out, float *w_out, void *stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!x || !idx_out || !w_out || T < 1 || T > h->dm.max_tokens) return MOE_EINVAL;
+    if (!aligned16(x)) return MOE_EALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t n = (size_t)T * h->dm.k;
+    cudaError_t e = moe::launch_router(h->dm, h->w, h->ws, (const uint16_t *)x, T, 1, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(idx_out, h->ws.topk_idx, 4 * n, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w_out, h->ws.topk_w, 4 * n, cudaMemcpyDeviceToDevice, st);
+    return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+extern "C" int moe_debug_active(moe_handle h, const void *x, int T, float tau, uint16_t *idx_out,
+                                int *cnt_out, void *out, void *stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!idx_out || !cnt_out) return MOE_EINVAL;
+    if (T < 1 || T > h->dm.max_tokens) return MOE_EINVAL;
+    rc = run_forward(h, x, T, tau, true, out ? out : (void *)h->ws.out_stage, stream, MOE_PATH_SPARSE);
+    if (rc) return rc;
+    cudaError_t e = moe::launch_mask_compact(h->ws, T * h->dm.k, h->dm.f, idx_out, cnt_out,
+                                             (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
+                                 void *stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!x || !tau_out || T < 1 || T > h->dm.max_tokens || std::isnan(sparsity)) return MOE_EINVAL;
+    if (!aligned16(x)) return MOE_EALIGN;
+    const moe::Dims &dm = h->dm;
+    const size_t n = (size_t)T * dm.k * dm.f;
+    if (sparsity <= 0.0) { *tau_out = 0.0f; return MOE_OK; }
+    const double kq = std::floor(sparsity * (double)n);
+    if (kq >= (double)n) { *tau_out = INFINITY; return MOE_OK; }
+    if (!h->scores) {
+        const size_t cap = (size_t)dm.max_tokens * dm.k * dm.f * sizeof(float);
+        if (cudaMalloc(&h->scores, cap) != cudaSuccess) { cudaGetLastError(); h->scores = nullptr; return MOE_ENOMEM; }
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    const uint16_t *xb = (const uint16_t *)x;
+    const int mt = moe::sparse_tile_tokens(T);
+    cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, mt, st);
+    if (e == cudaSuccess)
+        e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, mt,
+                                      h->grid_cap[mt_index(mt)], st, h->scores);
+    // exact selection of the kq-th smallest, 8 bits per pass, most significant first
+    unsigned long long want = (unsigned long long)kq;
+    uint32_t prefix = 0, pmask = 0;
+    for (int shift = 24; shift >= 0 && e == cudaSuccess; shift -= 8) {
+        unsigned hist[256];
+        e = moe::launch_radix_hist((const uint32_t *)h->scores, n, prefix, pmask, shift, h->hist, h->n_sm, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(hist, h->hist, sizeof hist, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) break;
+        unsigned long long below = 0;
+        int b = 0;
+        for (; b < 256; ++b) {
+            if (below + hist[b] > want) break;
+            below += hist[b];
+        }
+        if (b == 256) return MOE_ECUDA;   // counts do not add up: cannot happen for a consistent buffer
+        want -= below;
+        prefix |= (uint32_t)b << shift;
+        pmask |= 255u << shift;
+    }
+    if (e != cudaSuccess) return MOE_ECUDA;
+    float tau;
+    std::memcpy(&tau, &prefix, sizeof tau);
+    *tau_out = tau;
+    return MOE_OK;
+}
+
+extern "C" int moe_set_launch_events(moe_handle h, void *const *events, int n)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (!events || n == 0) { h->n_ev = 0; return MOE_OK; }
+    if (n != 3 || !events[0] || !events[1] || !events[2]) return MOE_EINVAL;
+    for (int i = 0; i < 3; ++i) h->ev[i] = (cudaEvent_t)events[i];
+    h->n_ev = 3;
+    return MOE_OK;
+}
+
+extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!st) return MOE_EINVAL;
+    std::memset(st, 0, sizeof *st);
+    const moe::Dims &dm = h->dm;
+    st->path = h->last_path;
+    st->n_tokens = h->last_T;
+    st->t_star = h->t_star;
+    if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
+    int err = 0;
+    if (cudaMemcpy(&err, h->ws.error_word, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
+    st->device_error = err;
+    if (h->last_T > 0) {
+        unsigned long long v[3] = {0, 0, 0};
+        if (moe::launch_stats(dm, h->ws, h->last_T, h->stats_dev, h->last_stream) != cudaSuccess ||
+            cudaMemcpyAsync(v, h->stats_dev, sizeof v, cudaMemcpyDeviceToHost, h->last_stream) != cudaSuccess ||
+            cudaStreamSynchronize(h->last_stream) != cudaSuccess)
+            return MOE_ECUDA;
+        const double d = dm.d, f = dm.f;
+        const bool masked = h->last_masked && h->last_path == MOE_PATH_SPARSE;
+        st->n_touched = (int)v[2];
+        st->n_active = masked ? (long long)v[0] : (long long)h->last_T * dm.k * dm.f;
+        st->n_union = masked ? (long long)v[1] : (long long)v[2] * dm.f;
+        const double fixed = dm.S * 3.0 * d * f * 2 + (double)dm.E * d * 2 + 2.0 * h->last_T * d * 2;
+        st->alg_bytes = st->n_touched * d * f * 2 + 2.0 * d * 2 * (double)st->n_union + fixed;
+        st->dense_bytes = st->n_touched * 3.0 * d * f * 2 + fixed;
+    }
+    return err ? MOE_EDEVICE : MOE_OK;
+}
+
+extern "C" const char *moe_strerror(int code)
+{
+    switch (code) {
+    case MOE_OK: return "success";
+    case MOE_EINVAL: return "invalid argument";
+    case MOE_ENOMEM: return "out of memory";
+    case MOE_ECUDA: return "CUDA runtime error";
+    case MOE_EALIGN: return "pointer not 16-byte aligned";
+    case MOE_EHANDLE: return "invalid or destroyed handle";
+    case MOE_EDEVICE: return "a kernel reported a device-side error";
+    case MOE_ENOTSUP: return "not supported by this build";
+    default: return "unknown error code";
+    }
+}

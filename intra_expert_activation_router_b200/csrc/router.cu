@@ -1,0 +1,217 @@
+// router.cu -- softmax top-k router and token-to-expert bucketing.
+//
+// "Uncovering Intra-expert Activation Sparsity for Efficient Mixture-of-Expert
+// Model Execution" (technical summary, Methodology item 3): the router is kept
+// unchanged -- logits = x Wr^T, p = softmax over all E experts, the top_k
+// experts by p are selected and weighted by p.  Ties go to the lower index.
+//
+// One launch does three things:
+//   1. logits: CTA (expert tile, token tile), one warp per expert, fp32
+//      accumulation of bf16 products; Wr rows stream once per token tile.
+//   2. the last CTA of each token tile (atomic ticket; no waiting) runs the
+//      softmax and the ordered top-k of its tokens, one warp per token.
+//   3. the last token tile builds the routing plan for the expert kernels:
+//      per-expert counts, offsets, a stable permutation of the pairs
+//      (t*k + rank) ordered by expert then token, the ascending list of
+//      touched experts and the work-item prefix sums of both paths.
+// Tickets reset themselves, so the launch can be replayed (graphs) without
+// host-side clears.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr int kRtTok = 8;   // tokens per router CTA
+constexpr int kRtExp = 8;   // experts per router CTA (one warp each)
+
+struct RouterArgs {
+    const uint16_t *x, *wr;
+    int T, d, E, k, mt, n_chunks;
+    Workspace ws;
+};
+
+__device__ __forceinline__ bool better(float v1, int i1, float v0, int i0)
+{
+    return v1 > v0 || (v1 == v0 && i1 < i0);
+}
+
+// Build the routing plan from topk_idx; executed by one whole CTA.
+__device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, P = a.T * a.k;
+    Plan *plan = a.ws.plan;
+    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    for (int p = tid; p < P; p += blockDim.x) atomicAdd(&s_cnt[__ldcg(&a.ws.topk_idx[p])], 1);
+    __syncthreads();
+    if (warp == 0) {
+        // exclusive scans over experts: positions, touched slots, work items, dense tiles
+        const int per = (E + 31) / 32;
+        const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+        int c_sum = 0, t_sum = 0, i_sum = 0, d_sum = 0;
+        for (int e = e0; e < e1; ++e) {
+            const int c = s_cnt[e];
+            c_sum += c;
+            if (c > 0) {
+                t_sum += 1;
+                i_sum += ((c + a.mt - 1) / a.mt) * a.n_chunks;
+                d_sum += (c + kDenseTileM - 1) / kDenseTileM;
+            }
+        }
+        int c_ex = c_sum, t_ex = t_sum, i_ex = i_sum, d_ex = d_sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int c = __shfl_up_sync(kFull, c_ex, o), t = __shfl_up_sync(kFull, t_ex, o);
+            int i = __shfl_up_sync(kFull, i_ex, o), dd = __shfl_up_sync(kFull, d_ex, o);
+            if (lane >= o) { c_ex += c; t_ex += t; i_ex += i; d_ex += dd; }
+        }
+        c_ex -= c_sum; t_ex -= t_sum; i_ex -= i_sum; d_ex -= d_sum;
+        for (int e = e0; e < e1; ++e) {
+            const int c = s_cnt[e];
+            plan->offsets[e] = c_ex;
+            s_cur[e] = c_ex;
+            if (c > 0) {
+                plan->touched[t_ex] = e;
+                plan->item_prefix[t_ex] = i_ex;
+                plan->tile_prefix[t_ex] = d_ex;
+                t_ex += 1;
+                i_ex += ((c + a.mt - 1) / a.mt) * a.n_chunks;
+                d_ex += (c + kDenseTileM - 1) / kDenseTileM;
+            }
+            c_ex += c;
+        }
+        if (lane == 31) {
+            plan->offsets[E] = c_ex;
+            plan->n_touched = t_ex;
+            plan->item_prefix[t_ex] = i_ex;
+            plan->tile_prefix[t_ex] = d_ex;
+            plan->n_routed_items = i_ex;
+            plan->n_dense_tiles = d_ex;
+        }
+        __syncwarp();
+        // stable scatter, 32 pairs at a time in pair order
+        for (int base = 0; base < P; base += 32) {
+            const int p = base + lane;
+            const int e = p < P ? __ldcg(&a.ws.topk_idx[p]) : -1 - lane;
+            const unsigned same = __match_any_sync(kFull, e);
+            const int rank = __popc(same & ((1u << lane) - 1));
+            int pos = 0;
+            if (p < P) pos = s_cur[e] + rank;
+            __syncwarp();
+            if (p < P && rank == 0) s_cur[e] += __popc(same);
+            if (p < P) a.ws.perm[pos] = p;
+            __syncwarp();
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) k_router(RouterArgs a)
+{
+    extern __shared__ float s_dyn[];   // kRtTok * E floats, reused as 2*E ints
+    __shared__ int s_last;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = blockIdx.y * kRtTok;
+    const int nt = min(kRtTok, a.T - t0);
+
+    // 1. logits
+    const int e = blockIdx.x * kRtExp + warp;
+    if (e < a.E) {
+        float acc[kRtTok];
+#pragma unroll
+        for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
+        const uint16_t *wrow = a.wr + (size_t)e * a.d;
+        for (int i = lane * 8; i < a.d; i += 256) {
+            const uint4 wv = ld_cached(wrow + i);
+#pragma unroll
+            for (int r = 0; r < kRtTok; ++r)
+                if (r < nt) acc[r] = dot8(wv, ld_cached(a.x + (size_t)(t0 + r) * a.d + i), acc[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
+        if (lane == 0)
+            for (int r = 0; r < nt; ++r) a.ws.logits[(size_t)(t0 + r) * a.E + e] = acc[r];
+    }
+
+    // 2. last CTA of this token tile: softmax + top-k
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int tk = atomicAdd(&a.ws.tile_ticket[blockIdx.y], 1);
+        s_last = (tk == (int)gridDim.x - 1);
+        if (s_last) a.ws.tile_ticket[blockIdx.y] = 0;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (warp < nt) {
+        const int t = t0 + warp;
+        float *row = s_dyn + warp * a.E;
+        float m = -INFINITY;
+        for (int j = lane; j < a.E; j += 32) {
+            const float v = __ldcg(&a.ws.logits[(size_t)t * a.E + j]);
+            row[j] = v;
+            m = fmaxf(m, v);
+        }
+        m = warp_max(m);
+        float s = 0.f;
+        for (int j = lane; j < a.E; j += 32) s += expf(row[j] - m);
+        s = warp_sum(s);
+        unsigned taken = 0;   // bit q: expert lane + 32q already selected
+        for (int r = 0; r < a.k; ++r) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int q = 0, j = lane; j < a.E; ++q, j += 32) {
+                if (taken & (1u << q)) continue;
+                const float v = row[j];
+                if (bi == 0x7fffffff || better(v, j, bv, bi)) { bv = v; bi = j; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, bv, o);
+                const int oi = __shfl_xor_sync(kFull, bi, o);
+                if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == 0) {
+                a.ws.topk_idx[(size_t)t * a.k + r] = bi;
+                a.ws.topk_w[(size_t)t * a.k + r] = expf(bv - m) / s;
+            }
+        }
+    }
+
+    // 3. last token tile: the routing plan
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int tk = atomicAdd(a.ws.done_ticket, 1);
+        s_last = (tk == (int)gridDim.y - 1);
+        if (s_last) *a.ws.done_ticket = 0;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    int *s_int = reinterpret_cast<int *>(s_dyn);
+    build_plan(a, s_int, s_int + a.E);
+}
+
+cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
+                          const uint16_t *x, int T, int mt, cudaStream_t st)
+{
+    RouterArgs a;
+    a.x = x;
+    a.wr = w.wr;
+    a.T = T;
+    a.d = dm.d;
+    a.E = dm.E;
+    a.k = dm.k;
+    a.mt = mt;
+    a.n_chunks = dm.f / kChunk;
+    a.ws = ws;
+    dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
+    size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // >= 2*E ints as well
+    k_router<<<grid, 256, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

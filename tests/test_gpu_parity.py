@@ -1,0 +1,228 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on the five workloads' shapes.
+
+Every comparison uses the same seeded bf16 inputs on both sides.  Small
+batches are compared token by token in full; the big batches (and the
+6.44 GB layer) on a seeded sample of tokens, which the oracle computes one
+by one -- tokens are independent, so a sampled token's expected output is
+exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+NTHREADS = 0   # oracle: all host cores
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+_layers = {}
+
+
+def layer_for(name, max_tokens=4096):
+    key = (name, max_tokens)
+    if key not in _layers:
+        for k_ in list(_layers):
+            if k_[0] != name:
+                _layers.pop(k_)[0].close()
+        torch.cuda.empty_cache()
+        sh = mi.SHAPES[name]
+        layer, W = pu.gpu_layer(sh, max_tokens=max_tokens)
+        _layers[key] = (layer, W, oracle.layer_inputs(W, torch.zeros(1, sh.d_model, dtype=torch.bfloat16)))
+    return _layers[key]
+
+
+def run_case(o, name, T, q, sample=None, check_lists=True):
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    # tau: the oracle's calibration on (at most) the first 64 tokens of the batch
+    cal = dict(inputs)
+    cal["x"] = inputs["x"][:64]
+    tau = pu.calibrate(o, cal, sh.top_k, q, NTHREADS)
+    # the GPU path on the whole batch
+    out = layer.forward(x, tau)
+    idx, w = layer.router(x)
+    lists, cnt = layer.active_lists(x, tau) if check_lists else (None, None)
+    torch.cuda.synchronize()
+    rows = np.arange(T) if sample is None else np.sort(
+        np.random.default_rng(1000 * T + int(q * 100)).choice(T, size=min(sample, T), replace=False))
+    sub = dict(inputs)
+    sub["x"] = inputs["x"][rows]
+    ref = o.forward(**sub, top_k=sh.top_k, tau=tau, nthreads=NTHREADS, want_scores=check_lists)
+    tie = pu.check_router(ref, idx.cpu().numpy()[rows], w.cpu().numpy()[rows], sh.top_k)
+    flipped = np.zeros(len(rows), bool)
+    if check_lists:
+        flipped, _ = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16)[rows],
+                                     cnt.cpu().numpy()[rows], tie)
+    worst = pu.check_output(ref.y, out[torch.as_tensor(rows, device="cuda")], tie | flipped)
+    assert (tie | flipped).sum() <= max(1, len(rows) // 50), "too many exempt tokens"
+    return tau, worst, layer
+
+
+def test_tiny(o):
+    tau, worst, _ = run_case(o, "tiny", 16, 0.9)
+    assert 0.5 < tau < 2.0
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+def test_olmoe(o, T):
+    run_case(o, "olmoe", T, 0.9)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+@pytest.mark.parametrize("q", [0.0, 0.5, 0.8, 0.9, 0.95])
+def test_dsv2lite(o, T, q):
+    run_case(o, "dsv2lite", T, q, sample=None if T <= 32 else 24)
+
+
+@pytest.mark.parametrize("T", [1, 16, 64])
+def test_large(o, T):
+    run_case(o, "large", T, 0.98, sample=None if T <= 16 else 12)
+
+
+@pytest.mark.parametrize("T", [3, 13, 100, 257, 1000, 4096])
+def test_crossover_sparse_sampled(o, T):
+    run_case(o, "crossover", T, 0.9, sample=None if T <= 13 else 12, check_lists=T <= 1000)
+
+
+def test_tau_extremes(o):
+    sh = mi.SHAPES["dsv2lite"]
+    layer, W, host = layer_for("dsv2lite")
+    x = mi.make_x(sh, 5, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    for tau in (0.0, -1.0, math.inf):
+        out = layer.forward(x, tau)
+        ref = o.forward(**inputs, top_k=sh.top_k, tau=tau, want_scores=False)
+        pu.check_output(ref.y, out)
+    # no shared expert and tau = +inf: exactly zero
+    layer2, W2, host2 = layer_for("olmoe")
+    x2 = mi.make_x(mi.SHAPES["olmoe"], 3, device="cuda")
+    out2 = layer2.forward(x2, math.inf)
+    assert not out2.float().abs().sum().item()
+
+
+def test_repeat_and_interleave(o):
+    """Workspace state (accumulators, tickets) resets itself between calls."""
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    xa, xb = mi.make_x(sh, 16, device="cuda"), mi.make_x(sh, 5, device="cuda", seed=99)
+    a1 = layer.forward(xa, 1.0).clone()
+    b1 = layer.forward(xb, 1.0).clone()
+    a2 = layer.forward(xa, 1.0).clone()
+    b2 = layer.forward(xb, 1.0).clone()
+    torch.cuda.synchronize()
+    for u, v in ((a1, a2), (b1, b2)):
+        d = (u.float() - v.float()).abs()
+        tol = u.float().abs() * 2.0 ** -7 + 1e-6     # fp32 atomics may reorder: <= 1 bf16 ulp
+        assert bool((d <= tol).all())
+
+
+def test_host_pointer_entry(o):
+    from intra_expert_activation_router_b200 import moe_sparse_forward_host
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    x = mi.make_x(sh, 7, device="cuda")
+    dev = layer.forward(x, 1.0)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    moe_sparse_forward_host(layer.h, xh, 7, 1.0, oh)
+    d = (oh.float() - dev.cpu().float()).abs()
+    assert bool((d <= dev.cpu().float().abs() * 2.0 ** -7 + 1e-6).all())
+
+
+def test_stats_match_oracle(o):
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    T = 16
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    tau = pu.calibrate(o, inputs, sh.top_k, 0.9)
+    layer.forward(x, tau)
+    st = layer.stats()
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=tau)
+    assert st["n_touched"] == len(np.unique(ref.topk_idx))
+    band = int((np.abs(ref.score - tau) <= pu.BAND_REL * tau).sum())
+    assert abs(st["n_active"] - int(ref.active.sum())) <= band
+    uni = 0
+    for e in np.unique(ref.topk_idx):
+        rows = np.argwhere(ref.topk_idx == e)
+        uni += int(np.any(ref.active[rows[:, 0], rows[:, 1]], axis=0).sum())
+    assert abs(st["n_union"] - uni) <= band
+    d, f = sh.d_model, sh.d_ff
+    want = st["n_touched"] * d * f * 2 + 4 * d * st["n_union"] + sh.n_experts * d * 2 + 4 * T * d
+    assert st["alg_bytes"] == pytest.approx(want)
+
+
+@pytest.mark.parametrize("dims", [
+    dict(d=264, E=4, f=32, k=4, S=0, T=9),     # E == k, one chunk, d not a multiple of 256
+    dict(d=64, E=16, f=96, k=1, S=1, T=37),    # top-1, ragged token count
+    dict(d=128, E=1024, f=64, k=2, S=0, T=5),  # the largest expert count
+    dict(d=2048, E=8, f=64, k=2, S=3, T=40),   # many shared experts, T == max_tokens
+])
+def test_edge_shapes(o, dims):
+    sh = mi.custom_shape(dims["d"], dims["E"], dims["f"], dims["k"], dims["S"])
+    W = mi.make_weights(sh, device="cuda")
+    from intra_expert_activation_router_b200 import MoESparseLayer
+    layer = MoESparseLayer.from_weights(W, sh.top_k, max_tokens=dims["T"])
+    x = mi.make_x(sh, dims["T"], device="cuda")
+    inputs = oracle.layer_inputs(W, x)
+    tau = pu.calibrate(o, inputs, sh.top_k, 0.7)
+    out = layer.forward(x, tau)
+    idx, w = layer.router(x)
+    lists, cnt = layer.active_lists(x, tau)
+    torch.cuda.synchronize()
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=tau)
+    tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
+    flipped, _ = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
+    pu.check_output(ref.y, out, tie | flipped)
+    layer.close()
+
+
+def test_argument_errors_live_handle():
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["tiny"]
+    layer, W, host = layer_for("tiny", max_tokens=32)
+    x = mi.make_x(sh, 4, device="cuda")
+    out = torch.empty_like(x)
+    for T in (0, -1, 33):
+        with pytest.raises(m.MoeError) as ei:
+            m.moe_sparse_forward(layer.h, x, T, 1.0, out)
+        assert ei.value.code == m.MOE_EINVAL
+    with pytest.raises(m.MoeError) as ei:
+        m.moe_sparse_forward(layer.h, x, 4, float("nan"), out)
+    assert ei.value.code == m.MOE_EINVAL
+    with pytest.raises(m.MoeError) as ei:
+        m.moe_sparse_forward(layer.h, x.data_ptr() + 2, 4, 1.0, out)
+    assert ei.value.code == m.MOE_EALIGN
+    with pytest.raises(m.MoeError) as ei:
+        m.moe_sparse_forward(layer.h, x, 4, 1.0, x)
+    assert ei.value.code == m.MOE_EINVAL
+    with pytest.raises(m.MoeError) as ei:
+        m.moe_set_path(layer.h, 7)
+    assert ei.value.code == m.MOE_EINVAL
+    # the handle still works after the rejected calls
+    layer.forward(x, 1.0)
+    torch.cuda.synchronize()
+    # destroyed handles are rejected, not dereferenced
+    h = m.moe_sparse_create(dict(w_router=W.w_router, w_gate=W.w_gate, w_up=W.w_up, w_down=W.w_down,
+                                 ws_gate=W.ws_gate, ws_up=W.ws_up, ws_down=W.ws_down),
+                            sh.n_experts, sh.top_k, sh.d_model, sh.d_ff, sh.n_shared, 8)
+    m.moe_sparse_destroy(h)
+    with pytest.raises(m.MoeError) as ei:
+        m.moe_sparse_forward(h, x, 4, 1.0, out)
+    assert ei.value.code == m.MOE_EHANDLE
