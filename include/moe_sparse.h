@@ -94,8 +94,8 @@ typedef struct {
  * memory (the caller may free its tensors afterwards) and allocates all
  * workspace for up to `max_tokens` tokens per call, so that forward calls
  * never allocate.  Synchronises the device before returning.
- * Requirements (else MOE_EINVAL): 1 <= top_k <= E <= 1024; d_model >= 8 and
- * d_model % 8 == 0; d_ff >= 32 and d_ff % 32 == 0; d_ff <= 65535;
+ * Requirements (else MOE_EINVAL): 1 <= top_k <= E <= 1024; 8 <= d_model <= 8192
+ * and d_model % 8 == 0; d_ff >= 32 and d_ff % 32 == 0; d_ff <= 65535;
  * 0 <= n_shared <= 8; 1 <= max_tokens <= 65536 (0 selects 4096).
  * Pointers must be 16-byte aligned (else MOE_EALIGN).  On failure *out is
  * set to NULL and nothing is leaked. */

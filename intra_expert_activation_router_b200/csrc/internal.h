@@ -50,6 +50,8 @@ struct Workspace {
     int *topk_idx;
     float *topk_w;
     int *perm;
+    int *perm_tok;      // [T*k] token of perm[i]
+    float *perm_w;      // [T*k] routing weight of perm[i]
     uint32_t *mask;
     float *y_acc;
     int *tok_cnt;
@@ -81,6 +83,6 @@ cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned lo
 cudaError_t launch_radix_hist(const uint32_t *v, size_t n, uint32_t prefix, uint32_t prefix_mask,
                               int shift, unsigned *hist, int n_sm, cudaStream_t st);
 
-int sparse_tile_tokens(int T);   // tokens per sparse work item for a batch of T
+int sparse_tile_tokens(int T, int d);   // tokens per sparse work item for a batch of T
 
 }  // namespace moe

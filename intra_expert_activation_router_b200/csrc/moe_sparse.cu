@@ -106,7 +106,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     if (!w) return MOE_EINVAL;
     if (max_tokens == 0) max_tokens = 4096;
     if (E < 1 || E > moe::kMaxExperts || top_k < 1 || top_k > E) return MOE_EINVAL;
-    if (d_model < 8 || d_model % 8 != 0) return MOE_EINVAL;
+    if (d_model < 8 || d_model % 8 != 0 || d_model > 8192) return MOE_EINVAL;
     if (d_ff < 32 || d_ff % 32 != 0 || d_ff > 65535) return MOE_EINVAL;
     if (n_shared < 0 || n_shared > 8 || max_tokens < 1 || max_tokens > 65536) return MOE_EINVAL;
     if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_EINVAL;
@@ -134,7 +134,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     const size_t fd = (size_t)d_ff * d_model;
     const size_t wbytes = 2 * ((size_t)E * d_model + 3 * E * fd + 3 * (size_t)n_shared * fd) + 16 * 256;
     const size_t T = max_tokens, P = T * top_k;
-    const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
+    const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
                            4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * P * d_model +
                            2 * P * d_ff + 2 * 2 * T * d_model + 64 + 1024 + 32 * 256;
     if (cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
@@ -158,6 +158,8 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.topk_idx = (int *)sb.take(4 * P);
     ws.topk_w = (float *)sb.take(4 * P);
     ws.perm = (int *)sb.take(4 * P);
+    ws.perm_tok = (int *)sb.take(4 * P);
+    ws.perm_w = (float *)sb.take(4 * P);
     ws.mask = (uint32_t *)sb.take(4 * P * (d_ff / 32));
     ws.y_acc = (float *)sb.take(4 * T * d_model);
     ws.tok_cnt = (int *)sb.take(4 * T);
@@ -228,7 +230,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     cudaError_t e = cudaSuccess;
     if (h->n_ev) e = cudaEventRecord(h->ev[0], st);
     if (path == MOE_PATH_SPARSE) {
-        const int mt = moe::sparse_tile_tokens(T);
+        const int mt = moe::sparse_tile_tokens(T, h->dm.d);
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, mt, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
         if (e == cudaSuccess)
@@ -338,7 +340,7 @@ extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double spar
     }
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
-    const int mt = moe::sparse_tile_tokens(T);
+    const int mt = moe::sparse_tile_tokens(T, dm.d);
     cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, mt, st);
     if (e == cudaSuccess)
         e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, mt,

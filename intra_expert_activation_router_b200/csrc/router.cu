@@ -7,7 +7,9 @@
 //
 // One launch does three things:
 //   1. logits: CTA (expert tile, token tile), one warp per expert, fp32
-//      accumulation of bf16 products; Wr rows stream once per token tile.
+//      accumulation of bf16 products; the tile's x rows are staged in shared
+//      memory and each warp's router row is loaded whole before the math, so
+//      the phase costs about one memory round trip.
 //   2. the last CTA of each token tile (atomic ticket; no waiting) runs the
 //      softmax and the ordered top-k of its tokens, one warp per token.
 //   3. the last token tile builds the routing plan for the expert kernels:
@@ -23,6 +25,7 @@ namespace moe {
 
 constexpr int kRtTok = 8;   // tokens per router CTA
 constexpr int kRtExp = 8;   // experts per router CTA (one warp each)
+constexpr int kStagePairs = 4096;   // plan built from shared memory up to this many pairs
 
 struct RouterArgs {
     const uint16_t *x, *wr;
@@ -36,14 +39,21 @@ __device__ __forceinline__ bool better(float v1, int i1, float v0, int i0)
 }
 
 // Build the routing plan from topk_idx; executed by one whole CTA.
-__device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur)
+__device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_idx, float *s_w)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, P = a.T * a.k;
+    const bool staged = s_idx != nullptr;   // top-k of all pairs held in shared memory
     Plan *plan = a.ws.plan;
     for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    if (staged)
+        for (int p = tid; p < P; p += blockDim.x) {
+            s_idx[p] = __ldcg(&a.ws.topk_idx[p]);
+            s_w[p] = __ldcg(&a.ws.topk_w[p]);
+        }
     __syncthreads();
-    for (int p = tid; p < P; p += blockDim.x) atomicAdd(&s_cnt[__ldcg(&a.ws.topk_idx[p])], 1);
+    for (int p = tid; p < P; p += blockDim.x)
+        atomicAdd(&s_cnt[staged ? s_idx[p] : __ldcg(&a.ws.topk_idx[p])], 1);
     __syncthreads();
     if (warp == 0) {
         // exclusive scans over experts: positions, touched slots, work items, dense tiles
@@ -93,14 +103,18 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur)
         // stable scatter, 32 pairs at a time in pair order
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
-            const int e = p < P ? __ldcg(&a.ws.topk_idx[p]) : -1 - lane;
+            const int e = p < P ? (staged ? s_idx[p] : __ldcg(&a.ws.topk_idx[p])) : -1 - lane;
             const unsigned same = __match_any_sync(kFull, e);
             const int rank = __popc(same & ((1u << lane) - 1));
             int pos = 0;
             if (p < P) pos = s_cur[e] + rank;
             __syncwarp();
             if (p < P && rank == 0) s_cur[e] += __popc(same);
-            if (p < P) a.ws.perm[pos] = p;
+            if (p < P) {
+                a.ws.perm[pos] = p;
+                a.ws.perm_tok[pos] = p / a.k;
+                a.ws.perm_w[pos] = staged ? s_w[p] : __ldcg(&a.ws.topk_w[p]);
+            }
             __syncwarp();
         }
     }
@@ -114,19 +128,43 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     const int t0 = blockIdx.y * kRtTok;
     const int nt = min(kRtTok, a.T - t0);
 
-    // 1. logits
+    // let the expert kernel launch now; it waits for this grid to finish
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    // 1. logits: the tile's x rows in shared memory (chunks of 2048), each
+    //    warp's router row in registers, all loads issued before any math
     const int e = blockIdx.x * kRtExp + warp;
-    if (e < a.E) {
-        float acc[kRtTok];
+    float acc[kRtTok];
 #pragma unroll
-        for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
-        const uint16_t *wrow = a.wr + (size_t)e * a.d;
-        for (int i = lane * 8; i < a.d; i += 256) {
-            const uint4 wv = ld_cached(wrow + i);
+    for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
+    uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);   // [kRtTok][256] 16-byte vectors
+    for (int c0 = 0; c0 < a.d; c0 += 2048) {
+        const int cv = min(2048, a.d - c0) / 8;
+        uint4 wv[8];
 #pragma unroll
-            for (int r = 0; r < kRtTok; ++r)
-                if (r < nt) acc[r] = dot8(wv, ld_cached(a.x + (size_t)(t0 + r) * a.d + i), acc[r]);
+        for (int q = 0; q < 8; ++q) {
+            const int v = lane + 32 * q;
+            wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
         }
+        __syncthreads();   // the previous chunk's x is no longer read
+        for (int i = threadIdx.x; i < nt * cv; i += blockDim.x) {
+            const int r = i / cv, v = i % cv;
+            xs[r * 256 + v] = ld_cached(a.x + (size_t)(t0 + r) * a.d + c0 + v * 8);
+        }
+        __syncthreads();
+        if (e < a.E) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int v = lane + 32 * q;
+                if (v < cv) {
+#pragma unroll
+                    for (int r = 0; r < kRtTok; ++r)
+                        if (r < nt) acc[r] = dot8(wv[q], xs[r * 256 + v], acc[r]);
+                }
+            }
+        }
+    }
+    if (e < a.E) {
 #pragma unroll
         for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
         if (lane == 0)
@@ -192,7 +230,10 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     if (!s_last) return;
     __threadfence();
     int *s_int = reinterpret_cast<int *>(s_dyn);
-    build_plan(a, s_int, s_int + a.E);
+    const int P = a.T * a.k;
+    const bool staged = P <= kStagePairs;
+    build_plan(a, s_int, s_int + a.E, staged ? s_int + 2 * a.E : nullptr,
+               staged ? reinterpret_cast<float *>(s_int + 2 * a.E + P) : nullptr);
 }
 
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
@@ -209,7 +250,12 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     a.n_chunks = dm.f / kChunk;
     a.ws = ws;
     dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
-    size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // >= 2*E ints as well
+    const size_t P = (size_t)T * dm.k;
+    size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // softmax rows
+    if (smem < 16 * (size_t)kRtTok * 256) smem = 16 * (size_t)kRtTok * 256;   // x chunk
+    size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (P <= kStagePairs ? 8 * P : 0);
+    if (plan_smem > smem) smem = plan_smem;
+    // at most max(32 KB, 2*1024*4 + 8*4096 = 40 KB): inside the default 48 KB window
     k_router<<<grid, 256, smem, st>>>(a);
     return cudaGetLastError();
 }

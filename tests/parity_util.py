@@ -2,13 +2,18 @@
 
 Acceptance rules (the layer's own stated bar):
   * router top-k indices equal, except tokens whose k-th and (k+1)-th oracle
-    logits are within 1e-4 * max|logit| (a near tie that fp32 may order
-    either way); such tokens are reported and excluded;
+    logits are within 1e-5 * max|logit| (a near tie that fp32 may order
+    either way -- 1e-5 is several hundred times the fp32 accumulation error of
+    a 4096-long dot product of these magnitudes); such tokens are excluded;
   * active-neuron sets equal, except neurons whose oracle score lies within
     1e-3 * tau of tau;
   * per token, ||y_gpu - y_oracle|| / ||y_oracle|| <= 1e-2, excluding tokens
     with a near-tie router or a band neuron decided differently; when the
     oracle output is exactly zero the GPU output must be exactly zero.
+A calibrated tau is itself the score of one routed neuron, so that neuron
+sits exactly on the threshold and either decision is correct; flips inside
+the band are therefore allowed (and their tokens excluded from the output
+comparison), while near ties must stay rare.
 """
 from __future__ import annotations
 
@@ -20,7 +25,7 @@ import torch
 import moe_inputs as mi
 import oracle
 
-TIE_REL = 1e-4
+TIE_REL = 1e-5
 BAND_REL = 1e-3
 OUT_REL_L2 = 1e-2
 
