@@ -94,8 +94,8 @@ typedef struct {
  * memory (the caller may free its tensors afterwards) and allocates all
  * workspace for up to `max_tokens` tokens per call, so that forward calls
  * never allocate.  Synchronises the device before returning.
- * Requirements (else MOE_EINVAL): 1 <= top_k <= E <= 1024; 8 <= d_model <= 8192
- * and d_model % 8 == 0; d_ff >= 32 and d_ff % 32 == 0; d_ff <= 65535;
+ * Requirements (else MOE_EINVAL): 1 <= top_k <= E <= 1024; 8 <= d_model <= 4096
+ * and d_model % 8 == 0 (eight gate rows must sit in at most two 32 KB stages); d_ff >= 32 and d_ff % 32 == 0; d_ff <= 65535;
  * 0 <= n_shared <= 8; 1 <= max_tokens <= 65536 (0 selects 4096).
  * Pointers must be 16-byte aligned (else MOE_EALIGN).  On failure *out is
  * set to NULL and nothing is leaked. */
@@ -160,6 +160,21 @@ int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float
  * events == NULL or n == 0 stops recording.  The handle keeps the three
  * handles, not the array. */
 int moe_set_launch_events(moe_handle h, void *const *events, int n);
+
+/* Tracing hook: when buf (DEVICE, 8-byte aligned, `bytes` long) is set, later
+ * forwards stamp the GPU global timer (ns) at phase boundaries of each CTA.
+ * The first half of the buffer holds 8 stamps per router CTA (CTA index
+ * y*gridDim.x + x): start, logits done, top-k start, top-k done, plan start,
+ * plan done (the last two only in the CTA that builds the plan).  The second
+ * half holds 64 per expert-kernel CTA: [0] start, [1] plan loaded, then for
+ * each of the CTA's first four items i, at 2 + 12*i: token rows in, the four
+ * 8-row gate groups in, gate done, mask done, gather issued, first gathered
+ * records in, up/down done, accumulator flushed (if it was); [50] end and
+ * [51] the CTA's item count; [52 + 2i], [53 + 2i] first and last gate stage
+ * of item i issued; [60 + i] token rows of item i issued; [40 + s] arrival
+ * of gate stage s, for the first ring-full of stages (at most 8).  Unwritten slots keep their old contents.
+ * buf == NULL turns tracing off. */
+int moe_set_trace(moe_handle h, void *buf, long long bytes);
 
 /* Statistics of the last forward.  Synchronises the stream of that forward
  * and reads device counters back; not for timed loops.  A nonzero device

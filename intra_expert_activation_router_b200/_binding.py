@@ -72,6 +72,7 @@ def _load():
         "moe_query_stats": (I, [P, ctypes.POINTER(moe_stats)]),
         "moe_calibrate_tau": (I, [P, P, I, ctypes.c_double, ctypes.POINTER(F), P]),
         "moe_set_launch_events": (I, [P, ctypes.POINTER(P), I]),
+        "moe_set_trace": (I, [P, P, ctypes.c_longlong]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -85,7 +86,7 @@ _lib = _load()
 EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_sparse_forward_host", "moe_sparse_destroy", "moe_set_path", "moe_set_t_star",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
-            "moe_calibrate_tau", "moe_set_launch_events")
+            "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace")
 
 
 def _addr(t):
@@ -192,6 +193,15 @@ def moe_set_launch_events(h, events):
     hs = [e if isinstance(e, int) else e.cuda_event for e in events]
     arr = (ctypes.c_void_p * len(hs))(*hs)
     _check(_lib.moe_set_launch_events(h, arr, len(hs)), "moe_set_launch_events")
+
+
+def moe_set_trace(h, buf, nbytes: int = 0):
+    """buf: an int64 CUDA tensor (or address) receiving phase timestamps; None turns tracing off."""
+    if buf is None:
+        _check(_lib.moe_set_trace(h, None, 0), "moe_set_trace")
+        return
+    n = nbytes or (buf.numel() * buf.element_size())
+    _check(_lib.moe_set_trace(h, _addr(buf), n), "moe_set_trace")
 
 
 def raw_call(name: str, *args) -> int:

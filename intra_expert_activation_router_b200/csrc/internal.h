@@ -1,11 +1,17 @@
 // internal.h -- data shared by the host library and the kernel launchers.
 //
 // Everything lives in device memory owned by the handle.  Layouts:
-//   repacked weights (neuron-major, so every neuron's row is contiguous):
-//     wg_n, wu_n   [E][f][d]      row j of expert e = the gate / up column j
-//     wd           [E][f][d]      row j = the down-projection row of neuron j
-//     wsg_n, wsu_n, wsd [S][f][d] the same for the shared experts
-//     wr           [E][d]
+//   repacked weights (neuron-major, so every neuron's data is contiguous):
+//     wg_n   [E][f][d]   row j = gate column j; inside every 128-byte group of a
+//                        row the eight 16-byte blocks are permuted b -> b ^ (j & 7)
+//                        (the 128-byte swizzle), so that eight consecutive rows
+//                        copied contiguously into shared memory are bank-conflict
+//                        free for tensor-core fragment loads; a tail of fewer than
+//                        eight blocks (d % 64 != 0) is stored unpermuted
+//     wud    [E][f][2d]  row j = [up column j | down row j]: one neuron's up and
+//                        down weights in a single contiguous 4d-byte record
+//     wsg_n, wsud        the same for the shared experts
+//     wr     [E][d]
 //   per-call workspace, sized for max_tokens:
 //     logits [T][E] fp32, topk_idx/topk_w [T][k], perm [T*k] (pair ids
 //     t*k+rank sorted by expert, stable), mask [T*k][f/32] uint32 (bit j of
@@ -41,9 +47,17 @@ struct Dims {
 
 struct DeviceWeights {
     const uint16_t *wr;
-    const uint16_t *wg_n, *wu_n, *wd;
-    const uint16_t *wsg_n, *wsu_n, *wsd;
+    const uint16_t *wg_n, *wud;
+    const uint16_t *wsg_n, *wsud;
 };
+
+// Position of element k inside a swizzled gate row j (see wg_n above).
+__host__ __device__ __forceinline__ int gate_pos(int j, int k, int d)
+{
+    const int b = k >> 3, full = (d >> 6) << 3;
+    const int sb = b < full ? (b ^ (j & 7)) : b;
+    return (sb << 3) | (k & 7);
+}
 
 struct Workspace {
     float *logits;
@@ -64,7 +78,18 @@ struct Workspace {
     uint16_t *h_perm;   // [T*k][f] bf16, masked SwiGLU activations
     // host-pointer entry
     uint16_t *x_stage, *out_stage;
+    // optional phase timestamps (moe_set_trace); nullptr when off
+    unsigned long long *trace_router;   // [router CTAs][8]
+    unsigned long long *trace_expert;   // [expert CTAs][16]
+    int trace_router_ctas, trace_expert_ctas;
 };
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 // Launchers (return cudaGetLastError()).
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
@@ -73,8 +98,13 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, int mt, int grid_cap, cudaStream_t st,
                                  float *score_out = nullptr);
-cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows,
-                                    int cols, cudaStream_t st);
+// dst[b][c][col_off + pos(c, r)] = src[b][r][c] with row stride ld (elements);
+// pos = gate_pos when swizzle, else r.
+cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
+                                    int ld, int col_off, bool swizzle, cudaStream_t st);
+// dst[b][r][col_off + c] = src[b][r][c] with row stride ld (elements).
+cudaError_t launch_repack_rows(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols, int ld,
+                               int col_off, cudaStream_t st);
 cudaError_t launch_mask_compact(const Workspace &ws, int n_pairs, int f, uint16_t *idx_out,
                                 int *cnt_out, cudaStream_t st);
 cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned long long *out3,

@@ -4,29 +4,55 @@
 
 namespace moe {
 
-// dst[b][c][r] = src[b][r][c]   (bf16 bits), 32x32 tiles through shared memory.
-__global__ void k_transpose(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, int rows,
-                            int cols)
+// dst[b][c][col_off + pos(c, r)] = src[b][r][c], 32x32 tiles through shared
+// memory; pos is the gate-row swizzle when `swizzle`, else the identity.
+__global__ void k_transpose(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, int rows, int cols,
+                            int ld, int col_off, int swizzle)
 {
     __shared__ uint16_t tile[32][33];
-    const size_t base = (size_t)blockIdx.z * rows * cols;
+    const size_t sbase = (size_t)blockIdx.z * rows * cols;
+    const size_t dbase = (size_t)blockIdx.z * cols * ld;
     const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int r = r0 + i, c = c0 + threadIdx.x;
-        if (r < rows && c < cols) tile[i][threadIdx.x] = src[base + (size_t)r * cols + c];
+        if (r < rows && c < cols) tile[i][threadIdx.x] = src[sbase + (size_t)r * cols + c];
     }
     __syncthreads();
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int c = c0 + i, r = r0 + threadIdx.x;
-        if (r < rows && c < cols) dst[base + (size_t)c * rows + r] = tile[threadIdx.x][i];
+        if (r < rows && c < cols) {
+            const int pos = swizzle ? gate_pos(c, r, rows) : r;
+            dst[dbase + (size_t)c * ld + col_off + pos] = tile[threadIdx.x][i];
+        }
     }
 }
 
-cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows,
-                                    int cols, cudaStream_t st)
+cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
+                                    int ld, int col_off, bool swizzle, cudaStream_t st)
 {
     dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches);
-    k_transpose<<<grid, dim3(32, 8), 0, st>>>(src, dst, rows, cols);
+    k_transpose<<<grid, dim3(32, 8), 0, st>>>(src, dst, rows, cols, ld, col_off, swizzle ? 1 : 0);
+    return cudaGetLastError();
+}
+
+__global__ void k_copy_rows(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, size_t n_rows, int cols,
+                            int ld, int col_off)
+{
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_rows * cols;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t r = i / cols;
+        const int c = (int)(i % cols);
+        dst[r * ld + col_off + c] = src[i];
+    }
+}
+
+cudaError_t launch_repack_rows(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols, int ld,
+                               int col_off, cudaStream_t st)
+{
+    const size_t n_rows = (size_t)batches * rows;
+    size_t blocks = (n_rows * cols + 255) / 256;
+    if (blocks > 65535 * 8) blocks = 65535 * 8;
+    k_copy_rows<<<(unsigned)blocks, 256, 0, st>>>(src, dst, n_rows, cols, ld, col_off);
     return cudaGetLastError();
 }
 

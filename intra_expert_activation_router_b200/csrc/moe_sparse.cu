@@ -106,7 +106,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     if (!w) return MOE_EINVAL;
     if (max_tokens == 0) max_tokens = 4096;
     if (E < 1 || E > moe::kMaxExperts || top_k < 1 || top_k > E) return MOE_EINVAL;
-    if (d_model < 8 || d_model % 8 != 0 || d_model > 8192) return MOE_EINVAL;
+    if (d_model < 8 || d_model % 8 != 0 || d_model > 4096) return MOE_EINVAL;
     if (d_ff < 32 || d_ff % 32 != 0 || d_ff > 65535) return MOE_EINVAL;
     if (n_shared < 0 || n_shared > 8 || max_tokens < 1 || max_tokens > 65536) return MOE_EINVAL;
     if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return MOE_EINVAL;
@@ -142,15 +142,14 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
 
     Block wb{(char *)h->weight_mem, 0, wbytes};
     uint16_t *wr = (uint16_t *)wb.take(2 * (size_t)E * d_model);
-    uint16_t *wg = (uint16_t *)wb.take(2 * E * fd), *wu = (uint16_t *)wb.take(2 * E * fd);
-    uint16_t *wd = (uint16_t *)wb.take(2 * E * fd);
-    uint16_t *wsg = nullptr, *wsu = nullptr, *wsd = nullptr;
+    uint16_t *wg = (uint16_t *)wb.take(2 * E * fd), *wud = (uint16_t *)wb.take(4 * E * fd);
+    uint16_t *wsg = nullptr, *wsud = nullptr;
     if (n_shared) {
         wsg = (uint16_t *)wb.take(2 * n_shared * fd);
-        wsu = (uint16_t *)wb.take(2 * n_shared * fd);
-        wsd = (uint16_t *)wb.take(2 * n_shared * fd);
+        wsud = (uint16_t *)wb.take(4 * n_shared * fd);
     }
-    h->w = {wr, wg, wu, wd, wsg, wsu, wsd};
+    if (!wr || !wg || !wud || (n_shared && (!wsg || !wsud))) { free_handle(h); return MOE_ENOMEM; }
+    h->w = {wr, wg, wud, wsg, wsud};
 
     Block sb{(char *)h->ws_mem, 0, wsbytes};
     moe::Workspace &ws = h->ws;
@@ -178,13 +177,14 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     cudaStream_t st = nullptr;
     bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
     ok = ok && cudaMemcpyAsync(wr, w->w_router, 2 * (size_t)E * d_model, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
-    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_gate, wg, E, d_model, d_ff, st) == cudaSuccess;
-    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wu, E, d_model, d_ff, st) == cudaSuccess;
-    ok = ok && cudaMemcpyAsync(wd, w->w_down, 2 * E * fd, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    const int d = d_model;
+    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_gate, wg, E, d, d_ff, d, 0, true, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wud, E, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_rows((const uint16_t *)w->w_down, wud, E, d_ff, d, 2 * d, d, st) == cudaSuccess;
     if (n_shared) {
-        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_gate, wsg, n_shared, d_model, d_ff, st) == cudaSuccess;
-        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsu, n_shared, d_model, d_ff, st) == cudaSuccess;
-        ok = ok && cudaMemcpyAsync(wsd, w->ws_down, 2 * n_shared * fd, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_gate, wsg, n_shared, d, d_ff, d, 0, true, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsud, n_shared, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_rows((const uint16_t *)w->ws_down, wsud, n_shared, d_ff, d, 2 * d, d, st) == cudaSuccess;
     }
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
@@ -379,6 +379,24 @@ extern "C" int moe_set_launch_events(moe_handle h, void *const *events, int n)
     if (n != 3 || !events[0] || !events[1] || !events[2]) return MOE_EINVAL;
     for (int i = 0; i < 3; ++i) h->ev[i] = (cudaEvent_t)events[i];
     h->n_ev = 3;
+    return MOE_OK;
+}
+
+extern "C" int moe_set_trace(moe_handle h, void *buf, long long bytes)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (!buf || bytes <= 0) {
+        h->ws.trace_router = h->ws.trace_expert = nullptr;
+        h->ws.trace_router_ctas = h->ws.trace_expert_ctas = 0;
+        return MOE_OK;
+    }
+    if (((uintptr_t)buf & 7u) != 0) return MOE_EALIGN;
+    const long long words = bytes / 8;
+    const long long router = words / 2;   // first half: router CTAs x 8 stamps
+    h->ws.trace_router = (unsigned long long *)buf;
+    h->ws.trace_router_ctas = (int)(router / 8);
+    h->ws.trace_expert = (unsigned long long *)buf + router;
+    h->ws.trace_expert_ctas = (int)((words - router) / 64);
     return MOE_OK;
 }
 

@@ -6,12 +6,14 @@
 // experts by p are selected and weighted by p.  Ties go to the lower index.
 //
 // One launch does three things:
-//   1. logits: CTA (expert tile, token tile), one warp per expert, fp32
-//      accumulation of bf16 products; the tile's x rows are staged in shared
-//      memory and each warp's router row is loaded whole before the math, so
-//      the phase costs about one memory round trip.
+//   1. logits: CTA (2 experts, 8 tokens), four warps per expert each taking a
+//      quarter of d, fp32 accumulation of bf16 products; the tile's x rows are
+//      staged in shared memory and the router rows loaded before the math, so
+//      the phase costs about one memory round trip on E/2 CTAs per tile.
 //   2. the last CTA of each token tile (atomic ticket; no waiting) runs the
-//      softmax and the ordered top-k of its tokens, one warp per token.
+//      softmax and the ordered top-k of its tokens, one warp per token: for
+//      E <= 256 every logit's rank is counted directly, above that k rounds of
+//      a warp arg-max select them.
 //   3. the last token tile builds the routing plan for the expert kernels:
 //      per-expert counts, offsets, a stable permutation of the pairs
 //      (t*k + rank) ordered by expert then token, the ascending list of
@@ -24,8 +26,9 @@
 namespace moe {
 
 constexpr int kRtTok = 8;   // tokens per router CTA
-constexpr int kRtExp = 8;   // experts per router CTA (one warp each)
+constexpr int kRtExp = 2;   // experts per router CTA (four warps each)
 constexpr int kStagePairs = 4096;   // plan built from shared memory up to this many pairs
+constexpr int kRankTopk = 256;      // up to this many experts, top-k by ranking all logits
 
 struct RouterArgs {
     const uint16_t *x, *wr;
@@ -130,20 +133,26 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
 
     // let the expert kernel launch now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;");
+    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    unsigned long long *tr = (a.ws.trace_router && cta < a.ws.trace_router_ctas) ? a.ws.trace_router + cta * 8 : nullptr;
+    if (tr && threadIdx.x == 0) tr[0] = global_ns();
 
-    // 1. logits: the tile's x rows in shared memory (chunks of 2048), each
-    //    warp's router row in registers, all loads issued before any math
-    const int e = blockIdx.x * kRtExp + warp;
+    // 1. logits: the tile's x rows in shared memory (chunks of 2048); warp w
+    //    takes expert blockIdx.x*2 + w/4 and a quarter of each chunk, so the
+    //    router spreads over E/2 CTAs per token tile; the four quarter sums
+    //    meet in shared memory
+    const int e = blockIdx.x * kRtExp + (warp >> 2);
+    const int quarter = warp & 3;
     float acc[kRtTok];
 #pragma unroll
     for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
     uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);   // [kRtTok][256] 16-byte vectors
     for (int c0 = 0; c0 < a.d; c0 += 2048) {
         const int cv = min(2048, a.d - c0) / 8;
-        uint4 wv[8];
+        uint4 wv[2];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int v = lane + 32 * q;
+        for (int q = 0; q < 2; ++q) {
+            const int v = quarter * 64 + lane + 32 * q;
             wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
         }
         __syncthreads();   // the previous chunk's x is no longer read
@@ -154,8 +163,8 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
         __syncthreads();
         if (e < a.E) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int v = lane + 32 * q;
+            for (int q = 0; q < 2; ++q) {
+                const int v = quarter * 64 + lane + 32 * q;
                 if (v < cv) {
 #pragma unroll
                     for (int r = 0; r < kRtTok; ++r)
@@ -164,14 +173,24 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
             }
         }
     }
-    if (e < a.E) {
 #pragma unroll
-        for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
-        if (lane == 0)
-            for (int r = 0; r < nt; ++r) a.ws.logits[(size_t)(t0 + r) * a.E + e] = acc[r];
+    for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
+    __syncthreads();   // x no longer needed: reuse shared memory for the quarter sums
+    float *qsum = s_dyn;   // [8 warps][kRtTok]
+    if (lane == 0)
+        for (int r = 0; r < kRtTok; ++r) qsum[warp * kRtTok + r] = acc[r];
+    __syncthreads();
+    if (threadIdx.x < kRtExp * kRtTok) {
+        const int ee = threadIdx.x / kRtTok, r = threadIdx.x % kRtTok;
+        const int eg = blockIdx.x * kRtExp + ee;
+        if (eg < a.E && r < nt) {
+            const float* q4 = qsum + (ee * 4) * kRtTok + r;
+            a.ws.logits[(size_t)(t0 + r) * a.E + eg] = q4[0] + q4[kRtTok] + q4[2 * kRtTok] + q4[3 * kRtTok];
+        }
     }
 
     // 2. last CTA of this token tile: softmax + top-k
+    if (tr && threadIdx.x == 0) tr[1] = global_ns();
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -182,6 +201,7 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    if (tr && threadIdx.x == 0) tr[2] = global_ns();
     if (warp < nt) {
         const int t = t0 + warp;
         float *row = s_dyn + warp * a.E;
@@ -195,45 +215,67 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
         float s = 0.f;
         for (int j = lane; j < a.E; j += 32) s += expf(row[j] - m);
         s = warp_sum(s);
-        unsigned taken = 0;   // bit q: expert lane + 32q already selected
-        for (int r = 0; r < a.k; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int q = 0, j = lane; j < a.E; ++q, j += 32) {
-                if (taken & (1u << q)) continue;
+        __syncwarp();
+        if (a.E <= kRankTopk) {
+            // rank of each logit = number of logits ranked before it (larger, or
+            // equal with a lower index); the ones with rank < k are the top-k,
+            // written straight to their rank -- no serial selection rounds
+            for (int j = lane; j < a.E; j += 32) {
                 const float v = row[j];
-                if (bi == 0x7fffffff || better(v, j, bv, bi)) { bv = v; bi = j; }
+                int rank = 0;
+                for (int i = 0; i < a.E; ++i) rank += better(row[i], i, v, j) ? 1 : 0;
+                if (rank < a.k) {
+                    a.ws.topk_idx[(size_t)t * a.k + rank] = j;
+                    a.ws.topk_w[(size_t)t * a.k + rank] = expf(v - m) / s;
+                }
             }
+        } else {
+            unsigned taken = 0;   // bit q: expert lane + 32q already selected
+            for (int r = 0; r < a.k; ++r) {
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+                for (int q = 0, j = lane; j < a.E; ++q, j += 32) {
+                    if (taken & (1u << q)) continue;
+                    const float v = row[j];
+                    if (bi == 0x7fffffff || better(v, j, bv, bi)) { bv = v; bi = j; }
+                }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(kFull, bv, o);
-                const int oi = __shfl_xor_sync(kFull, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-            }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (lane == 0) {
-                a.ws.topk_idx[(size_t)t * a.k + r] = bi;
-                a.ws.topk_w[(size_t)t * a.k + r] = expf(bv - m) / s;
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(kFull, bv, o);
+                    const int oi = __shfl_xor_sync(kFull, bi, o);
+                    if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+                }
+                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+                if (lane == 0) {
+                    a.ws.topk_idx[(size_t)t * a.k + r] = bi;
+                    a.ws.topk_w[(size_t)t * a.k + r] = expf(bv - m) / s;
+                }
             }
         }
     }
 
-    // 3. last token tile: the routing plan
+    // 3. last token tile: the routing plan (with a single tile, this CTA)
+    if (tr && threadIdx.x == 0) tr[3] = global_ns();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (gridDim.y > 1) {
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const int tk = atomicAdd(a.ws.done_ticket, 1);
+            s_last = (tk == (int)gridDim.y - 1);
+            if (s_last) *a.ws.done_ticket = 0;
+        }
+        __syncthreads();
+        if (!s_last) return;
         __threadfence();
-        const int tk = atomicAdd(a.ws.done_ticket, 1);
-        s_last = (tk == (int)gridDim.y - 1);
-        if (s_last) *a.ws.done_ticket = 0;
     }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
     int *s_int = reinterpret_cast<int *>(s_dyn);
     const int P = a.T * a.k;
     const bool staged = P <= kStagePairs;
+    if (tr && threadIdx.x == 0) tr[4] = global_ns();
     build_plan(a, s_int, s_int + a.E, staged ? s_int + 2 * a.E : nullptr,
                staged ? reinterpret_cast<float *>(s_int + 2 * a.E + P) : nullptr);
+    __syncthreads();
+    if (tr && threadIdx.x == 0) tr[5] = global_ns();
 }
 
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,

@@ -61,7 +61,7 @@ def _create(lib, w, E=8, k=2, d=256, f=512, S=0, maxT=16):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(E=0), -1), (dict(E=2000), -1), (dict(k=0), -1), (dict(k=9), -1),
-    (dict(d=260 - 1), -1), (dict(d=0), -1), (dict(f=48), -1), (dict(f=65536 + 32), -1),
+    (dict(d=260 - 1), -1), (dict(d=0), -1), (dict(d=4104), -1), (dict(f=48), -1), (dict(f=65536 + 32), -1),
     (dict(S=-1), -1), (dict(S=9), -1), (dict(maxT=-3), -1), (dict(maxT=70000), -1),
     (dict(S=1), -1),          # shared count without shared weights
 ])
