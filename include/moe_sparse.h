@@ -181,6 +181,34 @@ int moe_set_trace(moe_handle h, void *buf, long long bytes);
  * error word is reported in st->device_error and as MOE_EDEVICE. */
 int moe_query_stats(moe_handle h, moe_stats *st);
 
+/* Size of the fixed device scratch used by moe_router_topk_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (4 << 20)
+
+/* Router softmax top-k that allocates nothing, for callers that cannot call
+ * cudaMalloc: servers that reserve all device memory up front in their own
+ * arena, custom operators inside another framework that owns the allocator,
+ * and latency-critical paths where an allocation's implicit synchronisation
+ * is not acceptable.  The paper has no counterpart of this entry point; it
+ * computes the same routing as the router step of moe_sparse_forward (softmax
+ * over all E experts, top_k by probability, ties to the lower index, weight =
+ * probability) without a handle:
+ *   x        DEVICE [T][d_model] bf16, 16-byte aligned
+ *   w_router DEVICE [E][d_model] bf16, 16-byte aligned
+ *   idx_out  DEVICE [T][top_k] int32, w_out DEVICE [T][top_k] fp32, rank order
+ * Its scratch (the T*E fp32 logits, rounded up to 256 bytes, plus one int per
+ * 8 tokens) lives in a file-scope device array of MOE_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library keeps until the process exits; larger
+ * T*E (or more than 65535 tiles of 8 tokens) is rejected with MOE_ENOTSUP
+ * before anything is launched (e.g. E = 64 allows T up to 16352).  Other limits as moe_sparse_create: 1 <= top_k <= E
+ * <= 1024, d_model % 8 == 0.  The first call on a device looks up the array's
+ * device address with that device current, so make it before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU (on
+ * different streams) race and must be serialised by the caller.  Each call
+ * clears the tickets it needs with cudaMemsetAsync and calls no allocating
+ * routine.  Asynchronous on `stream`. */
+int moe_router_topk_noalloc(const void *x, int T, const void *w_router, int E, int d_model, int top_k,
+                            int *idx_out, float *w_out, void *stream);
+
 /* Static English text for an error code. */
 const char *moe_strerror(int code);
 

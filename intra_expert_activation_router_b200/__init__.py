@@ -13,7 +13,7 @@ _BINDING_NAMES = {
     "MoeError", "moe_debug_active", "moe_debug_router", "moe_dense_forward", "moe_query_stats",
     "moe_set_path", "moe_set_t_star", "moe_sparse_create", "moe_sparse_destroy",
     "moe_sparse_forward", "moe_sparse_forward_host", "moe_strerror", "raw_call",
-    "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace",
+    "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
 }
 
 

@@ -73,6 +73,7 @@ def _load():
         "moe_calibrate_tau": (I, [P, P, I, ctypes.c_double, ctypes.POINTER(F), P]),
         "moe_set_launch_events": (I, [P, ctypes.POINTER(P), I]),
         "moe_set_trace": (I, [P, P, ctypes.c_longlong]),
+        "moe_router_topk_noalloc": (I, [P, I, P, I, I, I, P, P, P]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -86,7 +87,7 @@ _lib = _load()
 EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_sparse_forward_host", "moe_sparse_destroy", "moe_set_path", "moe_set_t_star",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
-            "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace")
+            "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc")
 
 
 def _addr(t):
@@ -202,6 +203,13 @@ def moe_set_trace(h, buf, nbytes: int = 0):
         return
     n = nbytes or (buf.numel() * buf.element_size())
     _check(_lib.moe_set_trace(h, _addr(buf), n), "moe_set_trace")
+
+
+def moe_router_topk_noalloc(x, T: int, w_router, E: int, d_model: int, top_k: int, idx_out, w_out,
+                            stream=None):
+    """Router softmax top-k without a handle or any allocation (fixed device scratch)."""
+    _check(_lib.moe_router_topk_noalloc(_addr(x), T, _addr(w_router), E, d_model, top_k, _addr(idx_out),
+                                        _addr(w_out), _stream(stream)), "moe_router_topk_noalloc")
 
 
 def raw_call(name: str, *args) -> int:
