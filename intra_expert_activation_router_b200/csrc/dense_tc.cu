@@ -1,14 +1,388 @@
-// dense_tc.cu -- dense tensor-core (tcgen05) grouped-GEMM path.
+// dense_tc.cu -- the dense branch: the same masked layer through tcgen05
+// grouped GEMMs, for batches large enough that the union of active neurons
+// is dense ("Uncovering Intra-expert Activation Sparsity for Efficient
+// Mixture-of-Expert Model Execution", technical summary, Methodology item 3,
+// "Dynamic switching": sparse execution for small batches, dense for large).
+//
+//   gather   token rows in expert order (x_perm), and a copy of x for the
+//            shared experts, so every A tile is one TMA box
+//   GEMM1    per expert and 128-row tile of its tokens, per 128 neurons:
+//            D[128 x 256] = X_tile . [Wg rows | Wu rows]^T in TMEM (one
+//            M=128, N=256 MMA per 16 of K); epilogue h = silu(g) u, zeroed
+//            where |silu(g)| < tau on the masked path -> bf16 H
+//   GEMM2    per expert and tile, per 256 output dims:
+//            D[128 x 256] = H_tile . WdT rows^T; epilogue y_acc[token] +=
+//            w * D with fp32 vector atomics
+//   convert  out = bf16(y_acc), y_acc re-zeroed
+// Shared experts run as extra GEMM1/GEMM2 grids over all T tokens with the
+// mask off and weight 1.  Each GEMM CTA computes one tile: warp 0 issues the
+// TMA loads into a 4-stage ring, warp 1 issues the MMAs from one thread, all
+// four warps read the accumulator back for the epilogue.  Operands are K-major
+// with the 128-byte swizzle; the gate rows are stored pre-swizzled in HBM (see
+// gate_pos) and are copied with an unswizzled tensor map.
+#include <cuda.h>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace moe {
 
-bool dense_path_available() { return false; }
+constexpr int kBM = 128;            // token rows per tile
+constexpr int kBK = 64;             // K per stage (128 bytes of bf16)
+constexpr int kDStages = 4;
+constexpr int kDenseThreads = 128;
+constexpr int kATileBytes = kBM * kBK * 2;    // 16 KB
+constexpr int kBTileBytes = 256 * kBK * 2;    // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kDenseSmem = kDStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
 
-cudaError_t launch_dense(const Dims &, const DeviceWeights &, const Workspace &, const uint16_t *,
-                         int, float, bool, uint16_t *, int, cudaStream_t)
+enum DenseMode { kGateUp = 0, kDown = 1 };
+
+struct DenseArgs {
+    int mode;
+    int shared;        // 0: routed tiles from the plan; 1: shared expert `sidx` over all T tokens
+    int sidx;
+    int T, K, kb;      // tokens, contraction length, K blocks
+    int wrows;         // weight rows per expert (f for GEMM1, d for GEMM2)
+    int a_base;        // first A row of the launch (shared rows after the routed ones)
+    int h_base, h_ld;  // GEMM1: first H row, H row length (f)
+    float tau;
+    int use_mask;
+    const Plan *plan;
+    const int *perm_tok;
+    const float *perm_w;
+    uint16_t *h;       // GEMM1 output
+    float *y_acc;      // GEMM2 output
+    int d;
+    int *err;
+};
+
+// Token rows in expert order, plus the shared experts' copy of x.
+__global__ void k_dense_gather(const uint16_t *__restrict__ x, const int *__restrict__ perm_tok, int P, int T,
+                               int d8, int shared_base, uint16_t *__restrict__ x_perm)
 {
-    return cudaErrorNotSupported;
+    const size_t n = (size_t)(P + (shared_base >= 0 ? T : 0)) * d8;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = i / d8;
+        const int v = (int)(i % d8);
+        const int src = row < (size_t)P ? perm_tok[row] : (int)(row - P);
+        const size_t dst = row < (size_t)P ? row : (size_t)shared_base + (row - P);
+        reinterpret_cast<uint4 *>(x_perm)[dst * d8 + v] = ld_cached(x + ((size_t)src * d8 + v) * 8);
+    }
+}
+
+// out = bf16(y_acc) (round to nearest even), then y_acc = 0.
+__global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4)
+{
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = reinterpret_cast<const float4 *>(y_acc)[i];
+        uint2 p;
+        p.x = (uint32_t)f2bf_bits(v.x) | ((uint32_t)f2bf_bits(v.y) << 16);
+        p.y = (uint32_t)f2bf_bits(v.z) | ((uint32_t)f2bf_bits(v.w) << 16);
+        reinterpret_cast<uint2 *>(out)[i] = p;
+        reinterpret_cast<float4 *>(y_acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+}  // namespace moe
+
+namespace moe {
+
+__global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_constant__ DenseMaps maps, DenseArgs a)
+{
+    extern __shared__ uint8_t dsmem_raw[];
+    // the 128-byte swizzle needs 1024-byte aligned tiles
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDStages * kStageBytes);
+    uint64_t *empty = full + kDStages;
+    uint64_t *done = empty + kDStages;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(done + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- the tile: expert rows [row0, row0 + valid) of A, weight rows wrow0 + n0 ..
+    int row0, valid, wrow0;
+    if (!a.shared) {
+        const Plan *plan = a.plan;
+        const int n_tiles = plan->n_dense_tiles;
+        if ((int)blockIdx.x >= n_tiles) return;
+        const int mt = blockIdx.x;
+        int lo = 0, hi = plan->n_touched - 1;   // last slot with tile_prefix <= mt
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (plan->tile_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+        }
+        const int e = plan->touched[lo];
+        const int local = mt - plan->tile_prefix[lo];
+        const int off = plan->offsets[e], cnt = plan->offsets[e + 1] - off;
+        row0 = off + kBM * local;
+        valid = min(kBM, cnt - kBM * local);
+        wrow0 = e * a.wrows;
+    } else {
+        row0 = kBM * blockIdx.x;
+        valid = min(kBM, a.T - row0);
+        if (valid <= 0) return;
+        wrow0 = a.sidx * a.wrows;
+    }
+    const int ntile = a.mode == kGateUp ? 128 : 256;
+    const int n0 = blockIdx.y * ntile;
+
+    if (tid == 0) {
+        for (int s = 0; s < kDStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&maps.a);
+        tma_prefetch_desc(&maps.b0);
+        if (a.mode == kGateUp) tma_prefetch_desc(&maps.b1);
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0 && lane == 0) {
+        // ---- TMA producer
+        const uint32_t bytes = kATileBytes + (a.mode == kGateUp ? 2 * (kBTileBytes / 2) : kBTileBytes);
+        for (int kb = 0; kb < a.kb; ++kb) {
+            const int s = kb % kDStages;
+            mbar_wait(&empty[s], ((kb / kDStages) & 1) ^ 1, a.err, 31);
+            uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
+            mbar_arrive_expect_tx(&full[s], bytes);
+            tma_load_2d(A, &maps.a, kb * kBK, a.a_base + row0, &full[s]);
+            if (a.mode == kGateUp) {
+                tma_load_2d(B, &maps.b0, kb * kBK, wrow0 + n0, &full[s]);
+                tma_load_2d(B + kBTileBytes / 2, &maps.b1, kb * kBK, wrow0 + n0, &full[s]);
+            } else {
+                tma_load_2d(B, &maps.b0, kb * kBK, wrow0 + n0, &full[s]);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer: M = 128, N = 256, K = 16 per instruction
+        const uint32_t idesc = idesc_bf16_f32(kBM, 256);
+        for (int kb = 0; kb < a.kb; ++kb) {
+            const int s = kb % kDStages;
+            mbar_wait(&full[s], (kb / kDStages) & 1, a.err, 32);
+            tc_fence_after();
+            const uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+                umma_bf16(tmem, smem_desc_k_sw128(A + 32 * kk), smem_desc_k_sw128(B + 32 * kk), idesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+            umma_commit(&empty[s]);   // the stage is free once these MMAs have read it
+        }
+        umma_commit(done);
+    }
+    __syncwarp();
+
+    // ---- epilogue: thread = accumulator row (TMEM lane 32*warp + lane)
+    mbar_wait(done, 0, a.err, 33);
+    tc_fence_after();
+    const int row = warp * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    if (a.mode == kGateUp) {
+        uint16_t *hrow = a.h + (size_t)(a.h_base + row0 + row) * a.h_ld + n0;
+        for (int c = 0; c < 128; c += 16) {
+            float g[16], u[16];
+            tmem_ld16(tl + c, g);
+            tmem_ld16(tl + 128 + c, u);
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float hv[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float av = silu_f(g[2 * i + j]);
+                    const bool on = !a.use_mask || fabsf(av) >= a.tau;
+                    hv[j] = on ? av * u[2 * i + j] : 0.f;
+                }
+                pk[i] = (uint32_t)f2bf_bits(hv[0]) | ((uint32_t)f2bf_bits(hv[1]) << 16);
+            }
+            if (row < valid) {
+                reinterpret_cast<uint4 *>(hrow + c)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                reinterpret_cast<uint4 *>(hrow + c)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        }
+    } else {
+        int tok = 0;
+        float w = 1.f;
+        if (row < valid) {
+            tok = a.shared ? row0 + row : a.perm_tok[row0 + row];
+            w = a.shared ? 1.f : a.perm_w[row0 + row];
+        }
+        float *yrow = a.y_acc + (size_t)tok * a.d + n0;
+        for (int c = 0; c < 256; c += 16) {
+            float y[16];
+            tmem_ld16(tl + c, y);
+            if (row < valid) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 4)
+                    atomicAdd(reinterpret_cast<float4 *>(yrow + c + i),
+                              make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace moe
+
+namespace moe {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// A 2D bf16 matrix of `rows` rows of `cols` elements, `ld_bytes` apart; boxes of
+// 64 columns x box_rows rows.
+bool encode(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint64_t ld_bytes, uint32_t box_rows,
+            bool swizzle)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool dense_supported(const Dims &dm)
+{
+    return dm.d % 256 == 0 && dm.f % 128 == 0 && encode_fn() != nullptr;
+}
+
+bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st)
+{
+    st->ok = false;
+    if (!dense_supported(dm)) return true;   // not an error: the dense path is just unavailable
+    const uint64_t d = dm.d, f = dm.f, E = dm.E, S = dm.S;
+    const uint64_t Pm = (uint64_t)dm.max_tokens * dm.k, Tm = dm.max_tokens;
+    bool ok = true;
+    // GEMM1 routed / shared
+    ok = ok && encode(&st->g1r.a, ws.x_perm, d, Pm + Tm, 2 * d, kBM, true);
+    ok = ok && encode(&st->g1r.b0, w.wg_n, d, E * f, 2 * d, 128, false);
+    ok = ok && encode(&st->g1r.b1, w.wud, d, E * f, 4 * d, 128, true);
+    ok = ok && encode(&st->g2r.a, ws.h_perm, f, Pm + S * Tm, 2 * f, kBM, true);
+    ok = ok && encode(&st->g2r.b0, w.wdt, f, E * d, 2 * f, 256, true);
+    st->g2r.b1 = st->g2r.b0;
+    if (S > 0) {
+        st->g1s.a = st->g1r.a;
+        ok = ok && encode(&st->g1s.b0, w.wsg_n, d, S * f, 2 * d, 128, false);
+        ok = ok && encode(&st->g1s.b1, w.wsud, d, S * f, 4 * d, 128, true);
+        st->g2s.a = st->g2r.a;
+        ok = ok && encode(&st->g2s.b0, w.wsdt, f, S * d, 2 * f, 256, true);
+        st->g2s.b1 = st->g2s.b0;
+    }
+    st->ok = ok;
+    return ok;
+}
+
+cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s)
+{
+    if (!st.ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(k_dense_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kDenseSmem);
+    if (e != cudaSuccess) return e;
+    const int P = T * dm.k, Pm = dm.max_tokens * dm.k, Tm = dm.max_tokens;
+    const int d8 = dm.d / 8;
+    // gather
+    {
+        const size_t n = (size_t)(P + (dm.S > 0 ? T : 0)) * d8;
+        size_t blocks = (n + 255) / 256;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        k_dense_gather<<<(unsigned)blocks, 256, 0, s>>>(x, ws.perm_tok, P, T, d8, dm.S > 0 ? Pm : -1, ws.x_perm);
+    }
+    const int mbound = (P < dm.E ? P : dm.E) + P / kBM;
+    const int mshared = (T + kBM - 1) / kBM;
+    DenseArgs a = {};
+    a.T = T;
+    a.tau = tau;
+    a.use_mask = use_mask ? 1 : 0;
+    a.plan = ws.plan;
+    a.perm_tok = ws.perm_tok;
+    a.perm_w = ws.perm_w;
+    a.h = ws.h_perm;
+    a.h_ld = dm.f;
+    a.y_acc = ws.y_acc;
+    a.d = dm.d;
+    a.err = ws.error_word;
+    // GEMM1: gate | up with the mask epilogue
+    a.mode = kGateUp;
+    a.K = dm.d;
+    a.kb = dm.d / kBK;
+    a.wrows = dm.f;
+    a.shared = 0;
+    a.a_base = 0;
+    a.h_base = 0;
+    k_dense_gemm<<<dim3(mbound, dm.f / 128, 1), kDenseThreads, kDenseSmem, s>>>(st.g1r, a);
+    if (dm.S > 0) {
+        a.shared = 1;
+        a.a_base = Pm;
+        a.use_mask = 0;
+        for (int z = 0; z < dm.S; ++z) {
+            DenseArgs az = a;
+            az.sidx = z;
+            az.h_base = Pm + z * Tm;   // shared expert z's H rows
+            k_dense_gemm<<<dim3(mshared, dm.f / 128, 1), kDenseThreads, kDenseSmem, s>>>(st.g1s, az);
+        }
+    }
+    // GEMM2: down with the routing-weight epilogue
+    a.mode = kDown;
+    a.K = dm.f;
+    a.kb = dm.f / kBK;
+    a.wrows = dm.d;
+    a.shared = 0;
+    a.a_base = 0;
+    a.use_mask = use_mask ? 1 : 0;
+    k_dense_gemm<<<dim3(mbound, dm.d / 256, 1), kDenseThreads, kDenseSmem, s>>>(st.g2r, a);
+    for (int z = 0; z < dm.S; ++z) {
+        DenseArgs az = a;
+        az.shared = 1;
+        az.sidx = z;
+        az.a_base = Pm + z * Tm;
+        k_dense_gemm<<<dim3(mshared, dm.d / 256, 1), kDenseThreads, kDenseSmem, s>>>(st.g2s, az);
+    }
+    // convert
+    {
+        const size_t n4 = (size_t)T * dm.d / 4;
+        size_t blocks = (n4 + 255) / 256;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        k_dense_convert<<<(unsigned)blocks, 256, 0, s>>>(ws.y_acc, out, n4);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace moe

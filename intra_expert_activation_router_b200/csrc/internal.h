@@ -19,6 +19,7 @@
 //     calls), tok_cnt [T] (kept zero between calls), plan (below).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -49,6 +50,19 @@ struct DeviceWeights {
     const uint16_t *wr;
     const uint16_t *wg_n, *wud;
     const uint16_t *wsg_n, *wsud;
+    const uint16_t *wdt, *wsdt;   // dense branch only: down weights transposed, [E][d][f] / [S][d][f]
+};
+
+// Tensor maps of one dense GEMM launch (kernel parameters).
+struct DenseMaps {
+    CUtensorMap a;    // GEMM1: x_perm rows; GEMM2: H rows (128-byte swizzle, box 64 x 128)
+    CUtensorMap b0;   // GEMM1: gate rows (stored pre-swizzled, copied unswizzled); GEMM2: WdT rows (box 64 x 256)
+    CUtensorMap b1;   // GEMM1: up halves of the [up | down] records; GEMM2: unused
+};
+
+struct DenseState {
+    bool ok;                           // shape supported and maps encoded
+    DenseMaps g1r, g1s, g2r, g2s;      // GEMM1/GEMM2, routed/shared
 };
 
 // Position of element k inside a swizzled gate row j (see wg_n above).
@@ -74,8 +88,8 @@ struct Workspace {
     int *error_word;    // nonzero once a kernel reports an error
     Plan *plan;
     // dense path
-    uint16_t *x_perm;   // [T*k][d] bf16, tokens gathered in perm order
-    uint16_t *h_perm;   // [T*k][f] bf16, masked SwiGLU activations
+    uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts
+    uint16_t *h_perm;   // [T*k + S*T][f] bf16: masked SwiGLU activations, routed then shared
     // host-pointer entry
     uint16_t *x_stage, *out_stage;
     // optional phase timestamps (moe_set_trace); nullptr when off
@@ -112,6 +126,11 @@ cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned lo
 
 cudaError_t launch_radix_hist(const uint32_t *v, size_t n, uint32_t prefix, uint32_t prefix_mask,
                               int shift, unsigned *hist, int n_sm, cudaStream_t st);
+
+bool dense_supported(const Dims &dm);
+bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st);
+cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s);
 
 int sparse_tile_tokens(int T, int d);   // tokens per sparse work item for a batch of T
 

@@ -13,15 +13,12 @@
 
 namespace moe {
 int sparse_blocks_per_sm(int mt);
-bool dense_path_available();
-cudaError_t launch_dense(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                         const uint16_t *x, int T, float tau, bool use_mask, uint16_t *out,
-                         int n_sm, cudaStream_t st);
 }
 
 namespace {
 
 constexpr unsigned kMagic = 0x4d6f4553u;   // "MoES"
+constexpr int kDefaultTStar = 16;       // AUTO: sparse iff T <= this, when the dense branch exists
 
 struct Block {   // bump allocator over one cudaMalloc
     char *base = nullptr;
@@ -53,6 +50,7 @@ struct moe_sparse_s {
     // the last forward
     int last_T, last_path, last_masked;
     cudaStream_t last_stream;
+    moe::DenseState dense;   // tensor maps of the dense branch (dense.ok: available)
     cudaEvent_t ev[3];   // optional launch events (moe_set_launch_events)
     int n_ev;
     float *scores;       // calibration buffer, allocated by the first moe_calibrate_tau
@@ -121,7 +119,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     if (!h) return MOE_ENOMEM;
     h->magic = kMagic;
     h->path = MOE_PATH_AUTO;
-    h->t_star = moe::dense_path_available() ? 128 : INT_MAX;
+    h->t_star = INT_MAX;   // set below once the dense branch is known to be available
     if (cudaGetDevice(&h->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
         delete h;
@@ -132,11 +130,13 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     for (int i = 0; i < 4; ++i) h->grid_cap[i] = h->n_sm * moe::sparse_blocks_per_sm(1 << i);
 
     const size_t fd = (size_t)d_ff * d_model;
-    const size_t wbytes = 2 * ((size_t)E * d_model + 3 * E * fd + 3 * (size_t)n_shared * fd) + 16 * 256;
+    const bool dense = moe::dense_supported(dm);
+    const size_t wbytes = 2 * ((size_t)E * d_model + 3 * E * fd + 3 * (size_t)n_shared * fd) +
+                          (dense ? 2 * ((size_t)E + n_shared) * fd : 0) + 16 * 256;
     const size_t T = max_tokens, P = T * top_k;
     const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
-                           4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * P * d_model +
-                           2 * P * d_ff + 2 * 2 * T * d_model + 64 + 1024 + 32 * 256;
+                           4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * (P + T) * d_model +
+                           2 * (P + n_shared * T) * d_ff + 2 * 2 * T * d_model + 64 + 1024 + 32 * 256;
     if (cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
     if (cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
 
@@ -148,8 +148,16 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
         wsg = (uint16_t *)wb.take(2 * n_shared * fd);
         wsud = (uint16_t *)wb.take(4 * n_shared * fd);
     }
-    if (!wr || !wg || !wud || (n_shared && (!wsg || !wsud))) { free_handle(h); return MOE_ENOMEM; }
-    h->w = {wr, wg, wud, wsg, wsud};
+    uint16_t *wdt = nullptr, *wsdt = nullptr;
+    if (dense) {
+        wdt = (uint16_t *)wb.take(2 * E * fd);
+        if (n_shared) wsdt = (uint16_t *)wb.take(2 * n_shared * fd);
+    }
+    if (!wr || !wg || !wud || (n_shared && (!wsg || !wsud)) || (dense && (!wdt || (n_shared && !wsdt)))) {
+        free_handle(h);
+        return MOE_ENOMEM;
+    }
+    h->w = {wr, wg, wud, wsg, wsud, wdt, wsdt};
 
     Block sb{(char *)h->ws_mem, 0, wsbytes};
     moe::Workspace &ws = h->ws;
@@ -166,8 +174,8 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.done_ticket = (int *)sb.take(4);
     ws.error_word = (int *)sb.take(4);
     ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
-    ws.x_perm = (uint16_t *)sb.take(2 * P * d_model);
-    ws.h_perm = (uint16_t *)sb.take(2 * P * d_ff);
+    ws.x_perm = (uint16_t *)sb.take(2 * (P + T) * d_model);
+    ws.h_perm = (uint16_t *)sb.take(2 * (P + n_shared * T) * d_ff);
     ws.x_stage = (uint16_t *)sb.take(2 * T * d_model);
     ws.out_stage = (uint16_t *)sb.take(2 * T * d_model);
     h->stats_dev = (unsigned long long *)sb.take(64);
@@ -181,12 +189,21 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_gate, wg, E, d, d_ff, d, 0, true, st) == cudaSuccess;
     ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wud, E, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
     ok = ok && moe::launch_repack_rows((const uint16_t *)w->w_down, wud, E, d_ff, d, 2 * d, d, st) == cudaSuccess;
+    if (dense) {
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_down, wdt, E, d_ff, d, d_ff, 0, false, st) == cudaSuccess;
+        if (n_shared)
+            ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_down, wsdt, n_shared, d_ff, d, d_ff, 0, false, st) == cudaSuccess;
+    }
     if (n_shared) {
         ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_gate, wsg, n_shared, d, d_ff, d, 0, true, st) == cudaSuccess;
         ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsud, n_shared, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
         ok = ok && moe::launch_repack_rows((const uint16_t *)w->ws_down, wsud, n_shared, d_ff, d, 2 * d, d, st) == cudaSuccess;
     }
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    ok = ok && moe::dense_setup(h->dm, h->w, h->ws, &h->dense);
+    // measured on B200 at the OLMoE shape, 90 % sparsity: the sparse branch
+    // is faster through T = 16 tokens, the dense branch from T = 32 on
+    if (h->dense.ok) h->t_star = kDefaultTStar;
     if (!ok) {
         cudaGetLastError();
         free_handle(h);
@@ -223,7 +240,10 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     int path = forced_path;
     if (path == MOE_PATH_AUTO) path = h->path;
     if (path == MOE_PATH_AUTO) path = (T <= h->t_star) ? MOE_PATH_SPARSE : MOE_PATH_DENSE;
-    if (path == MOE_PATH_DENSE && !moe::dense_path_available()) return MOE_ENOTSUP;
+    if (path == MOE_PATH_DENSE && !h->dense.ok) {
+        if (forced_path == MOE_PATH_DENSE || h->path == MOE_PATH_DENSE) return MOE_ENOTSUP;
+        path = MOE_PATH_SPARSE;   // AUTO on a shape the dense branch does not cover
+    }
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
     uint16_t *ob = (uint16_t *)out;
@@ -240,7 +260,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
         if (e == cudaSuccess)
-            e = moe::launch_dense(h->dm, h->w, h->ws, xb, T, tau, masked, ob, h->n_sm, st);
+            e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st);
     }
     if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[2], st);
     h->last_T = T;
@@ -281,7 +301,7 @@ extern "C" int moe_set_path(moe_handle h, int path)
 {
     if (!is_live(h)) return MOE_EHANDLE;
     if (path != MOE_PATH_AUTO && path != MOE_PATH_SPARSE && path != MOE_PATH_DENSE) return MOE_EINVAL;
-    if (path == MOE_PATH_DENSE && !moe::dense_path_available()) return MOE_ENOTSUP;
+    if (path == MOE_PATH_DENSE && !h->dense.ok) return MOE_ENOTSUP;
     h->path = path;
     return MOE_OK;
 }

@@ -1,0 +1,142 @@
+"""The dense tensor-core branch (tcgen05 grouped GEMMs) against the CPU oracle
+and against the sparse branch, through the C ABI.
+
+The dense branch rounds h to bf16 before the down projection, so outputs are
+compared at the layer's 1e-2 relative-L2 bar.  Its mask is decided on
+tensor-core fp32 gate values; a token is exempt from the output check only
+if one of its neurons scores within 1e-5*tau of tau (where fp32 accumulation
+order may decide either way) or its router is a near tie.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def o():
+    return oracle.load()
+
+
+_cache = {}
+
+
+def layer_for(name):
+    if name not in _cache:
+        for k in list(_cache):
+            _cache.pop(k)[0].close()
+        torch.cuda.empty_cache()
+        sh = mi.SHAPES[name]
+        layer, W = pu.gpu_layer(sh, max_tokens=4096)
+        _cache[name] = (layer, W, oracle.layer_inputs(W, torch.zeros(1, sh.d_model, dtype=torch.bfloat16)))
+    return _cache[name]
+
+
+def run_dense(o, name, T, q, sample=None, masked=True):
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    cal = dict(inputs)
+    cal["x"] = inputs["x"][:64]
+    tau = pu.calibrate(o, cal, sh.top_k, q) if masked else 0.0
+    if masked:
+        layer.set_path(m.MOE_PATH_DENSE)
+        out = layer.forward(x, tau)
+        layer.set_path(m.MOE_PATH_AUTO)
+    else:
+        out = layer.dense_forward(x)
+    torch.cuda.synchronize()
+    st = layer.stats()
+    assert st["path"] == m.MOE_PATH_DENSE and st["device_error"] == 0
+    rows = np.arange(T) if sample is None else np.sort(
+        np.random.default_rng(7 * T + 1).choice(T, size=min(sample, T), replace=False))
+    sub = dict(inputs)
+    sub["x"] = inputs["x"][rows]
+    ref = o.forward(**sub, top_k=sh.top_k, tau=tau)
+    exempt = pu.near_tie_tokens(ref.logits, sh.top_k)
+    if masked and tau > 0:
+        exempt |= np.any(np.abs(ref.score - tau) <= 1e-5 * tau, axis=(1, 2))
+    assert exempt.sum() <= max(2, len(rows) // 20)
+    pu.check_output(ref.y, out[torch.as_tensor(rows, device="cuda")], exempt)
+    return layer, x, tau, out
+
+
+def test_tiny_dense_masked(o):
+    run_dense(o, "tiny", 16, 0.9)
+
+
+def test_tiny_dense_unmasked(o):
+    run_dense(o, "tiny", 16, 0.0, masked=False)
+
+
+@pytest.mark.parametrize("T", [1, 64, 257, 1000, 4096])
+def test_olmoe_dense(o, T):
+    run_dense(o, "olmoe", T, 0.9, sample=None if T <= 64 else 12)
+
+
+def test_olmoe_dense_unmasked_baseline(o):
+    run_dense(o, "olmoe", 300, 0.0, sample=12, masked=False)
+
+
+@pytest.mark.parametrize("T", [8, 128])
+def test_dsv2lite_dense_shared(o, T):
+    run_dense(o, "dsv2lite", T, 0.8, sample=None if T <= 8 else 12)
+
+
+def test_large_dense(o):
+    run_dense(o, "large", 64, 0.98, sample=8)
+
+
+def test_dense_matches_sparse(o):
+    """Both branches of the same layer at the same tau agree (up to h's bf16 rounding)."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    x = mi.make_x(sh, 48, device="cuda")
+    tau = layer.calibrate_tau(x, 0.9)
+    layer.set_path(m.MOE_PATH_SPARSE)
+    ys = layer.forward(x, tau).float()
+    layer.set_path(m.MOE_PATH_DENSE)
+    yd = layer.forward(x, tau).float()
+    layer.set_path(m.MOE_PATH_AUTO)
+    torch.cuda.synchronize()
+    rel = ((yd - ys).norm(dim=1) / ys.norm(dim=1)).cpu().numpy()
+    # a rare band neuron decided differently moves one token by a few percent
+    assert np.sum(rel > 1e-2) <= 2 and np.median(rel) < 5e-3
+
+
+def test_auto_switch_picks_by_batch(o):
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    layer.set_t_star(32)
+    for T, want in ((32, m.MOE_PATH_SPARSE), (33, m.MOE_PATH_DENSE)):
+        x = mi.make_x(sh, T, device="cuda")
+        layer.forward(x, 1.0)
+        assert layer.stats()["path"] == want
+    layer.set_t_star(16)
+
+
+def test_dense_unsupported_shape_rejected():
+    import intra_expert_activation_router_b200 as m
+    sh = mi.custom_shape(264, 4, 32, 4, 0)   # d not a multiple of 256: no dense branch
+    W = mi.make_weights(sh, device="cuda")
+    layer = m.MoESparseLayer.from_weights(W, 4, max_tokens=16)
+    x = mi.make_x(sh, 4, device="cuda")
+    with pytest.raises(m.MoeError) as ei:
+        layer.dense_forward(x)
+    assert ei.value.code == m.MOE_ENOTSUP
+    layer.set_t_star(0)          # AUTO above T* falls back to the sparse branch on such shapes
+    layer.forward(x, 0.5)
+    torch.cuda.synchronize()
+    assert layer.stats()["path"] == m.MOE_PATH_SPARSE
+    layer.close()

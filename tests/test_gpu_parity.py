@@ -52,8 +52,11 @@ def run_case(o, name, T, q, sample=None, check_lists=True):
     cal = dict(inputs)
     cal["x"] = inputs["x"][:64]
     tau = pu.calibrate(o, cal, sh.top_k, q, NTHREADS)
-    # the GPU path on the whole batch
+    # the sparse GPU path on the whole batch (large batches would otherwise switch to dense)
+    import intra_expert_activation_router_b200 as m
+    layer.set_path(m.MOE_PATH_SPARSE)
     out = layer.forward(x, tau)
+    layer.set_path(m.MOE_PATH_AUTO)
     idx, w = layer.router(x)
     lists, cnt = layer.active_lists(x, tau) if check_lists else (None, None)
     torch.cuda.synchronize()
