@@ -166,13 +166,16 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * The first half of the buffer holds 8 stamps per router CTA (CTA index
  * y*gridDim.x + x): start, logits done, top-k start, top-k done, plan start,
  * plan done (the last two only in the CTA that builds the plan).  The second
- * half holds 64 per expert-kernel CTA: [0] start, [1] plan loaded, then for
- * each of the CTA's first four items i, at 2 + 12*i: token rows in, the four
- * 8-row gate groups in, gate done, mask done, gather issued, first gathered
- * records in, up/down done, accumulator flushed (if it was); [50] end and
- * [51] the CTA's item count; [52 + 2i], [53 + 2i] first and last gate stage
- * of item i issued; [60 + i] token rows of item i issued; [40 + s] arrival
- * of gate stage s, for the first ring-full of stages (at most 8).  Unwritten slots keep their old contents.
+ * half holds 64 per expert-kernel CTA: [0] start, [1] plan loaded; for each
+ * of the CTA's first three items i, at 2 + 10*i: metadata ready, gate
+ * accumulator ready, mask read out (twice), mask step synchronised, mask and
+ * lists published, first gathered batch in, first batch consumed, last batch
+ * consumed, up/down done; [32 + 4u] for the gather of item u < 2: mask seen,
+ * then the issue times of its first three batches; [40 + g] issue of gate
+ * stage g < 8; [48 + q] token rows of tile q < 8 ready; [56 + 2i], [57 + 2i]
+ * first gate stage consumed and accumulator committed for item i < 3; [61]
+ * gathered records processed; [62] end; [63] the CTA's item count.  Unwritten
+ * slots keep their old contents.
  * buf == NULL turns tracing off. */
 int moe_set_trace(moe_handle h, void *buf, long long bytes);
 

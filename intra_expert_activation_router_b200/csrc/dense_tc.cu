@@ -18,8 +18,8 @@
 // mask off and weight 1.  Each GEMM CTA computes one tile: warp 0 issues the
 // TMA loads into a 4-stage ring, warp 1 issues the MMAs from one thread, all
 // four warps read the accumulator back for the epilogue.  Operands are K-major
-// with the 128-byte swizzle; the gate rows are stored pre-swizzled in HBM (see
-// gate_pos) and are copied with an unswizzled tensor map.
+// with the 128-byte swizzle; the gate weights are stored in HBM as exactly
+// these tiles (gate_tile_off), so each is one plain 16 KB bulk copy.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -46,6 +46,8 @@ struct DenseArgs {
     int T, K, kb;      // tokens, contraction length, K blocks
     int wrows;         // weight rows per expert (f for GEMM1, d for GEMM2)
     int a_base;        // first A row of the launch (shared rows after the routed ones)
+    const uint16_t *gate;   // GEMM1: gate tiles of the routed (or shared) experts
+    int n_kb, n_blk;        // GEMM1: gate tiles per 128-neuron block, blocks per expert
     int h_base, h_ld;  // GEMM1: first H row, H row length (f)
     float tau;
     int use_mask;
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- the tile: expert rows [row0, row0 + valid) of A, weight rows wrow0 + n0 ..
-    int row0, valid, wrow0;
+    int row0, valid, wrow0, ex;
     if (!a.shared) {
         const Plan *plan = a.plan;
         const int n_tiles = plan->n_dense_tiles;
@@ -118,11 +120,13 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
         row0 = off + kBM * local;
         valid = min(kBM, cnt - kBM * local);
         wrow0 = e * a.wrows;
+        ex = e;
     } else {
         row0 = kBM * blockIdx.x;
         valid = min(kBM, a.T - row0);
         if (valid <= 0) return;
         wrow0 = a.sidx * a.wrows;
+        ex = a.sidx;
     }
     const int ntile = a.mode == kGateUp ? 128 : 256;
     const int n0 = blockIdx.y * ntile;
@@ -135,8 +139,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
         mbar_init(done, 1);
         fence_mbar_init();
         tma_prefetch_desc(&maps.a);
-        tma_prefetch_desc(&maps.b0);
         if (a.mode == kGateUp) tma_prefetch_desc(&maps.b1);
+        else tma_prefetch_desc(&maps.b0);
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, 256);
@@ -157,7 +161,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
             mbar_arrive_expect_tx(&full[s], bytes);
             tma_load_2d(A, &maps.a, kb * kBK, a.a_base + row0, &full[s]);
             if (a.mode == kGateUp) {
-                tma_load_2d(B, &maps.b0, kb * kBK, wrow0 + n0, &full[s]);
+                const uint16_t *gt = a.gate + (((size_t)ex * a.n_blk + blockIdx.y) * a.n_kb + kb) * (kBM * kBK);
+                bulk_g2s(B, gt, kBTileBytes / 2, &full[s]);
                 tma_load_2d(B + kBTileBytes / 2, &maps.b1, kb * kBK, wrow0 + n0, &full[s]);
             } else {
                 tma_load_2d(B, &maps.b0, kb * kBK, wrow0 + n0, &full[s]);
@@ -293,15 +298,17 @@ bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, De
     bool ok = true;
     // GEMM1 routed / shared
     ok = ok && encode(&st->g1r.a, ws.x_perm, d, Pm + Tm, 2 * d, kBM, true);
-    ok = ok && encode(&st->g1r.b0, w.wg_n, d, E * f, 2 * d, 128, false);
     ok = ok && encode(&st->g1r.b1, w.wud, d, E * f, 4 * d, 128, true);
+    st->g1r.b0 = st->g1r.b1;   // unused: gate tiles are bulk copies
+    st->gate_r = w.wg_t;
+    st->gate_s = w.wsg_t;
     ok = ok && encode(&st->g2r.a, ws.h_perm, f, Pm + S * Tm, 2 * f, kBM, true);
     ok = ok && encode(&st->g2r.b0, w.wdt, f, E * d, 2 * f, 256, true);
     st->g2r.b1 = st->g2r.b0;
     if (S > 0) {
         st->g1s.a = st->g1r.a;
-        ok = ok && encode(&st->g1s.b0, w.wsg_n, d, S * f, 2 * d, 128, false);
         ok = ok && encode(&st->g1s.b1, w.wsud, d, S * f, 4 * d, 128, true);
+        st->g1s.b0 = st->g1s.b1;
         st->g2s.a = st->g2r.a;
         ok = ok && encode(&st->g2s.b0, w.wsdt, f, S * d, 2 * f, 256, true);
         st->g2s.b1 = st->g2s.b0;
@@ -341,6 +348,9 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     a.err = ws.error_word;
     // GEMM1: gate | up with the mask epilogue
     a.mode = kGateUp;
+    a.gate = st.gate_r;
+    a.n_kb = dm.n_kb;
+    a.n_blk = dm.n_blk;
     a.K = dm.d;
     a.kb = dm.d / kBK;
     a.wrows = dm.f;
@@ -352,6 +362,7 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
         a.shared = 1;
         a.a_base = Pm;
         a.use_mask = 0;
+        a.gate = st.gate_s;
         for (int z = 0; z < dm.S; ++z) {
             DenseArgs az = a;
             az.sidx = z;

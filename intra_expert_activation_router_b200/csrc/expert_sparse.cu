@@ -1,69 +1,93 @@
-// expert_sparse.cu -- fused gate projection, threshold mask, compaction and
-// gathered up/down projection for the routed experts (and the dense shared
-// experts): a persistent, warp-specialised kernel fed by bulk copies (TMA).
+// expert_sparse.cu -- the sparse branch: gate projection on the tensor cores,
+// threshold mask, compaction, and the gathered up/down projection of the
+// active neurons, in one persistent warp-specialised kernel.
 //
 // "Uncovering Intra-expert Activation Sparsity for Efficient Mixture-of-Expert
 // Model Execution" (technical summary, Methodology item 3):
 //   - gate projection, dense ("Gate projection" bullet): g = x Wg[e] for every
-//     neuron of the selected expert;
+//     neuron of the selected expert -- here a tcgen05 MMA per 128-neuron block:
+//     D[128 neurons x 16 columns] (TMEM) = Wg block . X tile^T, the block's
+//     gate tiles streamed through a ring of 32 KB stages (bulk copies), the
+//     tile's token rows resident in shared memory in the MMA's layout;
 //   - activation mask in one O(n) pass, no sort ("Activation masking"):
-//     active iff |silu(g)| >= tau -- a warp ballot over 32 neurons;
+//     active iff |silu(g)| >= tau -- a warp ballot over 32 neurons per token;
 //   - fused up-down projection over the active neurons only ("Fused up-down
 //     projection"): the active rows of Wu and Wd are gathered and packed
 //     densely in shared memory, h = silu(g) * (x Wu[:,j]) and y += w h Wd[j][:]
-//     (Hindi summary, "The skip": inactive neurons' weights are never loaded).
+//     (Hindi summary, "The skip": inactive neurons' weights are never loaded);
 //   - shared experts: the same code with the mask off and weight 1 (their
 //     execution is unchanged and always dense).
 //
-// Work items are (expert, token tile of up to MT of that expert's tokens,
-// chunk of 32 neurons), ordered expert, tile, chunk.  Each CTA (one per SM)
-// takes a contiguous range of items and runs three agents:
-//   gate/x lane (warp 8)  item metadata and the tile's token rows (copied only
-//                         when the (expert, tile) changes, into one of two
-//                         slots), and the chunk's gate rows in 32 KB stages
-//                         into a ring -- few, large bulk copies, since each
-//                         copy costs the issuing thread a fixed time;
-//   gather warp (warp 9)  once an item's mask is final, its union-active
-//                         neurons' [up | down] records (4d bytes each), in
-//                         batches, copies split over four lanes;
-//   consumers (warps 0-7) in the order G(0) M(0) | G(1) M(1) UD(0) | ..., so
-//                         the gather of item i lands while the gate rows of
-//                         item i+1 are reduced:
-//   G   each warp owns a slice of d, holds the tile's tokens for that slice in
-//       registers and, per group of 8 gate rows, accumulates fp32 dot
-//       products, then one transposed warp reduction leaves a partial per
-//       (row, token);
-//   M   the 8 slice partials are summed, silu and the threshold evaluated, a
-//       32-bit mask word balloted per token (written out as the pair's mask),
-//       and the union of the tile's words compacted into an ascending list;
-//   UD  up rows: the same slice dots give u, then h = bit ? silu(g) u : 0;
-//       down rows: each thread owns 8 output dims per pass and accumulates
-//       sum_j h_j Wd[j][:] in registers across consecutive items of the same
-//       (expert, tile); when that changes the partial goes to the fp32
-//       accumulator y_acc[token] with vector atomics and a per-token ticket
-//       counts the chunks; the token's last chunk converts y_acc to bf16 into
-//       `out` and re-zeroes its row and ticket.
-// The agents meet on mbarriers (copies, buffer reuse) and on monotonic
-// progress counters in shared memory; every wait is bounded.
+// Work items are (expert, tile of up to NT of its tokens, block of 128
+// neurons), ordered expert, tile, block; each CTA (one per SM) takes a
+// contiguous range.  Agents:
+//   gate lane (warp 8)     the item's gate tiles, 32 KB stages into the ring
+//   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of two
+//                          TMEM accumulators; owns the TMEM allocation
+//   x warp (warp 10)       per tile, the token rows into the MMA's K-major
+//                          128-byte-swizzled layout (cp.async), once the MMAs
+//                          of the previous tile are done
+//   gather warp (warp 11)  once an item's mask is final, the union-active
+//                          [up | down] records, in batches, two buffers
+//   consumers (warps 0-7)  M(i): warps 0-3 read the accumulator (one neuron per
+//                          thread), silu, threshold, ballot per token; the mask
+//                          words and, per pass of MT tokens, the ascending list
+//                          of union-active neurons; then UD(i-1) on the CUDA
+//                          cores: up dots (each warp a slice of d, one
+//                          transposed warp reduction per group of 4 rows), h,
+//                          down rows accumulated in registers across the
+//                          blocks of one (expert, tile); when that changes the
+//                          partial goes to the fp32 accumulator y_acc[token]
+//                          with vector atomics and a per-token ticket counts
+//                          the blocks; the token's last block converts y_acc
+//                          to bf16 into `out` and re-zeroes its row and ticket.
+// The agents meet on mbarriers (copies, MMA completion, buffer reuse) and on a
+// monotonic progress counter in shared memory; every wait is bounded.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 #include "tma.cuh"
 
 namespace moe {
 
 constexpr int kConsumerThreads = 256;
-constexpr int kSparseThreads = kConsumerThreads + 64;   // + gate/x producer warp + gather warp
-constexpr int kSparseSmemBudget = 220 * 1024;
-constexpr int kPrefetchStages = 1;   // next-item gate stages allowed before the previous gather starts
-constexpr int kGatherLanes = 4;      // lanes of the gather warp that issue copies
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpX = 10, kWarpGather = 11;
+constexpr int kSparseThreads = 384;
+constexpr int kGateTile = 16384;     // bytes of one gate tile: 128 neurons x 64 inputs
+constexpr int kStageBytes = 2 * kGateTile;
+constexpr int kMaxNT = 16;           // tokens per gate tile
+constexpr int kMaxSub = 4;           // passes of MT tokens per tile
+constexpr int kRows = 4;             // up rows per warp reduction
+constexpr int kMaxGB = 8;            // records per gather buffer
+constexpr int kAcc = 4;              // TMEM gate accumulators (the MMA runs up to kAcc items ahead)
+constexpr int kTmemCols = 16 * kAcc;
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kMaxNU = 6;            // gather buffers
+constexpr int kIdRing = 16;          // published work-item ids
+constexpr int kNumFixedBars = 2 * kAcc + 3;   // mbarriers besides the two rings': gdone, tfree, xfull, xfree, mdrain
 
-struct SparseLayout {   // byte offsets into dynamic shared memory
-    int ring_off, stage_bytes, rows_per_stage, n_stages, stages_per_chunk;
-    int gather_off, gather_rows, gpitch;   // neuron records [Wu row | Wd row] + 16-byte skew
-    int xbuf_off, xbuf_bytes, xpitch;      // token rows + 16-byte skew
-    int meta_off, meta_bytes;
-    int part_off, h_off, last_off, plan_off, bar_off;
-    int total;
+struct SparseLayout {   // byte offsets from the 1024-aligned base of dynamic shared memory
+    int xt_off, xt_kb;                      // token tile; bytes per 64-input block (nt * 128)
+    int ring_off, n_stages;
+    int ud_off, ud_buf_bytes, gb, gpitch;   // n_ud buffers of gb [up | down] records (+16-byte skew)
+    int n_ud;
+    int meta_off, part_off, h_off, last_off, ctr_off, plan_off, bar_off;
+    int total;                              // dynamic bytes to request (includes alignment slack)
+};
+
+struct ItemMeta {
+    const uint16_t *wud;          // the expert's [f][2d] up/down records
+    long long key;                // (expert slot or shared index, token tile)
+    int m, blk, masked, nsub;
+    int tok[kMaxNT];
+    int pair[kMaxNT];
+    float w[kMaxNT];
+    unsigned word[kMaxNT][4];     // mask words: token, 32-neuron quarter of the block
+    int n_uni[kMaxSub];
+    uint8_t uni[kMaxSub][kBlk];   // per pass: union-active neurons of the block, ascending
+    __half a[kMaxNT][kBlk];       // silu(g)
 };
 
 struct SparseArgs {
@@ -72,44 +96,96 @@ struct SparseArgs {
     DeviceWeights w;
     Workspace ws;
     int T, d, f, k, S;
+    int dp, n_kb, n_blk, n_chunks;
+    int nt;               // tokens per gate tile
+    int resident;         // T <= nt: the whole batch is the MMA's token operand, loaded once,
+                          // and work items are claimed dynamically, heaviest expert first
     float tau;
     int use_mask;
-    int n_chunks;
-    int n_tok_tiles;      // ceil(T / MT), for the shared experts
-    int n_shared_items;   // S * n_tok_tiles * n_chunks
-    int target;           // chunk contributions per token: (k + S) * n_chunks
+    int n_tok_tiles;      // ceil(T / nt), for the shared experts
+    int n_shared_items;   // S * n_tok_tiles * n_blk
+    int target;           // block contributions per token: (k + S) * n_blk
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f], no up/down
     SparseLayout L;
 };
 
-template <int MT>
-struct ItemMeta {
-    const uint16_t *wud;     // the expert's [f][2d] up/down records
-    long long key;           // (expert or shared index, token tile): items that share tokens
-    int xslot, xseq, xfirst; // token rows: slot, load sequence number, first item using them
-    int tok[MT];
-    int pair[MT];
-    float w[MT];
-    unsigned word[MT];
-    float a[kChunk][MT];     // silu(g) of the chunk's neurons
-    int uni[kChunk];         // union-active neuron offsets, ascending
-    int m, chunk, masked, n_uni;
+struct ItemPos {
+    int slot;   // routed expert slot, or -1 - s for shared expert s
+    int tile, blk;
 };
 
-// The tile's token rows, this lane's slice of d, widened to fp32 once per
-// phase: xf[p][r][e] = x_r[8 v + e] with v = warp*32 + lane + 256 p.
+struct PlanCache {      // the routing plan's per-slot arrays, copied to shared memory
+    const int *prefix, *expert, *off, *cnt;
+    const int *order;   // resident mode: slots by decreasing token count
+    int n_touched;
+};
+
+__device__ __forceinline__ ItemPos locate_item(const SparseArgs &a, const PlanCache &pc, int item)
+{
+    ItemPos p;
+    if (item < a.n_shared_items) {
+        const int per_s = a.n_tok_tiles * a.n_blk;
+        p.slot = -1 - item / per_s;
+        const int r0 = item % per_s;
+        p.tile = r0 / a.n_blk;
+        p.blk = r0 % a.n_blk;
+    } else if (a.resident) {   // one tile per expert, slots heaviest first
+        const int ir = item - a.n_shared_items;
+        p.slot = pc.order[min(ir / a.n_blk, pc.n_touched - 1)];
+        p.tile = 0;
+        p.blk = ir % a.n_blk;
+    } else {
+        const int ir = item - a.n_shared_items;
+        int lo = 0, hi = pc.n_touched - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pc.prefix[mid] <= ir) lo = mid; else hi = mid - 1;
+        }
+        const int local = ir - pc.prefix[lo];
+        p.slot = lo;
+        p.tile = local / a.n_blk;
+        p.blk = local % a.n_blk;
+    }
+    return p;
+}
+
+__device__ __forceinline__ long long item_key(const ItemPos &p)
+{
+    return ((long long)(p.slot < 0 ? p.slot : p.slot + 1) << 32) | (unsigned)p.tile;
+}
+
+// Tokens of the item's tile: count, and where token r comes from.
+__device__ __forceinline__ int tile_tokens(const SparseArgs &a, const PlanCache &pc, const ItemPos &p, int &base)
+{
+    if (p.slot < 0) {
+        base = p.tile * a.nt;   // token ids base .. base + m - 1
+        return max(1, min(a.nt, a.T - base));
+    }
+    base = pc.off[p.slot] + p.tile * a.nt;   // positions in perm
+    return max(1, min(a.nt, pc.cnt[p.slot] - p.tile * a.nt));
+}
+
+__device__ __forceinline__ int tile_token(const SparseArgs &a, const ItemPos &p, int base, int r)
+{
+    const int t = p.slot < 0 ? base + r : a.ws.perm_tok[base + r];
+    return min(max(t, 0), a.T - 1);
+}
+
+// The pass's token rows from global memory (L2-resident), this lane's slice
+// of d, widened to fp32: xf[p][r][e] = x_r[8 v + e] with v = warp*32 + lane + 256 p.
 template <int MT, int NP>
-__device__ __forceinline__ void load_x(const uint8_t *xb, int xpitch, int m, int d8, int warp, int lane,
+__device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m, int d, int warp, int lane,
                                        float (&xf)[NP][MT][8])
 {
+    const int d8 = d >> 3;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int v = warp * 32 + lane + 256 * p;
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
             if (r < m && v < d8) {
-                unpack8(*reinterpret_cast<const uint4 *>(xb + (size_t)r * xpitch + 16 * v), xf[p][r]);
+                unpack8(ld_cached(x + (size_t)tok[r] * d + 8 * v), xf[p][r]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) xf[p][r][e] = 0.f;
@@ -118,23 +194,17 @@ __device__ __forceinline__ void load_x(const uint8_t *xb, int xpitch, int m, int
     }
 }
 
-// Partial projections of a group of 8 weight rows over this warp's slice of
-// d: acc[q][r] = sum_{k in slice} w_q[k] x_r[k].  Row q lives at
-// lo + q * stride for q < split and at hi + (q - split) * stride after (a
-// group may straddle two ring stages).  When swz, the row's 16-byte blocks
-// are permuted b -> b ^ (q & 7) inside complete 128-byte groups (gate rows,
-// see gate_pos), otherwise stored in order.  All eight 16-byte loads are
-// issued before the math.  After one transposed warp reduction the warp-wide
-// sum for (q, r) sits in one lane, which stores it to
+// Partial up projections of kRows gathered rows over this warp's slice of d:
+// acc[q][r] = sum_{k in slice} w_q[k] x_r[k], rows q < nrows at lo + q*stride.
+// All row loads are issued before the math.  After one transposed warp
+// reduction the warp-wide sum for (q, r) sits in one lane, which stores it to
 // part_w[(row_off + q) * MT + r].
 template <int MT, int NP>
-__device__ __forceinline__ void group8(const uint8_t *lo, const uint8_t *hi, int split, int stride, bool swz,
-                                       int nrows, const float (&xf)[NP][MT][8], int d8, int warp, int lane,
-                                       float *part_w, int row_off)
+__device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nrows, const float (&xf)[NP][MT][8],
+                                           int d8, int warp, int lane, float *part_w, int row_off)
 {
-    constexpr int NV = 8 * MT;
+    constexpr int NV = kRows * MT;
     constexpr int SH = 5 - Log2<NV>::value;
-    const int full = (d8 >> 3) << 3;   // blocks in complete 128-byte groups
     float acc[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) acc[i] = 0.f;
@@ -142,16 +212,12 @@ __device__ __forceinline__ void group8(const uint8_t *lo, const uint8_t *hi, int
     for (int p = 0; p < NP; ++p) {
         const int v = warp * 32 + lane + 256 * p;
         if (v < d8) {
-            const bool sw = swz && v < full;
-            uint4 wv[8];
+            uint4 wv[kRows];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint8_t *row = q < split ? lo + q * stride : hi + (q - split) * stride;
-                const int pb = sw ? (v ^ q) : v;
-                wv[q] = q < nrows ? *reinterpret_cast<const uint4 *>(row + 16 * pb) : make_uint4(0, 0, 0, 0);
-            }
+            for (int q = 0; q < kRows; ++q)
+                wv[q] = q < nrows ? *reinterpret_cast<const uint4 *>(lo + q * stride + 16 * v) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < kRows; ++q) {
                 float wf[8];
                 unpack8(wv[q], wf);
 #pragma unroll
@@ -169,39 +235,56 @@ __device__ __forceinline__ void group8(const uint8_t *lo, const uint8_t *hi, int
     if ((lane & ((1 << SH) - 1)) == 0 && q < nrows) part_w[(row_off + q) * MT + r] = val;
 }
 
-template <int MT, int NP>
-__global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(SparseArgs a)
+// A bounded wait that does not give up early on another agent's error: used
+// only to drain copies before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
 {
-    extern __shared__ __align__(128) uint8_t smem[];
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return;
+}
+
+template <int MT, int NP>
+__global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
+{
+    extern __shared__ uint8_t dsm_raw[];
+    // the 128-byte swizzle of the MMA operands needs 1024-byte aligned tiles
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     const SparseLayout &L = a.L;
+    uint8_t *xt = smem + L.xt_off;
     uint8_t *ring = smem + L.ring_off;
-    uint8_t *gather = smem + L.gather_off;
-    ItemMeta<MT> *meta = reinterpret_cast<ItemMeta<MT> *>(smem + L.meta_off);
-    float *part = reinterpret_cast<float *>(smem + L.part_off);   // [8][32][MT]
-    float *hs = reinterpret_cast<float *>(smem + L.h_off);        // [GB][MT]
-    int *s_last = reinterpret_cast<int *>(smem + L.last_off);     // [MT]
-    // progress counters shared between the three agents (monotonic, so a
-    // reader can never mistake an old value for a new one):
-    //   mask_done   items whose mask and union list are final   (consumers)
-    //   pub_gi/xi   items whose gate stages / metadata are issued (gate lane)
-    //   pub_gstart  items whose gather has started                (gather warp)
-    volatile int *mask_done = reinterpret_cast<volatile int *>(s_last + 8);
-    volatile int *pub_gi = mask_done + 1, *pub_xi = mask_done + 2, *pub_gstart = mask_done + 3;
+    uint8_t *ud = smem + L.ud_off;
+    ItemMeta *meta = reinterpret_cast<ItemMeta *>(smem + L.meta_off);   // [2]
+    float *part = reinterpret_cast<float *>(smem + L.part_off);        // [8 warps][kMaxGB][MT]
+    float *hs = reinterpret_cast<float *>(smem + L.h_off);             // [kMaxGB][MT]
+    int *s_last = reinterpret_cast<int *>(smem + L.last_off);          // [MT]
+    // progress shared between the agents; monotonic, so a reader can never
+    // mistake an old value for a new one:
+    //   mask_done  items whose mask and union lists are final    (consumers)
+    //   pub_items  work-item ids published in s_items           (gate lane)
+    //   items_end  number of items of this CTA, once known      (consumers)
+    volatile int *mask_done = reinterpret_cast<volatile int *>(smem + L.ctr_off);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L.ctr_off + 16);
+    volatile int *pub_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 32);
+    volatile int *items_end = reinterpret_cast<volatile int *>(smem + L.ctr_off + 48);
+    volatile int *s_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 64);   // [kIdRing]
     int *s_prefix = reinterpret_cast<int *>(smem + L.plan_off);
     int *s_expert = s_prefix + a.max_touched + 1;
     int *s_off = s_expert + a.max_touched;
     int *s_cnt = s_off + a.max_touched;
+    int *s_order = s_cnt + a.max_touched;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     const int NS = L.n_stages;
-    uint64_t *full_g = bars, *empty_g = bars + NS;
-    uint64_t *mfull = bars + 2 * NS, *mempty = mfull + 3;      // item metadata, 3 deep
-    uint64_t *xfull = mempty + 3, *xempty = xfull + 2;         // token-row slots, by key
-    uint64_t *full_u = xempty + 2, *empty_u = full_u + 1;
+    uint64_t *full_g = bars, *empty_g = bars + NS;         // gate ring
+    uint64_t *gdone = bars + 2 * NS, *tfree = gdone + kAcc;   // TMEM accumulators
+    uint64_t *xfull = tfree + kAcc, *xfree = xfull + 1;       // token tile
+    uint64_t *mdrain = xfree + 1;
+    const int NU = L.n_ud;
+    uint64_t *full_u = mdrain + 1, *empty_u = full_u + NU;   // gather buffers
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const Plan *plan = a.ws.plan;
+    Plan *plan = a.ws.plan;
     int *err = a.ws.error_word;
-    const int d = a.d, row_bytes = 2 * d;
+    const int d = a.d;
     const bool score_mode = a.score_out != nullptr;
     unsigned long long *tr = (a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
                                  ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
@@ -210,24 +293,32 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(SparseArgs 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full_g[s], 1);
-            mbar_init(&empty_g[s], 8);
+            mbar_init(&empty_g[s], 1);
         }
-        for (int p = 0; p < 3; ++p) {
-            mbar_init(&mfull[p], 1);
-            mbar_init(&mempty[p], 1);
+        for (int b = 0; b < kAcc; ++b) {
+            mbar_init(&gdone[b], 1);
+            mbar_init(&tfree[b], 4);
         }
-        for (int p = 0; p < 2; ++p) {
-            mbar_init(&xfull[p], 1);
-            mbar_init(&xempty[p], 1);
+        for (int b = 0; b < NU; ++b) {
+            mbar_init(&full_u[b], 32);   // one cp.async arrival per gather lane
+            mbar_init(&empty_u[b], 1);
         }
-        mbar_init(full_u, 1);
-        mbar_init(empty_u, 1);
+        mbar_init(xfull, 1);
+        mbar_init(xfree, 1);
+        mbar_init(mdrain, 1);
         *mask_done = 0;
-        *pub_gi = 0;
-        *pub_xi = 0;
-        *pub_gstart = 0;
+        *pub_items = 0;
+        *items_end = 0x7fffffff;
         fence_mbar_init();
     }
+    if (warp == kWarpMma) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
     // everything above overlaps the router's tail (programmatic dependent
     // launch); the routing plan is read only after the router grid is done
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -243,217 +334,251 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(SparseArgs 
         }
     }
     __syncthreads();
+    if (a.resident) {
+        // slots by decreasing token count (ties by slot): claimed in this order,
+        // the most expensive items go first and the tail is made of cheap ones
+        for (int i = tid; i < n_touched; i += blockDim.x) {
+            const int c = s_cnt[i];
+            int r = 0;
+            for (int j = 0; j < n_touched; ++j) {
+                const int cj = s_cnt[j];
+                r += (cj > c) || (cj == c && j < i);
+            }
+            s_order[r] = i;
+        }
+        __syncthreads();
+    }
     if (tr && tid == 0) tr[1] = global_ns();
+    const PlanCache pc{s_prefix, s_expert, s_off, s_cnt, s_order, n_touched};
 
     const int n_items = a.n_shared_items + plan->n_routed_items;
+    // static ranges (token-tile mode): contiguous items per CTA
     const int G = gridDim.x, b = blockIdx.x;
     const int per = n_items / G, rem = n_items % G;
     const int first = b * per + min(b, rem);
     const int n_my = per + (b < rem ? 1 : 0);
-    const size_t fd = (size_t)a.f * d;
-
-    // item -> (expert slot or shared index, tile, chunk); routed slot found by
-    // binary search over the plan's per-slot item prefix
-    auto locate = [&](int item, int &slot, int &tile, int &chunk) {
-        if (item < a.n_shared_items) {
-            const int per_s = a.n_tok_tiles * a.n_chunks;
-            slot = -1 - item / per_s;
-            const int r0 = item % per_s;
-            tile = r0 / a.n_chunks;
-            chunk = r0 % a.n_chunks;
-        } else {
-            const int ir = item - a.n_shared_items;
-            int lo = 0, hi = n_touched - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_prefix[mid] <= ir) lo = mid; else hi = mid - 1;
+    const size_t gate_per_expert = (size_t)a.n_blk * a.n_kb * (kGateTile / 2);   // elements
+    const int spi = a.n_kb / 2;   // ring stages per item
+    auto gate_src = [&](const ItemPos &p) -> const uint16_t * {
+        const uint16_t *base = p.slot < 0 ? a.w.wsg_t + (size_t)(-1 - p.slot) * gate_per_expert
+                                          : a.w.wg_t + (size_t)pc.expert[p.slot] * gate_per_expert;
+        return base + (size_t)p.blk * a.n_kb * (kGateTile / 2);
+    };
+    // the id of this CTA's i-th work item (-1: no more), as published by the gate lane
+    auto get_item = [&](int i) -> int {
+        for (uint32_t spin = 0; *pub_items <= i; ++spin) {
+            if (spin > (kSpinLimit >> 4) || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                atomicCAS(err, 0, 50);
+                return -1;
             }
-            const int local = ir - s_prefix[lo];
-            slot = lo;
-            tile = local / a.n_chunks;
-            chunk = local % a.n_chunks;
+            __nanosleep(64);
         }
+        __threadfence_block();
+        return s_items[i % kIdRing];
     };
 
-    if (warp == 8) {
-        // ------------------------------------------------------- gate/x producer
-        // One lane polls two queues, so neither blocks the other:
-        //   metadata + token rows of item xi (at most one item ahead of the gate
-        //     cursor) once item xi-3 has released its metadata buffer; the token
-        //     rows are copied only when the (expert, tile) changes, into the slot
-        //     the tile before last has released
-        //   gate stages of item gi into free ring slots; at most
-        //     kPrefetchStages of an item before the previous item's gather has
-        //     started, so that gather is not queued behind them
-        if (lane == 0 && n_my > 0) {
+    if (warp == kWarpTma) {
+        // ------------------------------------------------------------ gate lane
+        // publishes the work-item ids (claimed from the plan's counter in
+        // resident mode, else the CTA's static range), then streams each
+        // item's gate tiles into the ring
+        if (lane == 0) {
             const uint64_t pol = policy_evict_first();
-            uint32_t g = 0, idle = 0;
-            int xi = 0, gi = 0, gs = 0, kseq = -1, cur_slot = 0;
-            long long prev_key = 0;
-            const uint16_t *g_src = nullptr;
-            while (gi < n_my || xi < n_my) {
-                bool prog = false;
-                if (xi < n_my && xi <= gi + 1 && mbar_test(&mempty[xi % 3], ((xi / 3) & 1) ^ 1)) {
-                    int slot, tile, chunk;
-                    locate(first + xi, slot, tile, chunk);
-                    const long long key = slot < 0 ? (((long long)slot << 32) | (unsigned)tile)
-                                                   : (((long long)(s_expert[slot] + 1) << 32) | (unsigned)tile);
-                    const bool newkey = score_mode || xi == 0 || key != prev_key;
-                    const int nslot = (kseq + 1) & 1;
-                    if (!newkey || mbar_test(&xempty[nslot], (((kseq + 1) >> 1) & 1) ^ 1)) {
-                        ItemMeta<MT> &M = meta[xi % 3];
-                        int m, tok0 = -1, off = 0;
-                        if (slot < 0) {
-                            const int s = -1 - slot;
-                            tok0 = tile * MT;
-                            m = min(MT, a.T - tok0);
-                            M.wud = a.w.wsud + 2 * s * fd;
-                            M.masked = 0;
-                        } else {
-                            m = min(MT, s_cnt[slot] - tile * MT);
-                            M.wud = a.w.wud + 2 * s_expert[slot] * fd;
-                            M.masked = a.use_mask;
-                            off = s_off[slot] + tile * MT;
-                        }
-                        m = min(max(m, 1), MT);
-                        M.key = key;
-                        M.m = m;
-                        M.chunk = chunk;
-                        for (int r = 0; r < m; ++r) {
-                            if (tok0 >= 0) {
-                                M.tok[r] = tok0 + r;
-                                M.pair[r] = -1;
-                                M.w[r] = 1.f;
-                            } else {
-                                M.pair[r] = min(max(a.ws.perm[off + r], 0), a.T * a.k - 1);
-                                M.tok[r] = min(max(a.ws.perm_tok[off + r], 0), a.T - 1);
-                                M.w[r] = a.ws.perm_w[off + r];
-                            }
-                        }
-                        if (newkey) {
-                            ++kseq;
-                            cur_slot = kseq & 1;
-                            uint8_t *xb = smem + L.xbuf_off + cur_slot * L.xbuf_bytes;
-                            if (tr && xi < 4) tr[60 + xi] = global_ns();
-                            mbar_arrive_expect_tx(&xfull[cur_slot], (uint32_t)(m * row_bytes));
-                            for (int r = 0; r < m; ++r)
-                                bulk_g2s(xb + (size_t)r * L.xpitch, a.x + (size_t)M.tok[r] * d, (uint32_t)row_bytes,
-                                         &xfull[cur_slot]);
-                        }
-                        M.xslot = cur_slot;
-                        M.xseq = kseq;
-                        M.xfirst = newkey ? 1 : 0;
-                        prev_key = key;
-                        mbar_arrive(&mfull[xi % 3]);
-                        ++xi;
-                        *pub_xi = xi;
-                        prog = true;
-                    }
-                }
-                if (gi < n_my && (score_mode || *pub_gstart >= gi || gs < kPrefetchStages)) {
-                    const int rslot = g % NS;
-                    if (mbar_test(&empty_g[rslot], ((g / NS) & 1) ^ 1)) {
-                        if (gs == 0) {
-                            int slot, tile, chunk;
-                            locate(first + gi, slot, tile, chunk);
-                            const uint16_t *wg = slot < 0 ? a.w.wsg_n + (-1 - slot) * fd
-                                                          : a.w.wg_n + s_expert[slot] * fd;
-                            g_src = wg + (size_t)chunk * kChunk * d;
-                        }
-                        if (tr && gi < 4 && (gs == 0 || gs == L.stages_per_chunk - 1))
-                            tr[52 + 2 * gi + (gs != 0)] = global_ns();
-                        mbar_arrive_expect_tx(&full_g[rslot], (uint32_t)L.stage_bytes);
-                        bulk_g2s_hint(ring + (size_t)rslot * L.stage_bytes,
-                                      g_src + (size_t)gs * L.rows_per_stage * d, (uint32_t)L.stage_bytes,
-                                      &full_g[rslot], pol);
-                        ++g;
-                        if (++gs == L.stages_per_chunk) {
-                            gs = 0;
-                            ++gi;
-                            *pub_gi = gi;
-                        }
-                        prog = true;
-                    }
-                }
-                if (prog) {
-                    idle = 0;
+            uint32_t g = 0;
+            int next = a.resident ? atomicAdd(&plan->next_item, 1) : 0;
+            for (int i = 0;; ++i) {
+                int id;
+                if (a.resident) {
+                    id = next < n_items ? next : -1;
+                    if (id >= 0) next = atomicAdd(&plan->next_item, 1);   // claimed early: the reply lands meanwhile
                 } else {
-                    if (++idle > kSpinLimit) {
-                        atomicCAS(err, 0, 12);
+                    id = i < n_my ? first + i : -1;
+                }
+                // ring slot i % kIdRing is free once the consumers have masked item i - kIdRing
+                for (uint32_t spin = 0; *mask_done < i - kIdRing + 1; ++spin) {
+                    if (spin > (kSpinLimit >> 4) || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                        atomicCAS(err, 0, 51);
+                        id = -1;
                         break;
                     }
-                    __nanosleep(32);
+                    __nanosleep(128);
+                }
+                s_items[i % kIdRing] = id;
+                __threadfence_block();
+                *pub_items = i + 1;
+                if (id < 0) break;
+                const uint16_t *src = gate_src(locate_item(a, pc, id));
+                bool ok = true;
+                for (int s = 0; s < spi; ++s, ++g) {
+                    const int slot = (int)(g % NS);
+                    if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
+                    if (tr && g < 8) tr[40 + g] = global_ns();
+                    mbar_arrive_expect_tx(&full_g[slot], kStageBytes);
+                    bulk_g2s_hint(ring + (size_t)slot * kStageBytes, src + (size_t)s * (kStageBytes / 2), kStageBytes,
+                                  &full_g[slot], pol);
+                }
+                if (!ok) {   // publish the end so that every agent stops
+                    s_items[(i + 1) % kIdRing] = -1;
+                    __threadfence_block();
+                    *pub_items = i + 2;
+                    break;
                 }
             }
-            // drain: every copy issued has landed before the CTA may exit
-            for (int s = 0; s < NS && (uint32_t)s < g; ++s) {
-                const uint32_t uses = (g - s + NS - 1) / NS;
-                mbar_wait(&full_g[s], (uses - 1) & 1, err, 15);
-            }
-            for (int p = 0; p < 2 && p <= kseq; ++p) {
-                const uint32_t uses = (kseq - p + 2) / 2;
-                mbar_wait(&xfull[p], (uses - 1) & 1, err, 17);
-            }
+            // every copy issued has landed before the CTA may exit
+            for (int s = 0; s < NS && (uint32_t)s < g; ++s) mbar_drain(&full_g[s], (((g - s + NS - 1) / NS) - 1) & 1);
         }
         __syncwarp();
-    } else if (warp == 9) {
-        // ------------------------------------------------------- gather producer
-        // Lanes 0..3: once the mask of item ui is final, its union-active up/down
-        // records are copied in batches of GB; lane 0 decides and waits for the
-        // buffer, the four lanes split each batch's copies.
-        if (lane < kGatherLanes && n_my > 0 && !score_mode) {
-            const uint64_t pol = policy_evict_first();
-            const unsigned lanes = (1u << kGatherLanes) - 1u;
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------------- MMA lane
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, 16);
+            uint32_t g = 0;
+            int q = -1;
+            long long prev_key = 0;
+            bool ok = true;
+            if (a.resident) ok = mbar_wait(xfull, 0, err, 31);   // the batch's token rows, once
+            for (int i = 0; ok; ++i) {
+                const int id = get_item(i);
+                if (id < 0) break;
+                const ItemPos p = locate_item(a, pc, id);
+                const long long key = item_key(p);
+                if (!a.resident && (i == 0 || key != prev_key)) {
+                    ++q;
+                    ok = mbar_wait(xfull, q & 1, err, 31);
+                }
+                const int bsel = i % kAcc;
+                ok = ok && mbar_wait(&tfree[bsel], ((i / kAcc) & 1) ^ 1, err, 32);
+                tc_fence_after();
+                const uint32_t dt = tmem + 16 * bsel;
+                for (int s = 0; s < spi && ok; ++s, ++g) {
+                    const int slot = (int)(g % NS);
+                    ok = mbar_wait(&full_g[slot], (g / NS) & 1, err, 33);
+                    tc_fence_after();
+                    if (tr && i < 3 && s == 0) tr[56 + 2 * i] = global_ns();
+                    const uint8_t *A = ring + (size_t)slot * kStageBytes;
+                    const uint8_t *B = xt + (size_t)(2 * s) * L.xt_kb;
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(dt, smem_desc_k_sw128(A + kb * kGateTile + 32 * kk),
+                                      smem_desc_k_sw128(B + kb * L.xt_kb + 32 * kk), idesc, (s | kb | kk) != 0 ? 1u : 0u);
+                    umma_commit(&empty_g[slot]);   // the stage is free once these MMAs have read it
+                }
+                umma_commit(&gdone[bsel]);
+                if (tr && i < 3) tr[57 + 2 * i] = global_ns();
+                if (!a.resident) {   // static ranges: the next id is first + i + 1
+                    const bool last_of_tile =
+                        i + 1 >= n_my || item_key(locate_item(a, pc, first + i + 1)) != key;
+                    if (last_of_tile) umma_commit(xfree);
+                }
+                prev_key = key;
+            }
+            umma_commit(mdrain);   // all MMAs complete before the accumulator is freed
+            mbar_drain(mdrain, 0);
+        }
+        __syncwarp();
+    } else if (warp == kWarpX) {
+        // --------------------------------------------------------------- x warp
+        // token rows into the MMA's K-major 128-byte-swizzled layout; inputs
+        // past d are the zero padding of the gate tiles
+        const int nck = a.dp >> 3;   // 16-byte chunks per padded row
+        auto load_rows = [&](int m, auto token_of) {
+            for (int r = 0; r < m; ++r) {
+                const uint16_t *xrow = a.x + (size_t)token_of(r) * d;
+                for (int c = lane; c < nck; c += 32) {
+                    const bool in = 8 * c < d;
+                    cp_async16(xt + (size_t)(c >> 3) * L.xt_kb + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                               in ? (const void *)(xrow + 8 * c) : (const void *)a.x, in ? 16u : 0u);
+                }
+            }
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+        };
+        if (a.resident) {
+            load_rows(a.T, [](int r) { return r; });   // column t of the MMA = token t
+            if (lane == 0) {
+                if (tr) tr[48] = global_ns();
+                mbar_arrive(xfull);
+            }
+        } else {
+            int q = -1;
+            long long prev_key = 0;
+            for (int i = 0; i < n_my; ++i) {
+                const ItemPos p = locate_item(a, pc, first + i);
+                const long long key = item_key(p);
+                if (i > 0 && key == prev_key) continue;
+                prev_key = key;
+                ++q;
+                if (q > 0 && !mbar_wait(xfree, (q - 1) & 1, err, 34)) break;
+                int base;
+                const int m = tile_tokens(a, pc, p, base);
+                load_rows(m, [&](int r) { return tile_token(a, p, base, r); });
+                if (lane == 0) {
+                    if (tr && q < 8) tr[48 + q] = global_ns();
+                    mbar_arrive(xfull);
+                }
+            }
+        }
+        cp_async_wait_all();
+        __syncwarp();
+    } else if (warp == kWarpGather) {
+        // ---------------------------------------------------------- gather warp
+        // once an item's mask is final, its union-active records into the
+        // gather buffers, batch by batch, as 16-byte cp.async copies spread
+        // over the 32 lanes: they take the load/store path, so they do not
+        // queue behind the gate stream's bulk copies in the SM's TMA unit
+        if (!score_mode) {
+            const int rec_ck = (4 * d) / 16;   // 16-byte chunks per [up | down] record (4d bytes)
             uint32_t ub = 0, idle = 0;
-            int ui = 0;
-            while (ui < n_my) {
+            for (int ui = 0;;) {
                 int go = 0;
-                if (lane == 0) go = ui < *pub_gi && ui < *pub_xi && *mask_done > ui;
-                go = __shfl_sync(lanes, go, 0);
-                if (!go) {
+                if (lane == 0)
+                    go = *mask_done > ui ? 1
+                                         : (*items_end <= ui || *reinterpret_cast<volatile int *>(err) != 0 ? -1 : 0);
+                go = __shfl_sync(kFull, go, 0);
+                if (go < 0) break;
+                if (go == 0) {
                     if (++idle > kSpinLimit) {
-                        if (lane == 0) atomicCAS(err, 0, 14);
+                        if (lane == 0) atomicCAS(err, 0, 35);
                         break;
                     }
-                    __nanosleep(64);
+                    __nanosleep(128);
                     continue;
                 }
                 idle = 0;
                 __threadfence_block();
-                const ItemMeta<MT> &M = meta[ui % 3];
-                const int n = min(max(M.n_uni, 0), kChunk);
-                const size_t j0 = (size_t)min(max(M.chunk, 0), a.n_chunks - 1) * kChunk;
-                if (n == 0 && lane == 0) *pub_gstart = ui + 1;
-                for (int b0 = 0; b0 < n; b0 += L.gather_rows, ++ub) {
-                    const int nb = min(L.gather_rows, n - b0);
-                    if (lane == 0) {
-                        mbar_wait(empty_u, (ub & 1) ^ 1, err, 14);
-                        if (tr && b0 == 0 && ui < 4) tr[9 + 12 * ui] = global_ns();
-                        mbar_arrive_expect_tx(full_u, (uint32_t)(nb * 2 * row_bytes));
+                const ItemMeta &M = meta[ui & 1];
+                unsigned long long *tg = (tr && ui < 2 && lane == 0) ? tr + 32 + 4 * ui : nullptr;
+                if (tg) tg[0] = global_ns();
+                int nbatch = 0;
+                const int nsub = min(max(M.nsub, 0), kMaxSub);
+                const size_t j0 = (size_t)M.blk * kBlk;
+                for (int s = 0; s < nsub; ++s) {
+                    const int n = min(max(M.n_uni[s], 0), kBlk);
+                    for (int b0 = 0; b0 < n; b0 += L.gb, ++ub) {
+                        const int nb = min(L.gb, n - b0);
+                        const int bi = (int)(ub % NU);
+                        mbar_wait(&empty_u[bi], ((ub / NU) & 1) ^ 1, err, 36);
+                        if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
+                        ++nbatch;
+                        uint8_t *dst = ud + (size_t)bi * L.ud_buf_bytes;
+                        for (int qq = 0; qq < nb; ++qq) {
+                            const size_t j = min(j0 + M.uni[s][b0 + qq], (size_t)a.f - 1);
+                            const uint16_t *src = M.wud + j * 2 * d;
+                            uint8_t *row = dst + (size_t)qq * L.gpitch;
+                            for (int cc = lane; cc < rec_ck; cc += 32) cp_async16(row + 16 * cc, src + 8 * cc, 16u);
+                        }
+                        cp_async_arrive_noinc(&full_u[bi]);   // one of the 32 expected arrivals
                     }
-                    __syncwarp(lanes);
-                    for (int q = lane; q < nb; q += kGatherLanes) {
-                        const size_t j = j0 + (M.uni[b0 + q] & (kChunk - 1));
-                        bulk_g2s_hint(gather + (size_t)q * L.gpitch, M.wud + j * 2 * d, (uint32_t)(2 * row_bytes),
-                                      full_u, pol);
-                    }
-                    __syncwarp(lanes);
-                    if (b0 == 0 && lane == 0) *pub_gstart = ui + 1;
                 }
                 ++ui;
             }
-            if (lane == 0 && ub > 0) mbar_wait(full_u, (ub - 1) & 1, err, 16);
-        }
-        if (tr && lane == 31 && n_my > 0) {
-            // trace observer: arrival time of the first ring-full of gate stages
-            const int n_obs = min(NS, min(8, n_my * L.stages_per_chunk));
-            for (int gg = 0; gg < n_obs; ++gg) {
-                mbar_wait(&full_g[gg], 0, err, 0x7f);
-                tr[40 + gg] = global_ns();
-            }
+            cp_async_wait_all();
         }
         __syncwarp();
-    } else if (n_my > 0) {
+    } else {
         // ------------------------------------------------------------ consumers
         const int ct = tid;   // 0..255
         const int d8 = d >> 3;
@@ -464,242 +589,291 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(SparseArgs 
             for (int e = 0; e < 8; ++e)
 #pragma unroll
                 for (int r = 0; r < MT; ++r) acc_y[p][e][r] = 0.f;
-        uint32_t g = 0, ub = 0;
-        int n_acc = 0;
-        const int spg = 8 / L.rows_per_stage;   // stages per group of 8 rows
-        for (int ii = 0; ii <= n_my; ++ii) {
-            if (ii < n_my) {
-                // G(ii): slice partials of the chunk's 32 gate rows, 8 at a time
-                const int par = ii % 3;
-                ItemMeta<MT> &M = meta[par];
-                mbar_wait(&mfull[par], (ii / 3) & 1, err, 20);
-                if (M.xfirst) mbar_wait(&xfull[M.xslot & 1], (M.xseq >> 1) & 1, err, 21);
-                if (tr && ct == 0 && ii < 4) tr[2 + 12 * ii] = global_ns();
-                const int m = M.m;
-                float xf[NP][MT][8];
-                load_x<MT, NP>(smem + L.xbuf_off + (M.xslot & 1) * L.xbuf_bytes, L.xpitch, m, d8, warp, lane, xf);
-                const int rs = L.rows_per_stage;   // a power of two; groups of 8 rows span spg stages
-                for (int grp = 0; grp < kChunk / 8; ++grp) {
-                    const uint32_t g0 = g + grp * spg;
-                    for (int j = 0; j < spg; ++j) {
-                        const uint32_t gg = g0 + j;
-                        mbar_wait(&full_g[gg % NS], (gg / NS) & 1, err, 22);
-                    }
-                    if (tr && ct == 0 && ii < 4) tr[3 + 12 * ii + grp] = global_ns();
-                    // rows 8*grp .. 8*grp+7: within one stage when rs >= 8, else spg stages of rs rows
-                    const int q0 = (8 * grp) & (rs - 1);
-                    const uint8_t *lo = ring + (size_t)(g0 % NS) * L.stage_bytes + (size_t)q0 * row_bytes;
-                    const uint8_t *hi = ring + (size_t)((g0 + 1) % NS) * L.stage_bytes;
-                    group8<MT, NP>(lo, hi, rs >= 8 ? 8 : rs, row_bytes, true, 8, xf, d8, warp, lane,
-                                   part + warp * kChunk * MT, 8 * grp);
-                    __syncwarp();
-                    if (lane == 0)
-                        for (int j = 0; j < spg; ++j) mbar_arrive(&empty_g[(g0 + j) % NS]);
-                }
-                g += L.stages_per_chunk;
-                consumer_sync(kConsumerThreads);
-                if (tr && ct == 0 && ii < 4) tr[7 + 12 * ii] = global_ns();
-                // M(ii): sum the slices, silu, threshold, ballot
-                for (int r = warp; r < MT; r += 8) {
-                    float gsum = 0.f;
-#pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8) gsum += part[(w8 * kChunk + lane) * MT + r];
-                    const float av = silu_f(gsum);
-                    const bool on = (r < m) && (!M.masked || fabsf(av) >= a.tau);
-                    const unsigned word = __ballot_sync(kFull, on);
-                    M.a[lane][r] = av;
-                    if (lane == 0) {
-                        M.word[r] = word;
-                        if (M.masked && r < m) a.ws.mask[(size_t)M.pair[r] * a.n_chunks + M.chunk] = word;
-                    }
-                    if (score_mode && r < m && M.pair[r] >= 0)
-                        a.score_out[(size_t)M.pair[r] * a.f + M.chunk * kChunk + lane] = fabsf(av);
-                }
-                consumer_sync(kConsumerThreads);
-                if (ct == 0) {
-                    unsigned uw = 0;
-                    for (int r = 0; r < m; ++r) uw |= M.word[r];
-                    int n = 0;
-                    for (unsigned bits = uw; bits; bits &= bits - 1) M.uni[n++] = __ffs(bits) - 1;
-                    M.n_uni = n;
-                    __threadfence_block();
-                    *mask_done = ii + 1;
-                    if (tr && ii < 4) tr[8 + 12 * ii] = global_ns();
-                    if (score_mode) {
-                        mbar_arrive(&mempty[par]);
-                        mbar_arrive(&xempty[M.xslot & 1]);
-                    }
+        uint32_t ub = 0;
+        int n_acc = 0, n_rec = 0, ii = 0;
+        unsigned long long t_wait = 0, t_ud = 0;   // trace only: time waiting for / spent on gathered batches
+        // ---- M(i): item metadata, accumulator -> silu, mask, union lists (all 256 threads)
+        auto do_mask = [&](int i, int id) {
+            ItemMeta &M = meta[i & 1];
+            const ItemPos p = locate_item(a, pc, id);
+            int base;
+            const int m = tile_tokens(a, pc, p, base);
+            if (ct < m) {
+                M.tok[ct] = tile_token(a, p, base, ct);
+                if (p.slot < 0) {
+                    M.pair[ct] = -1;
+                    M.w[ct] = 1.f;
+                } else {
+                    M.pair[ct] = min(max(a.ws.perm[base + ct], 0), a.T * a.k - 1);
+                    M.w[ct] = a.ws.perm_w[base + ct];
                 }
             }
-            if (ii >= 1 && !score_mode) {
-                // UD(ii-1): gathered up rows -> h, gathered down rows -> y
-                const int jj = ii - 1, pj = jj % 3;
-                ItemMeta<MT> &M = meta[pj];
-                consumer_sync(kConsumerThreads);
-                const int m = M.m, n_uni = min(max(M.n_uni, 0), kChunk);
-                float xf[NP][MT][8];
-                load_x<MT, NP>(smem + L.xbuf_off + (M.xslot & 1) * L.xbuf_bytes, L.xpitch, m, d8, warp, lane, xf);
-                for (int b0 = 0; b0 < n_uni; b0 += L.gather_rows, ++ub) {
-                    const int nb = min(L.gather_rows, n_uni - b0);
-                    mbar_wait(full_u, ub & 1, err, 23);
-                    if (tr && ct == 0 && jj < 4 && b0 == 0) tr[10 + 12 * jj] = global_ns();
-                    for (int grp = 0; grp * 8 < nb; ++grp) {
-                        const uint8_t *lo = gather + (size_t)(8 * grp) * L.gpitch;
-                        group8<MT, NP>(lo, lo, 8, L.gpitch, false, min(8, nb - 8 * grp), xf, d8, warp, lane,
-                                       part + warp * kChunk * MT, 8 * grp);
+            if (ct == 0) {
+                M.key = item_key(p);
+                M.m = m;
+                M.blk = p.blk;
+                M.masked = p.slot < 0 ? 0 : a.use_mask;
+                M.nsub = (m + MT - 1) / MT;
+                M.wud = p.slot < 0 ? a.w.wsud + (size_t)(-1 - p.slot) * 2 * a.f * d
+                                   : a.w.wud + (size_t)pc.expert[p.slot] * 2 * a.f * d;
+            }
+            consumer_sync(kConsumerThreads);
+            unsigned long long *ti = (tr && i < 3) ? tr + 2 + 10 * i : nullptr;   // per-item stamps
+            if (ti && ct == 0) ti[0] = global_ns();
+            if (warp < 4) {
+                const int bsel = i % kAcc;
+                mbar_wait(&gdone[bsel], (i / kAcc) & 1, err, 40);
+                tc_fence_after();
+                if (ti && ct == 0) ti[1] = global_ns();
+                const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + 16 * bsel;
+                const int jl = warp * 32 + lane;
+                const int j = M.blk * kBlk + jl;
+                const bool jv = j < a.f;
+                const int chunk = M.blk * 4 + warp;
+                const bool masked = M.masked != 0;
+                // a rolled loop over the tile's tokens: short code, one TMEM
+                // column each (the token's own column in resident mode)
+#pragma unroll 1
+                for (int t = 0; t < m; ++t) {
+                    const int col = a.resident ? M.tok[t] : t;
+                    const float av = silu_f(tmem_ld1(taddr + col));
+                    const bool on = jv && (!masked || fabsf(av) >= a.tau);
+                    const unsigned word = __ballot_sync(kFull, on);
+                    M.a[t][jl] = __float2half_rn(av);
+                    if (lane == 0) {
+                        M.word[t][warp] = word;
+                        if (masked && chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = word;
                     }
-                    consumer_sync(kConsumerThreads);
-                    for (int i = ct; i < nb * MT; i += kConsumerThreads) {
-                        const int q = i / MT, r = i % MT;
-                        float u = 0.f;
+                    if (score_mode && jv) a.score_out[(size_t)M.pair[t] * a.f + j] = fabsf(av);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tfree[bsel]);   // the MMA may overwrite this accumulator
+                if (ti && ct == 0) ti[2] = ti[3] = global_ns();
+            }
+            consumer_sync(kConsumerThreads);
+            if (ti && ct == 0) ti[4] = global_ns();
+            if (warp < M.nsub) {
+                // union of the pass's tokens, compacted in ascending neuron order
+                const int s = warp, t0 = s * MT, t1 = min(m, t0 + MT);
+                int n = 0;
 #pragma unroll
-                        for (int w8 = 0; w8 < 8; ++w8) u += part[(w8 * kChunk + q) * MT + r];
-                        const int jl = M.uni[b0 + q] & (kChunk - 1);
-                        const bool bit = (r < m) && ((M.word[r] >> jl) & 1u);
-                        hs[q * MT + r] = bit ? M.a[jl][r] * u : 0.f;
-                    }
-                    consumer_sync(kConsumerThreads);
+                for (int qw = 0; qw < 4; ++qw) {
+                    unsigned uw = 0;
+                    for (int t = t0; t < t1; ++t) uw |= M.word[t][qw];
+                    const bool on = (uw >> lane) & 1u;
+                    const unsigned bal = __ballot_sync(kFull, on);
+                    if (on) M.uni[s][n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)(qw * 32 + lane);
+                    n += __popc(bal);
+                }
+                if (lane == 0) M.n_uni[s] = n;
+            }
+            consumer_sync(kConsumerThreads);
+            if (ct == 0) {
+                __threadfence_block();
+                *mask_done = i + 1;
+                if (ti) ti[5] = global_ns();
+            }
+        };
+        for (;; ++ii) {
+            {
+                const int id = get_item(ii);
+                if (id < 0) {
+                    if (ct == 0) *items_end = ii;   // every item of this CTA has been masked
+                    break;
+                }
+                do_mask(ii, id);
+            }
+            if (!score_mode) {
+                // ---- UD(ii): gathered up rows -> h, gathered down rows -> y, while
+                // the tensor cores already reduce the next items' gate tiles
+                const int jj = ii;
+                const ItemMeta &M = meta[jj & 1];
+                // the next item (published by the gate lane well before this point)
+                // decides whether the down partial can stay in registers
+                const int nid = get_item(ii + 1);
+                const long long next_key = nid >= 0 ? item_key(locate_item(a, pc, nid)) : 0;
+                const int m = M.m, nsub = min(M.nsub, kMaxSub);
+                unsigned long long *tu = (tr && jj < 3) ? tr + 2 + 10 * jj : nullptr;
+                for (int s = 0; s < nsub; ++s) {
+                    const int r0 = s * MT, ms = min(MT, m - r0);
+                    float xf[NP][MT][8];
+                    load_x<MT, NP>(a.x, M.tok + r0, ms, d, warp, lane, xf);
+                    const int n_uni = min(max(M.n_uni[s], 0), kBlk);
+                    n_rec += n_uni;
+                    for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
+                        const int nb = min(L.gb, n_uni - b0);
+                        const int bi = (int)(ub % NU);
+                        const unsigned long long tw0 = tr ? global_ns() : 0;
+                        mbar_wait(&full_u[bi], (ub / NU) & 1, err, 41);
+                        const unsigned long long tw1 = tr ? global_ns() : 0;
+                        t_wait += tw1 - tw0;
+                        if (tu && ct == 0 && s == 0 && b0 == 0) tu[6] = global_ns();
+                        const uint8_t *buf = ud + (size_t)bi * L.ud_buf_bytes;
+                        for (int g0 = 0; g0 < nb; g0 += kRows)
+                            group_rows<MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0), xf, d8,
+                                               warp, lane, part + warp * kMaxGB * MT, g0);
+                        consumer_sync(kConsumerThreads);
+                        for (int i = ct; i < nb * MT; i += kConsumerThreads) {
+                            const int q = i / MT, r = i % MT;
+                            float u = 0.f;
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) {
-                        const int v = ct + 256 * p;
-                        if (v < d8) {
-                            for (int q = 0; q < nb; ++q) {
-                                float wf[8];
-                                unpack8(*reinterpret_cast<const uint4 *>(gather + (size_t)q * L.gpitch + row_bytes +
-                                                                         v * 16),
-                                        wf);
+                            for (int w8 = 0; w8 < 8; ++w8) u += part[(w8 * kMaxGB + q) * MT + r];
+                            const int jl = M.uni[s][b0 + q];
+                            const bool bit = (r < ms) && ((M.word[r0 + r][jl >> 5] >> (jl & 31)) & 1u);
+                            hs[q * MT + r] = bit ? __half2float(M.a[r0 + r][jl]) * u : 0.f;
+                        }
+                        consumer_sync(kConsumerThreads);
 #pragma unroll
-                                for (int r = 0; r < MT; ++r) {
-                                    const float hv = hs[q * MT + r];
+                        for (int p = 0; p < NP; ++p) {
+                            const int v = ct + 256 * p;
+                            if (v < d8) {
+                                for (int q = 0; q < nb; ++q) {
+                                    float wf[8];
+                                    unpack8(*reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d +
+                                                                             16 * v),
+                                            wf);
 #pragma unroll
-                                    for (int e = 0; e < 8; ++e) acc_y[p][e][r] = fmaf(hv, wf[e], acc_y[p][e][r]);
+                                    for (int r = 0; r < MT; ++r) {
+                                        const float hv = hs[q * MT + r];
+#pragma unroll
+                                        for (int e = 0; e < 8; ++e) acc_y[p][e][r] = fmaf(hv, wf[e], acc_y[p][e][r]);
+                                    }
                                 }
                             }
                         }
+                        consumer_sync(kConsumerThreads);
+                        if (ct == 0) {
+                            mbar_arrive(&empty_u[bi]);
+                            if (tu && s == 0 && b0 == 0) tu[7] = global_ns();
+                            if (tu) tu[8] = global_ns();
+                        }
+                        if (tr) t_ud += global_ns() - tw1;
                     }
-                    consumer_sync(kConsumerThreads);
-                    if (ct == 0) mbar_arrive(empty_u);
-                }
-                ++n_acc;
-                const bool flush = (jj == n_my - 1) || (meta[(jj + 1) % 3].key != M.key);
-                if (flush) {
+                    ++n_acc;
+                    // keep accumulating while the next item is the next block of the same tokens
+                    const bool cont = nsub == 1 && nid >= 0 && next_key == M.key;
+                    if (!cont) {
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) {
-                        const int v = ct + 256 * p;
+                        for (int p = 0; p < NP; ++p) {
+                            const int v = ct + 256 * p;
 #pragma unroll
-                        for (int r = 0; r < MT; ++r) {
-                            if (v < d8 && r < m) {
-                                const float wt = M.w[r];
-                                float4 *dst = reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r] * d + v * 8);
-                                atomicAdd(dst, make_float4(wt * acc_y[p][0][r], wt * acc_y[p][1][r],
-                                                           wt * acc_y[p][2][r], wt * acc_y[p][3][r]));
-                                atomicAdd(dst + 1, make_float4(wt * acc_y[p][4][r], wt * acc_y[p][5][r],
-                                                               wt * acc_y[p][6][r], wt * acc_y[p][7][r]));
+                            for (int r = 0; r < MT; ++r) {
+                                if (v < d8 && r < ms) {
+                                    const float wt = M.w[r0 + r];
+                                    float4 *dst =
+                                        reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
+                                    atomicAdd(dst, make_float4(wt * acc_y[p][0][r], wt * acc_y[p][1][r],
+                                                               wt * acc_y[p][2][r], wt * acc_y[p][3][r]));
+                                    atomicAdd(dst + 1, make_float4(wt * acc_y[p][4][r], wt * acc_y[p][5][r],
+                                                                   wt * acc_y[p][6][r], wt * acc_y[p][7][r]));
+                                }
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) acc_y[p][e][r] = 0.f;
                             }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) acc_y[p][e][r] = 0.f;
                         }
-                    }
-                    __threadfence();
-                    consumer_sync(kConsumerThreads);
-                    if (ct < m) {
-                        const int old = atomicAdd(&a.ws.tok_cnt[M.tok[ct]], n_acc);
-                        s_last[ct] = (old + n_acc == a.target);
-                    }
-                    consumer_sync(kConsumerThreads);
-                    for (int r = 0; r < m; ++r) {
-                        if (!s_last[r]) continue;
                         __threadfence();
-                        const int t = M.tok[r];
-                        float *yrow = a.ws.y_acc + (size_t)t * d;
-                        uint16_t *orow = a.out + (size_t)t * d;
-                        for (int i = ct * 4; i < d; i += kConsumerThreads * 4) {
-                            const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(yrow + i));
-                            uint2 packed;
-                            packed.x = (uint32_t)f2bf_bits(v4.x) | ((uint32_t)f2bf_bits(v4.y) << 16);
-                            packed.y = (uint32_t)f2bf_bits(v4.z) | ((uint32_t)f2bf_bits(v4.w) << 16);
-                            *reinterpret_cast<uint2 *>(orow + i) = packed;
-                            __stcg(reinterpret_cast<float4 *>(yrow + i), make_float4(0.f, 0.f, 0.f, 0.f));
+                        consumer_sync(kConsumerThreads);
+                        if (ct < ms) {
+                            const int old = atomicAdd(&a.ws.tok_cnt[M.tok[r0 + ct]], n_acc);
+                            s_last[ct] = (old + n_acc == a.target);
                         }
-                        if (ct == 0) a.ws.tok_cnt[t] = 0;
+                        consumer_sync(kConsumerThreads);
+                        for (int r = 0; r < ms; ++r) {
+                            if (!s_last[r]) continue;
+                            __threadfence();
+                            const int t = M.tok[r0 + r];
+                            float *yrow = a.ws.y_acc + (size_t)t * d;
+                            uint16_t *orow = a.out + (size_t)t * d;
+                            for (int i = ct * 4; i < d; i += kConsumerThreads * 4) {
+                                const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(yrow + i));
+                                uint2 packed;
+                                packed.x = (uint32_t)f2bf_bits(v4.x) | ((uint32_t)f2bf_bits(v4.y) << 16);
+                                packed.y = (uint32_t)f2bf_bits(v4.z) | ((uint32_t)f2bf_bits(v4.w) << 16);
+                                *reinterpret_cast<uint2 *>(orow + i) = packed;
+                                __stcg(reinterpret_cast<float4 *>(yrow + i), make_float4(0.f, 0.f, 0.f, 0.f));
+                            }
+                            if (ct == 0) a.ws.tok_cnt[t] = 0;
+                        }
+                        n_acc = 0;
+                        consumer_sync(kConsumerThreads);
                     }
-                    n_acc = 0;
-                    if (tr && ct == 0 && jj < 4) tr[12 + 12 * jj] = global_ns();
                 }
-                consumer_sync(kConsumerThreads);
-                if (ct == 0) {
-                    mbar_arrive(&mempty[pj]);
-                    if (flush) mbar_arrive(&xempty[M.xslot & 1]);
-                }
-                if (tr && ct == 0 && jj < 4) tr[11 + 12 * jj] = global_ns();
+                if (tu && ct == 0) tu[9] = global_ns();
+                consumer_sync(kConsumerThreads);   // this metadata slot is rewritten next iteration
             }
+        }
+        if (tr && ct == 0) {
+            tr[59] = t_wait;
+            tr[60] = t_ud;
+            tr[61] = (unsigned long long)n_rec;
+            tr[63] = (unsigned long long)ii;
         }
     }
     __syncthreads();
-    if (tr && tid == 0) {
-        tr[50] = global_ns();
-        tr[51] = (unsigned long long)n_my;
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
+    if (tr && tid == 0) tr[62] = global_ns();
 }
 
-// tokens per work item for a batch of T tokens and a model width d
-int sparse_tile_tokens(int T, int d)
+SparseTiling sparse_tiling(int T, int d)
 {
-    int mt = T <= 1 ? 1 : T <= 2 ? 2 : 4;
+    SparseTiling t;
     const int np = (d / 8 + 255) / 256;
-    while (mt > 1 && mt * np > 4) mt >>= 1;
-    return mt;
+    t.mt = T <= 1 ? 1 : T <= 2 ? 2 : 4;
+    while (t.mt > 1 && t.mt * np > 4) t.mt >>= 1;
+    const int dp = (d + 127) & ~127;
+    // 16-token tiles when they fit in 64 KB and the batch needs them: a batch
+    // of up to 16 tokens is resident as one tile; from 17 to 32 tokens an
+    // expert rarely gets more than 8 and the smaller tile leaves room for
+    // gather buffers
+    const bool fits16 = 16 * 2 * dp <= 64 * 1024 && 16 <= kMaxSub * t.mt;
+    t.nt = (fits16 && T > 8 && (T <= 16 || T > 32)) ? 16 : 8;
+    return t;
 }
 
-static int meta_size(int mt)
+static bool make_layout(int d, int dp, SparseTiling til, int max_touched, SparseLayout &L)
 {
-    switch (mt) {
-    case 1: return (int)sizeof(ItemMeta<1>);
-    case 2: return (int)sizeof(ItemMeta<2>);
-    default: return (int)sizeof(ItemMeta<4>);
-    }
-}
-
-static bool make_layout(int d, int mt, int max_touched, SparseLayout &L)
-{
-    const int row_bytes = 2 * d;
     auto up = [](int v) { return (v + 127) & ~127; };
-    int rs = 8;   // rows per ring stage: 8 or 4 (d <= 4096), one copy of <= 32 KB
-    while (rs > 4 && rs * row_bytes > 32 * 1024) rs >>= 1;
-    L.rows_per_stage = rs;
-    L.stage_bytes = rs * row_bytes;
-    L.stages_per_chunk = kChunk / rs;
-    L.gpitch = 2 * row_bytes + 16;
-    int gb = 65536 / (2 * row_bytes);
-    if (gb > kChunk) gb = kChunk;
-    if (gb < 1) gb = 1;
-    L.gather_rows = gb;
-    const int gather_bytes = up(gb * L.gpitch);
-    L.xpitch = row_bytes + 16;
-    L.xbuf_bytes = up(mt * L.xpitch);
-    L.meta_bytes = up(3 * meta_size(mt));
-    const int part_bytes = up(8 * kChunk * mt * 4);
-    const int h_bytes = up(kChunk * mt * 4);
-    const int last_bytes = 128;
-    const int plan_bytes = up(4 * (4 * max_touched + 1));
-    const int fixed = gather_bytes + 2 * L.xbuf_bytes + L.meta_bytes + part_bytes + h_bytes + last_bytes +
-                      plan_bytes + 1024;
-    int ns = (kSparseSmemBudget - fixed) / L.stage_bytes;
-    if (ns > 32) ns = 32;
-    if (ns < (rs >= 8 ? 1 : 8 / rs) + kPrefetchStages) return false;   // a group of 8 rows plus the prefetch
+    const int rec = 4 * d;
+    L.xt_kb = til.nt * 128;
+    const int xt_bytes = (dp / 64) * L.xt_kb;   // a multiple of 1024
+    L.gpitch = rec + 16;
+    const int meta_bytes = up(2 * (int)sizeof(ItemMeta));
+    const int part_bytes = up(8 * kMaxGB * til.mt * 4);
+    const int h_bytes = up(kMaxGB * til.mt * 4);
+    const int plan_bytes = up(4 * (5 * max_touched + 1));
+    const int fixed = xt_bytes + meta_bytes + part_bytes + h_bytes + 128 + 128 + plan_bytes +
+                      up((2 * 8 + 2 * kMaxNU + kNumFixedBars) * 8) + 1024 /* base alignment */;
+    // three gate stages, then as much gather buffering as fits: at least
+    // three buffers of at least two records where the records allow it
+    const int ns = 3;
+    const int room = kSmemLimit - fixed - ns * kStageBytes;
+    if (room < 2 * up(L.gpitch)) return false;
+    int gb = 32768 / rec;
+    gb = gb < 1 ? 1 : gb > 4 ? 4 : gb;
+    while (gb > 2 && room / up(gb * L.gpitch) < 3) --gb;
+    while (gb > 1 && room / up(gb * L.gpitch) < 2) --gb;
+    L.gb = gb;
+    L.ud_buf_bytes = up(gb * L.gpitch);
+    int nu = room / L.ud_buf_bytes;
+    L.n_ud = nu > kMaxNU ? kMaxNU : nu;
     L.n_stages = ns;
     int off = 0;
-    L.ring_off = off; off += up(ns * L.stage_bytes);
-    L.gather_off = off; off += gather_bytes;
-    L.xbuf_off = off; off += 2 * L.xbuf_bytes;
-    L.meta_off = off; off += L.meta_bytes;
+    L.xt_off = off; off += xt_bytes;
+    L.ring_off = off; off += ns * kStageBytes;
+    L.ud_off = off; off += L.n_ud * L.ud_buf_bytes;
+    L.meta_off = off; off += meta_bytes;
     L.part_off = off; off += part_bytes;
     L.h_off = off; off += h_bytes;
-    L.last_off = off; off += last_bytes;
+    L.last_off = off; off += 128;
+    L.ctr_off = off; off += 128;
     L.plan_off = off; off += plan_bytes;
-    L.bar_off = off; off += up((2 * ns + 12) * 8);
-    L.total = off;
-    return L.total <= 227 * 1024;
+    L.bar_off = off; off += up((2 * ns + 2 * L.n_ud + kNumFixedBars) * 8);
+    L.total = off + 1024;   // slack for aligning the base to 1024 bytes
+    return L.n_ud >= 2 && L.total <= kSmemLimit;
 }
 
 template <int MT, int NP>
@@ -725,7 +899,7 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
-                                 uint16_t *out, int mt, int grid_cap, cudaStream_t st,
+                                 uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
                                  float *score_out)
 {
     SparseArgs a;
@@ -738,21 +912,26 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.f = dm.f;
     a.k = dm.k;
     a.S = dm.S;
+    a.dp = dm.dp;
+    a.n_kb = dm.n_kb;
+    a.n_blk = dm.n_blk;
+    a.n_chunks = dm.f / kChunk;
+    a.nt = til.nt;
+    a.resident = T <= til.nt ? 1 : 0;
     a.tau = tau;
     a.use_mask = use_mask ? 1 : 0;
     a.score_out = score_out;
-    a.n_chunks = dm.f / kChunk;
-    a.n_tok_tiles = (T + mt - 1) / mt;
-    a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * a.n_chunks;
-    a.target = (dm.k + dm.S) * a.n_chunks;
+    a.n_tok_tiles = (T + til.nt - 1) / til.nt;
+    a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
+    a.target = (dm.k + dm.S) * dm.n_blk;
     const int pairs = T * dm.k;
     a.max_touched = pairs < dm.E ? pairs : dm.E;
-    if (!make_layout(dm.d, mt, a.max_touched, a.L)) return cudaErrorInvalidValue;
+    if (!make_layout(dm.d, dm.dp, til, a.max_touched, a.L)) return cudaErrorInvalidValue;
     const int np = (dm.d / 8 + 255) / 256;
-    const int bound = a.n_shared_items + (a.max_touched + pairs / mt) * a.n_chunks;
-    int grid = bound < grid_cap ? bound : grid_cap;
+    const long long bound = a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk;
+    int grid = bound < grid_cap ? (int)bound : grid_cap;
     if (grid < 1) grid = 1;
-    switch (np * 8 + mt) {
+    switch (np * 8 + til.mt) {
     case 8 + 1: return launch_mt<1, 1>(a, grid, st);
     case 8 + 2: return launch_mt<2, 1>(a, grid, st);
     case 8 + 4: return launch_mt<4, 1>(a, grid, st);
@@ -761,7 +940,5 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     default: return cudaErrorInvalidValue;
     }
 }
-
-int sparse_blocks_per_sm(int) { return 1; }
 
 }  // namespace moe

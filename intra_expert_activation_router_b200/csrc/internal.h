@@ -1,17 +1,19 @@
 // internal.h -- data shared by the host library and the kernel launchers.
 //
 // Everything lives in device memory owned by the handle.  Layouts:
-//   repacked weights (neuron-major, so every neuron's data is contiguous):
-//     wg_n   [E][f][d]   row j = gate column j; inside every 128-byte group of a
-//                        row the eight 16-byte blocks are permuted b -> b ^ (j & 7)
-//                        (the 128-byte swizzle), so that eight consecutive rows
-//                        copied contiguously into shared memory are bank-conflict
-//                        free for tensor-core fragment loads; a tail of fewer than
-//                        eight blocks (d % 64 != 0) is stored unpermuted
+//   repacked weights:
+//     wg_t   [E][fp/128][dp/64][128][64]  the gate weights as tensor-core tiles:
+//                        one 16 KB tile per (128 neurons, 64 inputs), row j of a
+//                        tile = neuron, 128 bytes of inputs with the 16-byte
+//                        blocks permuted b -> b ^ (j & 7) (the 128-byte swizzle
+//                        of the MMA's K-major shared-memory layout); dp, fp =
+//                        d and f rounded up to multiples of 128, padding zero.
+//                        A 128-neuron block is contiguous over all its inputs.
 //     wud    [E][f][2d]  row j = [up column j | down row j]: one neuron's up and
 //                        down weights in a single contiguous 4d-byte record
-//     wsg_n, wsud        the same for the shared experts
+//     wsg_t, wsud        the same for the shared experts
 //     wr     [E][d]
+//     wdt    [E][d][f]   dense branch only: down weights transposed (K-major)
 //   per-call workspace, sized for max_tokens:
 //     logits [T][E] fp32, topk_idx/topk_w [T][k], perm [T*k] (pair ids
 //     t*k+rank sorted by expert, stable), mask [T*k][f/32] uint32 (bit j of
@@ -26,7 +28,8 @@
 namespace moe {
 
 constexpr int kMaxExperts = 1024;
-constexpr int kChunk = 32;           // neurons per sparse work item (one mask word)
+constexpr int kChunk = 32;           // neurons per mask word
+constexpr int kBlk = 128;            // neurons per sparse work item (the gate MMA's M)
 constexpr int kDenseTileM = 128;     // tokens per dense GEMM tile
 
 // Routing plan written by the router's last CTA.
@@ -34,7 +37,7 @@ struct Plan {
     int n_touched;                    // distinct experts selected
     int n_routed_items;               // sparse work items over routed experts
     int n_dense_tiles;                // 128-token tiles over touched experts
-    int pad_;
+    int next_item;                    // sparse work-item counter (dynamic scheduling), reset here
     int touched[kMaxExperts];         // slot -> expert id (ascending)
     int offsets[kMaxExperts + 1];     // expert -> first position in perm
     int item_prefix[kMaxExperts + 1]; // slot -> first sparse work item
@@ -44,34 +47,44 @@ struct Plan {
 struct Dims {
     int E, k, d, f, S;
     int max_tokens;
+    int dp, fp;        // d and f rounded up to multiples of 128 (gate tile padding)
+    int n_kb, n_blk;   // dp / 64 input blocks, fp / 128 neuron blocks
 };
 
 struct DeviceWeights {
     const uint16_t *wr;
-    const uint16_t *wg_n, *wud;
-    const uint16_t *wsg_n, *wsud;
+    const uint16_t *wg_t, *wud;
+    const uint16_t *wsg_t, *wsud;
     const uint16_t *wdt, *wsdt;   // dense branch only: down weights transposed, [E][d][f] / [S][d][f]
 };
 
 // Tensor maps of one dense GEMM launch (kernel parameters).
 struct DenseMaps {
     CUtensorMap a;    // GEMM1: x_perm rows; GEMM2: H rows (128-byte swizzle, box 64 x 128)
-    CUtensorMap b0;   // GEMM1: gate rows (stored pre-swizzled, copied unswizzled); GEMM2: WdT rows (box 64 x 256)
+    CUtensorMap b0;   // GEMM1: unused (gate tiles are plain bulk copies); GEMM2: WdT rows (box 64 x 256)
     CUtensorMap b1;   // GEMM1: up halves of the [up | down] records; GEMM2: unused
 };
 
 struct DenseState {
     bool ok;                           // shape supported and maps encoded
     DenseMaps g1r, g1s, g2r, g2s;      // GEMM1/GEMM2, routed/shared
+    const uint16_t *gate_r, *gate_s;   // gate tiles, routed / shared experts
 };
 
-// Position of element k inside a swizzled gate row j (see wg_n above).
-__host__ __device__ __forceinline__ int gate_pos(int j, int k, int d)
+// Element offset of gate weight (neuron j, input k) inside one expert's tiles.
+__host__ __device__ __forceinline__ size_t gate_tile_off(int j, int k, int n_kb)
 {
-    const int b = k >> 3, full = (d >> 6) << 3;
-    const int sb = b < full ? (b ^ (j & 7)) : b;
-    return (sb << 3) | (k & 7);
+    const size_t tile = (size_t)(j >> 7) * n_kb + (k >> 6);
+    return tile * 8192 + (size_t)(j & 127) * 64 + ((((k & 63) >> 3) ^ (j & 7)) << 3) + (k & 7);
 }
+
+// Token tiling of the sparse branch for a batch of T tokens:
+//   nt  tokens per gate tile (8 or 16 of the gate MMA's 16 columns carry tokens)
+//   mt  tokens per up/down pass (held in registers; nt / mt <= 4)
+struct SparseTiling {
+    int nt, mt;
+};
+SparseTiling sparse_tiling(int T, int d);
 
 struct Workspace {
     float *logits;
@@ -94,7 +107,7 @@ struct Workspace {
     uint16_t *x_stage, *out_stage;
     // optional phase timestamps (moe_set_trace); nullptr when off
     unsigned long long *trace_router;   // [router CTAs][8]
-    unsigned long long *trace_expert;   // [expert CTAs][16]
+    unsigned long long *trace_expert;   // [expert CTAs][64]
     int trace_router_ctas, trace_expert_ctas;
 };
 
@@ -106,16 +119,20 @@ __device__ __forceinline__ unsigned long long global_ns()
 }
 
 // Launchers (return cudaGetLastError()).
+// Routing plan with sparse work items of (expert, tile of `tile_tokens`
+// tokens, 128-neuron block).
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int mt, cudaStream_t st);
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st);
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
-                                 uint16_t *out, int mt, int grid_cap, cudaStream_t st,
+                                 uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
                                  float *score_out = nullptr);
-// dst[b][c][col_off + pos(c, r)] = src[b][r][c] with row stride ld (elements);
-// pos = gate_pos when swizzle, else r.
+// dst[b][c][col_off + r] = src[b][r][c] with row stride ld (elements).
 cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
-                                    int ld, int col_off, bool swizzle, cudaStream_t st);
+                                    int ld, int col_off, cudaStream_t st);
+// Gate weights src[b][d][f] (x @ W layout) -> tiles (gate_tile_off); dst zeroed first.
+cudaError_t launch_repack_gate_tiles(const uint16_t *src, uint16_t *dst, int batches, const Dims &dm,
+                                     cudaStream_t st);
 // dst[b][r][col_off + c] = src[b][r][c] with row stride ld (elements).
 cudaError_t launch_repack_rows(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols, int ld,
                                int col_off, cudaStream_t st);
@@ -131,7 +148,5 @@ bool dense_supported(const Dims &dm);
 bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st);
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
                          float tau, bool use_mask, uint16_t *out, cudaStream_t s);
-
-int sparse_tile_tokens(int T, int d);   // tokens per sparse work item for a batch of T
 
 }  // namespace moe

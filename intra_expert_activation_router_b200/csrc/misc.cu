@@ -4,10 +4,9 @@
 
 namespace moe {
 
-// dst[b][c][col_off + pos(c, r)] = src[b][r][c], 32x32 tiles through shared
-// memory; pos is the gate-row swizzle when `swizzle`, else the identity.
+// dst[b][c][col_off + r] = src[b][r][c], 32x32 tiles through shared memory.
 __global__ void k_transpose(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, int rows, int cols,
-                            int ld, int col_off, int swizzle)
+                            int ld, int col_off)
 {
     __shared__ uint16_t tile[32][33];
     const size_t sbase = (size_t)blockIdx.z * rows * cols;
@@ -20,18 +19,46 @@ __global__ void k_transpose(const uint16_t *__restrict__ src, uint16_t *__restri
     __syncthreads();
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int c = c0 + i, r = r0 + threadIdx.x;
-        if (r < rows && c < cols) {
-            const int pos = swizzle ? gate_pos(c, r, rows) : r;
-            dst[dbase + (size_t)c * ld + col_off + pos] = tile[threadIdx.x][i];
-        }
+        if (r < rows && c < cols) dst[dbase + (size_t)c * ld + col_off + r] = tile[threadIdx.x][i];
     }
 }
 
 cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
-                                    int ld, int col_off, bool swizzle, cudaStream_t st)
+                                    int ld, int col_off, cudaStream_t st)
 {
     dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches);
-    k_transpose<<<grid, dim3(32, 8), 0, st>>>(src, dst, rows, cols, ld, col_off, swizzle ? 1 : 0);
+    k_transpose<<<grid, dim3(32, 8), 0, st>>>(src, dst, rows, cols, ld, col_off);
+    return cudaGetLastError();
+}
+
+// Gate weights src[b][k][j] (input k, neuron j) -> the tensor-core tile layout
+// (gate_tile_off), 32x32 tiles through shared memory.
+__global__ void k_gate_tiles(const uint16_t *__restrict__ src, uint16_t *__restrict__ dst, int d, int f,
+                             int n_kb, size_t per_expert)
+{
+    __shared__ uint16_t tile[32][33];
+    const size_t sbase = (size_t)blockIdx.z * d * f;
+    uint16_t *dexp = dst + (size_t)blockIdx.z * per_expert;
+    const int j0 = blockIdx.x * 32, k0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int k = k0 + i, j = j0 + threadIdx.x;
+        if (k < d && j < f) tile[i][threadIdx.x] = src[sbase + (size_t)k * f + j];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int j = j0 + i, k = k0 + threadIdx.x;
+        if (k < d && j < f) dexp[gate_tile_off(j, k, n_kb)] = tile[threadIdx.x][i];
+    }
+}
+
+cudaError_t launch_repack_gate_tiles(const uint16_t *src, uint16_t *dst, int batches, const Dims &dm,
+                                     cudaStream_t st)
+{
+    const size_t per_expert = (size_t)dm.fp * dm.dp;
+    cudaError_t e = cudaMemsetAsync(dst, 0, 2 * per_expert * batches, st);
+    if (e != cudaSuccess) return e;
+    dim3 grid((dm.f + 31) / 32, (dm.d + 31) / 32, batches);
+    k_gate_tiles<<<grid, dim3(32, 8), 0, st>>>(src, dst, dm.d, dm.f, dm.n_kb, per_expert);
     return cudaGetLastError();
 }
 

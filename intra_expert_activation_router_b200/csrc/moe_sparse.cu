@@ -12,7 +12,6 @@
 #include "internal.h"
 
 namespace moe {
-int sparse_blocks_per_sm(int mt);
 }
 
 namespace {
@@ -46,7 +45,6 @@ struct moe_sparse_s {
     void *ws_mem;
     int path;
     int t_star;
-    int grid_cap[4];   // sparse kernel CTAs that fit at once, per token-tile size
     // the last forward
     int last_T, last_path, last_masked;
     cudaStream_t last_stream;
@@ -94,7 +92,6 @@ static void free_handle(moe_handle h)
     delete h;
 }
 
-static int mt_index(int mt) { return mt <= 1 ? 0 : mt <= 2 ? 1 : mt <= 4 ? 2 : 3; }
 
 extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_model, int d_ff,
                                  int n_shared, int max_tokens, moe_handle *out)
@@ -127,11 +124,15 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     }
     moe::Dims &dm = h->dm;
     dm.E = E; dm.k = top_k; dm.d = d_model; dm.f = d_ff; dm.S = n_shared; dm.max_tokens = max_tokens;
-    for (int i = 0; i < 4; ++i) h->grid_cap[i] = h->n_sm * moe::sparse_blocks_per_sm(1 << i);
+    dm.dp = (d_model + 127) & ~127;
+    dm.fp = (d_ff + 127) & ~127;
+    dm.n_kb = dm.dp / 64;
+    dm.n_blk = dm.fp / 128;
 
     const size_t fd = (size_t)d_ff * d_model;
     const bool dense = moe::dense_supported(dm);
-    const size_t wbytes = 2 * ((size_t)E * d_model + 3 * E * fd + 3 * (size_t)n_shared * fd) +
+    const size_t gd = (size_t)dm.fp * dm.dp;   // gate tiles per expert (elements)
+    const size_t wbytes = 2 * ((size_t)E * d_model + E * (gd + 2 * fd) + (size_t)n_shared * (gd + 2 * fd)) +
                           (dense ? 2 * ((size_t)E + n_shared) * fd : 0) + 16 * 256;
     const size_t T = max_tokens, P = T * top_k;
     const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
@@ -142,10 +143,10 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
 
     Block wb{(char *)h->weight_mem, 0, wbytes};
     uint16_t *wr = (uint16_t *)wb.take(2 * (size_t)E * d_model);
-    uint16_t *wg = (uint16_t *)wb.take(2 * E * fd), *wud = (uint16_t *)wb.take(4 * E * fd);
+    uint16_t *wg = (uint16_t *)wb.take(2 * E * gd), *wud = (uint16_t *)wb.take(4 * E * fd);
     uint16_t *wsg = nullptr, *wsud = nullptr;
     if (n_shared) {
-        wsg = (uint16_t *)wb.take(2 * n_shared * fd);
+        wsg = (uint16_t *)wb.take(2 * n_shared * gd);
         wsud = (uint16_t *)wb.take(4 * n_shared * fd);
     }
     uint16_t *wdt = nullptr, *wsdt = nullptr;
@@ -186,17 +187,17 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
     ok = ok && cudaMemcpyAsync(wr, w->w_router, 2 * (size_t)E * d_model, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
     const int d = d_model;
-    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_gate, wg, E, d, d_ff, d, 0, true, st) == cudaSuccess;
-    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wud, E, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_gate_tiles((const uint16_t *)w->w_gate, wg, E, dm, st) == cudaSuccess;
+    ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_up, wud, E, d, d_ff, 2 * d, 0, st) == cudaSuccess;
     ok = ok && moe::launch_repack_rows((const uint16_t *)w->w_down, wud, E, d_ff, d, 2 * d, d, st) == cudaSuccess;
     if (dense) {
-        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_down, wdt, E, d_ff, d, d_ff, 0, false, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->w_down, wdt, E, d_ff, d, d_ff, 0, st) == cudaSuccess;
         if (n_shared)
-            ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_down, wsdt, n_shared, d_ff, d, d_ff, 0, false, st) == cudaSuccess;
+            ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_down, wsdt, n_shared, d_ff, d, d_ff, 0, st) == cudaSuccess;
     }
     if (n_shared) {
-        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_gate, wsg, n_shared, d, d_ff, d, 0, true, st) == cudaSuccess;
-        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsud, n_shared, d, d_ff, 2 * d, 0, false, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_gate_tiles((const uint16_t *)w->ws_gate, wsg, n_shared, dm, st) == cudaSuccess;
+        ok = ok && moe::launch_repack_transpose((const uint16_t *)w->ws_up, wsud, n_shared, d, d_ff, 2 * d, 0, st) == cudaSuccess;
         ok = ok && moe::launch_repack_rows((const uint16_t *)w->ws_down, wsud, n_shared, d_ff, d, 2 * d, d, st) == cudaSuccess;
     }
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
@@ -250,12 +251,11 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     cudaError_t e = cudaSuccess;
     if (h->n_ev) e = cudaEventRecord(h->ev[0], st);
     if (path == MOE_PATH_SPARSE) {
-        const int mt = moe::sparse_tile_tokens(T, h->dm.d);
-        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, mt, st);
+        const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
+        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
         if (e == cudaSuccess)
-            e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, mt,
-                                          h->grid_cap[mt_index(mt)], st);
+            e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st);
     } else {
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
@@ -360,11 +360,11 @@ extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double spar
     }
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
-    const int mt = moe::sparse_tile_tokens(T, dm.d);
-    cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, mt, st);
+    const moe::SparseTiling til = moe::sparse_tiling(T, dm.d);
+    cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, til.nt, st);
     if (e == cudaSuccess)
-        e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, mt,
-                                      h->grid_cap[mt_index(mt)], st, h->scores);
+        e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, til, h->n_sm, st,
+                                      h->scores);
     // exact selection of the kq-th smallest, 8 bits per pass, most significant first
     unsigned long long want = (unsigned long long)kq;
     uint32_t prefix = 0, pmask = 0;

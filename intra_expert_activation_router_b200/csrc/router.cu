@@ -32,7 +32,8 @@ constexpr int kRankTopk = 256;      // up to this many experts, top-k by ranking
 
 struct RouterArgs {
     const uint16_t *x, *wr;
-    int T, d, E, k, mt, n_chunks;
+    int T, d, E, k;
+    int mt, n_chunks;   // sparse work items per expert: ceil(tokens / mt) * n_chunks
     Workspace ws;
 };
 
@@ -101,6 +102,7 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
             plan->tile_prefix[t_ex] = d_ex;
             plan->n_routed_items = i_ex;
             plan->n_dense_tiles = d_ex;
+            plan->next_item = 0;
         }
         __syncwarp();
         // stable scatter, 32 pairs at a time in pair order
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
 }
 
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int mt, cudaStream_t st)
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st)
 {
     RouterArgs a;
     a.x = x;
@@ -288,8 +290,8 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     a.d = dm.d;
     a.E = dm.E;
     a.k = dm.k;
-    a.mt = mt;
-    a.n_chunks = dm.f / kChunk;
+    a.mt = tile_tokens;
+    a.n_chunks = dm.n_blk;
     a.ws = ws;
     dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
     const size_t P = (size_t)T * dm.k;

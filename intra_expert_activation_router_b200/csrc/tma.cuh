@@ -1,6 +1,7 @@
 // tma.cuh -- mbarrier and bulk-copy (TMA, non-tensor) helpers, inline PTX for sm_100a.
 //
-// Every wait is bounded: after kSpinLimit failed polls the waiter records an
+// Every wait is bounded: after kSpinLimit failed polls (each a suspended wait
+// of up to kSuspendNs, or a short sleep) the waiter records an
 // error code in the handle's device error word and carries on, so a broken
 // pipeline ends the kernel with a reported error instead of a hang.  All
 // addresses a kernel computes come from item metadata, never from loaded
@@ -11,7 +12,7 @@
 
 namespace moe {
 
-constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kSpinLimit = 1u << 20;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -40,15 +41,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// The waiting thread is suspended in hardware until the phase completes or
+// kSuspendNs pass, so a waiting warp does not spin on the issue slots that the
+// working warps of its scheduler need.
+constexpr uint32_t kSuspendNs = 1000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -67,11 +73,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; bounded.
+// Wait for the phase with the given parity to complete; bounded.  Once any
+// agent of the kernel has reported an error the wait gives up early, so a
+// broken pipeline unwinds in one timeout rather than one per remaining wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code)
 {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *reinterpret_cast<volatile int *>(err) != 0) return false;
+    }
     atomicCAS(err, 0, code);
     return false;
 }
