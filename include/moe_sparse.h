@@ -172,10 +172,11 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * lists published, first gathered batch in, first batch consumed, last batch
  * consumed, up/down done; [32 + 4u] for the gather of item u < 2: mask seen,
  * then the issue times of its first three batches; [40 + g] issue of gate
- * stage g < 8; [48 + q] token rows of tile q < 8 ready; [56 + 2i], [57 + 2i]
- * first gate stage consumed and accumulator committed for item i < 3; [61]
- * gathered records processed; [62] end; [63] the CTA's item count.  Unwritten
- * slots keep their old contents.
+ * stage g < 8; [48 + q] token rows of tile q < 8 ready; [56], [57] first gate
+ * stage consumed and accumulator committed for item 0; [59], [60] the
+ * consumers' total time waiting for and working on gathered batches (ns);
+ * [61] gathered records processed; [62] end; [63] the CTA's item count.
+ * Unwritten slots keep their old contents.
  * buf == NULL turns tracing off. */
 int moe_set_trace(moe_handle h, void *buf, long long bytes);
 

@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const int slot = (int)(g % NS);
                     ok = mbar_wait(&full_g[slot], (g / NS) & 1, err, 33);
                     tc_fence_after();
-                    if (tr && i < 3 && s == 0) tr[56 + 2 * i] = global_ns();
+                    if (tr && i == 0 && s == 0) tr[56] = global_ns();
                     const uint8_t *A = ring + (size_t)slot * kStageBytes;
                     const uint8_t *B = xt + (size_t)(2 * s) * L.xt_kb;
 #pragma unroll
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     umma_commit(&empty_g[slot]);   // the stage is free once these MMAs have read it
                 }
                 umma_commit(&gdone[bsel]);
-                if (tr && i < 3) tr[57 + 2 * i] = global_ns();
+                if (tr && i == 0) tr[57] = global_ns();
                 if (!a.resident) {   // static ranges: the next id is first + i + 1
                     const bool last_of_tile =
                         i + 1 >= n_my || item_key(locate_item(a, pc, first + i + 1)) != key;
