@@ -418,9 +418,9 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * shape.d_model * 2,
                     "d2h_bytes_per_step": T * shape.d_model * 2},
-            # sparse: router + expert kernel; dense: router, gather, GEMM1 and GEMM2 per
+            # sparse: router, expert kernel, y conversion; dense: router, gather, GEMM1 and GEMM2 per
             # routed/shared group, convert
-            "gpu_launches": (2 if path == "sparse" else 5 + 2 * shape.n_shared) * args.steps,
+            "gpu_launches": (3 if path == "sparse" else 5 + 2 * shape.n_shared) * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"]},
             "stats": {"n_touched": st["n_touched"], "n_active": st["n_active"], "n_union": st["n_union"]},

@@ -19,30 +19,33 @@
 //     execution is unchanged and always dense).
 //
 // Work items are (expert, tile of up to NT of its tokens, block of 128
-// neurons), ordered expert, tile, block; each CTA (one per SM) takes a
-// contiguous range.  Agents:
-//   gate lane (warp 8)     the item's gate tiles, 32 KB stages into the ring
-//   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of two
-//                          TMEM accumulators; owns the TMEM allocation
-//   x warp (warp 10)       per tile, the token rows into the MMA's K-major
-//                          128-byte-swizzled layout (cp.async), once the MMAs
-//                          of the previous tile are done
+// neurons).  With T <= NT ("resident" mode) the whole batch is the gate MMA's
+// token operand, loaded once, and items are claimed from a counter in the
+// plan, the experts with most tokens first; otherwise each CTA takes a
+// contiguous range of items and loads each tile's token rows.  Agents, one
+// CTA per SM:
+//   gate lane (warp 8)     publishes item ids; the item's gate tiles, 32 KB
+//                          stages into the ring
+//   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of
+//                          four TMEM accumulators; owns the TMEM allocation
+//   x warp (warp 10)       token rows into the MMA's K-major 128-byte-swizzled
+//                          layout (cp.async)
 //   gather warp (warp 11)  once an item's mask is final, the union-active
-//                          [up | down] records, in batches, two buffers
-//   consumers (warps 0-7)  M(i): warps 0-3 read the accumulator (one neuron per
-//                          thread), silu, threshold, ballot per token; the mask
-//                          words and, per pass of MT tokens, the ascending list
-//                          of union-active neurons; then UD(i-1) on the CUDA
-//                          cores: up dots (each warp a slice of d, one
-//                          transposed warp reduction per group of 4 rows), h,
-//                          down rows accumulated in registers across the
-//                          blocks of one (expert, tile); when that changes the
-//                          partial goes to the fp32 accumulator y_acc[token]
-//                          with vector atomics and a per-token ticket counts
-//                          the blocks; the token's last block converts y_acc
-//                          to bf16 into `out` and re-zeroes its row and ticket.
-// The agents meet on mbarriers (copies, MMA completion, buffer reuse) and on a
-// monotonic progress counter in shared memory; every wait is bounded.
+//                          [up | down] records into a ring of buffers
+//                          (cp.async: off the TMA unit's queue)
+//   up warps (0-3)         M(i): the accumulator (one neuron per thread),
+//                          silu, threshold, ballot per token, the union per
+//                          pass of MT tokens; then per gathered batch the up
+//                          dots (each thread holds slices of d of the pass's
+//                          tokens, one transposed warp reduction per 4 rows)
+//                          and h = silu(g) u where the bit is set
+//   down warps (4-7)       per batch, h x the gathered down rows into
+//                          per-thread registers kept across consecutive blocks
+//                          of the same tokens, then fp32 vector atomics into
+//                          y_acc; a small kernel after this one converts y_acc
+//                          to bf16 into `out` and re-zeroes it.
+// The agents meet on mbarriers (copies, MMA completion, buffer and h hand-off)
+// and on monotonic progress counters in shared memory; every wait is bounded.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -52,7 +55,8 @@
 
 namespace moe {
 
-constexpr int kConsumerThreads = 256;
+constexpr int kUpThreads = 128;     // warps 0-3: mask and up projection
+constexpr int kDownThreads = 128;   // warps 4-7: down projection and flush
 constexpr int kWarpTma = 8, kWarpMma = 9, kWarpX = 10, kWarpGather = 11;
 constexpr int kSparseThreads = 384;
 constexpr int kGateTile = 16384;     // bytes of one gate tile: 128 neurons x 64 inputs
@@ -66,7 +70,9 @@ constexpr int kTmemCols = 16 * kAcc;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
-constexpr int kNumFixedBars = 2 * kAcc + 3;   // mbarriers besides the two rings': gdone, tfree, xfull, xfree, mdrain
+// mbarriers besides the two rings': gdone, tfree (kAcc each), xfull, xfree,
+// mdrain, hsfull, hsfree (2 each)
+constexpr int kNumFixedBars = 2 * kAcc + 7;
 
 struct SparseLayout {   // byte offsets from the 1024-aligned base of dynamic shared memory
     int xt_off, xt_kb;                      // token tile; bytes per 64-input block (nt * 128)
@@ -104,7 +110,6 @@ struct SparseArgs {
     int use_mask;
     int n_tok_tiles;      // ceil(T / nt), for the shared experts
     int n_shared_items;   // S * n_tok_tiles * n_blk
-    int target;           // block contributions per token: (k + S) * n_blk
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f], no up/down
     SparseLayout L;
@@ -172,16 +177,17 @@ __device__ __forceinline__ int tile_token(const SparseArgs &a, const ItemPos &p,
     return min(max(t, 0), a.T - 1);
 }
 
-// The pass's token rows from global memory (L2-resident), this lane's slice
-// of d, widened to fp32: xf[p][r][e] = x_r[8 v + e] with v = warp*32 + lane + 256 p.
+// The pass's token rows from global memory (L2-resident), this thread's
+// slice of d, widened to fp32: xf[p][r][e] = x_r[8 v + e] with
+// v = t128 + 128 p (t128: the thread's index among the four up warps).
 template <int MT, int NP>
-__device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m, int d, int warp, int lane,
+__device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m, int d, int t128,
                                        float (&xf)[NP][MT][8])
 {
     const int d8 = d >> 3;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-        const int v = warp * 32 + lane + 256 * p;
+        const int v = t128 + 128 * p;
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
             if (r < m && v < d8) {
@@ -194,30 +200,54 @@ __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m,
     }
 }
 
-// Partial up projections of kRows gathered rows over this warp's slice of d:
+// The same from the resident token tile in shared memory (the MMA's K-major
+// 128-byte-swizzled layout, token t in row t).
+template <int MT, int NP>
+__device__ __forceinline__ void load_x_tile(const uint8_t *xt, int xt_kb, const int *row, int m, int d8, int t128,
+                                            float (&xf)[NP][MT][8])
+{
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const int v = t128 + 128 * p;
+#pragma unroll
+        for (int r = 0; r < MT; ++r) {
+            if (r < m && v < d8) {
+                const int rr = row[r];
+                unpack8(*reinterpret_cast<const uint4 *>(xt + (size_t)(v >> 3) * xt_kb + rr * 128 +
+                                                         (((v & 7) ^ (rr & 7)) << 4)),
+                        xf[p][r]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xf[p][r][e] = 0.f;
+            }
+        }
+    }
+}
+
+// Partial up projections of R gathered rows over this warp's slices of d:
 // acc[q][r] = sum_{k in slice} w_q[k] x_r[k], rows q < nrows at lo + q*stride.
 // All row loads are issued before the math.  After one transposed warp
 // reduction the warp-wide sum for (q, r) sits in one lane, which stores it to
 // part_w[(row_off + q) * MT + r].
-template <int MT, int NP>
+template <int R, int MT, int NP>
 __device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nrows, const float (&xf)[NP][MT][8],
-                                           int d8, int warp, int lane, float *part_w, int row_off)
+                                           int d8, int t128, int lane, float *part_w, int row_off)
 {
-    constexpr int NV = kRows * MT;
+    constexpr int NV = R * MT;
     constexpr int SH = 5 - Log2<NV>::value;
     float acc[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-        const int v = warp * 32 + lane + 256 * p;
+        const int v = t128 + 128 * p;
         if (v < d8) {
-            uint4 wv[kRows];
+            uint4 wv[R];
 #pragma unroll
-            for (int q = 0; q < kRows; ++q)
+            for (int q = 0; q < R; ++q)
                 wv[q] = q < nrows ? *reinterpret_cast<const uint4 *>(lo + q * stride + 16 * v) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int q = 0; q < kRows; ++q) {
+            for (int q = 0; q < R; ++q) {
                 float wf[8];
                 unpack8(wv[q], wf);
 #pragma unroll
@@ -254,9 +284,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     uint8_t *ring = smem + L.ring_off;
     uint8_t *ud = smem + L.ud_off;
     ItemMeta *meta = reinterpret_cast<ItemMeta *>(smem + L.meta_off);   // [2]
-    float *part = reinterpret_cast<float *>(smem + L.part_off);        // [8 warps][kMaxGB][MT]
-    float *hs = reinterpret_cast<float *>(smem + L.h_off);             // [kMaxGB][MT]
-    int *s_last = reinterpret_cast<int *>(smem + L.last_off);          // [MT]
+    float *part = reinterpret_cast<float *>(smem + L.part_off);        // [2][4 up warps][kMaxGB][MT]
+    float *hs = reinterpret_cast<float *>(smem + L.h_off);             // [2][kMaxGB][MT]
     // progress shared between the agents; monotonic, so a reader can never
     // mistake an old value for a new one:
     //   mask_done  items whose mask and union lists are final    (consumers)
@@ -266,6 +295,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L.ctr_off + 16);
     volatile int *pub_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 32);
     volatile int *items_end = reinterpret_cast<volatile int *>(smem + L.ctr_off + 48);
+    // items whose down projection and flush are done (down warps)
+    volatile int *down_done = reinterpret_cast<volatile int *>(smem + L.ctr_off + 52);
     volatile int *s_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 64);   // [kIdRing]
     int *s_prefix = reinterpret_cast<int *>(smem + L.plan_off);
     int *s_expert = s_prefix + a.max_touched + 1;
@@ -280,6 +311,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     uint64_t *mdrain = xfree + 1;
     const int NU = L.n_ud;
     uint64_t *full_u = mdrain + 1, *empty_u = full_u + NU;   // gather buffers
+    uint64_t *hsfull = empty_u + NU, *hsfree = hsfull + 2;   // h of a batch, up warps -> down warps
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     Plan *plan = a.ws.plan;
@@ -306,6 +338,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         mbar_init(xfull, 1);
         mbar_init(xfree, 1);
         mbar_init(mdrain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&hsfull[b], 1);
+            mbar_init(&hsfree[b], 1);
+        }
+        *down_done = 0;
         *mask_done = 0;
         *pub_items = 0;
         *items_end = 0x7fffffff;
@@ -375,6 +412,64 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         }
         __threadfence_block();
         return s_items[i % kIdRing];
+    };
+
+    // The gather: once an item's mask is final, its union-active records into
+    // the gather buffers, batch by batch, as 16-byte cp.async copies spread
+    // over a warp's 32 lanes (they take the load/store path and so do not
+    // queue behind the gate stream's bulk copies in the SM's TMA unit).  A
+    // warp's batch is handed over with cp.async.mbarrier.arrive, which in
+    // practice holds the warp's next copies back until its earlier ones have
+    // landed; so `owners` warps take turns, batch ub belonging to warp
+    // ub % owners, and that many batches are in flight.
+    auto gather_loop = [&](int owner, int owners) {
+            const int rec_ck = (4 * d) / 16;   // 16-byte chunks per [up | down] record (4d bytes)
+            uint32_t ub = 0, idle = 0;
+            for (int ui = 0;;) {
+                int go = 0;
+                if (lane == 0)
+                    go = *mask_done > ui ? 1
+                                         : (*items_end <= ui || *reinterpret_cast<volatile int *>(err) != 0 ? -1 : 0);
+                go = __shfl_sync(kFull, go, 0);
+                if (go < 0) break;
+                if (go == 0) {
+                    if (++idle > kSpinLimit) {
+                        if (lane == 0) atomicCAS(err, 0, 35);
+                        break;
+                    }
+                    __nanosleep(128);
+                    continue;
+                }
+                idle = 0;
+                __threadfence_block();
+                const ItemMeta &M = meta[ui & 1];
+                unsigned long long *tg = (tr && ui < 2 && lane == 0 && owner == 0) ? tr + 32 + 4 * ui : nullptr;
+                if (tg) tg[0] = global_ns();
+                int nbatch = 0;
+                const int nsub = min(max(M.nsub, 0), kMaxSub);
+                const size_t j0 = (size_t)M.blk * kBlk;
+                for (int s = 0; s < nsub; ++s) {
+                    const int n = min(max(M.n_uni[s], 0), kBlk);
+                    for (int b0 = 0; b0 < n; b0 += L.gb, ++ub) {
+                        const int nb = min(L.gb, n - b0);
+                        const int bi = (int)(ub % NU);
+                        if ((int)(ub % (uint32_t)owners) != owner) continue;   // another gather warp's batch
+                        mbar_wait(&empty_u[bi], ((ub / NU) & 1) ^ 1, err, 36);
+                        if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
+                        ++nbatch;
+                        uint8_t *dst = ud + (size_t)bi * L.ud_buf_bytes;
+                        for (int qq = 0; qq < nb; ++qq) {
+                            const size_t j = min(j0 + M.uni[s][b0 + qq], (size_t)a.f - 1);
+                            const uint16_t *src = M.wud + j * 2 * d;
+                            uint8_t *row = dst + (size_t)qq * L.gpitch;
+                            for (int cc = lane; cc < rec_ck; cc += 32) cp_async16(row + 16 * cc, src + 8 * cc, 16u);
+                        }
+                        cp_async_arrive_noinc(&full_u[bi]);   // one of the 32 expected arrivals
+                    }
+                }
+                ++ui;
+            }
+            cp_async_wait_all();
     };
 
     if (warp == kWarpTma) {
@@ -502,6 +597,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (tr) tr[48] = global_ns();
                 mbar_arrive(xfull);
             }
+            if (!score_mode) gather_loop(1, 2);   // then the second gather warp
         } else {
             int q = -1;
             long long prev_key = 0;
@@ -525,74 +621,21 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         __syncwarp();
     } else if (warp == kWarpGather) {
         // ---------------------------------------------------------- gather warp
-        // once an item's mask is final, its union-active records into the
-        // gather buffers, batch by batch, as 16-byte cp.async copies spread
-        // over the 32 lanes: they take the load/store path, so they do not
-        // queue behind the gate stream's bulk copies in the SM's TMA unit
-        if (!score_mode) {
-            const int rec_ck = (4 * d) / 16;   // 16-byte chunks per [up | down] record (4d bytes)
-            uint32_t ub = 0, idle = 0;
-            for (int ui = 0;;) {
-                int go = 0;
-                if (lane == 0)
-                    go = *mask_done > ui ? 1
-                                         : (*items_end <= ui || *reinterpret_cast<volatile int *>(err) != 0 ? -1 : 0);
-                go = __shfl_sync(kFull, go, 0);
-                if (go < 0) break;
-                if (go == 0) {
-                    if (++idle > kSpinLimit) {
-                        if (lane == 0) atomicCAS(err, 0, 35);
-                        break;
-                    }
-                    __nanosleep(128);
-                    continue;
-                }
-                idle = 0;
-                __threadfence_block();
-                const ItemMeta &M = meta[ui & 1];
-                unsigned long long *tg = (tr && ui < 2 && lane == 0) ? tr + 32 + 4 * ui : nullptr;
-                if (tg) tg[0] = global_ns();
-                int nbatch = 0;
-                const int nsub = min(max(M.nsub, 0), kMaxSub);
-                const size_t j0 = (size_t)M.blk * kBlk;
-                for (int s = 0; s < nsub; ++s) {
-                    const int n = min(max(M.n_uni[s], 0), kBlk);
-                    for (int b0 = 0; b0 < n; b0 += L.gb, ++ub) {
-                        const int nb = min(L.gb, n - b0);
-                        const int bi = (int)(ub % NU);
-                        mbar_wait(&empty_u[bi], ((ub / NU) & 1) ^ 1, err, 36);
-                        if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
-                        ++nbatch;
-                        uint8_t *dst = ud + (size_t)bi * L.ud_buf_bytes;
-                        for (int qq = 0; qq < nb; ++qq) {
-                            const size_t j = min(j0 + M.uni[s][b0 + qq], (size_t)a.f - 1);
-                            const uint16_t *src = M.wud + j * 2 * d;
-                            uint8_t *row = dst + (size_t)qq * L.gpitch;
-                            for (int cc = lane; cc < rec_ck; cc += 32) cp_async16(row + 16 * cc, src + 8 * cc, 16u);
-                        }
-                        cp_async_arrive_noinc(&full_u[bi]);   // one of the 32 expected arrivals
-                    }
-                }
-                ++ui;
-            }
-            cp_async_wait_all();
-        }
+        if (!score_mode) gather_loop(0, a.resident ? 2 : 1);
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ consumers
-        const int ct = tid;   // 0..255
+    } else if (warp < 4) {
+        // ------------------------------------------------ up warps: mask and up
+        // M(i): metadata, the gate accumulator (one neuron per thread), silu,
+        // threshold, ballot per token, the union per pass of MT tokens; then,
+        // batch by batch, the gathered up rows against the pass's tokens (each
+        // thread holds its slices of d in registers), one transposed warp
+        // reduction per 4 rows, the four warps' partials summed by warp 0 into
+        // h = silu(g) u where the bit is set, handed to the down warps
+        const int ct = tid;   // 0..127
         const int d8 = d >> 3;
-        float acc_y[NP][8][MT];
-#pragma unroll
-        for (int p = 0; p < NP; ++p)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-#pragma unroll
-                for (int r = 0; r < MT; ++r) acc_y[p][e][r] = 0.f;
         uint32_t ub = 0;
-        int n_acc = 0, n_rec = 0, ii = 0;
-        unsigned long long t_wait = 0, t_ud = 0;   // trace only: time waiting for / spent on gathered batches
-        // ---- M(i): item metadata, accumulator -> silu, mask, union lists (all 256 threads)
+        int n_rec = 0, ii = 0;
+        unsigned long long t_wait = 0, t_work = 0;   // trace only
         auto do_mask = [&](int i, int id) {
             ItemMeta &M = meta[i & 1];
             const ItemPos p = locate_item(a, pc, id);
@@ -617,7 +660,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 M.wud = p.slot < 0 ? a.w.wsud + (size_t)(-1 - p.slot) * 2 * a.f * d
                                    : a.w.wud + (size_t)pc.expert[p.slot] * 2 * a.f * d;
             }
-            consumer_sync(kConsumerThreads);
+            consumer_sync(kUpThreads);
             unsigned long long *ti = (tr && i < 3) ? tr + 2 + 10 * i : nullptr;   // per-item stamps
             if (ti && ct == 0) ti[0] = global_ns();
             if (warp < 4) {
@@ -629,7 +672,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const int jl = warp * 32 + lane;
                 const int j = M.blk * kBlk + jl;
                 const bool jv = j < a.f;
-                const int chunk = M.blk * 4 + warp;
                 const bool masked = M.masked != 0;
                 // a rolled loop over the tile's tokens: short code, one TMEM
                 // column each (the token's own column in resident mode)
@@ -640,10 +682,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const bool on = jv && (!masked || fabsf(av) >= a.tau);
                     const unsigned word = __ballot_sync(kFull, on);
                     M.a[t][jl] = __float2half_rn(av);
-                    if (lane == 0) {
-                        M.word[t][warp] = word;
-                        if (masked && chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = word;
-                    }
+                    if (lane == 0) M.word[t][warp] = word;
                     if (score_mode && jv) a.score_out[(size_t)M.pair[t] * a.f + j] = fabsf(av);
                 }
                 tc_fence_before();
@@ -651,7 +690,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (lane == 0) mbar_arrive(&tfree[bsel]);   // the MMA may overwrite this accumulator
                 if (ti && ct == 0) ti[2] = ti[3] = global_ns();
             }
-            consumer_sync(kConsumerThreads);
+            consumer_sync(kUpThreads);
             if (ti && ct == 0) ti[4] = global_ns();
             if (warp < M.nsub) {
                 // union of the pass's tokens, compacted in ascending neuron order
@@ -668,146 +707,190 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 }
                 if (lane == 0) M.n_uni[s] = n;
             }
-            consumer_sync(kConsumerThreads);
+            consumer_sync(kUpThreads);
             if (ct == 0) {
                 __threadfence_block();
                 *mask_done = i + 1;
                 if (ti) ti[5] = global_ns();
             }
+            // the pairs' mask words for statistics and the debug lists: written
+            // after the publication, off the gather's critical path
+            if (M.masked && ct < m * 4) {
+                const int t = ct >> 2, qw = ct & 3, chunk = M.blk * 4 + qw;
+                if (chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = M.word[t][qw];
+            }
         };
         for (;; ++ii) {
-            {
-                const int id = get_item(ii);
-                if (id < 0) {
-                    if (ct == 0) *items_end = ii;   // every item of this CTA has been masked
+            const int id = get_item(ii);
+            if (id < 0) {
+                if (ct == 0) *items_end = ii;   // every item of this CTA has been masked
+                break;
+            }
+            // this metadata slot held item ii - 2: the down warps must be done with it
+            for (uint32_t spin = 0; !score_mode && ii >= 2 && *down_done < ii - 1; ++spin) {
+                if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                    atomicCAS(err, 0, 53);
                     break;
                 }
-                do_mask(ii, id);
+                __nanosleep(64);
             }
-            if (!score_mode) {
-                // ---- UD(ii): gathered up rows -> h, gathered down rows -> y, while
-                // the tensor cores already reduce the next items' gate tiles
-                const int jj = ii;
-                const ItemMeta &M = meta[jj & 1];
-                // the next item (published by the gate lane well before this point)
-                // decides whether the down partial can stay in registers
-                const int nid = get_item(ii + 1);
-                const long long next_key = nid >= 0 ? item_key(locate_item(a, pc, nid)) : 0;
-                const int m = M.m, nsub = min(M.nsub, kMaxSub);
-                unsigned long long *tu = (tr && jj < 3) ? tr + 2 + 10 * jj : nullptr;
-                for (int s = 0; s < nsub; ++s) {
-                    const int r0 = s * MT, ms = min(MT, m - r0);
-                    float xf[NP][MT][8];
-                    load_x<MT, NP>(a.x, M.tok + r0, ms, d, warp, lane, xf);
-                    const int n_uni = min(max(M.n_uni[s], 0), kBlk);
-                    n_rec += n_uni;
-                    for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
-                        const int nb = min(L.gb, n_uni - b0);
-                        const int bi = (int)(ub % NU);
-                        const unsigned long long tw0 = tr ? global_ns() : 0;
-                        mbar_wait(&full_u[bi], (ub / NU) & 1, err, 41);
-                        const unsigned long long tw1 = tr ? global_ns() : 0;
-                        t_wait += tw1 - tw0;
-                        if (tu && ct == 0 && s == 0 && b0 == 0) tu[6] = global_ns();
-                        const uint8_t *buf = ud + (size_t)bi * L.ud_buf_bytes;
+            do_mask(ii, id);
+            if (score_mode) continue;
+            const ItemMeta &M = meta[ii & 1];
+            const int m = M.m, nsub = min(M.nsub, kMaxSub);
+            unsigned long long *tu = (tr && ii < 3) ? tr + 2 + 10 * ii : nullptr;
+            for (int s = 0; s < nsub; ++s) {
+                const int r0 = s * MT, ms = min(MT, m - r0);
+                float xf[NP][MT][8];
+                if (a.resident)   // the batch never leaves shared memory
+                    load_x_tile<MT, NP>(xt, L.xt_kb, M.tok + r0, ms, d8, ct, xf);
+                else              // the tile's rows may be replaced by the next tile's
+                    load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);
+                const int n_uni = min(max(M.n_uni[s], 0), kBlk);
+                n_rec += n_uni;
+                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
+                    const int nb = min(L.gb, n_uni - b0);
+                    const int bi = (int)(ub % NU), hb = (int)(ub & 1);
+                    const unsigned long long tw0 = tr ? global_ns() : 0;
+                    mbar_wait(&full_u[bi], (ub / NU) & 1, err, 41);
+                    const unsigned long long tw1 = tr ? global_ns() : 0;
+                    t_wait += tw1 - tw0;
+                    if (tu && ct == 0 && s == 0 && b0 == 0) tu[6] = global_ns();
+                    const uint8_t *buf = ud + (size_t)bi * L.ud_buf_bytes;
+                    float *pw = part + (size_t)((hb * 4 + warp) * kMaxGB) * MT;
+                    if (L.gb <= 2)   // rows per reduction matched to the batch: no empty rows reduced
+                        group_rows<2, MT, NP>(buf, L.gpitch, nb, xf, d8, ct, lane, pw, 0);
+                    else
                         for (int g0 = 0; g0 < nb; g0 += kRows)
-                            group_rows<MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0), xf, d8,
-                                               warp, lane, part + warp * kMaxGB * MT, g0);
-                        consumer_sync(kConsumerThreads);
-                        for (int i = ct; i < nb * MT; i += kConsumerThreads) {
+                            group_rows<kRows, MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0), xf,
+                                                      d8, ct, lane, pw, g0);
+                    consumer_sync(kUpThreads);   // the four warps' partials are in
+                    if (warp == 0) {
+                        mbar_wait(&hsfree[hb], ((ub >> 1) & 1) ^ 1, err, 44);   // the down warps read this slot out
+                        for (int i = lane; i < nb * MT; i += 32) {
                             const int q = i / MT, r = i % MT;
                             float u = 0.f;
 #pragma unroll
-                            for (int w8 = 0; w8 < 8; ++w8) u += part[(w8 * kMaxGB + q) * MT + r];
+                            for (int w4 = 0; w4 < 4; ++w4) u += part[((hb * 4 + w4) * kMaxGB + q) * MT + r];
                             const int jl = M.uni[s][b0 + q];
                             const bool bit = (r < ms) && ((M.word[r0 + r][jl >> 5] >> (jl & 31)) & 1u);
-                            hs[q * MT + r] = bit ? __half2float(M.a[r0 + r][jl]) * u : 0.f;
+                            hs[(hb * kMaxGB + q) * MT + r] = bit ? __half2float(M.a[r0 + r][jl]) * u : 0.f;
                         }
-                        consumer_sync(kConsumerThreads);
-#pragma unroll
-                        for (int p = 0; p < NP; ++p) {
-                            const int v = ct + 256 * p;
-                            if (v < d8) {
-                                for (int q = 0; q < nb; ++q) {
-                                    float wf[8];
-                                    unpack8(*reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d +
-                                                                             16 * v),
-                                            wf);
-#pragma unroll
-                                    for (int r = 0; r < MT; ++r) {
-                                        const float hv = hs[q * MT + r];
-#pragma unroll
-                                        for (int e = 0; e < 8; ++e) acc_y[p][e][r] = fmaf(hv, wf[e], acc_y[p][e][r]);
-                                    }
-                                }
-                            }
-                        }
-                        consumer_sync(kConsumerThreads);
-                        if (ct == 0) {
-                            mbar_arrive(&empty_u[bi]);
-                            if (tu && s == 0 && b0 == 0) tu[7] = global_ns();
-                            if (tu) tu[8] = global_ns();
-                        }
-                        if (tr) t_ud += global_ns() - tw1;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&hsfull[hb]);
                     }
-                    ++n_acc;
-                    // keep accumulating while the next item is the next block of the same tokens
-                    const bool cont = nsub == 1 && nid >= 0 && next_key == M.key;
-                    if (!cont) {
+                    if (tr) t_work += global_ns() - tw1;
+                }
+            }
+            if (tu && ct == 0) tu[8] = global_ns();
+        }
+        if (tr && ct == 0) {
+            tr[52] = t_wait;
+            tr[53] = t_work;
+            tr[61] = (unsigned long long)n_rec;
+            tr[63] = (unsigned long long)ii;
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------ down warps: down and flush
+        // batch by batch, h x the gathered down rows into per-thread registers
+        // (each thread owns NP x 8 outputs for the pass's tokens), kept across
+        // consecutive blocks of the same tokens; then into y_acc by fp32
+        // vector atomics
+        const int ct = tid - kUpThreads;   // 0..127
+        const int d8 = d >> 3;
+        float acc_y[NP][8][MT];
 #pragma unroll
-                        for (int p = 0; p < NP; ++p) {
-                            const int v = ct + 256 * p;
+        for (int p = 0; p < NP; ++p)
 #pragma unroll
-                            for (int r = 0; r < MT; ++r) {
-                                if (v < d8 && r < ms) {
-                                    const float wt = M.w[r0 + r];
-                                    float4 *dst =
-                                        reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
-                                    atomicAdd(dst, make_float4(wt * acc_y[p][0][r], wt * acc_y[p][1][r],
-                                                               wt * acc_y[p][2][r], wt * acc_y[p][3][r]));
-                                    atomicAdd(dst + 1, make_float4(wt * acc_y[p][4][r], wt * acc_y[p][5][r],
-                                                                   wt * acc_y[p][6][r], wt * acc_y[p][7][r]));
+            for (int e = 0; e < 8; ++e)
+#pragma unroll
+                for (int r = 0; r < MT; ++r) acc_y[p][e][r] = 0.f;
+        uint32_t ub = 0;
+        unsigned long long t_wait = 0, t_work = 0;   // trace only
+        for (int ii = 0; !score_mode; ++ii) {
+            bool have = false;
+            for (uint32_t spin = 0; spin < kSpinLimit; ++spin) {
+                if (*mask_done > ii) { have = true; break; }
+                if (*items_end <= ii || *reinterpret_cast<volatile int *>(err) != 0) break;
+                __nanosleep(64);
+            }
+            if (!have) break;
+            __threadfence_block();
+            const ItemMeta &M = meta[ii & 1];
+            // the next item decides whether the down partial can stay in registers
+            const int nid = get_item(ii + 1);
+            const long long next_key = nid >= 0 ? item_key(locate_item(a, pc, nid)) : 0;
+            const int m = M.m, nsub = min(M.nsub, kMaxSub);
+            unsigned long long *tu = (tr && ii < 3) ? tr + 2 + 10 * ii : nullptr;
+            for (int s = 0; s < nsub; ++s) {
+                const int r0 = s * MT, ms = min(MT, m - r0);
+                const int n_uni = min(max(M.n_uni[s], 0), kBlk);
+                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
+                    const int nb = min(L.gb, n_uni - b0);
+                    const int bi = (int)(ub % NU), hb = (int)(ub & 1);
+                    const unsigned long long tw0 = tr ? global_ns() : 0;
+                    mbar_wait(&hsfull[hb], (ub >> 1) & 1, err, 45);
+                    const unsigned long long tw1 = tr ? global_ns() : 0;
+                    t_wait += tw1 - tw0;
+                    if (tu && ct == 0 && s == 0 && b0 == 0) tu[7] = global_ns();
+                    const uint8_t *buf = ud + (size_t)bi * L.ud_buf_bytes;
+                    const float *hq = hs + (size_t)(hb * kMaxGB) * MT;
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) {
+                        const int v = ct + 128 * p;
+                        if (v < d8) {
+                            for (int q = 0; q < nb; ++q) {
+                                float wf[8];
+                                unpack8(*reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d + 16 * v),
+                                        wf);
+#pragma unroll
+                                for (int r = 0; r < MT; ++r) {
+                                    const float hv = hq[q * MT + r];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) acc_y[p][e][r] = fmaf(hv, wf[e], acc_y[p][e][r]);
                                 }
+                            }
+                        }
+                    }
+                    group_sync(2, kDownThreads);
+                    if (ct == 0) {
+                        mbar_arrive(&hsfree[hb]);   // h slot and gather buffer are free again
+                        mbar_arrive(&empty_u[bi]);
+                    }
+                    if (tr) t_work += global_ns() - tw1;
+                }
+                // keep accumulating while the next item is the next block of the same tokens
+                const bool cont = nsub == 1 && nid >= 0 && next_key == M.key;
+                if (!cont) {
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) acc_y[p][e][r] = 0.f;
+                    for (int p = 0; p < NP; ++p) {
+                        const int v = ct + 128 * p;
+#pragma unroll
+                        for (int r = 0; r < MT; ++r) {
+                            if (v < d8 && r < ms) {
+                                const float wt = M.w[r0 + r];
+                                float4 *dst = reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
+                                atomicAdd(dst, make_float4(wt * acc_y[p][0][r], wt * acc_y[p][1][r],
+                                                           wt * acc_y[p][2][r], wt * acc_y[p][3][r]));
+                                atomicAdd(dst + 1, make_float4(wt * acc_y[p][4][r], wt * acc_y[p][5][r],
+                                                               wt * acc_y[p][6][r], wt * acc_y[p][7][r]));
                             }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc_y[p][e][r] = 0.f;
                         }
-                        __threadfence();
-                        consumer_sync(kConsumerThreads);
-                        if (ct < ms) {
-                            const int old = atomicAdd(&a.ws.tok_cnt[M.tok[r0 + ct]], n_acc);
-                            s_last[ct] = (old + n_acc == a.target);
-                        }
-                        consumer_sync(kConsumerThreads);
-                        for (int r = 0; r < ms; ++r) {
-                            if (!s_last[r]) continue;
-                            __threadfence();
-                            const int t = M.tok[r0 + r];
-                            float *yrow = a.ws.y_acc + (size_t)t * d;
-                            uint16_t *orow = a.out + (size_t)t * d;
-                            for (int i = ct * 4; i < d; i += kConsumerThreads * 4) {
-                                const float4 v4 = __ldcg(reinterpret_cast<const float4 *>(yrow + i));
-                                uint2 packed;
-                                packed.x = (uint32_t)f2bf_bits(v4.x) | ((uint32_t)f2bf_bits(v4.y) << 16);
-                                packed.y = (uint32_t)f2bf_bits(v4.z) | ((uint32_t)f2bf_bits(v4.w) << 16);
-                                *reinterpret_cast<uint2 *>(orow + i) = packed;
-                                __stcg(reinterpret_cast<float4 *>(yrow + i), make_float4(0.f, 0.f, 0.f, 0.f));
-                            }
-                            if (ct == 0) a.ws.tok_cnt[t] = 0;
-                        }
-                        n_acc = 0;
-                        consumer_sync(kConsumerThreads);
                     }
                 }
-                if (tu && ct == 0) tu[9] = global_ns();
-                consumer_sync(kConsumerThreads);   // this metadata slot is rewritten next iteration
+            }
+            group_sync(2, kDownThreads);
+            if (ct == 0) {
+                __threadfence_block();
+                *down_done = ii + 1;   // this item's metadata slot may be reused
+                if (tu) tu[9] = global_ns();
             }
         }
         if (tr && ct == 0) {
-            tr[59] = t_wait;
-            tr[60] = t_ud;
-            tr[61] = (unsigned long long)n_rec;
-            tr[63] = (unsigned long long)ii;
+            tr[54] = t_wait;
+            tr[55] = t_work;
         }
     }
     __syncthreads();
@@ -821,9 +904,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
 SparseTiling sparse_tiling(int T, int d)
 {
     SparseTiling t;
-    const int np = (d / 8 + 255) / 256;
+    const int np = (d / 8 + 127) / 128;   // 16-byte slices of d per up/down thread
     t.mt = T <= 1 ? 1 : T <= 2 ? 2 : 4;
-    while (t.mt > 1 && t.mt * np > 4) t.mt >>= 1;
+    while (t.mt > 1 && t.mt * np > 8) t.mt >>= 1;
     const int dp = (d + 127) & ~127;
     // 16-token tiles when they fit in 64 KB and the batch needs them: a batch
     // of up to 16 tokens is resident as one tile; from 17 to 32 tokens an
@@ -842,19 +925,20 @@ static bool make_layout(int d, int dp, SparseTiling til, int max_touched, Sparse
     const int xt_bytes = (dp / 64) * L.xt_kb;   // a multiple of 1024
     L.gpitch = rec + 16;
     const int meta_bytes = up(2 * (int)sizeof(ItemMeta));
-    const int part_bytes = up(8 * kMaxGB * til.mt * 4);
-    const int h_bytes = up(kMaxGB * til.mt * 4);
+    const int part_bytes = up(2 * 4 * kMaxGB * til.mt * 4);
+    const int h_bytes = up(2 * kMaxGB * til.mt * 4);
     const int plan_bytes = up(4 * (5 * max_touched + 1));
     const int fixed = xt_bytes + meta_bytes + part_bytes + h_bytes + 128 + 128 + plan_bytes +
                       up((2 * 8 + 2 * kMaxNU + kNumFixedBars) * 8) + 1024 /* base alignment */;
-    // three gate stages, then as much gather buffering as fits: at least
-    // three buffers of at least two records where the records allow it
-    const int ns = 3;
-    const int room = kSmemLimit - fixed - ns * kStageBytes;
-    if (room < 2 * up(L.gpitch)) return false;
+    // gather buffers of up to four records (rows per up reduction), at least
+    // two of them; three gate stages when that leaves room, else two (with
+    // every SM streaming, 64 KB in flight per SM still saturate HBM)
     int gb = 32768 / rec;
     gb = gb < 1 ? 1 : gb > 4 ? 4 : gb;
-    while (gb > 2 && room / up(gb * L.gpitch) < 3) --gb;
+    int ns = 3;
+    if ((kSmemLimit - fixed - ns * kStageBytes) / up(gb * L.gpitch) < 2) ns = 2;
+    const int room = kSmemLimit - fixed - ns * kStageBytes;
+    if (room < 2 * up(L.gpitch)) return false;
     while (gb > 1 && room / up(gb * L.gpitch) < 2) --gb;
     L.gb = gb;
     L.ud_buf_bytes = up(gb * L.gpitch);
@@ -874,6 +958,40 @@ static bool make_layout(int d, int dp, SparseTiling til, int max_touched, Sparse
     L.bar_off = off; off += up((2 * ns + 2 * L.n_ud + kNumFixedBars) * 8);
     L.total = off + 1024;   // slack for aligning the base to 1024 bytes
     return L.n_ud >= 2 && L.total <= kSmemLimit;
+}
+
+// out = bf16(y_acc) (round to nearest even), then y_acc = 0; launched after
+// the expert kernel as its programmatic dependent.
+__global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(y_acc) + i);
+        uint2 p;
+        p.x = (uint32_t)f2bf_bits(v.x) | ((uint32_t)f2bf_bits(v.y) << 16);
+        p.y = (uint32_t)f2bf_bits(v.z) | ((uint32_t)f2bf_bits(v.w) << 16);
+        reinterpret_cast<uint2 *>(out)[i] = p;
+        __stcg(reinterpret_cast<float4 *>(y_acc) + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
+}
+
+static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm, cudaStream_t st)
+{
+    size_t blocks = (n4 + 255) / 256;
+    if (blocks > (size_t)n_sm * 4) blocks = (size_t)n_sm * 4;
+    if (blocks < 1) blocks = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_y_out, y_acc, out, n4);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 template <int MT, int NP>
@@ -923,22 +1041,27 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.score_out = score_out;
     a.n_tok_tiles = (T + til.nt - 1) / til.nt;
     a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
-    a.target = (dm.k + dm.S) * dm.n_blk;
     const int pairs = T * dm.k;
     a.max_touched = pairs < dm.E ? pairs : dm.E;
     if (!make_layout(dm.d, dm.dp, til, a.max_touched, a.L)) return cudaErrorInvalidValue;
-    const int np = (dm.d / 8 + 255) / 256;
+    const int np = (dm.d / 8 + 127) / 128;
     const long long bound = a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
     if (grid < 1) grid = 1;
+    cudaError_t e;
     switch (np * 8 + til.mt) {
-    case 8 + 1: return launch_mt<1, 1>(a, grid, st);
-    case 8 + 2: return launch_mt<2, 1>(a, grid, st);
-    case 8 + 4: return launch_mt<4, 1>(a, grid, st);
-    case 16 + 1: return launch_mt<1, 2>(a, grid, st);
-    case 16 + 2: return launch_mt<2, 2>(a, grid, st);
+    case 8 + 1: e = launch_mt<1, 1>(a, grid, st); break;
+    case 8 + 2: e = launch_mt<2, 1>(a, grid, st); break;
+    case 8 + 4: e = launch_mt<4, 1>(a, grid, st); break;
+    case 16 + 1: e = launch_mt<1, 2>(a, grid, st); break;
+    case 16 + 2: e = launch_mt<2, 2>(a, grid, st); break;
+    case 16 + 4: e = launch_mt<4, 2>(a, grid, st); break;
+    case 32 + 1: e = launch_mt<1, 4>(a, grid, st); break;
+    case 32 + 2: e = launch_mt<2, 4>(a, grid, st); break;
     default: return cudaErrorInvalidValue;
     }
+    if (e != cudaSuccess || score_out) return e;
+    return launch_y_out(ws.y_acc, out, (size_t)T * dm.d / 4, grid_cap, st);
 }
 
 }  // namespace moe

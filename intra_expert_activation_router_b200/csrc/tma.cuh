@@ -115,10 +115,16 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
-// Barrier among the consumer warps only (id 1); the producer warp never joins it.
+// Barriers among a subset of the CTA's warps (named barriers 1 and 2); the
+// other warps never join them.
 __device__ __forceinline__ void consumer_sync(int n_threads)
 {
     asm volatile("bar.sync 1, %0;" ::"r"(n_threads) : "memory");
+}
+
+__device__ __forceinline__ void group_sync(int id, int n_threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n_threads) : "memory");
 }
 
 }  // namespace moe
