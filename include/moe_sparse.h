@@ -169,12 +169,13 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * half holds 64 per expert-kernel CTA: [0] start, [1] plan loaded; for each
  * of the CTA's first three items i, at 2 + 10*i: metadata ready, gate
  * accumulator ready, mask read out (twice), mask step synchronised, mask and
- * lists published, first gathered batch in, first batch consumed, last batch
- * consumed, up/down done; [32 + 4u] for the gather of item u < 2: mask seen,
- * then the issue times of its first three batches; [40 + g] issue of gate
- * stage g < 8; [48 + q] token rows of tile q < 8 ready; [56], [57] first gate
- * stage consumed and accumulator committed for item 0; [59], [60] the
- * consumers' total time waiting for and working on gathered batches (ns);
+ * lists published, first gathered batch in (up warps), first h in (down
+ * warps), up projection done, down projection and flush done; [32 + 4u] for
+ * the gather of item u < 2: mask seen, then the issue times of its first
+ * three batches; [40 + g] issue of gate stage g < 8; [48 + q] token rows of
+ * tile q < 4 ready; [52], [53] the up warps' total time waiting for and
+ * working on gathered batches, [54], [55] the same for the down warps (ns);
+ * [56], [57] first gate stage consumed and accumulator committed for item 0;
  * [61] gathered records processed; [62] end; [63] the CTA's item count.
  * Unwritten slots keep their old contents.
  * buf == NULL turns tracing off. */

@@ -612,7 +612,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const int m = tile_tokens(a, pc, p, base);
                 load_rows(m, [&](int r) { return tile_token(a, p, base, r); });
                 if (lane == 0) {
-                    if (tr && q < 8) tr[48 + q] = global_ns();
+                    if (tr && q < 4) tr[48 + q] = global_ns();
                     mbar_arrive(xfull);
                 }
             }
