@@ -36,6 +36,30 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
     f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
 }
 
+// Two fp32 lanes in one 64-bit register (element 0 in the low half), for the
+// packed fp32 FMA of sm_100 (fma.rn.f32x2: each lane an ordinary fma.rn).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// bf16 pair (low half = element 0) -> the two floats, packed.  Exact widening.
+__device__ __forceinline__ uint64_t bf16x2_f2(uint32_t v) { return f2_pack(bf16_lo(v), bf16_hi(v)); }
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b, float acc)
 {
     acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);

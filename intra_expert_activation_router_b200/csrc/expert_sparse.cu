@@ -21,9 +21,13 @@
 // Work items are (expert, tile of up to NT of its tokens, block of 128
 // neurons).  With T <= NT ("resident" mode) the whole batch is the gate MMA's
 // token operand, loaded once, and items are claimed from a counter in the
-// plan, the experts with most tokens first; otherwise each CTA takes a
-// contiguous range of items and loads each tile's token rows.  Agents, one
-// CTA per SM:
+// plan, the experts with most tokens first.  A CTA claims its next item only
+// once its previous one is masked and at most kClaimBacklog of its gathered
+// records are still to be projected: an item's up/down cost (its active
+// records) varies several-fold and is known only after its mask, so claims
+// paced by the gate stream alone leave some CTAs with three heavy items and
+// others idle.  Otherwise each CTA takes a contiguous range of items and
+// loads each tile's token rows.  Agents, one CTA per SM:
 //   gate lane (warp 8)     publishes item ids; the item's gate tiles, 32 KB
 //                          stages into the ring
 //   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of
@@ -70,6 +74,7 @@ constexpr int kTmemCols = 16 * kAcc;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
+constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
 // mbarriers besides the two rings': gdone, tfree (kAcc each), xfull, xfree,
 // mdrain, hsfull, hsfree (2 each)
 constexpr int kNumFixedBars = 2 * kAcc + 7;
@@ -178,11 +183,12 @@ __device__ __forceinline__ int tile_token(const SparseArgs &a, const ItemPos &p,
 }
 
 // The pass's token rows from global memory (L2-resident), this thread's
-// slice of d, widened to fp32: xf[p][r][e] = x_r[8 v + e] with
-// v = t128 + 128 p (t128: the thread's index among the four up warps).
+// slices of d, widened to fp32 and packed in pairs: xf[p][r][i] holds
+// x_r[8 v + 2i] and x_r[8 v + 2i + 1] with v = t128 + 128 p (t128: the
+// thread's index among the four up warps).
 template <int MT, int NP>
 __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m, int d, int t128,
-                                       float (&xf)[NP][MT][8])
+                                       uint64_t (&xf)[NP][MT][4])
 {
     const int d8 = d >> 3;
 #pragma unroll
@@ -190,12 +196,11 @@ __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m,
         const int v = t128 + 128 * p;
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
-            if (r < m && v < d8) {
-                unpack8(ld_cached(x + (size_t)tok[r] * d + 8 * v), xf[p][r]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xf[p][r][e] = 0.f;
-            }
+            const uint4 xv = (r < m && v < d8) ? ld_cached(x + (size_t)tok[r] * d + 8 * v) : make_uint4(0, 0, 0, 0);
+            xf[p][r][0] = bf16x2_f2(xv.x);
+            xf[p][r][1] = bf16x2_f2(xv.y);
+            xf[p][r][2] = bf16x2_f2(xv.z);
+            xf[p][r][3] = bf16x2_f2(xv.w);
         }
     }
 }
@@ -204,40 +209,42 @@ __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m,
 // 128-byte-swizzled layout, token t in row t).
 template <int MT, int NP>
 __device__ __forceinline__ void load_x_tile(const uint8_t *xt, int xt_kb, const int *row, int m, int d8, int t128,
-                                            float (&xf)[NP][MT][8])
+                                            uint64_t (&xf)[NP][MT][4])
 {
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int v = t128 + 128 * p;
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
+            uint4 xv = make_uint4(0, 0, 0, 0);
             if (r < m && v < d8) {
                 const int rr = row[r];
-                unpack8(*reinterpret_cast<const uint4 *>(xt + (size_t)(v >> 3) * xt_kb + rr * 128 +
-                                                         (((v & 7) ^ (rr & 7)) << 4)),
-                        xf[p][r]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xf[p][r][e] = 0.f;
+                xv = *reinterpret_cast<const uint4 *>(xt + (size_t)(v >> 3) * xt_kb + rr * 128 +
+                                                      (((v & 7) ^ (rr & 7)) << 4));
             }
+            xf[p][r][0] = bf16x2_f2(xv.x);
+            xf[p][r][1] = bf16x2_f2(xv.y);
+            xf[p][r][2] = bf16x2_f2(xv.z);
+            xf[p][r][3] = bf16x2_f2(xv.w);
         }
     }
 }
 
 // Partial up projections of R gathered rows over this warp's slices of d:
-// acc[q][r] = sum_{k in slice} w_q[k] x_r[k], rows q < nrows at lo + q*stride.
-// All row loads are issued before the math.  After one transposed warp
-// reduction the warp-wide sum for (q, r) sits in one lane, which stores it to
+// acc[q][r] = sum_{k in slices} w_q[k] x_r[k], rows q < nrows at lo + q*stride,
+// even and odd k in the two lanes of packed fp32 FMAs.  All row loads are
+// issued before the math.  After one transposed warp reduction the warp-wide
+// sum for (q, r) sits in one lane, which stores it to
 // part_w[(row_off + q) * MT + r].
 template <int R, int MT, int NP>
-__device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nrows, const float (&xf)[NP][MT][8],
+__device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nrows, const uint64_t (&xf)[NP][MT][4],
                                            int d8, int t128, int lane, float *part_w, int row_off)
 {
     constexpr int NV = R * MT;
     constexpr int SH = 5 - Log2<NV>::value;
-    float acc[NV];
+    uint64_t acc2[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) acc[i] = 0.f;
+    for (int i = 0; i < NV; ++i) acc2[i] = 0ull;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int v = t128 + 128 * p;
@@ -248,17 +255,24 @@ __device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nr
                 wv[q] = q < nrows ? *reinterpret_cast<const uint4 *>(lo + q * stride + 16 * v) : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int q = 0; q < R; ++q) {
-                float wf[8];
-                unpack8(wv[q], wf);
+                const uint64_t w2[4] = {bf16x2_f2(wv[q].x), bf16x2_f2(wv[q].y), bf16x2_f2(wv[q].z),
+                                        bf16x2_f2(wv[q].w)};
 #pragma unroll
                 for (int r = 0; r < MT; ++r) {
-                    float s = acc[q * MT + r];
+                    uint64_t a2 = acc2[q * MT + r];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s = fmaf(wf[e], xf[p][r][e], s);
-                    acc[q * MT + r] = s;
+                    for (int i = 0; i < 4; ++i) a2 = ffma2(w2[i], xf[p][r][i], a2);
+                    acc2[q * MT + r] = a2;
                 }
             }
         }
+    }
+    float acc[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        float e0, e1;
+        f2_unpack(acc2[i], e0, e1);
+        acc[i] = e0 + e1;
     }
     const float val = transpose_reduce<NV>(acc, lane);
     const int vi = lane >> SH, q = vi / MT, r = vi % MT;
@@ -297,6 +311,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     volatile int *items_end = reinterpret_cast<volatile int *>(smem + L.ctr_off + 48);
     // items whose down projection and flush are done (down warps)
     volatile int *down_done = reinterpret_cast<volatile int *>(smem + L.ctr_off + 52);
+    // records of the masked items (up warps) and records projected (down warps)
+    volatile int *rec_masked = reinterpret_cast<volatile int *>(smem + L.ctr_off + 36);
+    volatile int *rec_done = reinterpret_cast<volatile int *>(smem + L.ctr_off + 40);
     volatile int *s_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 64);   // [kIdRing]
     int *s_prefix = reinterpret_cast<int *>(smem + L.plan_off);
     int *s_expert = s_prefix + a.max_touched + 1;
@@ -344,6 +361,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         }
         *down_done = 0;
         *mask_done = 0;
+        *rec_masked = 0;
+        *rec_done = 0;
         *pub_items = 0;
         *items_end = 0x7fffffff;
         fence_mbar_init();
@@ -484,8 +503,25 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int i = 0;; ++i) {
                 int id;
                 if (a.resident) {
+                    if (i > 0 && next < n_items) {
+                        // item i - 1 masked and the up/down backlog short: claim the
+                        // next item (its gate streams while the backlog drains)
+                        bool ok = true;
+                        for (uint32_t spin = 0;; ++spin) {
+                            if (*mask_done >= i) {
+                                __threadfence_block();
+                                if (score_mode || *rec_masked - *rec_done <= kClaimBacklog) break;
+                            }
+                            if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                                atomicCAS(err, 0, 54);
+                                ok = false;
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                        next = ok ? atomicAdd(&plan->next_item, 1) : n_items;
+                    }
                     id = next < n_items ? next : -1;
-                    if (id >= 0) next = atomicAdd(&plan->next_item, 1);   // claimed early: the reply lands meanwhile
                 } else {
                     id = i < n_my ? first + i : -1;
                 }
@@ -709,6 +745,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             }
             consumer_sync(kUpThreads);
             if (ct == 0) {
+                if (!score_mode) {
+                    int total = 0;
+                    for (int s = 0; s < min(M.nsub, kMaxSub); ++s) total += min(max(M.n_uni[s], 0), kBlk);
+                    *rec_masked = *rec_masked + total;
+                }
                 __threadfence_block();
                 *mask_done = i + 1;
                 if (ti) ti[5] = global_ns();
@@ -741,7 +782,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             unsigned long long *tu = (tr && ii < 3) ? tr + 2 + 10 * ii : nullptr;
             for (int s = 0; s < nsub; ++s) {
                 const int r0 = s * MT, ms = min(MT, m - r0);
-                float xf[NP][MT][8];
+                uint64_t xf[NP][MT][4];
                 if (a.resident)   // the batch never leaves shared memory
                     load_x_tile<MT, NP>(xt, L.xt_kb, M.tok + r0, ms, d8, ct, xf);
                 else              // the tile's rows may be replaced by the next tile's
@@ -798,13 +839,13 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         // vector atomics
         const int ct = tid - kUpThreads;   // 0..127
         const int d8 = d >> 3;
-        float acc_y[NP][8][MT];
+        uint64_t acc_y[NP][4][MT];   // output pairs (8 v + 2i, 8 v + 2i + 1) of each token, packed
 #pragma unroll
         for (int p = 0; p < NP; ++p)
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int r = 0; r < MT; ++r) acc_y[p][e][r] = 0.f;
+                for (int r = 0; r < MT; ++r) acc_y[p][i][r] = 0ull;
         uint32_t ub = 0;
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         for (int ii = 0; !score_mode; ++ii) {
@@ -817,9 +858,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             if (!have) break;
             __threadfence_block();
             const ItemMeta &M = meta[ii & 1];
-            // the next item decides whether the down partial can stay in registers
-            const int nid = get_item(ii + 1);
-            const long long next_key = nid >= 0 ? item_key(locate_item(a, pc, nid)) : 0;
             const int m = M.m, nsub = min(M.nsub, kMaxSub);
             unsigned long long *tu = (tr && ii < 3) ? tr + 2 + 10 * ii : nullptr;
             for (int s = 0; s < nsub; ++s) {
@@ -840,14 +878,16 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                         const int v = ct + 128 * p;
                         if (v < d8) {
                             for (int q = 0; q < nb; ++q) {
-                                float wf[8];
-                                unpack8(*reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d + 16 * v),
-                                        wf);
+                                const uint4 wv =
+                                    *reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d + 16 * v);
+                                const uint64_t w2[4] = {bf16x2_f2(wv.x), bf16x2_f2(wv.y), bf16x2_f2(wv.z),
+                                                        bf16x2_f2(wv.w)};
 #pragma unroll
                                 for (int r = 0; r < MT; ++r) {
                                     const float hv = hq[q * MT + r];
+                                    const uint64_t h2 = f2_pack(hv, hv);
 #pragma unroll
-                                    for (int e = 0; e < 8; ++e) acc_y[p][e][r] = fmaf(hv, wf[e], acc_y[p][e][r]);
+                                    for (int i = 0; i < 4; ++i) acc_y[p][i][r] = ffma2(w2[i], h2, acc_y[p][i][r]);
                                 }
                             }
                         }
@@ -856,11 +896,18 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     if (ct == 0) {
                         mbar_arrive(&hsfree[hb]);   // h slot and gather buffer are free again
                         mbar_arrive(&empty_u[bi]);
+                        *rec_done = *rec_done + nb;
                     }
                     if (tr) t_work += global_ns() - tw1;
                 }
-                // keep accumulating while the next item is the next block of the same tokens
-                const bool cont = nsub == 1 && nid >= 0 && next_key == M.key;
+                // keep accumulating while the next item is the next block of the
+                // same tokens (looked up only now: in resident mode the next item
+                // is claimed once this one's backlog has drained)
+                bool cont = false;
+                if (nsub == 1) {
+                    const int nid = get_item(ii + 1);
+                    cont = nid >= 0 && item_key(locate_item(a, pc, nid)) == M.key;
+                }
                 if (!cont) {
 #pragma unroll
                     for (int p = 0; p < NP; ++p) {
@@ -869,14 +916,15 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                         for (int r = 0; r < MT; ++r) {
                             if (v < d8 && r < ms) {
                                 const float wt = M.w[r0 + r];
+                                float y[8];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) f2_unpack(acc_y[p][i][r], y[2 * i], y[2 * i + 1]);
                                 float4 *dst = reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
-                                atomicAdd(dst, make_float4(wt * acc_y[p][0][r], wt * acc_y[p][1][r],
-                                                           wt * acc_y[p][2][r], wt * acc_y[p][3][r]));
-                                atomicAdd(dst + 1, make_float4(wt * acc_y[p][4][r], wt * acc_y[p][5][r],
-                                                               wt * acc_y[p][6][r], wt * acc_y[p][7][r]));
+                                atomicAdd(dst, make_float4(wt * y[0], wt * y[1], wt * y[2], wt * y[3]));
+                                atomicAdd(dst + 1, make_float4(wt * y[4], wt * y[5], wt * y[6], wt * y[7]));
                             }
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) acc_y[p][e][r] = 0.f;
+                            for (int i = 0; i < 4; ++i) acc_y[p][i][r] = 0ull;
                         }
                     }
                 }
