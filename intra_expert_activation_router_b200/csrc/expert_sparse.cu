@@ -8,7 +8,7 @@
 //     neuron of the selected expert -- here a tcgen05 MMA per 128-neuron block:
 //     D[128 neurons x 16 columns] (TMEM) = Wg block . X tile^T, the block's
 //     gate tiles streamed through a ring of 32 KB stages (bulk copies), the
-//     tile's token rows resident in shared memory in the MMA's layout;
+//     token operand in the MMA's K-major swizzled layout;
 //   - activation mask in one O(n) pass, no sort ("Activation masking"):
 //     active iff |silu(g)| >= tau -- a warp ballot over 32 neurons per token;
 //   - fused up-down projection over the active neurons only ("Fused up-down
@@ -20,8 +20,11 @@
 //
 // Work items are (expert, tile of up to NT of its tokens, block of 128
 // neurons).  With T <= NT ("resident" mode) the whole batch is the gate MMA's
-// token operand, loaded once, and items are claimed from a counter in the
-// plan, the experts with most tokens first.  A CTA claims its next item only
+// token operand: the router writes it in the MMA's layout, and each ring
+// stage carries its two 64-input blocks (2 or 4 KB, re-read from L2 per
+// item) next to the 32 KB of gate tiles, which leaves the shared memory of a
+// resident token tile to the gather buffers.  Items are claimed from a
+// counter in the plan, the experts with most tokens first.  A CTA claims its next item only
 // once its previous one is masked and at most kClaimBacklog of its gathered
 // records are still to be projected: an item's up/down cost (its active
 // records) varies several-fold and is known only after its mask, so claims
@@ -29,11 +32,13 @@
 // others idle.  Otherwise each CTA takes a contiguous range of items and
 // loads each tile's token rows.  Agents, one CTA per SM:
 //   gate lane (warp 8)     publishes item ids; the item's gate tiles, 32 KB
-//                          stages into the ring
+//                          stages into the ring (with the token operand's
+//                          blocks in resident mode)
 //   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of
 //                          four TMEM accumulators; owns the TMEM allocation
-//   x warp (warp 10)       token rows into the MMA's K-major 128-byte-swizzled
-//                          layout (cp.async)
+//   x warp (warp 10)       tile mode: token rows into the MMA's K-major
+//                          128-byte-swizzled layout (cp.async); resident
+//                          mode: a second gather warp
 //   gather warp (warp 11)  once an item's mask is final, the union-active
 //                          [up | down] records into a ring of buffers
 //                          (cp.async: off the TMA unit's queue)
@@ -80,7 +85,9 @@ constexpr int kClaimBacklog = 24;    // resident mode: records still to project 
 constexpr int kNumFixedBars = 2 * kAcc + 7;
 
 struct SparseLayout {   // byte offsets from the 1024-aligned base of dynamic shared memory
-    int xt_off, xt_kb;                      // token tile; bytes per 64-input block (nt * 128)
+    int xt_off, xt_kb;                      // token tile (tile mode); bytes per 64-input block (nt * 128)
+    int stage_pitch, xs_bytes;              // ring stage: 32 KB of gate tiles, then (resident mode) the
+                                            // stage's two 64-input blocks of the token operand
     int ring_off, n_stages;
     int ud_off, ud_buf_bytes, gb, gpitch;   // n_ud buffers of gb [up | down] records (+16-byte skew)
     int n_ud;
@@ -197,31 +204,6 @@ __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m,
 #pragma unroll
         for (int r = 0; r < MT; ++r) {
             const uint4 xv = (r < m && v < d8) ? ld_cached(x + (size_t)tok[r] * d + 8 * v) : make_uint4(0, 0, 0, 0);
-            xf[p][r][0] = bf16x2_f2(xv.x);
-            xf[p][r][1] = bf16x2_f2(xv.y);
-            xf[p][r][2] = bf16x2_f2(xv.z);
-            xf[p][r][3] = bf16x2_f2(xv.w);
-        }
-    }
-}
-
-// The same from the resident token tile in shared memory (the MMA's K-major
-// 128-byte-swizzled layout, token t in row t).
-template <int MT, int NP>
-__device__ __forceinline__ void load_x_tile(const uint8_t *xt, int xt_kb, const int *row, int m, int d8, int t128,
-                                            uint64_t (&xf)[NP][MT][4])
-{
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-        const int v = t128 + 128 * p;
-#pragma unroll
-        for (int r = 0; r < MT; ++r) {
-            uint4 xv = make_uint4(0, 0, 0, 0);
-            if (r < m && v < d8) {
-                const int rr = row[r];
-                xv = *reinterpret_cast<const uint4 *>(xt + (size_t)(v >> 3) * xt_kb + rr * 128 +
-                                                      (((v & 7) ^ (rr & 7)) << 4));
-            }
             xf[p][r][0] = bf16x2_f2(xv.x);
             xf[p][r][1] = bf16x2_f2(xv.y);
             xf[p][r][2] = bf16x2_f2(xv.z);
@@ -544,8 +526,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const int slot = (int)(g % NS);
                     if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
                     if (tr && g < 8) tr[40 + g] = global_ns();
-                    mbar_arrive_expect_tx(&full_g[slot], kStageBytes);
-                    bulk_g2s_hint(ring + (size_t)slot * kStageBytes, src + (size_t)s * (kStageBytes / 2), kStageBytes,
+                    uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
+                    mbar_arrive_expect_tx(&full_g[slot], kStageBytes + L.xs_bytes);
+                    if (L.xs_bytes)   // the token operand's blocks 2s, 2s+1 (L2-resident, re-read per item)
+                        bulk_g2s(stage + kStageBytes, a.ws.x_tiles + (size_t)s * (L.xs_bytes / 2), L.xs_bytes,
+                                 &full_g[slot]);
+                    bulk_g2s_hint(stage, src + (size_t)s * (kStageBytes / 2), kStageBytes,
                                   &full_g[slot], pol);
                 }
                 if (!ok) {   // publish the end so that every agent stops
@@ -567,7 +553,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             int q = -1;
             long long prev_key = 0;
             bool ok = true;
-            if (a.resident) ok = mbar_wait(xfull, 0, err, 31);   // the batch's token rows, once
             for (int i = 0; ok; ++i) {
                 const int id = get_item(i);
                 if (id < 0) break;
@@ -586,8 +571,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     ok = mbar_wait(&full_g[slot], (g / NS) & 1, err, 33);
                     tc_fence_after();
                     if (tr && i == 0 && s == 0) tr[56] = global_ns();
-                    const uint8_t *A = ring + (size_t)slot * kStageBytes;
-                    const uint8_t *B = xt + (size_t)(2 * s) * L.xt_kb;
+                    const uint8_t *A = ring + (size_t)slot * L.stage_pitch;
+                    const uint8_t *B = L.xs_bytes ? A + kStageBytes : xt + (size_t)(2 * s) * L.xt_kb;
 #pragma unroll
                     for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
@@ -628,12 +613,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             __syncwarp();
         };
         if (a.resident) {
-            load_rows(a.T, [](int r) { return r; });   // column t of the MMA = token t
-            if (lane == 0) {
-                if (tr) tr[48] = global_ns();
-                mbar_arrive(xfull);
-            }
-            if (!score_mode) gather_loop(1, 2);   // then the second gather warp
+            // the token operand streams with the gate tiles: this warp is the
+            // second gather warp
+            if (!score_mode) gather_loop(1, 2);
         } else {
             int q = -1;
             long long prev_key = 0;
@@ -783,10 +765,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int s = 0; s < nsub; ++s) {
                 const int r0 = s * MT, ms = min(MT, m - r0);
                 uint64_t xf[NP][MT][4];
-                if (a.resident)   // the batch never leaves shared memory
-                    load_x_tile<MT, NP>(xt, L.xt_kb, M.tok + r0, ms, d8, ct, xf);
-                else              // the tile's rows may be replaced by the next tile's
-                    load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);
+                load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);   // the pass's token rows (L2-resident)
                 const int n_uni = min(max(M.n_uni[s], 0), kBlk);
                 n_rec += n_uni;
                 for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
@@ -965,12 +944,16 @@ SparseTiling sparse_tiling(int T, int d)
     return t;
 }
 
-static bool make_layout(int d, int dp, SparseTiling til, int max_touched, SparseLayout &L)
+static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_touched, SparseLayout &L)
 {
     auto up = [](int v) { return (v + 127) & ~127; };
     const int rec = 4 * d;
     L.xt_kb = til.nt * 128;
-    const int xt_bytes = (dp / 64) * L.xt_kb;   // a multiple of 1024
+    // resident mode streams the token operand with the gate stages; tile mode
+    // keeps the tile's rows in shared memory
+    const int xt_bytes = resident ? 0 : (dp / 64) * L.xt_kb;   // a multiple of 1024
+    L.xs_bytes = resident ? 2 * L.xt_kb : 0;
+    L.stage_pitch = kStageBytes + L.xs_bytes;                  // a multiple of 1024
     L.gpitch = rec + 16;
     const int meta_bytes = up(2 * (int)sizeof(ItemMeta));
     const int part_bytes = up(2 * 4 * kMaxGB * til.mt * 4);
@@ -979,13 +962,12 @@ static bool make_layout(int d, int dp, SparseTiling til, int max_touched, Sparse
     const int fixed = xt_bytes + meta_bytes + part_bytes + h_bytes + 128 + 128 + plan_bytes +
                       up((2 * 8 + 2 * kMaxNU + kNumFixedBars) * 8) + 1024 /* base alignment */;
     // gather buffers of up to four records (rows per up reduction), at least
-    // two of them; three gate stages when that leaves room, else two (with
-    // every SM streaming, 64 KB in flight per SM still saturate HBM)
+    // two of them; three gate stages when that leaves two buffers, else two
     int gb = 32768 / rec;
     gb = gb < 1 ? 1 : gb > 4 ? 4 : gb;
     int ns = 3;
-    if ((kSmemLimit - fixed - ns * kStageBytes) / up(gb * L.gpitch) < 2) ns = 2;
-    const int room = kSmemLimit - fixed - ns * kStageBytes;
+    if ((kSmemLimit - fixed - ns * L.stage_pitch) / up(gb * L.gpitch) < 2) ns = 2;
+    const int room = kSmemLimit - fixed - ns * L.stage_pitch;
     if (room < 2 * up(L.gpitch)) return false;
     while (gb > 1 && room / up(gb * L.gpitch) < 2) --gb;
     L.gb = gb;
@@ -995,7 +977,7 @@ static bool make_layout(int d, int dp, SparseTiling til, int max_touched, Sparse
     L.n_stages = ns;
     int off = 0;
     L.xt_off = off; off += xt_bytes;
-    L.ring_off = off; off += ns * kStageBytes;
+    L.ring_off = off; off += ns * L.stage_pitch;
     L.ud_off = off; off += L.n_ud * L.ud_buf_bytes;
     L.meta_off = off; off += meta_bytes;
     L.part_off = off; off += part_bytes;
@@ -1091,7 +1073,7 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
     const int pairs = T * dm.k;
     a.max_touched = pairs < dm.E ? pairs : dm.E;
-    if (!make_layout(dm.d, dm.dp, til, a.max_touched, a.L)) return cudaErrorInvalidValue;
+    if (!make_layout(dm.d, dm.dp, til, a.resident != 0, a.max_touched, a.L)) return cudaErrorInvalidValue;
     const int np = (dm.d / 8 + 127) / 128;
     const long long bound = a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk;
     int grid = bound < grid_cap ? (int)bound : grid_cap;

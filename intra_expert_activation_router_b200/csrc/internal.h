@@ -102,6 +102,11 @@ struct Workspace {
     Plan *plan;
     // dense path
     uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts
+    // batches of T <= nt <= 16 tokens: x as the gate MMA's token operand,
+    // [dp/64][nt][64] bf16 with the 16-byte blocks of row t permuted
+    // b -> b ^ (t & 7) (128-byte swizzle), rows t >= T and inputs past d zero;
+    // written by the router, streamed by the sparse kernel with the gate tiles
+    uint16_t *x_tiles;
     uint16_t *h_perm;   // [T*k + S*T][f] bf16: masked SwiGLU activations, routed then shared
     // host-pointer entry
     uint16_t *x_stage, *out_stage;

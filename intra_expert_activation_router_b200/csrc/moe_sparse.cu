@@ -137,7 +137,8 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     const size_t T = max_tokens, P = T * top_k;
     const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
                            4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * (P + T) * d_model +
-                           2 * (P + n_shared * T) * d_ff + 2 * 2 * T * d_model + 64 + 1024 + 32 * 256;
+                           2 * (P + n_shared * T) * d_ff + 2 * 2 * T * d_model + 32 * (size_t)dm.dp + 64 + 1024 +
+                           33 * 256;
     if (cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
     if (cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
 
@@ -179,9 +180,10 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.h_perm = (uint16_t *)sb.take(2 * (P + n_shared * T) * d_ff);
     ws.x_stage = (uint16_t *)sb.take(2 * T * d_model);
     ws.out_stage = (uint16_t *)sb.take(2 * T * d_model);
+    ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist) { free_handle(h); return MOE_ENOMEM; }
+    if (!h->stats_dev || !h->hist || !ws.x_tiles) { free_handle(h); return MOE_ENOMEM; }
 
     cudaStream_t st = nullptr;
     bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;

@@ -34,6 +34,8 @@ struct RouterArgs {
     const uint16_t *x, *wr;
     int T, d, E, k;
     int mt, n_chunks;   // sparse work items per expert: ceil(tokens / mt) * n_chunks
+    int dp;             // d rounded up to 128
+    int xtile;          // T <= xtile <= 16: also write x into ws.x_tiles with xtile rows; else 0
     Workspace ws;
 };
 
@@ -163,6 +165,17 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
             xs[r * 256 + v] = ld_cached(a.x + (size_t)(t0 + r) * a.d + c0 + v * 8);
         }
         __syncthreads();
+        if (a.xtile > 0 && blockIdx.x == 0) {   // the tile's rows of the swizzled token operand
+            for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
+                const int r = i / cv, v = i % cv, t = t0 + r;
+                if (t < a.xtile) {
+                    const int cc = c0 / 8 + v;   // 16-byte block of the row
+                    *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
+                                               (((cc & 7) ^ (t & 7)) << 3)) =
+                        r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
         if (e < a.E) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -173,6 +186,15 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
                         if (r < nt) acc[r] = dot8(wv[q], xs[r * 256 + v], acc[r]);
                 }
             }
+        }
+    }
+    if (a.xtile > 0 && blockIdx.x == 0) {   // inputs past d: zero
+        const int npad = (a.dp - a.d) / 8;
+        for (int i = threadIdx.x; i < kRtTok * npad; i += blockDim.x) {
+            const int r = i / npad, t = t0 + r, cc = a.d / 8 + i % npad;
+            if (t < a.xtile)
+                *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
+                                           (((cc & 7) ^ (t & 7)) << 3)) = make_uint4(0, 0, 0, 0);
         }
     }
 #pragma unroll
@@ -292,6 +314,8 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     a.k = dm.k;
     a.mt = tile_tokens;
     a.n_chunks = dm.n_blk;
+    a.dp = dm.dp;
+    a.xtile = (T <= tile_tokens && tile_tokens <= 16) ? tile_tokens : 0;
     a.ws = ws;
     dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
     const size_t P = (size_t)T * dm.k;
