@@ -173,7 +173,9 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * warps), up projection done, down projection and flush done; [32 + 4u] for
  * the gather of item u < 2: mask seen, then the issue times of its first
  * three batches; [40 + g] issue of gate stage g < 8; [48 + q] token rows of
- * tile q < 4 ready; [52], [53] the up warps' total time waiting for and
+ * tile q < 4 ready (batches of more than 16 tokens; smaller batches stream
+ * the token operand with the gate stages); [52], [53] the up warps' total
+ * time waiting for and
  * working on gathered batches, [54], [55] the same for the down warps (ns);
  * [56], [57] first gate stage consumed and accumulator committed for item 0;
  * [61] gathered records processed; [62] end; [63] the CTA's item count.
