@@ -175,6 +175,23 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(value, device=None):
+    """The largest of each rank's `value` over the default process group
+    (the value itself when there is none or it has one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank, seconds):
+    """Units all ranks processed per second of the slowest rank (weak scaling)."""
+    return world * units_per_rank / seconds
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -323,13 +340,9 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1000)
+    value = whole_job_rate(world, T * args.steps, total_ms / 1000)
     st = layer.stats()
     path = "sparse" if st["path"] == m.MOE_PATH_SPARSE else "dense"
     alg = st["alg_bytes"] if path == "sparse" else st["dense_bytes"]
@@ -353,12 +366,8 @@ def run_ours(args):
         t0 = time.perf_counter()
         m.moe_sparse_forward_host(layer.h, xh, T, tau, oh)
         e2e_t.append(time.perf_counter() - t0)
-    e2e_total = sum(e2e_t)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = world * T * e2e_steps / e2e_total
+    e2e_total = max_over_ranks(sum(e2e_t), dev)
+    e2e_value = whole_job_rate(world, T * e2e_steps, e2e_total)
 
     sweep = []
     if rank == 0 and sweep_T:
