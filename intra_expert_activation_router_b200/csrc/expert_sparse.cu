@@ -116,7 +116,7 @@ struct SparseArgs {
     int T, d, f, k, S;
     int dp, n_kb, n_blk, n_chunks;
     int nt;               // tokens per gate tile
-    int resident;         // T <= nt: the whole batch is the MMA's token operand, loaded once,
+    int resident;         // T <= nt: the whole batch is the MMA's token operand (x_tiles),
                           // and work items are claimed dynamically, heaviest expert first
     float tau;
     int use_mask;
