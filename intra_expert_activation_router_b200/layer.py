@@ -41,15 +41,25 @@ class MoESparseLayer:
         if x.dim() != 2 or x.shape[1] != self.d_model:
             raise ValueError(f"x must be [T][{self.d_model}]")
 
+    @staticmethod
+    def _out_like(x, out):
+        """`out`, or a new tensor like x; the library writes T x d_model bf16 values there."""
+        if out is None:
+            return torch.empty_like(x)
+        if (out.dtype != torch.bfloat16 or out.device != x.device or not out.is_contiguous()
+                or out.shape != x.shape):
+            raise ValueError(f"out must be a contiguous bf16 tensor of shape {tuple(x.shape)} on {x.device}")
+        return out
+
     def forward(self, x, tau: float, out=None, stream=None):
         self._check_x(x)
-        out = torch.empty_like(x) if out is None else out
+        out = self._out_like(x, out)
         B.moe_sparse_forward(self.h, x, x.shape[0], float(tau), out, stream)
         return out
 
     def dense_forward(self, x, out=None, stream=None):
         self._check_x(x)
-        out = torch.empty_like(x) if out is None else out
+        out = self._out_like(x, out)
         B.moe_dense_forward(self.h, x, x.shape[0], out, stream)
         return out
 
@@ -72,6 +82,7 @@ class MoESparseLayer:
         T = x.shape[0]
         idx = torch.empty((T, self.top_k, self.d_ff), dtype=torch.int16, device=x.device)
         cnt = torch.empty((T, self.top_k), dtype=torch.int32, device=x.device)
+        out = None if out is None else self._out_like(x, out)
         B.moe_debug_active(self.h, x, T, float(tau), idx, cnt, out, stream)
         return idx, cnt
 

@@ -219,6 +219,13 @@ def test_argument_errors_live_handle():
     with pytest.raises(m.MoeError) as ei:
         m.moe_set_path(layer.h, 7)
     assert ei.value.code == m.MOE_EINVAL
+    # the layer class rejects an output it cannot fill, before any launch
+    for bad in (torch.empty(3, sh.d_model, dtype=torch.bfloat16, device="cuda"),
+                torch.empty(4, sh.d_model, dtype=torch.float32, device="cuda"),
+                torch.empty(4, sh.d_model, dtype=torch.bfloat16),
+                torch.empty(sh.d_model, 4, dtype=torch.bfloat16, device="cuda").t()):
+        with pytest.raises(ValueError):
+            layer.forward(x, 1.0, out=bad)
     # the handle still works after the rejected calls
     layer.forward(x, 1.0)
     torch.cuda.synchronize()
