@@ -93,3 +93,16 @@ def test_create_without_gpu_reports_cuda_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _create(lib, _weights(lib)) == lib.MOE_ECUDA
+
+
+def test_layer_output_check_on_host(lib):
+    """The layer class checks `out` before any launch (CPU tensors stand in)."""
+    import torch
+    x = torch.zeros(4, 8, dtype=torch.bfloat16)
+    good = torch.empty_like(x)
+    assert lib.MoESparseLayer._out_like(x, good) is good
+    assert lib.MoESparseLayer._out_like(x, None).shape == x.shape
+    for bad in (torch.empty(3, 8, dtype=torch.bfloat16), torch.empty(4, 8, dtype=torch.float32),
+                torch.empty(8, 4, dtype=torch.bfloat16).t()):
+        with pytest.raises(ValueError):
+            lib.MoESparseLayer._out_like(x, bad)
