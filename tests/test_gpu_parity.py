@@ -86,6 +86,16 @@ def test_olmoe(o, T):
     run_case(o, "olmoe", T, 0.9)
 
 
+@pytest.mark.parametrize("name,T", [("tiny", 1), ("tiny", 2), ("tiny", 9), ("olmoe", 2), ("olmoe", 9),
+                                    ("olmoe", 17), ("olmoe", 33)])
+def test_tiling_boundaries(o, name, T):
+    """The kernel's (tokens per pass, 16-byte slices per thread) instantiations
+    not reached above, and the batch sizes where the token tiling changes:
+    one token tile up to 16 tokens, 8-token tiles from 17, 16-token tiles
+    again from 33."""
+    run_case(o, name, T, 0.9)
+
+
 @pytest.mark.parametrize("T", [1, 8, 32, 128])
 @pytest.mark.parametrize("q", [0.0, 0.5, 0.8, 0.9, 0.95])
 def test_dsv2lite(o, T, q):
