@@ -65,7 +65,7 @@ class Oracle:
         f.restype = ctypes.c_int
         f.argtypes = [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                       ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, ctypes.c_int,
-                      _P, _P, _P, _P, _P, _P]
+                      _P, _P, _P, _P, _P, _P, _P]
         c = self._lib.oracle_calibrate_tau
         c.restype = ctypes.c_double
         c.argtypes = [_P, ctypes.c_long, ctypes.c_double]
@@ -76,8 +76,13 @@ class Oracle:
 
     def forward(self, x, w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None,
                 ws_down=None, *, top_k: int, tau: float, want_scores: bool = True,
-                nthreads: int = 0) -> OracleResult:
-        """All weight/x arguments are uint16 numpy arrays of bf16 bits (x @ W layout)."""
+                nthreads: int = 0, active=None) -> OracleResult:
+        """All weight/x arguments are uint16 numpy arrays of bf16 bits (x @ W layout).
+
+        ``active``: optional [T][top_k][d_ff] mask (nonzero = active) that
+        replaces the threshold decision for each (token, rank) pair; ``tau``
+        is then unused.  It evaluates the layer under a given decision, e.g.
+        the CUDA path's for neurons whose score sits on the threshold."""
         arrs = [np.ascontiguousarray(a, dtype=np.uint16) if a is not None else None
                 for a in (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)]
         x, wr, wg, wu, wd, wsg, wsu, wsd = arrs
@@ -92,11 +97,16 @@ class Oracle:
         lg = np.zeros((T, E), np.float64)
         sc = np.zeros((T, k, f), np.float64) if want_scores else None
         ac = np.zeros((T, k, f), np.uint8) if want_scores else None
+        ain = None
+        if active is not None:
+            ain = np.ascontiguousarray(np.asarray(active) != 0, dtype=np.uint8)
+            if ain.shape != (T, k, f):
+                raise ValueError(f"active must be [{T}][{k}][{f}], got {ain.shape}")
         rc = self._lib.oracle_moe_forward(
             self._ptr(x), T, d, f, E, k, S, self._ptr(wr), self._ptr(wg), self._ptr(wu),
             self._ptr(wd), self._ptr(wsg), self._ptr(wsu), self._ptr(wsd),
             ctypes.c_float(tau), int(nthreads), self._ptr(y), self._ptr(idx), self._ptr(w),
-            self._ptr(lg), self._ptr(sc), self._ptr(ac))
+            self._ptr(lg), self._ptr(sc), self._ptr(ac), self._ptr(ain))
         if rc != 0:
             raise RuntimeError(f"oracle_moe_forward failed ({rc})")
         return OracleResult(y, idx, w, lg, sc, ac)

@@ -110,13 +110,19 @@ static void gate_up(const uint16_t *xt, int d, int f, const uint16_t *wg, const 
  *   logits     [T][E]   router logits
  *   score      [T][k][f] s = |silu(g)| of each selected pair
  *   active     [T][k][f] 1 where s >= tau (decided in float)
+ * Optional input:
+ *   active_in  [T][k][f] when not NULL, neuron j of the pair (t, rank r) is
+ *              active iff active_in[t][r][j] != 0, in place of the threshold
+ *              decision (tau is then unused).  This evaluates the layer under
+ *              a given mask, e.g. one whose neurons at the threshold went the
+ *              other way; `active` then echoes active_in.
  * Returns 0, or -1 on bad sizes / allocation failure. */
 int oracle_moe_forward(const uint16_t *x, int T, int d, int f, int E, int k, int S,
                        const uint16_t *wr, const uint16_t *wg, const uint16_t *wu,
                        const uint16_t *wd, const uint16_t *wsg, const uint16_t *wsu,
                        const uint16_t *wsd, float tau, int nthreads,
                        double *y, int *topk_idx, double *topk_w, double *logits,
-                       double *score, uint8_t *active)
+                       double *score, uint8_t *active, const uint8_t *active_in)
 {
     if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0 || k > E || S < 0) return -1;
     if (S > 0 && (!wsg || !wsu || !wsd)) return -1;
@@ -159,8 +165,9 @@ int oracle_moe_forward(const uint16_t *x, int T, int d, int f, int E, int k, int
                 for (int j = 0; j < f; ++j) {
                     double a = silu(g[j]);
                     double s = fabs(a);
-                    int on = ((float)s >= tau);
                     size_t o = ((size_t)t * k + r) * f + j;
+                    int on = ((float)s >= tau);
+                    if (active_in) on = (active_in[o] != 0);
                     if (score) score[o] = s;
                     if (active) active[o] = (uint8_t)on;
                     if (!on) continue;

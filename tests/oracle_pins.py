@@ -52,9 +52,9 @@ def _rand_layer(seed, d, E, f, k, S, T, scale_x=1.0):
     return x, W
 
 
-def _call(o, x, W, k, tau):
+def _call(o, x, W, k, tau, active=None):
     args = {n: _bits(t) for n, t in W.items()}
-    return o.forward(_bits(x), **args, top_k=k, tau=tau)
+    return o.forward(_bits(x), **args, top_k=k, tau=tau, active=active)
 
 
 def _torch_dense(x, W, k, with_routed=True, with_shared=True):
@@ -191,6 +191,54 @@ def pin_bruteforce(o):
     assert _rel(r.y, np.array(y)) < 1e-12, ("y", _rel(r.y, np.array(y)))
 
 
+def pin_mask_override(o):
+    """A given mask replaces the threshold: scalar-Python enumeration under an
+    arbitrary seeded mask (unrelated to any threshold), on a tiny layer."""
+    d, E, f, k, S, T = 16, 4, 8, 2, 1, 3
+    x, W = _rand_layer(33, d, E, f, k, S, T, scale_x=1.0)
+    X = x.float().double().tolist()
+    Wr = W["w_router"].double().tolist()
+    Wg, Wu, Wd = (W["w_gate"].double().tolist(), W["w_up"].double().tolist(),
+                  W["w_down"].double().tolist())
+    Sg, Su, Sd = (W["ws_gate"].double().tolist(), W["ws_up"].double().tolist(),
+                  W["ws_down"].double().tolist())
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    mask = (np.random.default_rng(34).random((T, k, f)) < 0.5).astype(np.uint8)
+    mask[0, 0, :] = 1          # one pair fully on, one fully off
+    mask[1, 1, :] = 0
+    y = [[0.0] * d for _ in range(T)]
+    want_score = np.zeros((T, k, f))
+    for t in range(T):
+        lg = [sum(X[t][i] * Wr[e][i] for i in range(d)) for e in range(E)]
+        m = max(lg)
+        ex = [math.exp(v - m) for v in lg]
+        p = [v / sum(ex) for v in ex]
+        chosen = sorted(range(E), key=lambda e: (-p[e], e))[:k]
+        for r_, e in enumerate(chosen):
+            for j in range(f):
+                g = sum(X[t][i] * Wg[e][i][j] for i in range(d))
+                u = sum(X[t][i] * Wu[e][i][j] for i in range(d))
+                want_score[t, r_, j] = abs(silu(g))
+                if mask[t, r_, j]:
+                    for i in range(d):
+                        y[t][i] += p[e] * silu(g) * u * Wd[e][j][i]
+        for s_ in range(S):
+            for j in range(f):
+                g = sum(X[t][i] * Sg[s_][i][j] for i in range(d))
+                u = sum(X[t][i] * Su[s_][i][j] for i in range(d))
+                for i in range(d):
+                    y[t][i] += silu(g) * u * Sd[s_][j][i]
+    # tau = 0 would keep every neuron and +inf none: the mask alone must decide
+    for tau in (0.0, math.inf):
+        r = _call(o, x, W, k, tau, active=mask)
+        assert np.array_equal(r.active, mask), ("active echo", tau)
+        assert np.allclose(r.score, want_score, rtol=1e-12, atol=1e-15), "scores"
+        assert _rel(r.y, np.array(y)) < 1e-12, ("y", tau, _rel(r.y, np.array(y)))
+
+
 def pin_nested_masks(o):
     """tau1 < tau2  =>  A(tau2) is a subset of A(tau1), for every pair."""
     x, W = _rand_layer(41, d=64, E=8, f=64, k=2, S=1, T=6)
@@ -262,7 +310,8 @@ def pin_calibration(o):
 
 
 ALL_PINS = [pin_handworked, pin_tau0_is_dense, pin_tauinf_is_shared_only, pin_bruteforce,
-            pin_nested_masks, pin_threshold_decomposition, pin_router_ranking, pin_calibration]
+            pin_mask_override, pin_nested_masks, pin_threshold_decomposition, pin_router_ranking,
+            pin_calibration]
 
 
 def run_all(o):

@@ -33,6 +33,8 @@ MUTANTS = [
     ("calibration_off_by_one", "double tau = c[m];", "double tau = c[m > 0 ? m - 1 : 0];"),
     ("up_from_gate", "for (int j = 0; j < f; ++j) u[j] += xi * bf16_to_double(ru[j]);",
      "for (int j = 0; j < f; ++j) u[j] += xi * bf16_to_double(rg[j]);"),
+    ("mask_input_ignored", "if (active_in) on = (active_in[o] != 0);", ";"),
+    ("mask_input_inverted", "if (active_in) on = (active_in[o] != 0);", "if (active_in) on = (active_in[o] == 0);"),
     ("shared_weighted", "for (int i = 0; i < d; ++i) yt[i] += h * bf16_to_double(down[(size_t)j * d + i]);",
      "for (int i = 0; i < d; ++i) yt[i] += 0.5 * h * bf16_to_double(down[(size_t)j * d + i]);"),
 ]
