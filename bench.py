@@ -2,7 +2,7 @@
 """Benchmark of the routed-expert MoE layer with intra-expert activation sparsity.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload olmoe] [--T 16] [--sparsity 0.9] [--no-sweep]
+                    [--workload olmoe] [--T 16] [--sparsity 0.9] [--sweep full|quick|none]
 
 One step is one forward of the whole layer (router + bucketing, gate
 projection, threshold mask and compaction, gathered up/down projection,
@@ -16,8 +16,16 @@ Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
 replica of the layer on its own GPU ("replicas only": the layer has no
 exchange step); the step time is the max over ranks.
 
+The JSON line's ``sweep`` holds one row per (workload, batch size, sparsity):
+the sparse path, the dense path and AUTO each timed the same way, with the
+expert kernel's roofline fraction and AUTO's choice.  It covers the tiny
+layer, the OLMoE-shaped layer at T = 1, 4, 16, 64, the DeepSeek-V2-Lite-shaped
+layer at T = 1, 8, 32, 128 and sparsity 0/50/80/90/95 %, the large layer at
+T = 1, 16, 64 and a 2 % keep rate, and the crossover sweep T = 1 ... 4096.
+
 ``--impl reference`` times the CPU oracle (the plain fp64 definition of the
-layer) on the host cores instead -- rank 0 only.
+layer) on the host cores instead -- rank 0 only -- on the same inputs (drawn
+on the GPU when there is one, as the GPU arm does, then copied to the host).
 """
 from __future__ import annotations
 
@@ -62,7 +70,8 @@ def parse():
     p.add_argument("--T", type=int, default=16)
     p.add_argument("--sparsity", type=float, default=0.9)
     p.add_argument("--path", choices=["auto", "sparse", "dense"], default="auto")
-    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--sweep", choices=["full", "quick", "none"], default="full")
+    p.add_argument("--no-sweep", action="store_true", help="same as --sweep none")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     return p.parse_args()
@@ -199,18 +208,35 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def oracle_time_sample(shape, W_host, x_host, T, target_s, nthreads):
-    """The CPU oracle on repeats of the batch for about target_s seconds (rank 0, N=1)."""
+def bench_config(args, world):
+    """The workload description both arms print (identical dicts)."""
+    return {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": args.T,
+            "sparsity": args.sparsity, "parallelism": f"replicas{world}",
+            "l2": "flushed before every timed step (2x L2 written, then read back, outside the step events)"}
+
+
+def draw_inputs(shape, T, device):
+    """The workload's weights and batch, drawn on `device` from the seeded
+    generators (the GPU arm draws on its GPU; the reference arm draws the
+    same values there too when a GPU is present, then copies them)."""
+    import moe_inputs as mi
+    return mi.make_weights(shape, device=device), mi.make_x(shape, T, device=device)
+
+
+def oracle_time_sample(shape, W_host, x_host, tau, target_s, nthreads):
+    """The CPU oracle at threshold tau on repeats of the batch for about
+    target_s seconds (rank 0, N = 1).  Returns (tokens/s, repeats, seconds)."""
     import oracle
     o = oracle.Oracle()
     inputs = oracle.layer_inputs(W_host, x_host)
+    T = x_host.shape[0]
     t0 = time.perf_counter()
-    o.forward(**inputs, top_k=shape.top_k, tau=1.0, want_scores=False, nthreads=nthreads)
+    o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=nthreads)
     one = time.perf_counter() - t0
     reps = max(1, min(500, int(math.ceil(target_s / max(one, 1e-6)))))
     t0 = time.perf_counter()
     for _ in range(reps):
-        o.forward(**inputs, top_k=shape.top_k, tau=1.0, want_scores=False, nthreads=nthreads)
+        o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=nthreads)
     el = time.perf_counter() - t0
     return reps * T / el, reps, el
 
@@ -223,8 +249,9 @@ def run_reference(args):
     import moe_inputs as mi
     import oracle
     shape = mi.SHAPES[args.workload]
-    W = mi.make_weights(shape, device="cpu")
-    x = mi.make_x(shape, args.T, device="cpu")
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    W, x = draw_inputs(shape, args.T, gen_dev)
+    W, x = W.to("cpu"), x.cpu()
     o = oracle.Oracle()
     inputs = oracle.layer_inputs(W, x)
     cores = cpu_cores()
@@ -249,14 +276,13 @@ def run_reference(args):
         times.append(time.perf_counter() - t0)
     ms = 1000 * statistics.mean(times)
     value = n_tok / (ms / 1000)
-    sample = f"{n_tok} of the {args.T} tokens per step, {args.steps} steps"
+    sample = (f"{n_tok} of the {args.T} tokens per step, {args.steps} steps; inputs drawn on "
+              f"{'the GPU' if gen_dev == 'cuda' else 'the CPU'} and copied to the host")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": args.T,
-                   "sparsity": args.sparsity, "tau": tau},
+        "data": "synthetic", "config": bench_config(args, world), "tau": tau,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -301,6 +327,74 @@ def time_steps(layer, x, tau, out, flush, steps, events=True, dense=False):
     return step_ms, router_ms, expert_ms
 
 
+# (workload, batch sizes, sparsities) of the sweep; "quick" keeps one point per workload
+SWEEP_FULL = [
+    ("tiny", (16,), (0.9,)),
+    ("olmoe", (1, 4, 16, 64), (0.9,)),
+    ("dsv2lite", (1, 8, 32, 128), (0.0, 0.5, 0.8, 0.9, 0.95)),
+    ("large", (1, 16, 64), (0.98,)),
+    ("crossover", (1, 2, 4, 8, 16, 24, 32, 48, 64, 128, 256, 512, 1024, 2048, 4096), (0.9,)),
+]
+SWEEP_QUICK = [("tiny", (16,), (0.9,)), ("olmoe", (1, 16), (0.9,)), ("dsv2lite", (8,), (0.9,)),
+               ("large", (1,), (0.98,))]
+
+
+def sweep_rows(dev, kind, peak, flush, steps=20):
+    """One row per (workload, T, sparsity): sparse, dense and AUTO timed alike."""
+    import torch
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    rows = []
+    plan = SWEEP_FULL if kind == "full" else SWEEP_QUICK
+    for name, Ts, qs in plan:
+        shape = mi.SHAPES[name]
+        W = mi.make_weights(shape, device=dev)
+        layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max(Ts))
+        del W
+        for T in Ts:
+            x = mi.make_x(shape, T, device=dev)
+            out = torch.empty_like(x)
+            for q in qs:
+                tau = layer.calibrate_tau(x, q)
+                row = {"workload": name, "T": T, "sparsity": q, "tau": tau}
+                for mode, path in (("sparse", m.MOE_PATH_SPARSE), ("dense", m.MOE_PATH_DENSE),
+                                   ("auto", m.MOE_PATH_AUTO)):
+                    try:
+                        layer.set_path(path)
+                    except m.MoeError:
+                        row[f"{mode}_us"] = None
+                        continue
+                    for _ in range(3):
+                        layer.forward(x, tau, out=out)
+                    sm_, rm_, em_ = time_steps(layer, x, tau, out, flush, steps)
+                    st = layer.stats()
+                    used = "sparse" if st["path"] == m.MOE_PATH_SPARSE else "dense"
+                    b = st["alg_bytes"] if used == "sparse" else st["dense_bytes"]
+                    us = 1000 * statistics.mean(sm_)
+                    kus = 1000 * statistics.mean(em_)
+                    kb = b - shape.n_experts * shape.d_model * 2 - T * shape.d_model * 2
+                    row[f"{mode}_us"] = us
+                    row[f"{mode}_tokens_per_s"] = T / (us * 1e-6)
+                    if mode == "auto":
+                        row["auto_path"] = used
+                        continue
+                    row[f"{mode}_kernels_us"] = kus
+                    row[f"{mode}_alg_bytes"] = b
+                    row[f"{mode}_gbs"] = b / (us * 1e-6) / 1e9
+                    row[f"{mode}_kernel_frac"] = kb / (kus * 1e-6) / 1e9 / peak
+                    if mode == "sparse":
+                        row["n_active"], row["n_union"], row["n_touched"] = (
+                            st["n_active"], st["n_union"], st["n_touched"])
+                best = min(v for v in (row.get("sparse_us"), row.get("dense_us")) if v is not None)
+                row["auto_over_best"] = row["auto_us"] / best
+                layer.set_path(m.MOE_PATH_AUTO)
+                rows.append(row)
+                log(json.dumps({k: (round(v, 2) if isinstance(v, float) else v) for k, v in row.items()}))
+        layer.close()
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -317,13 +411,11 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     shape = mi.SHAPES[args.workload]
     T = args.T
-    sweep_T = [] if args.no_sweep or world > 1 else [t for t in shape.t_values]
-    max_tokens = max([T] + sweep_T + [64])
-    W = mi.make_weights(shape, device=dev)
-    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max_tokens)
+    sweep_kind = "none" if args.no_sweep or world > 1 else args.sweep
+    W, x = draw_inputs(shape, T, dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max(T, 64))
     if args.path != "auto":
         layer.set_path({"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
-    x = mi.make_x(shape, T, device=dev)
     out = torch.empty_like(x)
     tau = layer.calibrate_tau(x, args.sparsity)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -368,41 +460,21 @@ def run_ours(args):
         e2e_t.append(time.perf_counter() - t0)
     e2e_total = max_over_ranks(sum(e2e_t), dev)
     e2e_value = whole_job_rate(world, T * e2e_steps, e2e_total)
+    layer.close()
 
-    sweep = []
-    if rank == 0 and sweep_T:
-        for Ts in sweep_T:
-            xs = mi.make_x(shape, Ts, device=dev)
-            outs = torch.empty_like(xs)
-            taus = layer.calibrate_tau(xs, args.sparsity)
-            row = {"T": Ts, "tau": taus}
-            for mode in ("sparse", "dense"):
-                try:
-                    layer.set_path(m.MOE_PATH_SPARSE if mode == "sparse" else m.MOE_PATH_DENSE)
-                except m.MoeError:
-                    row[f"{mode}_us"] = None
-                    continue
-                for _ in range(3):
-                    layer.forward(xs, taus, out=outs)
-                sm_, rm_, em_ = time_steps(layer, xs, taus, outs, flush, 30)
-                s2 = layer.stats()
-                b = s2["alg_bytes"] if mode == "sparse" else s2["dense_bytes"]
-                row[f"{mode}_us"] = 1000 * statistics.mean(sm_)
-                row[f"{mode}_expert_us"] = 1000 * statistics.mean(em_)
-                row[f"{mode}_alg_bytes"] = b
-                row[f"{mode}_gbs"] = b / (statistics.mean(sm_) / 1000) / 1e9
-            layer.set_path(m.MOE_PATH_AUTO if args.path == "auto" else
-                           {"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
-            sweep.append(row)
+    sweep = sweep_rows(dev, sweep_kind, peak, flush) if rank == 0 and sweep_kind != "none" else []
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = cpu_cores()
-        W_host = W.to("cpu")
-        tps, reps, el = oracle_time_sample(shape, W_host, x.cpu(), T, args.cpu_seconds, cores)
+        W_host, x_host = W.to("cpu"), x.cpu()
+        tps, reps, el = oracle_time_sample(shape, W_host, x_host, tau, args.cpu_seconds, cores)
+        tps1, reps1, el1 = oracle_time_sample(shape, W_host, x_host[:4], tau, args.cpu_seconds / 2, 1)
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{reps} repeats of the {T}-token batch ({el:.1f} s, fp64 oracle, "
-                         f"OpenMP over tokens)"}
+               "sample": f"{reps} repeats of the {T}-token batch ({el:.1f} s, fp64 oracle at the bench's "
+                         f"tau, OpenMP over tokens on {cores} threads)",
+               "single_thread": {"value": tps1, "unit": "tokens/s", "cores": 1,
+                                 "sample": f"{reps1} repeats of the batch's first 4 tokens ({el1:.1f} s)"}}
 
     if rank == 0:
         clocks = clk.summary()
@@ -410,11 +482,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": T,
-                       "sparsity": args.sparsity, "tau": tau, "path": path,
-                       "parallelism": f"replicas{world}",
-                       "l2": "flushed before every timed step (2x L2 written, then read back, outside the step events)"},
+            "data": "synthetic", "config": bench_config(args, world), "tau": tau, "path": path,
             "hbm_gbs": alg / (ms / 1000) / 1e9,
             "latency_us": 1000 * ms,
             "alg_bytes_per_step": alg,
@@ -422,7 +490,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         if peak_kind == "measured" else "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)",
                          "alg_bytes_per_launch": expert_bytes},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * shape.d_model * 2,
@@ -436,7 +504,6 @@ def run_ours(args):
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         torch.distributed.destroy_process_group()
 

@@ -45,8 +45,11 @@ extern "C" {
 #define MOE_ECUDA (-3)    /* a CUDA runtime call or kernel launch failed     */
 #define MOE_EALIGN (-4)   /* a pointer is not 16-byte aligned                */
 #define MOE_EHANDLE (-5)  /* NULL or destroyed handle                        */
-#define MOE_EDEVICE (-6)  /* a kernel reported an error word (e.g. a bounded
-                             wait ran out); the handle stays usable           */
+#define MOE_EDEVICE (-6)  /* a kernel reported an error (e.g. a bounded wait
+                             ran out); read by moe_query_stats.  The forward
+                             in which it happened produced wrong output;
+                             later forwards start with a clear error state
+                             and are unaffected                              */
 #define MOE_ENOTSUP (-7)  /* shape or path not supported by this build       */
 
 /* Path selection (moe_set_path). */
@@ -184,9 +187,29 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
 int moe_set_trace(moe_handle h, void *buf, long long bytes);
 
 /* Statistics of the last forward.  Synchronises the stream of that forward
- * and reads device counters back; not for timed loops.  A nonzero device
- * error word is reported in st->device_error and as MOE_EDEVICE. */
+ * and reads device counters back; not for timed loops.
+ * Device errors: forward calls do not synchronise, so they cannot report
+ * what their kernels find (a bounded wait that ran out, error codes >= 30).
+ * Each forward starts with a clear error state, so an error affects only the
+ * forward it happened in (whose output is then wrong).  This call reports
+ * the FIRST device error code since its previous call in st->device_error,
+ * returns MOE_EDEVICE for it, and clears it; 0 / MOE_OK when there was none. */
 int moe_query_stats(moe_handle h, moe_stats *st);
+
+/* Test-only fault injection (no GPU fault, trap or hang is involved).
+ * MOE_INJECT_WITHHOLD_ITEMS: in the next sparse-path forward the expert
+ * kernel's gate lane publishes no work item and issues no copy, so the other
+ * agents' bounded waits for work run out (after about 10 ms); the kernel
+ * records error code 50 and returns, that forward's output is wrong (zero),
+ * and moe_query_stats then returns MOE_EDEVICE.  Applies once.
+ * MOE_INJECT_NONE cancels a pending injection.
+ * Separately, when the environment variable MOE_INJECT_ALLOC_FAIL is
+ * "weights" or "workspace", moe_sparse_create treats that device allocation
+ * as failed (MOE_ENOMEM, nothing leaked); "scores" does the same for the
+ * first moe_calibrate_tau's score buffer. */
+#define MOE_INJECT_NONE 0
+#define MOE_INJECT_WITHHOLD_ITEMS 1
+int moe_debug_inject(moe_handle h, int kind);
 
 /* Size of the fixed device scratch used by moe_router_topk_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (4 << 20)
@@ -209,7 +232,12 @@ int moe_query_stats(moe_handle h, moe_stats *st);
  * before anything is launched (e.g. E = 64 allows T up to 16352).  Other limits as moe_sparse_create: 1 <= top_k <= E
  * <= 1024, d_model % 8 == 0.  The first call on a device looks up the array's
  * device address with that device current, so make it before any stream
- * capture.  All calls share the array: calls that overlap on the GPU (on
+ * capture.  Under CUDA's lazy module loading (the default) that first call is
+ * also when the library's device code and this array are loaded onto the
+ * device, which needs MOE_NOALLOC_SCRATCH_BYTES plus the code of free device
+ * memory: a caller whose own arena takes all device memory should make one
+ * call at initialisation, before reserving it (or load modules eagerly with
+ * CUDA_MODULE_LOADING=EAGER), after which calls need no free memory.  All calls share the array: calls that overlap on the GPU (on
  * different streams) race and must be serialised by the caller.  Each call
  * clears the tickets it needs with cudaMemsetAsync and calls no allocating
  * routine.  Asynchronous on `stream`. */

@@ -25,6 +25,9 @@ MOE_EHANDLE = -5
 MOE_EDEVICE = -6
 MOE_ENOTSUP = -7
 
+MOE_INJECT_NONE = 0
+MOE_INJECT_WITHHOLD_ITEMS = 1
+
 MOE_PATH_AUTO = 0
 MOE_PATH_SPARSE = 1
 MOE_PATH_DENSE = 2
@@ -74,6 +77,7 @@ def _load():
         "moe_set_launch_events": (I, [P, ctypes.POINTER(P), I]),
         "moe_set_trace": (I, [P, P, ctypes.c_longlong]),
         "moe_router_topk_noalloc": (I, [P, I, P, I, I, I, P, P, P]),
+        "moe_debug_inject": (I, [P, I]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -87,7 +91,8 @@ _lib = _load()
 EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_sparse_forward_host", "moe_sparse_destroy", "moe_set_path", "moe_set_t_star",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
-            "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc")
+            "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
+            "moe_debug_inject")
 
 
 def _addr(t):
@@ -210,6 +215,11 @@ def moe_router_topk_noalloc(x, T: int, w_router, E: int, d_model: int, top_k: in
     """Router softmax top-k without a handle or any allocation (fixed device scratch)."""
     _check(_lib.moe_router_topk_noalloc(_addr(x), T, _addr(w_router), E, d_model, top_k, _addr(idx_out),
                                         _addr(w_out), _stream(stream)), "moe_router_topk_noalloc")
+
+
+def moe_debug_inject(h, kind: int):
+    """Test-only fault for the next sparse forward (MOE_INJECT_*)."""
+    _check(_lib.moe_debug_inject(h, kind), "moe_debug_inject")
 
 
 def raw_call(name: str, *args) -> int:

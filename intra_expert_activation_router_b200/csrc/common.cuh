@@ -28,6 +28,9 @@ __device__ __forceinline__ uint4 ld_cached(const void *p)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// One bf16 (its 16 bits) -> float.  Exact widening.
+__device__ __forceinline__ float bf16_f(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
 {
     f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);

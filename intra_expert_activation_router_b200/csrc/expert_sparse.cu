@@ -55,8 +55,6 @@
 //                          to bf16 into `out` and re-zeroes it.
 // The agents meet on mbarriers (copies, MMA completion, buffer and h hand-off)
 // and on monotonic progress counters in shared memory; every wait is bounded.
-#include <cuda_fp16.h>
-
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -105,7 +103,7 @@ struct ItemMeta {
     unsigned word[kMaxNT][4];     // mask words: token, 32-neuron quarter of the block
     int n_uni[kMaxSub];
     uint8_t uni[kMaxSub][kBlk];   // per pass: union-active neurons of the block, ascending
-    __half a[kMaxNT][kBlk];       // silu(g)
+    uint16_t a[kMaxNT][kBlk];     // silu(g) as bf16 (RNE): fp32's range, relative error <= 2^-9
 };
 
 struct SparseArgs {
@@ -124,6 +122,7 @@ struct SparseArgs {
     int n_shared_items;   // S * n_tok_tiles * n_blk
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f], no up/down
+    int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
     SparseLayout L;
 };
 
@@ -478,7 +477,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         // publishes the work-item ids (claimed from the plan's counter in
         // resident mode, else the CTA's static range), then streams each
         // item's gate tiles into the ring
-        if (lane == 0) {
+        if (lane == 0 && a.inject != 1) {
             const uint64_t pol = policy_evict_first();
             uint32_t g = 0;
             int next = a.resident ? atomicAdd(&plan->next_item, 1) : 0;
@@ -699,7 +698,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const float av = silu_f(tmem_ld1(taddr + col));
                     const bool on = jv && (!masked || fabsf(av) >= a.tau);
                     const unsigned word = __ballot_sync(kFull, on);
-                    M.a[t][jl] = __float2half_rn(av);
+                    M.a[t][jl] = f2bf_bits(av);
                     if (lane == 0) M.word[t][warp] = word;
                     if (score_mode && jv) a.score_out[(size_t)M.pair[t] * a.f + j] = fabsf(av);
                 }
@@ -794,7 +793,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                             for (int w4 = 0; w4 < 4; ++w4) u += part[((hb * 4 + w4) * kMaxGB + q) * MT + r];
                             const int jl = M.uni[s][b0 + q];
                             const bool bit = (r < ms) && ((M.word[r0 + r][jl >> 5] >> (jl & 31)) & 1u);
-                            hs[(hb * kMaxGB + q) * MT + r] = bit ? __half2float(M.a[r0 + r][jl]) * u : 0.f;
+                            hs[(hb * kMaxGB + q) * MT + r] = bit ? bf16_f(M.a[r0 + r][jl]) * u : 0.f;
                         }
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&hsfull[hb]);
@@ -1048,7 +1047,7 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out)
+                                 float *score_out, int inject)
 {
     SparseArgs a;
     a.x = x;
@@ -1069,6 +1068,7 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.tau = tau;
     a.use_mask = use_mask ? 1 : 0;
     a.score_out = score_out;
+    a.inject = inject;
     a.n_tok_tiles = (T + til.nt - 1) / til.nt;
     a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
     const int pairs = T * dm.k;

@@ -98,7 +98,14 @@ struct Workspace {
     int *tok_cnt;
     int *tile_ticket;   // one per router token tile, kept zero between calls
     int *done_ticket;   // one, kept zero between calls
-    int *error_word;    // nonzero once a kernel reports an error
+    // device errors (a bounded wait that ran out, ...): kernels of a forward
+    // record their first code in error_word, which the router -- the first
+    // kernel of every forward, running after all earlier kernels -- folds
+    // into error_sticky and clears, so one forward's error never cuts short a
+    // later forward; error_sticky keeps the first code until moe_query_stats
+    // reads and clears it
+    int *error_word;
+    int *error_sticky;
     Plan *plan;
     // dense path
     uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts
@@ -128,10 +135,12 @@ __device__ __forceinline__ unsigned long long global_ns()
 // tokens, 128-neuron block).
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                           const uint16_t *x, int T, int tile_tokens, cudaStream_t st);
+// inject: test-only fault (MOE_INJECT_WITHHOLD_ITEMS: the gate lane publishes
+// no work item, so the consumers' bounded waits run out), 0 otherwise.
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out = nullptr);
+                                 float *score_out = nullptr, int inject = 0);
 // dst[b][c][col_off + r] = src[b][r][c] with row stride ld (elements).
 cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
                                     int ld, int col_off, cudaStream_t st);

@@ -53,9 +53,19 @@ struct moe_sparse_s {
     int n_ev;
     float *scores;       // calibration buffer, allocated by the first moe_calibrate_tau
     unsigned *hist;      // 256 bins, inside the workspace
+    int inject_next;     // test-only fault for the next sparse forward (moe_debug_inject)
 };
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Host-side fault injection for tests: MOE_INJECT_ALLOC_FAIL=<what> makes the
+// named device allocation ("weights", "workspace" or "scores") report failure
+// without being attempted, so the error paths can be exercised on a live GPU.
+static bool inject_alloc_fail(const char *what)
+{
+    const char *v = std::getenv("MOE_INJECT_ALLOC_FAIL");
+    return v && std::strcmp(v, what) == 0;
+}
 
 // Live handles, so that a NULL, foreign or destroyed handle is an error code
 // rather than a dereference of freed memory.
@@ -138,9 +148,19 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
                            4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * (P + T) * d_model +
                            2 * (P + n_shared * T) * d_ff + 2 * 2 * T * d_model + 32 * (size_t)dm.dp + 64 + 1024 +
-                           33 * 256;
-    if (cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
-    if (cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) { cudaGetLastError(); free_handle(h); return MOE_ENOMEM; }
+                           64 + 40 * 256;
+    if (inject_alloc_fail("weights") || cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) {
+        cudaGetLastError();
+        h->weight_mem = nullptr;
+        free_handle(h);
+        return MOE_ENOMEM;
+    }
+    if (inject_alloc_fail("workspace") || cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) {
+        cudaGetLastError();
+        h->ws_mem = nullptr;
+        free_handle(h);
+        return MOE_ENOMEM;
+    }
 
     Block wb{(char *)h->weight_mem, 0, wbytes};
     uint16_t *wr = (uint16_t *)wb.take(2 * (size_t)E * d_model);
@@ -175,6 +195,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.tile_ticket = (int *)sb.take(4 * ((T + 7) / 8));
     ws.done_ticket = (int *)sb.take(4);
     ws.error_word = (int *)sb.take(4);
+    ws.error_sticky = (int *)sb.take(4);
     ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
     ws.x_perm = (uint16_t *)sb.take(2 * (P + T) * d_model);
     ws.h_perm = (uint16_t *)sb.take(2 * (P + n_shared * T) * d_ff);
@@ -183,7 +204,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist || !ws.x_tiles) { free_handle(h); return MOE_ENOMEM; }
+    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky) { free_handle(h); return MOE_ENOMEM; }
 
     cudaStream_t st = nullptr;
     bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
@@ -257,7 +278,9 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
         if (e == cudaSuccess)
-            e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st);
+            e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
+                                          h->inject_next);
+        h->inject_next = 0;
     } else {
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
@@ -358,7 +381,11 @@ extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double spar
     if (kq >= (double)n) { *tau_out = INFINITY; return MOE_OK; }
     if (!h->scores) {
         const size_t cap = (size_t)dm.max_tokens * dm.k * dm.f * sizeof(float);
-        if (cudaMalloc(&h->scores, cap) != cudaSuccess) { cudaGetLastError(); h->scores = nullptr; return MOE_ENOMEM; }
+        if (inject_alloc_fail("scores") || cudaMalloc(&h->scores, cap) != cudaSuccess) {
+            cudaGetLastError();
+            h->scores = nullptr;
+            return MOE_ENOMEM;
+        }
     }
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
@@ -433,8 +460,17 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
     st->n_tokens = h->last_T;
     st->t_star = h->t_star;
     if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
-    int err = 0;
-    if (cudaMemcpy(&err, h->ws.error_word, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
+    // the first error code since the previous call: an earlier forward's (kept
+    // in the sticky word by the router of the next forward), else the last
+    // forward's own; both are cleared
+    int words[2] = {0, 0};
+    if (cudaMemcpy(&words[0], h->ws.error_sticky, 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(&words[1], h->ws.error_word, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ECUDA;
+    const int err = words[0] != 0 ? words[0] : words[1];
+    if (err != 0 && (cudaMemset(h->ws.error_sticky, 0, 4) != cudaSuccess ||
+                     cudaMemset(h->ws.error_word, 0, 4) != cudaSuccess))
+        return MOE_ECUDA;
     st->device_error = err;
     if (h->last_T > 0) {
         unsigned long long v[3] = {0, 0, 0};
@@ -452,6 +488,14 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
         st->dense_bytes = st->n_touched * 3.0 * d * f * 2 + fixed;
     }
     return err ? MOE_EDEVICE : MOE_OK;
+}
+
+extern "C" int moe_debug_inject(moe_handle h, int kind)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (kind != MOE_INJECT_NONE && kind != MOE_INJECT_WITHHOLD_ITEMS) return MOE_EINVAL;
+    h->inject_next = kind;
+    return MOE_OK;
 }
 
 extern "C" const char *moe_strerror(int code)

@@ -137,6 +137,15 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
 
     // let the expert kernel launch now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;");
+    // every kernel of earlier calls has finished: keep their error code and
+    // give this forward a clear error word (read only after this grid ends)
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        const int e0 = *a.ws.error_word;
+        if (e0 != 0) {
+            atomicCAS(a.ws.error_sticky, 0, e0);
+            *a.ws.error_word = 0;
+        }
+    }
     const int cta = blockIdx.y * gridDim.x + blockIdx.x;
     unsigned long long *tr = (a.ws.trace_router && cta < a.ws.trace_router_ctas) ? a.ws.trace_router + cta * 8 : nullptr;
     if (tr && threadIdx.x == 0) tr[0] = global_ns();

@@ -32,7 +32,7 @@ def test_reference_line_contract():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
-    assert d["config"]["T"] == 16 and d["config"]["tau"] > 0
+    assert d["config"]["T"] == 16 and d["tau"] > 0
 
 
 def test_reference_other_ranks_exit_without_work():

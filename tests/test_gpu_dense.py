@@ -3,9 +3,10 @@ and against the sparse branch, through the C ABI.
 
 The dense branch rounds h to bf16 before the down projection, so outputs are
 compared at the layer's 1e-2 relative-L2 bar.  Its mask is decided on
-tensor-core fp32 gate values; a token is exempt from the output check only
-if one of its neurons scores within 1e-5*tau of tau (where fp32 accumulation
-order may decide either way) or its router is a near tie.
+tensor-core fp32 gate values, where a neuron scoring within 1e-5*tau of tau
+may go either way; such a token must match the oracle under one of the
+decisions of its band neurons (every combination is evaluated).  Only
+near-tie router tokens are left out of the output check.
 """
 
 import numpy as np
@@ -17,6 +18,11 @@ import oracle
 from tests import parity_util as pu
 
 pytestmark = pytest.mark.gpu
+
+# the dense branch's mask is decided on tensor-core fp32 gate values (sums of
+# 2048 to 4096 products in a different order from the oracle's fp64 sums):
+# neurons this close to tau may go either way
+DENSE_BAND_REL = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -62,11 +68,11 @@ def run_dense(o, name, T, q, sample=None, masked=True):
     sub = dict(inputs)
     sub["x"] = inputs["x"][rows]
     ref = o.forward(**sub, top_k=sh.top_k, tau=tau)
-    exempt = pu.near_tie_tokens(ref.logits, sh.top_k)
-    if masked and tau > 0:
-        exempt |= np.any(np.abs(ref.score - tau) <= 1e-5 * tau, axis=(1, 2))
-    assert exempt.sum() <= max(2, len(rows) // 20)
-    pu.check_output(ref.y, out[torch.as_tensor(rows, device="cuda")], exempt)
+    tie = pu.near_tie_tokens(ref.logits, sh.top_k)
+    assert tie.sum() <= max(1, len(rows) // 50)
+    band = DENSE_BAND_REL if masked and 0 < tau < np.inf else 0.0
+    pu.check_output_any_band_decision(o, sub, sh.top_k, tau, ref, out[torch.as_tensor(rows, device="cuda")],
+                                      tie, band)
     return layer, x, tau, out
 
 

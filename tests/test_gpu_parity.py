@@ -58,7 +58,8 @@ def run_case(o, name, T, q, sample=None, check_lists=True):
     out = layer.forward(x, tau)
     layer.set_path(m.MOE_PATH_AUTO)
     idx, w = layer.router(x)
-    lists, cnt = layer.active_lists(x, tau) if check_lists else (None, None)
+    out_dbg = torch.empty_like(x)
+    lists, cnt = layer.active_lists(x, tau, out=out_dbg) if check_lists else (None, None)
     torch.cuda.synchronize()
     rows = np.arange(T) if sample is None else np.sort(
         np.random.default_rng(1000 * T + int(q * 100)).choice(T, size=min(sample, T), replace=False))
@@ -66,11 +67,17 @@ def run_case(o, name, T, q, sample=None, check_lists=True):
     sub["x"] = inputs["x"][rows]
     ref = o.forward(**sub, top_k=sh.top_k, tau=tau, nthreads=NTHREADS, want_scores=check_lists)
     tie = pu.check_router(ref, idx.cpu().numpy()[rows], w.cpu().numpy()[rows], sh.top_k)
+    y_expect = ref.y
     flipped = np.zeros(len(rows), bool)
+    trows = torch.as_tensor(rows, device="cuda")
     if check_lists:
-        flipped, _ = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16)[rows],
-                                     cnt.cpu().numpy()[rows], tie)
-    worst = pu.check_output(ref.y, out[torch.as_tensor(rows, device="cuda")], tie | flipped)
+        flipped, _, gmask = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16)[rows],
+                                            cnt.cpu().numpy()[rows], tie)
+        # a token whose threshold-band neuron the GPU decided the other way is
+        # checked against the oracle under the GPU's mask, not dropped
+        y_expect = pu.expected_under_gpu_mask(o, sub, sh.top_k, tau, ref, gmask, flipped, tie, NTHREADS)
+        pu.check_output(y_expect, out_dbg[trows], tie)
+    worst = pu.check_output(y_expect, out[trows], tie)
     assert tie.sum() <= max(1, len(rows) // 50), "too many near-tie tokens"
     assert flipped.sum() <= max(2, len(rows) // 20), "too many band flips"
     return tau, worst, layer
@@ -110,6 +117,68 @@ def test_large(o, T):
 @pytest.mark.parametrize("T", [3, 13, 100, 257, 1000, 4096])
 def test_crossover_sparse_sampled(o, T):
     run_case(o, "crossover", T, 0.9, sample=None if T <= 13 else 12, check_lists=T <= 1000)
+
+
+@pytest.mark.parametrize("name,T,qs", [
+    ("tiny", 16, (0.5, 0.9, 0.98)),
+    ("olmoe", 16, (0.5, 0.9, 0.98)),
+    ("dsv2lite", 8, (0.5, 0.8, 0.9, 0.95)),
+    ("large", 1, (0.98,)),
+])
+def test_calibrate_tau_matches_oracle(o, name, T, qs):
+    """The library's on-GPU threshold (an exact radix select over its fp32
+    scores) against the oracle's order statistic of its fp64 scores."""
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=math.inf, nthreads=NTHREADS)
+    idx, w = layer.router(x)
+    torch.cuda.synchronize()
+    tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
+    assert not tie.any(), "a near-tie token would make the two populations differ"
+    s = np.sort(ref.score.reshape(-1))
+    N = s.size
+    eps = 1e-4   # fp32 gate sums of up to 4096 products against fp64 ones
+    for q in qs:
+        tau_g = layer.calibrate_tau(x, q)
+        m = int(math.floor(q * N))
+        # the GPU's tau is the m-th smallest score, up to the fp32 noise of the scores
+        lo, hi = tau_g * (1 - eps), tau_g * (1 + eps)
+        assert np.sum(s < lo) <= m < np.sum(s <= hi), (q, tau_g, s[m])
+        assert abs(tau_g - o.calibrate_tau(ref.score, q)) <= 2 * eps * tau_g + (s[min(m + 1, N - 1)] - s[m])
+        # about 1 - q of the routed neurons are kept
+        band = int(np.sum((s >= lo) & (s <= hi)))
+        assert abs(int(np.sum(s >= tau_g)) - (N - m)) <= 1 + band
+    assert layer.calibrate_tau(x, 0.0) == 0.0
+    assert layer.calibrate_tau(x, -0.5) == 0.0
+    assert math.isinf(layer.calibrate_tau(x, 1.0))
+
+
+def test_gate_values_beyond_fp16_range(o):
+    """|g| up to ~1e6, far above the fp16 range: the sparse path keeps silu(g)
+    finite and matches the oracle (routed and shared experts)."""
+    from intra_expert_activation_router_b200 import MoESparseLayer
+    sh = mi.custom_shape(256, 8, 64, 2, 1, seed_base=7300)
+    W = mi.make_weights(sh, device="cuda")
+    W.w_gate = (W.w_gate.float() * 2e5).to(torch.bfloat16)
+    W.ws_gate = (W.ws_gate.float() * 2e5).to(torch.bfloat16)
+    layer = MoESparseLayer.from_weights(W, sh.top_k, max_tokens=16)
+    x = mi.make_x(sh, 16, device="cuda")
+    inputs = oracle.layer_inputs(W, x)
+    tau = pu.calibrate(o, inputs, sh.top_k, 0.7)
+    assert tau > 65504.0
+    out = layer.forward(x, tau)
+    idx, w = layer.router(x)
+    lists, cnt = layer.active_lists(x, tau)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out.float()).all())
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=tau)
+    tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
+    flipped, _, gmask = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
+    pu.check_output(pu.expected_under_gpu_mask(o, inputs, sh.top_k, tau, ref, gmask, flipped, tie), out, tie)
+    layer.close()
 
 
 def test_tau_extremes(o):
@@ -202,8 +271,8 @@ def test_edge_shapes(o, dims):
     torch.cuda.synchronize()
     ref = o.forward(**inputs, top_k=sh.top_k, tau=tau)
     tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
-    flipped, _ = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
-    pu.check_output(ref.y, out, tie | flipped)
+    flipped, _, gmask = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
+    pu.check_output(pu.expected_under_gpu_mask(o, inputs, sh.top_k, tau, ref, gmask, flipped, tie), out, tie)
     layer.close()
 
 

@@ -1,7 +1,8 @@
-"""The allocation-free router entry point (for callers that cannot call
-cudaMalloc: servers with a pre-reserved memory arena, custom operators inside a
-framework that owns the allocator, latency-critical paths) against the
-handle-based router of the same library.
+"""The allocation-free router entry point, for callers that cannot call
+cudaMalloc (servers that reserve all device memory up front in their own
+arena, custom operators inside a framework that owns the allocator, paths
+that cannot afford an allocation's implicit synchronisation), against the
+handle-based router of the same library and against the CPU oracle.
 
 Kept in its own file, collected last, so a failure here comes after every
 other test has run.  It creates its own inputs and passes when run alone.
@@ -11,14 +12,24 @@ import pytest
 import torch
 
 import moe_inputs as mi
+import oracle
+from tests import parity_util as pu
 
 pytestmark = pytest.mark.gpu
 
+SHAPES = {
+    "tiny": mi.SHAPES["tiny"],
+    "olmoe": mi.SHAPES["olmoe"],
+    "large": mi.SHAPES["large"],
+    # the largest expert count: the selection's 32-bit "taken" mask is full
+    "e1024": mi.custom_shape(128, 1024, 32, 8, 0, name="e1024"),
+}
 
-@pytest.mark.parametrize("name,T", [("tiny", 16), ("olmoe", 37), ("large", 5)])
-def test_noalloc_router_matches_handle_router(name, T):
+
+@pytest.mark.parametrize("name,T", [("tiny", 16), ("olmoe", 37), ("large", 5), ("e1024", 9)])
+def test_noalloc_router_matches_handle_router_and_oracle(name, T):
     import intra_expert_activation_router_b200 as m
-    sh = mi.SHAPES[name]
+    sh = SHAPES[name]
     g = torch.Generator(device="cuda").manual_seed(11 + T)
     w_router = (torch.randn(sh.n_experts, sh.d_model, generator=g, device="cuda") * sh.d_model ** -0.5).to(torch.bfloat16)
     # a handle with the same router (the expert weights do not affect routing)
@@ -32,6 +43,12 @@ def test_noalloc_router_matches_handle_router(name, T):
         idx_ref = torch.empty(T, sh.top_k, dtype=torch.int32, device="cuda")
         w_ref = torch.empty(T, sh.top_k, dtype=torch.float32, device="cuda")
         m.moe_debug_router(h, x, T, idx_ref, w_ref)
+        torch.cuda.synchronize()
+        # the oracle's routing of the same bf16 inputs (near-tie tokens excluded)
+        zh = np.zeros((sh.n_experts, sh.d_model, f), np.uint16)
+        ref = oracle.load().forward(mi.bf16_bits(x), mi.bf16_bits(w_router), zh, zh,
+                                    np.zeros((sh.n_experts, f, sh.d_model), np.uint16),
+                                    top_k=sh.top_k, tau=float("inf"), want_scores=False)
         for _call in range(2):   # two calls in a row share the fixed scratch
             idx = torch.full((T, sh.top_k), -1, dtype=torch.int32, device="cuda")
             w = torch.full((T, sh.top_k), -1.0, dtype=torch.float32, device="cuda")
@@ -40,6 +57,8 @@ def test_noalloc_router_matches_handle_router(name, T):
             assert torch.equal(idx.cpu(), idx_ref.cpu())
             wr, wn = w_ref.cpu().numpy(), w.cpu().numpy()
             assert np.abs(wr - wn).max() <= 1e-5 + 1e-4 * np.abs(wr).max()
+            tie = pu.check_router(ref, idx.cpu().numpy(), wn, sh.top_k)
+            assert tie.sum() <= 1
     finally:
         m.moe_sparse_destroy(h)
 
