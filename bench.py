@@ -297,30 +297,49 @@ def l2_flush(buf):
     buf.sum()
 
 
-def time_steps(layer, x, tau, out, flush, steps, events=True, dense=False):
-    """Per-step CUDA-event timing with an L2 flush before each step (outside the events)."""
+def time_steps(layer, x, tau, out, flush, steps, graph=True):
+    """Per-step CUDA-event timing with an L2 flush before each step (outside the events).
+
+    graph=True (the default): the K steps -- flush, start event, forward (whose
+    kernels record the launch events), end event -- are captured into one CUDA
+    graph and replayed once, so the host's enqueue cost cannot leave the GPU
+    idle inside a step; the device does exactly the same work.  graph=False
+    enqueues the steps one by one from Python (eager)."""
     import torch
     from intra_expert_activation_router_b200 import moe_set_launch_events
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True, external=True)
+
+    starts = [ev() for _ in range(steps)]
+    ends = [ev() for _ in range(steps)]
+    kev = [[ev() for _ in range(3)] for _ in range(steps)]
     st = torch.cuda.current_stream()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for trio in kev:   # create the CUDA events before the library records them
         for e in trio:
             e.record(st)
     torch.cuda.synchronize()
-    for i in range(steps):
-        l2_flush(flush)
-        starts[i].record(st)
-        if events:
+
+    def body():
+        for i in range(steps):
+            l2_flush(flush)
+            starts[i].record()
             moe_set_launch_events(layer.h, kev[i])
-        if dense:
-            layer.dense_forward(x, out=out)
-        else:
             layer.forward(x, tau, out=out)
-        ends[i].record(st)
-    moe_set_launch_events(layer.h, None)
-    torch.cuda.synchronize()
+            ends[i].record()
+        moe_set_launch_events(layer.h, None)
+
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        del g
+    else:
+        body()
+        torch.cuda.synchronize()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     router_ms = [t[0].elapsed_time(t[1]) for t in kev]
     expert_ms = [t[1].elapsed_time(t[2]) for t in kev]
@@ -368,11 +387,13 @@ def sweep_rows(dev, kind, peak, flush, steps=20):
                         layer.forward(x, tau, out=out)
                     sm_, rm_, em_ = time_steps(layer, x, tau, out, flush, steps)
                     st = layer.stats()
+                    if st["device_error"]:
+                        row[f"{mode}_device_error"] = st["device_error"]
                     used = "sparse" if st["path"] == m.MOE_PATH_SPARSE else "dense"
                     b = st["alg_bytes"] if used == "sparse" else st["dense_bytes"]
                     us = 1000 * statistics.mean(sm_)
                     kus = 1000 * statistics.mean(em_)
-                    kb = b - shape.n_experts * shape.d_model * 2 - T * shape.d_model * 2
+                    kb = b - (0 if st["fused_router"] else shape.n_experts * shape.d_model * 2 + T * shape.d_model * 2)
                     row[f"{mode}_us"] = us
                     row[f"{mode}_tokens_per_s"] = T / (us * 1e-6)
                     if mode == "auto":
@@ -436,9 +457,13 @@ def run_ours(args):
     ms = total_ms / args.steps
     value = whole_job_rate(world, T * args.steps, total_ms / 1000)
     st = layer.stats()
+    # the same steps enqueued one by one from Python, for comparison
+    eager_ms, _, _ = time_steps(layer, x, tau, out, flush, args.steps, graph=False)
+    eager_ms = max_over_ranks(sum(eager_ms), dev) / args.steps
     path = "sparse" if st["path"] == m.MOE_PATH_SPARSE else "dense"
     alg = st["alg_bytes"] if path == "sparse" else st["dense_bytes"]
-    router_bytes = shape.n_experts * shape.d_model * 2 + T * shape.d_model * 2
+    # the router's bytes belong to the expert kernel when it routes the batch itself
+    router_bytes = 0 if st["fused_router"] else shape.n_experts * shape.d_model * 2 + T * shape.d_model * 2
     expert_bytes = alg - router_bytes
     expert_ms_mean = statistics.mean(expert_ms)
     peaks, peak_kind = measured_peaks()
@@ -485,6 +510,11 @@ def run_ours(args):
             "data": "synthetic", "config": bench_config(args, world), "tau": tau, "path": path,
             "hbm_gbs": alg / (ms / 1000) / 1e9,
             "latency_us": 1000 * ms,
+            "timing": "K steps captured in one CUDA graph and replayed once (device work identical; "
+                      "no host enqueue gaps); eager_latency_us: the same steps enqueued one by one",
+            "eager_latency_us": 1000 * eager_ms,
+            "device_error": st["device_error"],
+            "fused_router": st["fused_router"],
             "alg_bytes_per_step": alg,
             "kernels_us": {"router": 1000 * statistics.mean(router_ms), kname: 1000 * expert_ms_mean},
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
@@ -495,9 +525,10 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * shape.d_model * 2,
                     "d2h_bytes_per_step": T * shape.d_model * 2},
-            # sparse: router, expert kernel, y conversion; dense: router, gather, GEMM1 and GEMM2 per
-            # routed/shared group, convert
-            "gpu_launches": (3 if path == "sparse" else 5 + 2 * shape.n_shared) * args.steps,
+            # sparse: router (unless routed in the expert kernel), expert kernel, y conversion;
+            # dense: router, gather, GEMM1 and GEMM2 per routed/shared group, convert
+            "gpu_launches": ((2 if st["fused_router"] else 3) if path == "sparse"
+                             else 5 + 2 * shape.n_shared) * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"]},
             "stats": {"n_touched": st["n_touched"], "n_active": st["n_active"], "n_union": st["n_union"]},

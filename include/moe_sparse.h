@@ -90,7 +90,10 @@ typedef struct {
                               union-active neuron + shared experts + router +
                               x and out                                          */
     double dense_bytes;    /* the same for the dense path (all neurons)          */
-    int device_error;      /* last error word read back from the device (0 ok)  */
+    int device_error;      /* first device error code since the previous
+                              moe_query_stats (0: none)                          */
+    int fused_router;      /* 1 if the last forward routed the batch inside the
+                              expert kernel (no separate router launch)          */
 } moe_stats;
 
 /* Create a layer.  Copies and repacks the weights into library-owned device
@@ -132,6 +135,19 @@ int moe_set_path(moe_handle h, int path);
 /* Set the switch point T* of MOE_PATH_AUTO (sparse iff T <= t_star). */
 int moe_set_t_star(moe_handle h, int t_star);
 
+/* Decode batches on the sparse path (T within one token tile of the expert
+ * kernel: up to 16 tokens for d_model <= 2048, up to 8 above; T * top_k <= 128,
+ * T * E <= 8192, d_model >= 64) normally route inside the expert kernel: each
+ * CTA computes some experts' logits, all CTAs then select the top-k and build
+ * the plan themselves, so no router kernel and no plan hand-off precede the
+ * gate stream.  enable = 0 uses the separate router kernel instead (same
+ * results up to the order of fp32 sums in the logits); 1 restores the
+ * default.  This assumes every CTA of the expert kernel (at most one per SM)
+ * can be resident at once, which holds unless the context is restricted to
+ * fewer SMs than the device has; otherwise the routing wait runs out and
+ * reports error code 55. */
+int moe_set_fused_router(moe_handle h, int enable);
+
 /* Router only: idx_out [T][top_k] int32 and w_out [T][top_k] fp32, both
  * DEVICE pointers, in rank order.  Asynchronous. */
 int moe_debug_router(moe_handle h, const void *x, int T, int *idx_out, float *w_out, void *stream);
@@ -159,9 +175,11 @@ int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float
 /* Timing hook for benchmarks: on every later forward, record caller-owned CUDA
  * events (cudaEvent_t cast to void*, created on the handle's device) on the
  * forward's stream -- events[0] before the router kernel, events[1] between
- * the router and the expert kernel(s), events[2] after them.  n must be 3;
- * events == NULL or n == 0 stops recording.  The handle keeps the three
- * handles, not the array. */
+ * the router and the expert kernel(s), events[2] after them; when the batch
+ * is routed inside the expert kernel, events[1] directly follows events[0].
+ * They are recorded with cudaEventRecordExternal, so a forward captured into
+ * a CUDA graph records them on every replay.  n must be 3; events == NULL or
+ * n == 0 stops recording.  The handle keeps the three handles, not the array. */
 int moe_set_launch_events(moe_handle h, void *const *events, int n);
 
 /* Tracing hook: when buf (DEVICE, 8-byte aligned, `bytes` long) is set, later
@@ -175,12 +193,16 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * lists published, first gathered batch in (up warps), first h in (down
  * warps), up projection done, down projection and flush done; [32 + 4u] for
  * the gather of item u < 2: mask seen, then the issue times of its first
- * three batches; [40 + g] issue of gate stage g < 8; [48 + q] token rows of
+ * three batches; [40 + g] issue of gate stage g < 4; [44]..[47] routing
+ * inside the kernel: start, own logits computed, logits staged, plan built;
+ * [48 + q] token rows of
  * tile q < 4 ready (batches of more than 16 tokens; smaller batches stream
  * the token operand with the gate stages); [52], [53] the up warps' total
  * time waiting for and
  * working on gathered batches, [54], [55] the same for the down warps (ns);
  * [56], [57] first gate stage consumed and accumulator committed for item 0;
+ * [58], [59], [60] routing inside the kernel: this CTA's logits published,
+ * every expert's logits available, top-k selected;
  * [61] gathered records processed; [62] end; [63] the CTA's item count.
  * Unwritten slots keep their old contents.
  * buf == NULL turns tracing off. */

@@ -50,7 +50,8 @@ class moe_stats(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("n_tokens", ctypes.c_int), ("n_touched", ctypes.c_int),
                 ("t_star", ctypes.c_int), ("n_active", ctypes.c_longlong),
                 ("n_union", ctypes.c_longlong), ("alg_bytes", ctypes.c_double),
-                ("dense_bytes", ctypes.c_double), ("device_error", ctypes.c_int)]
+                ("dense_bytes", ctypes.c_double), ("device_error", ctypes.c_int),
+                ("fused_router", ctypes.c_int)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -78,6 +79,7 @@ def _load():
         "moe_set_trace": (I, [P, P, ctypes.c_longlong]),
         "moe_router_topk_noalloc": (I, [P, I, P, I, I, I, P, P, P]),
         "moe_debug_inject": (I, [P, I]),
+        "moe_set_fused_router": (I, [P, I]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -92,7 +94,7 @@ EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_sparse_forward_host", "moe_sparse_destroy", "moe_set_path", "moe_set_t_star",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
             "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
-            "moe_debug_inject")
+            "moe_debug_inject", "moe_set_fused_router")
 
 
 def _addr(t):
@@ -215,6 +217,10 @@ def moe_router_topk_noalloc(x, T: int, w_router, E: int, d_model: int, top_k: in
     """Router softmax top-k without a handle or any allocation (fixed device scratch)."""
     _check(_lib.moe_router_topk_noalloc(_addr(x), T, _addr(w_router), E, d_model, top_k, _addr(idx_out),
                                         _addr(w_out), _stream(stream)), "moe_router_topk_noalloc")
+
+
+def moe_set_fused_router(h, enable: int):
+    _check(_lib.moe_set_fused_router(h, int(enable)), "moe_set_fused_router")
 
 
 def moe_debug_inject(h, kind: int):

@@ -74,9 +74,19 @@ __global__ void k_dense_gather(const uint16_t *__restrict__ x, const int *__rest
     }
 }
 
-// out = bf16(y_acc) (round to nearest even), then y_acc = 0.
-__global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4)
+// out = bf16(y_acc) (round to nearest even), then y_acc = 0.  The last kernel
+// of a dense forward: it also moves the forward's error code into the sticky
+// word and clears its own word (as the sparse path's conversion kernel does).
+__global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4, int *error_word,
+                                int *error_sticky)
 {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const int e0 = *error_word;
+        if (e0 != 0) {
+            atomicCAS(error_sticky, 0, e0);
+            *error_word = 0;
+        }
+    }
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const float4 v = reinterpret_cast<const float4 *>(y_acc)[i];
         uint2 p;
@@ -266,8 +276,10 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+}  // namespace
+
 // A 2D bf16 matrix of `rows` rows of `cols` elements, `ld_bytes` apart; boxes of
-// 64 columns x box_rows rows.
+// 64 columns x box_rows rows; elements outside the matrix read as zero.
 bool encode(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint64_t ld_bytes, uint32_t box_rows,
             bool swizzle)
 {
@@ -281,8 +293,6 @@ bool encode(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, ui
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 bool dense_supported(const Dims &dm)
 {
@@ -321,7 +331,8 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
                          float tau, bool use_mask, uint16_t *out, cudaStream_t s)
 {
     if (!st.ok) return cudaErrorNotSupported;
-    cudaError_t e = cudaFuncSetAttribute(k_dense_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, kDenseSmem);
+    static int smem_set[kMaxDevices] = {};
+    cudaError_t e = ensure_dynamic_smem(k_dense_gemm, kDenseSmem, smem_set);
     if (e != cudaSuccess) return e;
     const int P = T * dm.k, Pm = dm.max_tokens * dm.k, Tm = dm.max_tokens;
     const int d8 = dm.d / 8;
@@ -391,7 +402,7 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
         const size_t n4 = (size_t)T * dm.d / 4;
         size_t blocks = (n4 + 255) / 256;
         if (blocks > 148 * 16) blocks = 148 * 16;
-        k_dense_convert<<<(unsigned)blocks, 256, 0, s>>>(ws.y_acc, out, n4);
+        k_dense_convert<<<(unsigned)blocks, 256, 0, s>>>(ws.y_acc, out, n4, ws.error_word, ws.error_sticky);
     }
     return cudaGetLastError();
 }

@@ -78,6 +78,8 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
 constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
+constexpr int kMaxFusedPairs = 128;  // fused routing: (token, expert) pairs kept in shared memory
+constexpr int kMaxFusedLogits = 8192;   // fused routing: T * E logits staged in the gate ring
 // mbarriers besides the two rings': gdone, tfree (kAcc each), xfull, xfree,
 // mdrain, hsfull, hsfree (2 each)
 constexpr int kNumFixedBars = 2 * kAcc + 7;
@@ -89,7 +91,7 @@ struct SparseLayout {   // byte offsets from the 1024-aligned base of dynamic sh
     int ring_off, n_stages;
     int ud_off, ud_buf_bytes, gb, gpitch;   // n_ud buffers of gb [up | down] records (+16-byte skew)
     int n_ud;
-    int meta_off, part_off, h_off, last_off, ctr_off, plan_off, bar_off;
+    int meta_off, part_off, h_off, last_off, ctr_off, plan_off, perm_off, bar_off;
     int total;                              // dynamic bytes to request (includes alignment slack)
 };
 
@@ -107,6 +109,7 @@ struct ItemMeta {
 };
 
 struct SparseArgs {
+    CUtensorMap xmap;     // fused mode: x [T][d] as the MMA's token operand (box 64 x nt, 128-byte swizzle)
     const uint16_t *x;
     uint16_t *out;
     DeviceWeights w;
@@ -123,6 +126,10 @@ struct SparseArgs {
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f], no up/down
     int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
+    int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
+    const uint16_t *wr;   // fused: router weights [E][d]
+    int E;
+    int max_pairs;        // fused: T * k (permutation arrays kept in shared memory)
     SparseLayout L;
 };
 
@@ -135,6 +142,10 @@ struct PlanCache {      // the routing plan's per-slot arrays, copied to shared 
     const int *prefix, *expert, *off, *cnt;
     const int *order;   // resident mode: slots by decreasing token count
     int n_touched;
+    // the permutation of (token, rank) pairs by expert: the workspace's, or in
+    // fused mode this CTA's own copy in shared memory
+    const int *perm, *perm_tok;
+    const float *perm_w;
 };
 
 __device__ __forceinline__ ItemPos locate_item(const SparseArgs &a, const PlanCache &pc, int item)
@@ -182,9 +193,10 @@ __device__ __forceinline__ int tile_tokens(const SparseArgs &a, const PlanCache 
     return max(1, min(a.nt, pc.cnt[p.slot] - p.tile * a.nt));
 }
 
-__device__ __forceinline__ int tile_token(const SparseArgs &a, const ItemPos &p, int base, int r)
+__device__ __forceinline__ int tile_token(const SparseArgs &a, const PlanCache &pc, const ItemPos &p, int base,
+                                          int r)
 {
-    const int t = p.slot < 0 ? base + r : a.ws.perm_tok[base + r];
+    const int t = p.slot < 0 ? base + r : pc.perm_tok[base + r];
     return min(max(t, 0), a.T - 1);
 }
 
@@ -266,6 +278,215 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
 {
     for (uint32_t i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(bar, parity)) return;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ bool route_better(float v1, int i1, float v0, int i0)
+{
+    return v1 > v0 || (v1 == v0 && i1 < i0);
+}
+
+// Routing inside the expert kernel, for batches it takes as one token tile
+// (the decode path).  It is the router of the technical summary ("Uncovering
+// Intra-expert Activation Sparsity ...", Methodology item 3: the router logic
+// is kept unchanged): logits = x Wr^T with fp32 accumulation, softmax over all
+// E experts, the top_k experts by probability (ties to the lower index),
+// weight = probability.  Computing it here removes the router launch and the
+// grid-wide hand-off of its plan from the front of the gate stream:
+//   1. CTA b computes the logits of experts b, b + G, ... for all T tokens and
+//      publishes them with a release-ordered count;
+//   2. once all E experts are counted (bounded wait), every CTA reads the
+//      T x E logits and selects each token's top_k (one warp per token, k
+//      rounds of a warp arg-max);
+//   3. every CTA builds the plan -- per-expert counts, the ascending list of
+//      touched experts, their offsets and the stable permutation of the pairs
+//      (expert, then token) -- in its own shared memory; CTA 0 also writes it
+//      to the workspace, where the statistics and debug calls read it.
+// `scratch` (the gate ring, idle until the plan exists) holds the
+// temporaries.  Called by every thread of the CTA.
+__device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scratch, int *s_prefix, int *s_expert,
+                                             int *s_off, int *s_cnt, int *s_perm, int *s_perm_tok, float *s_perm_w,
+                                             volatile int *s_ntouched)
+{
+    constexpr int NW = kSparseThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = a.T, E = a.E, k = a.k, d = a.d, d8 = d >> 3, P = T * k;
+    float *red = reinterpret_cast<float *>(scratch);                   // [NW][kMaxNT]
+    float *lg = reinterpret_cast<float *>(scratch + 1024);             // [T][E]
+    int *tk_idx = reinterpret_cast<int *>(lg + (size_t)T * E);          // [P]
+    float *tk_w = reinterpret_cast<float *>(tk_idx + P);                // [P]
+    int *ecnt = reinterpret_cast<int *>(tk_w + P);                      // [E]
+    int *ecur = ecnt + E;                                               // [E]
+    Plan *plan = a.ws.plan;
+
+    unsigned long long *tr = (a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
+                                 ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
+    if (tr && tid == 0) tr[44] = global_ns();
+    // 1. this CTA's experts' logits
+    int mine = 0;
+    for (int e = blockIdx.x; e < E; e += gridDim.x, ++mine) {
+        float acc[kMaxNT];
+#pragma unroll
+        for (int r = 0; r < kMaxNT; ++r) acc[r] = 0.f;
+        const uint16_t *wrow = a.wr + (size_t)e * d;
+        for (int v = tid; v < d8; v += kSparseThreads) {
+            const uint4 wv = ld_cached(wrow + 8 * v);
+#pragma unroll
+            for (int r = 0; r < kMaxNT; ++r)
+                if (r < T) acc[r] = dot8(wv, ld_cached(a.x + (size_t)r * d + 8 * v), acc[r]);
+        }
+        const float val = transpose_reduce<kMaxNT>(acc, lane);   // lanes 2r, 2r + 1: token r
+        if ((lane & 1) == 0) red[warp * kMaxNT + (lane >> 1)] = val;
+        __syncthreads();
+        if (tid < T) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) sum += red[w * kMaxNT + tid];
+            a.ws.logits[(size_t)tid * E + e] = sum;
+            __threadfence();
+        }
+        __syncthreads();
+    }
+    if (tr && tid == 0) tr[45] = global_ns();
+    if (tid == 0 && mine > 0) {
+        __threadfence();
+        atomicAdd(a.ws.route_count, mine);
+    }
+    if (tr && tid == 0) tr[58] = global_ns();
+    // 2. every expert's logits, then each token's top_k
+    if (tid == 0) {
+        for (uint32_t spin = 0; ld_acquire_gpu(a.ws.route_count) < E; ++spin) {
+            if (spin > kSpinLimit) {
+                atomicCAS(a.ws.error_word, 0, 55);
+                break;
+            }
+            __nanosleep(32);
+        }
+    }
+    __syncthreads();
+    if (tr && tid == 0) tr[59] = global_ns();
+    for (int i = tid; i < T * E; i += kSparseThreads) lg[i] = __ldcg(&a.ws.logits[i]);
+    for (int e = tid; e < E; e += kSparseThreads) ecnt[e] = 0;
+    __syncthreads();
+    if (tr && tid == 0) tr[46] = global_ns();
+    for (int t = warp; t < T; t += NW) {
+        const float *row = lg + (size_t)t * E;
+        float m = -INFINITY;
+        for (int j = lane; j < E; j += 32) m = fmaxf(m, row[j]);
+        m = warp_max(m);
+        float sum = 0.f;
+        for (int j = lane; j < E; j += 32) sum += expf(row[j] - m);
+        sum = warp_sum(sum);
+        unsigned taken = 0;   // bit q: expert lane + 32 q already selected
+        for (int r = 0; r < k; ++r) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int q = 0, j = lane; j < E; ++q, j += 32) {
+                if (taken & (1u << q)) continue;
+                const float v = row[j];
+                if (bi == 0x7fffffff || route_better(v, j, bv, bi)) { bv = v; bi = j; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFull, bv, o);
+                const int oi = __shfl_xor_sync(kFull, bi, o);
+                if (oi != 0x7fffffff && (bi == 0x7fffffff || route_better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+            }
+            bi = min(max(bi, 0), E - 1);   // only non-finite logits could leave it unset
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == 0) {
+                tk_idx[t * k + r] = bi;
+                tk_w[t * k + r] = expf(bv - m) / sum;
+            }
+        }
+    }
+    __syncthreads();
+    if (tr && tid == 0) tr[60] = global_ns();
+    // 3. the plan
+    for (int p = tid; p < P; p += kSparseThreads) atomicAdd(&ecnt[tk_idx[p]], 1);
+    __syncthreads();
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+        int c_sum = 0, t_sum = 0;
+        for (int e = e0; e < e1; ++e) {
+            c_sum += ecnt[e];
+            t_sum += ecnt[e] > 0 ? 1 : 0;
+        }
+        int c_ex = c_sum, t_ex = t_sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int c = __shfl_up_sync(kFull, c_ex, o), t = __shfl_up_sync(kFull, t_ex, o);
+            if (lane >= o) { c_ex += c; t_ex += t; }
+        }
+        c_ex -= c_sum;
+        t_ex -= t_sum;
+        for (int e = e0; e < e1; ++e) {
+            const int c = ecnt[e];
+            ecur[e] = c_ex;
+            if (c > 0) {
+                s_expert[t_ex] = e;
+                s_off[t_ex] = c_ex;
+                s_cnt[t_ex] = c;
+                s_prefix[t_ex] = t_ex * a.n_blk;
+                ++t_ex;
+            }
+            c_ex += c;
+        }
+        if (lane == 31) {
+            *s_ntouched = t_ex;
+            s_prefix[t_ex] = t_ex * a.n_blk;
+        }
+        __syncwarp();
+        // stable scatter, 32 pairs at a time in pair order
+        for (int base = 0; base < P; base += 32) {
+            const int p = base + lane;
+            const int e = p < P ? tk_idx[p] : -1 - lane;
+            const unsigned same = __match_any_sync(kFull, e);
+            const int rank = __popc(same & ((1u << lane) - 1u));
+            int pos = 0;
+            if (p < P) pos = ecur[e] + rank;
+            __syncwarp();
+            if (p < P && rank == 0) ecur[e] += __popc(same);
+            if (p < P) {
+                s_perm[pos] = p;
+                s_perm_tok[pos] = p / k;
+                s_perm_w[pos] = tk_w[p];
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    if (tr && tid == 0) tr[47] = global_ns();
+    if (blockIdx.x == 0) {   // the workspace copy for statistics and debug calls
+        const int n_t = *s_ntouched;
+        for (int p = tid; p < P; p += kSparseThreads) {
+            a.ws.topk_idx[p] = tk_idx[p];
+            a.ws.topk_w[p] = tk_w[p];
+            a.ws.perm[p] = s_perm[p];
+            a.ws.perm_tok[p] = s_perm_tok[p];
+            a.ws.perm_w[p] = s_perm_w[p];
+        }
+        for (int e = tid; e < E; e += kSparseThreads) plan->offsets[e] = ecur[e] - ecnt[e];
+        for (int i = tid; i <= n_t; i += kSparseThreads) {
+            if (i < n_t) plan->touched[i] = s_expert[i];
+            plan->item_prefix[i] = s_prefix[i];
+        }
+        if (tid == 0) {
+            plan->offsets[E] = P;
+            plan->n_touched = n_t;
+            plan->n_routed_items = n_t * a.n_blk;
+        }
+    }
+    // the gate ring is written by the copy engine from here on
+    fence_proxy_async_smem();
+    __syncthreads();
 }
 
 template <int MT, int NP>
@@ -360,17 +581,30 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     // launch); the routing plan is read only after the router grid is done
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    const int n_touched = plan->n_touched;
-    for (int i = tid; i <= n_touched; i += blockDim.x) {
-        s_prefix[i] = plan->item_prefix[i];
-        if (i < n_touched) {
-            const int e = plan->touched[i];
-            s_expert[i] = e;
-            s_off[i] = plan->offsets[e];
-            s_cnt[i] = plan->offsets[e + 1] - plan->offsets[e];
+    // fused mode: this CTA's copy of the permutation of pairs
+    int *s_perm = reinterpret_cast<int *>(smem + L.perm_off);
+    int *s_perm_tok = s_perm + a.max_pairs;
+    float *s_perm_w = reinterpret_cast<float *>(s_perm_tok + a.max_pairs);
+    volatile int *s_ntouched = reinterpret_cast<volatile int *>(smem + L.ctr_off + 56);
+    int n_touched, n_routed_items;
+    if (a.fused) {
+        route_in_kernel(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched);
+        n_touched = *s_ntouched;
+        n_routed_items = n_touched * a.n_blk;
+    } else {
+        n_touched = plan->n_touched;
+        n_routed_items = plan->n_routed_items;
+        for (int i = tid; i <= n_touched; i += blockDim.x) {
+            s_prefix[i] = plan->item_prefix[i];
+            if (i < n_touched) {
+                const int e = plan->touched[i];
+                s_expert[i] = e;
+                s_off[i] = plan->offsets[e];
+                s_cnt[i] = plan->offsets[e + 1] - plan->offsets[e];
+            }
         }
+        __syncthreads();
     }
-    __syncthreads();
     if (a.resident) {
         // slots by decreasing token count (ties by slot): claimed in this order,
         // the most expensive items go first and the tail is made of cheap ones
@@ -386,9 +620,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         __syncthreads();
     }
     if (tr && tid == 0) tr[1] = global_ns();
-    const PlanCache pc{s_prefix, s_expert, s_off, s_cnt, s_order, n_touched};
+    const PlanCache pc{s_prefix, s_expert, s_off, s_cnt, s_order, n_touched,
+                       a.fused ? s_perm : a.ws.perm, a.fused ? s_perm_tok : a.ws.perm_tok,
+                       a.fused ? s_perm_w : a.ws.perm_w};
 
-    const int n_items = a.n_shared_items + plan->n_routed_items;
+    const int n_items = a.n_shared_items + n_routed_items;
     // static ranges (token-tile mode): contiguous items per CTA
     const int G = gridDim.x, b = blockIdx.x;
     const int per = n_items / G, rem = n_items % G;
@@ -524,12 +760,16 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 for (int s = 0; s < spi; ++s, ++g) {
                     const int slot = (int)(g % NS);
                     if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
-                    if (tr && g < 8) tr[40 + g] = global_ns();
+                    if (tr && g < 4) tr[40 + g] = global_ns();
                     uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
                     mbar_arrive_expect_tx(&full_g[slot], kStageBytes + L.xs_bytes);
-                    if (L.xs_bytes)   // the token operand's blocks 2s, 2s+1 (L2-resident, re-read per item)
+                    if (a.fused) {   // the token operand's blocks 2s, 2s+1 straight from x (L2-resident)
+                        tma_load_2d(stage + kStageBytes, &a.xmap, 128 * s, 0, &full_g[slot]);
+                        tma_load_2d(stage + kStageBytes + L.xt_kb, &a.xmap, 128 * s + 64, 0, &full_g[slot]);
+                    } else if (L.xs_bytes) {   // the same, pre-swizzled by the router
                         bulk_g2s(stage + kStageBytes, a.ws.x_tiles + (size_t)s * (L.xs_bytes / 2), L.xs_bytes,
                                  &full_g[slot]);
+                    }
                     bulk_g2s_hint(stage, src + (size_t)s * (kStageBytes / 2), kStageBytes,
                                   &full_g[slot], pol);
                 }
@@ -627,7 +867,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (q > 0 && !mbar_wait(xfree, (q - 1) & 1, err, 34)) break;
                 int base;
                 const int m = tile_tokens(a, pc, p, base);
-                load_rows(m, [&](int r) { return tile_token(a, p, base, r); });
+                load_rows(m, [&](int r) { return tile_token(a, pc, p, base, r); });
                 if (lane == 0) {
                     if (tr && q < 4) tr[48 + q] = global_ns();
                     mbar_arrive(xfull);
@@ -659,13 +899,13 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             int base;
             const int m = tile_tokens(a, pc, p, base);
             if (ct < m) {
-                M.tok[ct] = tile_token(a, p, base, ct);
+                M.tok[ct] = tile_token(a, pc, p, base, ct);
                 if (p.slot < 0) {
                     M.pair[ct] = -1;
                     M.w[ct] = 1.f;
                 } else {
-                    M.pair[ct] = min(max(a.ws.perm[base + ct], 0), a.T * a.k - 1);
-                    M.w[ct] = a.ws.perm_w[base + ct];
+                    M.pair[ct] = min(max(pc.perm[base + ct], 0), a.T * a.k - 1);
+                    M.w[ct] = pc.perm_w[base + ct];
                 }
             }
             if (ct == 0) {
@@ -927,6 +1167,15 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     if (tr && tid == 0) tr[62] = global_ns();
 }
 
+// Routing inside the expert kernel needs: the batch as one token tile
+// (resident mode), the permutation (T * k pairs) in shared memory, the T x E
+// logits in the idle gate ring, and x at least one 64-input box wide.
+bool fused_possible(const Dims &dm, int T)
+{
+    const SparseTiling t = sparse_tiling(T, dm.d);
+    return T <= t.nt && T * dm.k <= kMaxFusedPairs && T * dm.E <= kMaxFusedLogits && dm.d >= 64;
+}
+
 SparseTiling sparse_tiling(int T, int d)
 {
     SparseTiling t;
@@ -943,7 +1192,8 @@ SparseTiling sparse_tiling(int T, int d)
     return t;
 }
 
-static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_touched, SparseLayout &L)
+static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_touched, int perm_pairs,
+                        SparseLayout &L)
 {
     auto up = [](int v) { return (v + 127) & ~127; };
     const int rec = 4 * d;
@@ -958,7 +1208,8 @@ static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_
     const int part_bytes = up(2 * 4 * kMaxGB * til.mt * 4);
     const int h_bytes = up(2 * kMaxGB * til.mt * 4);
     const int plan_bytes = up(4 * (5 * max_touched + 1));
-    const int fixed = xt_bytes + meta_bytes + part_bytes + h_bytes + 128 + 128 + plan_bytes +
+    const int perm_bytes = up(12 * perm_pairs);   // fused mode: perm, perm_tok, perm_w
+    const int fixed = xt_bytes + meta_bytes + part_bytes + h_bytes + 128 + 128 + plan_bytes + perm_bytes +
                       up((2 * 8 + 2 * kMaxNU + kNumFixedBars) * 8) + 1024 /* base alignment */;
     // gather buffers of up to four records (rows per up reduction), at least
     // two of them; three gate stages when that leaves two buffers, else two
@@ -984,16 +1235,31 @@ static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_
     L.last_off = off; off += 128;
     L.ctr_off = off; off += 128;
     L.plan_off = off; off += plan_bytes;
+    L.perm_off = off; off += perm_bytes;
     L.bar_off = off; off += up((2 * ns + 2 * L.n_ud + kNumFixedBars) * 8);
     L.total = off + 1024;   // slack for aligning the base to 1024 bytes
     return L.n_ud >= 2 && L.total <= kSmemLimit;
 }
 
 // out = bf16(y_acc) (round to nearest even), then y_acc = 0; launched after
-// the expert kernel as its programmatic dependent.
-__global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4)
+// the expert kernel as its programmatic dependent.  It also ends the forward
+// for the next one: the work-item and route counters go back to zero (CUDA
+// graph replays included), and the forward's error code is moved into the
+// sticky word and its own word cleared, so a later forward is not cut short.
+// With n4 = 0 it only does that.
+__global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4,
+                                               int *route_count, int *next_item, int *error_word, int *error_sticky)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *route_count = 0;
+        *next_item = 0;
+        const int e0 = *error_word;
+        if (e0 != 0) {
+            atomicCAS(error_sticky, 0, e0);
+            *error_word = 0;
+        }
+    }
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const float4 v = __ldcg(reinterpret_cast<const float4 *>(y_acc) + i);
         uint2 p;
@@ -1004,7 +1270,8 @@ __global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16
     }
 }
 
-static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm, cudaStream_t st)
+static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm, const Workspace &ws,
+                                cudaStream_t st)
 {
     size_t blocks = (n4 + 255) / 256;
     if (blocks > (size_t)n_sm * 4) blocks = (size_t)n_sm * 4;
@@ -1018,7 +1285,8 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_y_out, y_acc, out, n4);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_y_out, y_acc, out, n4, ws.route_count, &ws.plan->next_item,
+                                       ws.error_word, ws.error_sticky);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1027,7 +1295,8 @@ template <int MT, int NP>
 static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 {
     auto kern = k_expert_sparse<MT, NP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.L.total);
+    static int smem_set[kMaxDevices] = {};
+    cudaError_t e = ensure_dynamic_smem(kern, a.L.total, smem_set);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1047,7 +1316,7 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out, int inject)
+                                 float *score_out, int inject, bool fused)
 {
     SparseArgs a;
     a.x = x;
@@ -1069,11 +1338,16 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.use_mask = use_mask ? 1 : 0;
     a.score_out = score_out;
     a.inject = inject;
+    a.fused = (fused && !score_out && fused_possible(dm, T)) ? 1 : 0;
+    a.wr = w.wr;
+    a.E = dm.E;
+    a.max_pairs = a.fused ? T * dm.k : 0;
+    if (a.fused && !encode(&a.xmap, x, dm.d, T, 2ull * dm.d, til.nt, true)) return cudaErrorInvalidValue;
     a.n_tok_tiles = (T + til.nt - 1) / til.nt;
     a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
     const int pairs = T * dm.k;
     a.max_touched = pairs < dm.E ? pairs : dm.E;
-    if (!make_layout(dm.d, dm.dp, til, a.resident != 0, a.max_touched, a.L)) return cudaErrorInvalidValue;
+    if (!make_layout(dm.d, dm.dp, til, a.resident != 0, a.max_touched, a.max_pairs, a.L)) return cudaErrorInvalidValue;
     const int np = (dm.d / 8 + 127) / 128;
     const long long bound = a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
@@ -1090,8 +1364,9 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     case 32 + 2: e = launch_mt<2, 4>(a, grid, st); break;
     default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess || score_out) return e;
-    return launch_y_out(ws.y_acc, out, (size_t)T * dm.d / 4, grid_cap, st);
+    if (e != cudaSuccess) return e;
+    // score mode writes no output: only the counters are reset
+    return launch_y_out(ws.y_acc, out, score_out ? 0 : (size_t)T * dm.d / 4, grid_cap, ws, st);
 }
 
 }  // namespace moe

@@ -106,6 +106,10 @@ struct Workspace {
     // reads and clears it
     int *error_word;
     int *error_sticky;
+    // the fused decode path's count of experts whose logits are written; like
+    // the plan's work-item counter it is zero when a forward starts (the
+    // conversion kernel that ends every forward resets both)
+    int *route_count;
     Plan *plan;
     // dense path
     uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts
@@ -123,6 +127,22 @@ struct Workspace {
     int trace_router_ctas, trace_expert_ctas;
 };
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device
+// rather than on every launch: `done` is a per-kernel array of the largest
+// size set so far on each device (the caller keeps one array per kernel).
+constexpr int kMaxDevices = 64;
+template <typename Kern>
+inline cudaError_t ensure_dynamic_smem(Kern kern, int bytes, int (&done)[kMaxDevices])
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (__atomic_load_n(&done[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) __atomic_store_n(&done[dev], bytes, __ATOMIC_RELEASE);
+    return e;
+}
+
 __device__ __forceinline__ unsigned long long global_ns()
 {
     unsigned long long t;
@@ -137,10 +157,14 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
                           const uint16_t *x, int T, int tile_tokens, cudaStream_t st);
 // inject: test-only fault (MOE_INJECT_WITHHOLD_ITEMS: the gate lane publishes
 // no work item, so the consumers' bounded waits run out), 0 otherwise.
+// fused: the kernel routes the batch itself (no router launch before it);
+// only when fused_possible() holds.  *fused_used reports whether it did.
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out = nullptr, int inject = 0);
+                                 float *score_out = nullptr, int inject = 0, bool fused = false);
+// Whether a sparse forward of T tokens can route inside the expert kernel.
+bool fused_possible(const Dims &dm, int T);
 // dst[b][c][col_off + r] = src[b][r][c] with row stride ld (elements).
 cudaError_t launch_repack_transpose(const uint16_t *src, uint16_t *dst, int batches, int rows, int cols,
                                     int ld, int col_off, cudaStream_t st);
@@ -157,6 +181,13 @@ cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned lo
 
 cudaError_t launch_radix_hist(const uint32_t *v, size_t n, uint32_t prefix, uint32_t prefix_mask,
                               int shift, unsigned *hist, int n_sm, cudaStream_t st);
+
+// Tensor map of a 2D bf16 matrix (`rows` rows of `cols` elements, `ld_bytes`
+// apart), boxes of 64 columns x box_rows rows, optionally with the 128-byte
+// swizzle; reads outside the matrix return zero.  False if the driver
+// rejects it.
+bool encode(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint64_t ld_bytes, uint32_t box_rows,
+            bool swizzle);
 
 bool dense_supported(const Dims &dm);
 bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st);

@@ -54,6 +54,8 @@ struct moe_sparse_s {
     float *scores;       // calibration buffer, allocated by the first moe_calibrate_tau
     unsigned *hist;      // 256 bins, inside the workspace
     int inject_next;     // test-only fault for the next sparse forward (moe_debug_inject)
+    int fused_router;    // route decode batches inside the expert kernel (moe_set_fused_router)
+    int last_fused;      // the last forward routed inside the expert kernel
 };
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -196,6 +198,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.done_ticket = (int *)sb.take(4);
     ws.error_word = (int *)sb.take(4);
     ws.error_sticky = (int *)sb.take(4);
+    ws.route_count = (int *)sb.take(4);
     ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
     ws.x_perm = (uint16_t *)sb.take(2 * (P + T) * d_model);
     ws.h_perm = (uint16_t *)sb.take(2 * (P + n_shared * T) * d_ff);
@@ -204,7 +207,10 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky) { free_handle(h); return MOE_ENOMEM; }
+    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count) {
+        free_handle(h);
+        return MOE_ENOMEM;
+    }
 
     cudaStream_t st = nullptr;
     bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
@@ -233,6 +239,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
         free_handle(h);
         return MOE_ECUDA;
     }
+    h->fused_router = 1;
     h->last_T = 0;
     h->last_path = MOE_PATH_SPARSE;
     h->last_masked = 1;
@@ -272,25 +279,34 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     const uint16_t *xb = (const uint16_t *)x;
     uint16_t *ob = (uint16_t *)out;
     cudaError_t e = cudaSuccess;
-    if (h->n_ev) e = cudaEventRecord(h->ev[0], st);
+    // inside a stream capture the launch events must be external nodes, so that
+    // every replay records them; outside a capture a plain record
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (h->n_ev && cudaStreamIsCapturing(st, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusNone;
+    const unsigned ev_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    if (h->n_ev) e = cudaEventRecordWithFlags(h->ev[0], st, ev_flags);
+    bool fused = false;
     if (path == MOE_PATH_SPARSE) {
         const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
-        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
-        if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
+        // decode batches route inside the expert kernel: no router launch
+        fused = h->fused_router && moe::fused_possible(h->dm, T);
+        if (e == cudaSuccess && !fused) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
+        if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
             e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
-                                          h->inject_next);
+                                          h->inject_next, fused);
         h->inject_next = 0;
     } else {
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
-        if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[1], st);
+        if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
             e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st);
     }
-    if (e == cudaSuccess && h->n_ev) e = cudaEventRecord(h->ev[2], st);
+    if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[2], st, ev_flags);
     h->last_T = T;
     h->last_path = path;
     h->last_masked = masked;
+    h->last_fused = fused ? 1 : 0;
     h->last_stream = st;
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -459,6 +475,7 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
     st->path = h->last_path;
     st->n_tokens = h->last_T;
     st->t_star = h->t_star;
+    st->fused_router = h->last_fused;
     if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
     // the first error code since the previous call: an earlier forward's (kept
     // in the sticky word by the router of the next forward), else the last
@@ -488,6 +505,14 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
         st->dense_bytes = st->n_touched * 3.0 * d * f * 2 + fixed;
     }
     return err ? MOE_EDEVICE : MOE_OK;
+}
+
+extern "C" int moe_set_fused_router(moe_handle h, int enable)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (enable != 0 && enable != 1) return MOE_EINVAL;
+    h->fused_router = enable;
+    return MOE_OK;
 }
 
 extern "C" int moe_debug_inject(moe_handle h, int kind)

@@ -69,6 +69,9 @@ class MoESparseLayer:
     def set_t_star(self, t_star: int):
         B.moe_set_t_star(self.h, t_star)
 
+    def set_fused_router(self, enable: bool):
+        B.moe_set_fused_router(self.h, 1 if enable else 0)
+
     def router(self, x, stream=None):
         self._check_x(x)
         T = x.shape[0]

@@ -103,6 +103,36 @@ def test_tiling_boundaries(o, name, T):
     run_case(o, name, T, 0.9)
 
 
+@pytest.mark.parametrize("name,T,q", [("olmoe", 1, 0.9), ("olmoe", 4, 0.9), ("olmoe", 16, 0.9), ("tiny", 16, 0.9),
+                                      ("dsv2lite", 8, 0.9), ("large", 1, 0.98), ("large", 8, 0.98)])
+def test_router_kernel_path(o, name, T, q):
+    """Decode batches route inside the expert kernel by default; the same
+    batches through the separate router kernel must match the oracle too."""
+    layer, W, host = layer_for(name)
+    layer.set_fused_router(False)
+    try:
+        run_case(o, name, T, q)
+        assert layer.stats()["fused_router"] == 0
+    finally:
+        layer.set_fused_router(True)
+
+
+def test_in_kernel_routing_is_used_for_decode_batches(o):
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    for T, want in ((1, 1), (16, 1), (17, 0)):
+        x = mi.make_x(sh, T, device="cuda")
+        layer.forward(x, 1.0)
+        st = layer.stats()
+        assert st["fused_router"] == want and st["rc"] == 0, (T, st)
+    # the workspace copy of the plan that the statistics use is the kernel's own
+    x = mi.make_x(sh, 16, device="cuda")
+    idx, _ = layer.router(x)
+    layer.forward(x, 1.0)
+    st = layer.stats()
+    assert st["n_touched"] == len(np.unique(idx.cpu().numpy()))
+
+
 @pytest.mark.parametrize("T", [1, 8, 32, 128])
 @pytest.mark.parametrize("q", [0.0, 0.5, 0.8, 0.9, 0.95])
 def test_dsv2lite(o, T, q):
