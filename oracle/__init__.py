@@ -49,6 +49,7 @@ class OracleResult:
     logits: np.ndarray       # [T][E] float64
     score: np.ndarray | None   # [T][k][f] float64
     active: np.ndarray | None  # [T][k][f] uint8
+    score_shared: np.ndarray | None = None   # [T][S][f] float64
 
 
 class Oracle:
@@ -64,8 +65,8 @@ class Oracle:
         f = self._lib.oracle_moe_forward
         f.restype = ctypes.c_int
         f.argtypes = [_P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                      ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, ctypes.c_int,
-                      _P, _P, _P, _P, _P, _P, _P]
+                      ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, ctypes.c_float,
+                      ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, _P]
         c = self._lib.oracle_calibrate_tau
         c.restype = ctypes.c_double
         c.argtypes = [_P, ctypes.c_long, ctypes.c_double]
@@ -76,13 +77,16 @@ class Oracle:
 
     def forward(self, x, w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None,
                 ws_down=None, *, top_k: int, tau: float, want_scores: bool = True,
-                nthreads: int = 0, active=None) -> OracleResult:
+                nthreads: int = 0, active=None, tau_shared: float = 0.0) -> OracleResult:
         """All weight/x arguments are uint16 numpy arrays of bf16 bits (x @ W layout).
 
         ``active``: optional [T][top_k][d_ff] mask (nonzero = active) that
         replaces the threshold decision for each (token, rank) pair; ``tau``
         is then unused.  It evaluates the layer under a given decision, e.g.
-        the CUDA path's for neurons whose score sits on the threshold."""
+        the CUDA path's for neurons whose score sits on the threshold.
+
+        ``tau_shared``: shared-expert neurons count iff |silu(g)| >= tau_shared
+        (<= 0, the default: every shared neuron)."""
         arrs = [np.ascontiguousarray(a, dtype=np.uint16) if a is not None else None
                 for a in (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)]
         x, wr, wg, wu, wd, wsg, wsu, wsd = arrs
@@ -97,6 +101,7 @@ class Oracle:
         lg = np.zeros((T, E), np.float64)
         sc = np.zeros((T, k, f), np.float64) if want_scores else None
         ac = np.zeros((T, k, f), np.uint8) if want_scores else None
+        ssh = np.zeros((T, S, f), np.float64) if (want_scores and S > 0) else None
         ain = None
         if active is not None:
             ain = np.ascontiguousarray(np.asarray(active) != 0, dtype=np.uint8)
@@ -105,11 +110,11 @@ class Oracle:
         rc = self._lib.oracle_moe_forward(
             self._ptr(x), T, d, f, E, k, S, self._ptr(wr), self._ptr(wg), self._ptr(wu),
             self._ptr(wd), self._ptr(wsg), self._ptr(wsu), self._ptr(wsd),
-            ctypes.c_float(tau), int(nthreads), self._ptr(y), self._ptr(idx), self._ptr(w),
-            self._ptr(lg), self._ptr(sc), self._ptr(ac), self._ptr(ain))
+            ctypes.c_float(tau), ctypes.c_float(tau_shared), int(nthreads), self._ptr(y), self._ptr(idx),
+            self._ptr(w), self._ptr(lg), self._ptr(sc), self._ptr(ac), self._ptr(ain), self._ptr(ssh))
         if rc != 0:
             raise RuntimeError(f"oracle_moe_forward failed ({rc})")
-        return OracleResult(y, idx, w, lg, sc, ac)
+        return OracleResult(y, idx, w, lg, sc, ac, ssh)
 
     def calibrate_tau(self, scores: np.ndarray, sparsity: float) -> float:
         """tau = the floor(q*N)-th smallest of the routed pairs' scores s = |silu(g)|.

@@ -22,10 +22,14 @@
  *               h_j = silu(g_j) u_j,  y += p_e h_j Wd[e][j][:]
  *               ("Fused up-down projection" bullet; inactive neurons are not
  *               loaded, Hindi summary "The skip").
- *   shared      y += sum_j silu(gs_j) us_j Wds[j][:]  over all neurons of each
- *               shared expert, never masked and not weighted (shared experts
- *               are always on and their execution is unchanged, Methodology
- *               items 1-3).
+ *   shared      y += sum_j silu(gs_j) us_j Wds[j][:]  over the neurons of each
+ *               shared expert, not weighted (shared experts are always on and
+ *               their execution is unchanged, Methodology items 1-3).  By
+ *               default every shared neuron counts; a separate shared
+ *               threshold tau_s > 0 keeps only shared neurons with
+ *               |silu(gs_j)| >= tau_s (Methodology item 1: shared neurons
+ *               matter more per neuron than routed ones, so they take their
+ *               own, looser threshold).
  *
  * Precision: bf16 inputs are widened exactly; every product and sum is in
  * double.  The mask decision compares the score rounded to float with the
@@ -110,6 +114,9 @@ static void gate_up(const uint16_t *xt, int d, int f, const uint16_t *wg, const 
  *   logits     [T][E]   router logits
  *   score      [T][k][f] s = |silu(g)| of each selected pair
  *   active     [T][k][f] 1 where s >= tau (decided in float)
+ *   score_shared [T][S][f] |silu(gs)| of each shared neuron
+ * tau_shared: shared neuron j counts iff (float)|silu(gs_j)| >= tau_shared;
+ * tau_shared <= 0 keeps every shared neuron (the default layer).
  * Optional input:
  *   active_in  [T][k][f] when not NULL, neuron j of the pair (t, rank r) is
  *              active iff active_in[t][r][j] != 0, in place of the threshold
@@ -120,9 +127,9 @@ static void gate_up(const uint16_t *xt, int d, int f, const uint16_t *wg, const 
 int oracle_moe_forward(const uint16_t *x, int T, int d, int f, int E, int k, int S,
                        const uint16_t *wr, const uint16_t *wg, const uint16_t *wu,
                        const uint16_t *wd, const uint16_t *wsg, const uint16_t *wsu,
-                       const uint16_t *wsd, float tau, int nthreads,
+                       const uint16_t *wsd, float tau, float tau_shared, int nthreads,
                        double *y, int *topk_idx, double *topk_w, double *logits,
-                       double *score, uint8_t *active, const uint8_t *active_in)
+                       double *score, uint8_t *active, const uint8_t *active_in, double *score_shared)
 {
     if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0 || k > E || S < 0) return -1;
     if (S > 0 && (!wsg || !wsu || !wsd)) return -1;
@@ -148,12 +155,17 @@ int oracle_moe_forward(const uint16_t *x, int T, int d, int f, int E, int k, int
             if (logits) memcpy(logits + (size_t)t * E, lg, sizeof(double) * E);
             if (topk_idx) memcpy(topk_idx + (size_t)t * k, idx, sizeof(int) * k);
             if (topk_w) memcpy(topk_w + (size_t)t * k, w, sizeof(double) * k);
-            /* shared experts: dense SwiGLU, every neuron, unweighted */
+            /* shared experts: SwiGLU, unweighted; every neuron unless a
+               shared threshold is given */
             for (int s = 0; s < S; ++s) {
                 gate_up(xt, d, f, wsg + (size_t)s * d * f, wsu + (size_t)s * d * f, g, u);
                 const uint16_t *down = wsd + (size_t)s * f * d;
                 for (int j = 0; j < f; ++j) {
-                    double h = silu(g[j]) * u[j];
+                    double as = silu(g[j]);
+                    double ss = fabs(as);
+                    if (score_shared) score_shared[((size_t)t * S + s) * f + j] = ss;
+                    if (!((float)ss >= tau_shared)) continue;
+                    double h = as * u[j];
                     for (int i = 0; i < d; ++i) yt[i] += h * bf16_to_double(down[(size_t)j * d + i]);
                 }
             }

@@ -52,9 +52,9 @@ def _rand_layer(seed, d, E, f, k, S, T, scale_x=1.0):
     return x, W
 
 
-def _call(o, x, W, k, tau, active=None):
+def _call(o, x, W, k, tau, active=None, tau_shared=0.0):
     args = {n: _bits(t) for n, t in W.items()}
-    return o.forward(_bits(x), **args, top_k=k, tau=tau, active=active)
+    return o.forward(_bits(x), **args, top_k=k, tau=tau, active=active, tau_shared=tau_shared)
 
 
 def _torch_dense(x, W, k, with_routed=True, with_shared=True):
@@ -239,6 +239,60 @@ def pin_mask_override(o):
         assert _rel(r.y, np.array(y)) < 1e-12, ("y", tau, _rel(r.y, np.array(y)))
 
 
+def pin_shared_threshold(o):
+    """The shared-expert threshold: +inf removes the shared experts (torch fp64
+    routed-only layer); tau_s equal to a shared neuron's own score keeps it (>=);
+    scalar-Python enumeration at that tau_s; shared scores = |silu(x Ws_g)|."""
+    d, E, f, k, S, T = 16, 4, 8, 2, 2, 3
+    x, W = _rand_layer(35, d, E, f, k, S, T, scale_x=1.0)
+    r_inf = _call(o, x, W, k, 0.0, tau_shared=math.inf)
+    y_routed, *_ = _torch_dense(x, W, k, with_shared=False)
+    assert _rel(r_inf.y, y_routed) < 1e-12, ("tau_s=inf", _rel(r_inf.y, y_routed))
+    X = x.float().double().tolist()
+    Wr = W["w_router"].double().tolist()
+    Wg, Wu, Wd = (W["w_gate"].double().tolist(), W["w_up"].double().tolist(),
+                  W["w_down"].double().tolist())
+    Sg, Su, Sd = (W["ws_gate"].double().tolist(), W["ws_up"].double().tolist(),
+                  W["ws_down"].double().tolist())
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    sh = []   # (t, s, j, silu(g), u)
+    for t in range(T):
+        for s_ in range(S):
+            for j in range(f):
+                g = sum(X[t][i] * Sg[s_][i][j] for i in range(d))
+                u = sum(X[t][i] * Su[s_][i][j] for i in range(d))
+                sh.append((t, s_, j, silu(g), u))
+    scores = sorted(abs(a) for (_, _, _, a, _) in sh)
+    tau_s = float(np.float32(scores[len(scores) // 2]))   # one shared neuron sits exactly on it
+    y = [[0.0] * d for _ in range(T)]
+    for t in range(T):
+        lg = [sum(X[t][i] * Wr[e][i] for i in range(d)) for e in range(E)]
+        m = max(lg)
+        ex = [math.exp(v - m) for v in lg]
+        p = [v / sum(ex) for v in ex]
+        for e in sorted(range(E), key=lambda e: (-p[e], e))[:k]:   # tau = 0: every routed neuron
+            for j in range(f):
+                g = sum(X[t][i] * Wg[e][i][j] for i in range(d))
+                u = sum(X[t][i] * Wu[e][i][j] for i in range(d))
+                for i in range(d):
+                    y[t][i] += p[e] * silu(g) * u * Wd[e][j][i]
+    kept = 0
+    for (t, s_, j, a, u) in sh:
+        if np.float32(abs(a)) >= np.float32(tau_s):
+            kept += 1
+            for i in range(d):
+                y[t][i] += a * u * Sd[s_][j][i]
+    assert 0 < kept < len(sh)
+    r = _call(o, x, W, k, 0.0, tau_shared=tau_s)
+    assert _rel(r.y, np.array(y)) < 1e-12, ("y", _rel(r.y, np.array(y)))
+    want = np.array([[[abs(silu(sum(X[t][i] * Sg[s_][i][j] for i in range(d)))) for j in range(f)]
+                      for s_ in range(S)] for t in range(T)])
+    assert np.allclose(r.score_shared, want, rtol=1e-12, atol=1e-15), "shared scores"
+
+
 def pin_nested_masks(o):
     """tau1 < tau2  =>  A(tau2) is a subset of A(tau1), for every pair."""
     x, W = _rand_layer(41, d=64, E=8, f=64, k=2, S=1, T=6)
@@ -310,8 +364,8 @@ def pin_calibration(o):
 
 
 ALL_PINS = [pin_handworked, pin_tau0_is_dense, pin_tauinf_is_shared_only, pin_bruteforce,
-            pin_mask_override, pin_nested_masks, pin_threshold_decomposition, pin_router_ranking,
-            pin_calibration]
+            pin_mask_override, pin_shared_threshold, pin_nested_masks, pin_threshold_decomposition,
+            pin_router_ranking, pin_calibration]
 
 
 def run_all(o):

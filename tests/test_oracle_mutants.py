@@ -35,6 +35,10 @@ MUTANTS = [
      "for (int j = 0; j < f; ++j) u[j] += xi * bf16_to_double(rg[j]);"),
     ("mask_input_ignored", "if (active_in) on = (active_in[o] != 0);", ";"),
     ("mask_input_inverted", "if (active_in) on = (active_in[o] != 0);", "if (active_in) on = (active_in[o] == 0);"),
+    ("shared_mask_ignored", "if (!((float)ss >= tau_shared)) continue;", ";"),
+    ("shared_mask_uses_routed_tau", "if (!((float)ss >= tau_shared)) continue;",
+     "if (!((float)ss >= tau)) continue;"),
+    ("shared_mask_strict", "if (!((float)ss >= tau_shared)) continue;", "if (!((float)ss > tau_shared)) continue;"),
     ("shared_weighted", "for (int i = 0; i < d; ++i) yt[i] += h * bf16_to_double(down[(size_t)j * d + i]);",
      "for (int i = 0; i < d; ++i) yt[i] += 0.5 * h * bf16_to_double(down[(size_t)j * d + i]);"),
 ]
