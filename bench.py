@@ -70,6 +70,8 @@ def parse():
     p.add_argument("--T", type=int, default=16)
     p.add_argument("--sparsity", type=float, default=0.9)
     p.add_argument("--path", choices=["auto", "sparse", "dense"], default="auto")
+    p.add_argument("--router", choices=["fused", "kernel"], default="fused",
+                   help="decode batches: route inside the expert kernel (default) or with the router kernel")
     p.add_argument("--sweep", choices=["full", "quick", "none"], default="full")
     p.add_argument("--no-sweep", action="store_true", help="same as --sweep none")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -370,12 +372,15 @@ def sweep_rows(dev, kind, peak, flush, steps=20):
         W = mi.make_weights(shape, device=dev)
         layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max(Ts))
         del W
-        for T in Ts:
-            x = mi.make_x(shape, T, device=dev)
-            out = torch.empty_like(x)
-            for q in qs:
+        x_max = mi.make_x(shape, max(Ts), device=dev)
+        for q in qs:
+            # AUTO's switch point for this layer and sparsity, measured on the device
+            t_star = layer.tune_t_star(x_max, layer.calibrate_tau(x_max, q))
+            for T in Ts:
+                x = mi.make_x(shape, T, device=dev)
+                out = torch.empty_like(x)
                 tau = layer.calibrate_tau(x, q)
-                row = {"workload": name, "T": T, "sparsity": q, "tau": tau}
+                row = {"workload": name, "T": T, "sparsity": q, "tau": tau, "t_star": t_star}
                 for mode, path in (("sparse", m.MOE_PATH_SPARSE), ("dense", m.MOE_PATH_DENSE),
                                    ("auto", m.MOE_PATH_AUTO)):
                     try:
@@ -437,6 +442,7 @@ def run_ours(args):
     layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max(T, 64))
     if args.path != "auto":
         layer.set_path({"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
+    layer.set_fused_router(args.router == "fused")
     out = torch.empty_like(x)
     tau = layer.calibrate_tau(x, args.sparsity)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size

@@ -135,6 +135,21 @@ int moe_set_path(moe_handle h, int path);
 /* Set the switch point T* of MOE_PATH_AUTO (sparse iff T <= t_star). */
 int moe_set_t_star(moe_handle h, int t_star);
 
+/* Measure the switch point of MOE_PATH_AUTO on this device for this layer:
+ * for batch sizes 1, 2, 3, 4, 6, 8, 12, 16, 24, ... up to T_max, the first T
+ * rows of x (DEVICE [T_max][d_model] bf16, a representative batch) run through
+ * both branches at threshold tau (the sparse branch's cost depends on it),
+ * each timed on the device (median of five, L2 flushed before every run);
+ * T* becomes the largest measured T at which the sparse branch was not
+ * slower, and is stored in the handle and in *t_star_out (HOST pointer).
+ * ("Uncovering Intra-expert Activation Sparsity...", technical summary,
+ * Methodology item 3, "Dynamic switching": sparse for small batches, dense
+ * for large.)  Allocates and frees a 2 x L2-sized flush buffer; synchronises
+ * `stream`; the launch events of moe_set_launch_events are not recorded
+ * meanwhile.  Without a dense branch T* becomes INT_MAX.  Until this is
+ * called, T* is 16 (measured on the OLMoE-shaped layer at 90% sparsity). */
+int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau, int *t_star_out, void *stream);
+
 /* Decode batches on the sparse path (T within one token tile of the expert
  * kernel: up to 16 tokens for d_model <= 2048, up to 8 above; T * top_k <= 128,
  * T * E <= 8192, d_model >= 64) normally route inside the expert kernel: each
@@ -167,10 +182,30 @@ int moe_debug_active(moe_handle h, const void *x, int T, float tau, uint16_t *id
  * floor(q*N) >= N gives +inf.  About 1 - q of the routed neurons then have
  * s >= tau ("Uncovering Intra-expert Activation Sparsity...", Results:
  * per-model sparsity cutoffs are set as a fraction of neurons kept).
- * The first call allocates a score buffer of max_tokens*top_k*d_ff floats
- * that the handle keeps (MOE_ENOMEM if that fails).  Synchronises `stream`. */
+ * The first call allocates a score buffer of max_tokens*max(top_k, n_shared)*d_ff
+ * floats that the handle keeps (MOE_ENOMEM if that fails).  Synchronises
+ * `stream`. */
 int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
                       void *stream);
+
+/* The shared experts' own threshold ("Uncovering Intra-expert Activation
+ * Sparsity...", technical summary, Methodology item 1: shared-expert neurons
+ * matter more per neuron than routed ones, so they take a separate, looser
+ * threshold).  On later masked forwards (moe_sparse_forward, either path) a
+ * shared neuron j counts iff |silu(x Ws_g[:,j])| >= tau_shared; tau_shared
+ * <= 0 (the default) keeps every shared neuron, +inf none.  moe_dense_forward
+ * stays unmasked.  NaN is MOE_EINVAL.  moe_query_stats' byte counts still
+ * count the shared experts in full. */
+int moe_set_shared_tau(moe_handle h, float tau_shared);
+
+/* As moe_calibrate_tau, over the N = T*n_shared*d_ff scores of the shared
+ * experts' neurons: the floor(q*N)-th smallest |silu(x Ws_g)| (0-based, exact
+ * selection); q <= 0 gives 0 and floor(q*N) >= N gives +inf.  MOE_EINVAL when
+ * the layer has no shared expert.  Shares the score buffer of
+ * moe_calibrate_tau (allocated by the first of the two calls).  Synchronises
+ * `stream`. */
+int moe_calibrate_tau_shared(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
+                             void *stream);
 
 /* Timing hook for benchmarks: on every later forward, record caller-owned CUDA
  * events (cudaEvent_t cast to void*, created on the handle's device) on the

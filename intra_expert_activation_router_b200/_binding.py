@@ -80,6 +80,9 @@ def _load():
         "moe_router_topk_noalloc": (I, [P, I, P, I, I, I, P, P, P]),
         "moe_debug_inject": (I, [P, I]),
         "moe_set_fused_router": (I, [P, I]),
+        "moe_set_shared_tau": (I, [P, F]),
+        "moe_calibrate_tau_shared": (I, [P, P, I, ctypes.c_double, ctypes.POINTER(F), P]),
+        "moe_tune_t_star": (I, [P, P, I, F, ctypes.POINTER(I), P]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -94,7 +97,8 @@ EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_sparse_forward_host", "moe_sparse_destroy", "moe_set_path", "moe_set_t_star",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
             "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
-            "moe_debug_inject", "moe_set_fused_router")
+            "moe_debug_inject", "moe_set_fused_router", "moe_set_shared_tau", "moe_calibrate_tau_shared",
+            "moe_tune_t_star")
 
 
 def _addr(t):
@@ -217,6 +221,25 @@ def moe_router_topk_noalloc(x, T: int, w_router, E: int, d_model: int, top_k: in
     """Router softmax top-k without a handle or any allocation (fixed device scratch)."""
     _check(_lib.moe_router_topk_noalloc(_addr(x), T, _addr(w_router), E, d_model, top_k, _addr(idx_out),
                                         _addr(w_out), _stream(stream)), "moe_router_topk_noalloc")
+
+
+def moe_set_shared_tau(h, tau_shared: float):
+    _check(_lib.moe_set_shared_tau(h, float(tau_shared)), "moe_set_shared_tau")
+
+
+def moe_calibrate_tau_shared(h, x, T: int, sparsity: float, stream=None) -> float:
+    tau = ctypes.c_float()
+    _check(_lib.moe_calibrate_tau_shared(h, _addr(x), T, float(sparsity), ctypes.byref(tau), _stream(stream)),
+           "moe_calibrate_tau_shared")
+    return tau.value
+
+
+def moe_tune_t_star(h, x, T_max: int, tau: float, stream=None) -> int:
+    """Measure both branches at batch sizes up to T_max and set the AUTO switch point; returns it."""
+    t = ctypes.c_int()
+    _check(_lib.moe_tune_t_star(h, _addr(x), T_max, float(tau), ctypes.byref(t), _stream(stream)),
+           "moe_tune_t_star")
+    return t.value
 
 
 def moe_set_fused_router(h, enable: int):

@@ -113,12 +113,18 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- the tile: expert rows [row0, row0 + valid) of A, weight rows wrow0 + n0 ..
+    // The grid is flat with the output block fastest, so that the CTAs of one
+    // wave cover a few token tiles completely: a tile's activations are read by
+    // its output blocks from L2, an expert's weights by its token tiles at about
+    // the same time.
+    const int n_out = a.mode == kGateUp ? a.wrows / 128 : a.wrows / 256;   // output blocks
+    const int bx = (int)(blockIdx.x % (unsigned)n_out), by = (int)(blockIdx.x / (unsigned)n_out);
     int row0, valid, wrow0, ex;
     if (!a.shared) {
         const Plan *plan = a.plan;
         const int n_tiles = plan->n_dense_tiles;
-        if ((int)blockIdx.x >= n_tiles) return;
-        const int mt = blockIdx.x;
+        if (by >= n_tiles) return;
+        const int mt = by;
         int lo = 0, hi = plan->n_touched - 1;   // last slot with tile_prefix <= mt
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -132,14 +138,14 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
         wrow0 = e * a.wrows;
         ex = e;
     } else {
-        row0 = kBM * blockIdx.x;
+        row0 = kBM * by;
         valid = min(kBM, a.T - row0);
         if (valid <= 0) return;
         wrow0 = a.sidx * a.wrows;
         ex = a.sidx;
     }
     const int ntile = a.mode == kGateUp ? 128 : 256;
-    const int n0 = blockIdx.y * ntile;
+    const int n0 = bx * ntile;
 
     if (tid == 0) {
         for (int s = 0; s < kDStages; ++s) {
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
             mbar_arrive_expect_tx(&full[s], bytes);
             tma_load_2d(A, &maps.a, kb * kBK, a.a_base + row0, &full[s]);
             if (a.mode == kGateUp) {
-                const uint16_t *gt = a.gate + (((size_t)ex * a.n_blk + blockIdx.y) * a.n_kb + kb) * (kBM * kBK);
+                const uint16_t *gt = a.gate + (((size_t)ex * a.n_blk + bx) * a.n_kb + kb) * (kBM * kBK);
                 bulk_g2s(B, gt, kBTileBytes / 2, &full[s]);
                 tma_load_2d(B + kBTileBytes / 2, &maps.b1, kb * kBK, wrow0 + n0, &full[s]);
             } else {
@@ -328,7 +334,7 @@ bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, De
 }
 
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
-                         float tau, bool use_mask, uint16_t *out, cudaStream_t s)
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared)
 {
     if (!st.ok) return cudaErrorNotSupported;
     static int smem_set[kMaxDevices] = {};
@@ -368,34 +374,36 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     a.shared = 0;
     a.a_base = 0;
     a.h_base = 0;
-    k_dense_gemm<<<dim3(mbound, dm.f / 128, 1), kDenseThreads, kDenseSmem, s>>>(st.g1r, a);
+    k_dense_gemm<<<(unsigned)(dm.f / 128) * mbound, kDenseThreads, kDenseSmem, s>>>(st.g1r, a);
     if (dm.S > 0) {
         a.shared = 1;
         a.a_base = Pm;
-        a.use_mask = 0;
+        a.use_mask = (use_mask && tau_shared > 0.f) ? 1 : 0;   // the shared experts' own threshold
+        a.tau = tau_shared;
         a.gate = st.gate_s;
         for (int z = 0; z < dm.S; ++z) {
             DenseArgs az = a;
             az.sidx = z;
             az.h_base = Pm + z * Tm;   // shared expert z's H rows
-            k_dense_gemm<<<dim3(mshared, dm.f / 128, 1), kDenseThreads, kDenseSmem, s>>>(st.g1s, az);
+            k_dense_gemm<<<(unsigned)(dm.f / 128) * mshared, kDenseThreads, kDenseSmem, s>>>(st.g1s, az);
         }
     }
     // GEMM2: down with the routing-weight epilogue
     a.mode = kDown;
+    a.tau = tau;
     a.K = dm.f;
     a.kb = dm.f / kBK;
     a.wrows = dm.d;
     a.shared = 0;
     a.a_base = 0;
     a.use_mask = use_mask ? 1 : 0;
-    k_dense_gemm<<<dim3(mbound, dm.d / 256, 1), kDenseThreads, kDenseSmem, s>>>(st.g2r, a);
+    k_dense_gemm<<<(unsigned)(dm.d / 256) * mbound, kDenseThreads, kDenseSmem, s>>>(st.g2r, a);
     for (int z = 0; z < dm.S; ++z) {
         DenseArgs az = a;
         az.shared = 1;
         az.sidx = z;
         az.a_base = Pm + z * Tm;
-        k_dense_gemm<<<dim3(mshared, dm.d / 256, 1), kDenseThreads, kDenseSmem, s>>>(st.g2s, az);
+        k_dense_gemm<<<(unsigned)(dm.d / 256) * mshared, kDenseThreads, kDenseSmem, s>>>(st.g2s, az);
     }
     // convert
     {

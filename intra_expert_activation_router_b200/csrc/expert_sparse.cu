@@ -37,11 +37,11 @@
 //   MMA lane (warp 9)      per stage 8 MMAs (M 128, N 16, K 16) into one of
 //                          four TMEM accumulators; owns the TMEM allocation
 //   x warp (warp 10)       tile mode: token rows into the MMA's K-major
-//                          128-byte-swizzled layout (cp.async); resident
-//                          mode: a second gather warp
+//                          128-byte-swizzled layout (cp.async); idle in
+//                          resident mode
 //   gather warp (warp 11)  once an item's mask is final, the union-active
-//                          [up | down] records into a ring of buffers
-//                          (cp.async: off the TMA unit's queue)
+//                          [up | down] records into a ring of buffers, one
+//                          bulk copy per record
 //   up warps (0-3)         M(i): the accumulator (one neuron per thread),
 //                          silu, threshold, ballot per token, the union per
 //                          pass of MT tokens; then per gathered batch the up
@@ -55,6 +55,9 @@
 //                          to bf16 into `out` and re-zeroes it.
 // The agents meet on mbarriers (copies, MMA completion, buffer and h hand-off)
 // and on monotonic progress counters in shared memory; every wait is bounded.
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -80,6 +83,7 @@ constexpr int kIdRing = 16;          // published work-item ids
 constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
 constexpr int kMaxFusedPairs = 128;  // fused routing: (token, expert) pairs kept in shared memory
 constexpr int kMaxFusedLogits = 8192;   // fused routing: T * E logits staged in the gate ring
+constexpr int kMaxFusedExperts = 256;   // fused routing: rank counting costs E per logit
 // mbarriers besides the two rings': gdone, tfree (kAcc each), xfull, xfree,
 // mdrain, hsfull, hsfree (2 each)
 constexpr int kNumFixedBars = 2 * kAcc + 7;
@@ -99,6 +103,8 @@ struct ItemMeta {
     const uint16_t *wud;          // the expert's [f][2d] up/down records
     long long key;                // (expert slot or shared index, token tile)
     int m, blk, masked, nsub;
+    int sidx;                     // shared expert of the item, -1 for a routed expert
+    int part;                     // gate split: 0 owner (masks, projects), > 0 publishes partial sums only
     int tok[kMaxNT];
     int pair[kMaxNT];
     float w[kMaxNT];
@@ -120,12 +126,16 @@ struct SparseArgs {
     int resident;         // T <= nt: the whole batch is the MMA's token operand (x_tiles),
                           // and work items are claimed dynamically, heaviest expert first
     float tau;
+    float tau_shared;     // shared experts' threshold (masked forwards); <= 0: every shared neuron
     int use_mask;
+    int score_shared;     // score mode over the shared experts' neurons instead of the routed pairs'
     int n_tok_tiles;      // ceil(T / nt), for the shared experts
     int n_shared_items;   // S * n_tok_tiles * n_blk
     int max_touched;      // plan cache capacity
-    float *score_out;     // score mode: write |silu(g)| [pair][f], no up/down
+    float *score_out;     // score mode: write |silu(g)| [pair][f] (or [token][S][f]), no up/down
     int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
+    int gate_yield;       // resident mode: pause the gate stream while more records than this await projection (0: never)
+    int n_parts;          // gate split: parts per item (1: none); part 0, claimed last, owns the item
     int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
     const uint16_t *wr;   // fused: router weights [E][d]
     int E;
@@ -180,6 +190,20 @@ __device__ __forceinline__ ItemPos locate_item(const SparseArgs &a, const PlanCa
 __device__ __forceinline__ long long item_key(const ItemPos &p)
 {
     return ((long long)(p.slot < 0 ? p.slot : p.slot + 1) << 32) | (unsigned)p.tile;
+}
+
+// Gate split: claim id -> (item, part).  An item's parts are claimed in the
+// order n_parts - 1, ..., 1, 0, so the owner (part 0), which waits for the
+// others' partial sums, is always claimed after them: every wait points to an
+// earlier claim, which its CTA publishes before it reaches any later wait.
+__device__ __forceinline__ int split_item(const SparseArgs &a, int id) { return id / a.n_parts; }
+__device__ __forceinline__ int split_part(const SparseArgs &a, int id) { return a.n_parts - 1 - id % a.n_parts; }
+
+// Stages [lo, hi) of the item's spi gate stages that a part streams.
+__device__ __forceinline__ void part_stages(int spi, int n_parts, int part, int &lo, int &hi)
+{
+    lo = spi * part / n_parts;
+    hi = spi * (part + 1) / n_parts;
 }
 
 // Tokens of the item's tile: count, and where token r comes from.
@@ -312,41 +336,60 @@ __device__ __forceinline__ bool route_better(float v1, int i1, float v0, int i0)
 // temporaries.  Called by every thread of the CTA.
 __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scratch, int *s_prefix, int *s_expert,
                                              int *s_off, int *s_cnt, int *s_perm, int *s_perm_tok, float *s_perm_w,
-                                             volatile int *s_ntouched)
+                                             volatile int *s_ntouched, uint64_t *xbar)
 {
+    // written as short loops: this runs once per forward, so its code is
+    // fetched cold -- few instructions matter more than unrolled ones
     constexpr int NW = kSparseThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = a.T, E = a.E, k = a.k, d = a.d, d8 = d >> 3, P = T * k;
-    float *red = reinterpret_cast<float *>(scratch);                   // [NW][kMaxNT]
-    float *lg = reinterpret_cast<float *>(scratch + 1024);             // [T][E]
-    int *tk_idx = reinterpret_cast<int *>(lg + (size_t)T * E);          // [P]
-    float *tk_w = reinterpret_cast<float *>(tk_idx + P);                // [P]
-    int *ecnt = reinterpret_cast<int *>(tk_w + P);                      // [E]
-    int *ecur = ecnt + E;                                               // [E]
+    uint4 *xs = reinterpret_cast<uint4 *>(scratch);                  // [T][d8] the batch's rows
+    float *red = reinterpret_cast<float *>(xs + (size_t)T * d8);     // [NW][kMaxNT]
+    float *lg = red + NW * kMaxNT;                                    // [T][E]
+    int *tk_idx = reinterpret_cast<int *>(lg + (size_t)T * E);        // [P]
+    float *tk_w = reinterpret_cast<float *>(tk_idx + P);              // [P]
+    int *ecnt = reinterpret_cast<int *>(tk_w + P);                    // [E] pairs per expert
+    int *eoff = ecnt + E;                                             // [E] first position per expert
     Plan *plan = a.ws.plan;
-
     unsigned long long *tr = (a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
                                  ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
     if (tr && tid == 0) tr[44] = global_ns();
-    // 1. this CTA's experts' logits
+
+    // 1. this CTA's experts' logits (fp32 accumulation of bf16 products); the
+    //    batch's rows arrive by one bulk copy (x is [T][d], contiguous)
     int mine = 0;
-    for (int e = blockIdx.x; e < E; e += gridDim.x, ++mine) {
-        float acc[kMaxNT];
-#pragma unroll
-        for (int r = 0; r < kMaxNT; ++r) acc[r] = 0.f;
-        const uint16_t *wrow = a.wr + (size_t)e * d;
-        for (int v = tid; v < d8; v += kSparseThreads) {
-            const uint4 wv = ld_cached(wrow + 8 * v);
-#pragma unroll
-            for (int r = 0; r < kMaxNT; ++r)
-                if (r < T) acc[r] = dot8(wv, ld_cached(a.x + (size_t)r * d + 8 * v), acc[r]);
+    if ((int)blockIdx.x < E) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(xbar, (uint32_t)(T * d * 2));
+            bulk_g2s(xs, a.x, (uint32_t)(T * d * 2), xbar);
         }
-        const float val = transpose_reduce<kMaxNT>(acc, lane);   // lanes 2r, 2r + 1: token r
-        if ((lane & 1) == 0) red[warp * kMaxNT + (lane >> 1)] = val;
+        mbar_wait(xbar, 0, a.ws.error_word, 57);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int e = blockIdx.x; e < E; e += gridDim.x, ++mine) {
+        const uint16_t *wrow = a.wr + (size_t)e * d;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        const uint4 w0 = tid < d8 ? ld_cached(wrow + 8 * tid) : z;
+        const uint4 w1 = tid + kSparseThreads < d8 ? ld_cached(wrow + 8 * (tid + kSparseThreads)) : z;
+#pragma unroll 1
+        for (int t0 = 0; t0 < T; t0 += 4) {   // four tokens per transposed warp reduction
+            float acc[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                acc[u] = 0.f;
+                if (t0 + u < T) {
+                    if (tid < d8) acc[u] = dot8(w0, xs[(t0 + u) * d8 + tid], acc[u]);
+                    if (tid + kSparseThreads < d8) acc[u] = dot8(w1, xs[(t0 + u) * d8 + tid + kSparseThreads], acc[u]);
+                }
+            }
+            const float v = transpose_reduce<4>(acc, lane);   // lanes 8u .. 8u + 7: token t0 + u
+            if ((lane & 7) == 0 && t0 + (lane >> 3) < T) red[warp * kMaxNT + t0 + (lane >> 3)] = v;
+        }
         __syncthreads();
         if (tid < T) {
             float sum = 0.f;
-#pragma unroll
+#pragma unroll 1
             for (int w = 0; w < NW; ++w) sum += red[w * kMaxNT + tid];
             a.ws.logits[(size_t)tid * E + e] = sum;
             __threadfence();
@@ -371,101 +414,101 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
     }
     __syncthreads();
     if (tr && tid == 0) tr[59] = global_ns();
+#pragma unroll 4
     for (int i = tid; i < T * E; i += kSparseThreads) lg[i] = __ldcg(&a.ws.logits[i]);
+#pragma unroll 1
     for (int e = tid; e < E; e += kSparseThreads) ecnt[e] = 0;
+#pragma unroll 1
+    for (int p = tid; p < P; p += kSparseThreads) {   // valid defaults: only non-finite logits could
+        tk_idx[p] = 0;                                 // leave a rank unwritten
+        tk_w[p] = 0.f;
+    }
     __syncthreads();
     if (tr && tid == 0) tr[46] = global_ns();
-    for (int t = warp; t < T; t += NW) {
+#pragma unroll 1
+    for (int t = warp; t < T; t += NW) {   // each token's softmax max and sum (one warp per token)
         const float *row = lg + (size_t)t * E;
         float m = -INFINITY;
+#pragma unroll 1
         for (int j = lane; j < E; j += 32) m = fmaxf(m, row[j]);
         m = warp_max(m);
         float sum = 0.f;
+#pragma unroll 1
         for (int j = lane; j < E; j += 32) sum += expf(row[j] - m);
         sum = warp_sum(sum);
-        unsigned taken = 0;   // bit q: expert lane + 32 q already selected
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int q = 0, j = lane; j < E; ++q, j += 32) {
-                if (taken & (1u << q)) continue;
-                const float v = row[j];
-                if (bi == 0x7fffffff || route_better(v, j, bv, bi)) { bv = v; bi = j; }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(kFull, bv, o);
-                const int oi = __shfl_xor_sync(kFull, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || route_better(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-            }
-            bi = min(max(bi, 0), E - 1);   // only non-finite logits could leave it unset
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (lane == 0) {
-                tk_idx[t * k + r] = bi;
-                tk_w[t * k + r] = expf(bv - m) / sum;
-            }
+        if (lane == 0) {
+            red[2 * t] = m;
+            red[2 * t + 1] = sum;
+        }
+    }
+    __syncthreads();
+    // the rank of each logit within its token's row: the logits before it
+    // (larger, or equal with a lower index); ranks below k are the top_k, in
+    // rank order.  One (token, expert) pair per thread at a time.
+#pragma unroll 1
+    for (int i = tid; i < T * E; i += kSparseThreads) {
+        const int t = i / E, j = i - t * E;
+        const float *row = lg + (size_t)t * E;
+        const float v = row[j];
+        int rank = 0;
+#pragma unroll 4
+        for (int q = 0; q < E; ++q) rank += route_better(row[q], q, v, j) ? 1 : 0;
+        if (rank < k) {
+            tk_idx[t * k + rank] = j;
+            tk_w[t * k + rank] = expf(v - red[2 * t]) / red[2 * t + 1];
         }
     }
     __syncthreads();
     if (tr && tid == 0) tr[60] = global_ns();
-    // 3. the plan
-    for (int p = tid; p < P; p += kSparseThreads) atomicAdd(&ecnt[tk_idx[p]], 1);
+    // 3. the plan: counts, offsets and ascending touched list, stable permutation
+#pragma unroll 1
+    for (int p = tid; p < P; p += kSparseThreads) atomicAdd(&ecnt[min(max(tk_idx[p], 0), E - 1)], 1);
     __syncthreads();
     if (warp == 0) {
-        const int per = (E + 31) / 32;
-        const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-        int c_sum = 0, t_sum = 0;
-        for (int e = e0; e < e1; ++e) {
-            c_sum += ecnt[e];
-            t_sum += ecnt[e] > 0 ? 1 : 0;
-        }
-        int c_ex = c_sum, t_ex = t_sum;
+        int run_c = 0, run_t = 0;
+#pragma unroll 1
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = e < E ? ecnt[e] : 0, on = c > 0 ? 1 : 0;
+            int ic = c, it = on;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int c = __shfl_up_sync(kFull, c_ex, o), t = __shfl_up_sync(kFull, t_ex, o);
-            if (lane >= o) { c_ex += c; t_ex += t; }
-        }
-        c_ex -= c_sum;
-        t_ex -= t_sum;
-        for (int e = e0; e < e1; ++e) {
-            const int c = ecnt[e];
-            ecur[e] = c_ex;
-            if (c > 0) {
-                s_expert[t_ex] = e;
-                s_off[t_ex] = c_ex;
-                s_cnt[t_ex] = c;
-                s_prefix[t_ex] = t_ex * a.n_blk;
-                ++t_ex;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int uc = __shfl_up_sync(kFull, ic, o), ut = __shfl_up_sync(kFull, it, o);
+                if (lane >= o) { ic += uc; it += ut; }
             }
-            c_ex += c;
-        }
-        if (lane == 31) {
-            *s_ntouched = t_ex;
-            s_prefix[t_ex] = t_ex * a.n_blk;
-        }
-        __syncwarp();
-        // stable scatter, 32 pairs at a time in pair order
-        for (int base = 0; base < P; base += 32) {
-            const int p = base + lane;
-            const int e = p < P ? tk_idx[p] : -1 - lane;
-            const unsigned same = __match_any_sync(kFull, e);
-            const int rank = __popc(same & ((1u << lane) - 1u));
-            int pos = 0;
-            if (p < P) pos = ecur[e] + rank;
-            __syncwarp();
-            if (p < P && rank == 0) ecur[e] += __popc(same);
-            if (p < P) {
-                s_perm[pos] = p;
-                s_perm_tok[pos] = p / k;
-                s_perm_w[pos] = tk_w[p];
+            const int off = run_c + ic - c, slot = run_t + it - on;
+            if (e < E) eoff[e] = off;
+            if (on) {
+                s_expert[slot] = e;
+                s_off[slot] = off;
+                s_cnt[slot] = c;
+                s_prefix[slot] = slot * a.n_blk;
             }
-            __syncwarp();
+            run_c += __shfl_sync(kFull, ic, 31);
+            run_t += __shfl_sync(kFull, it, 31);
         }
+        if (lane == 0) {
+            *s_ntouched = run_t;
+            s_prefix[run_t] = run_t * a.n_blk;
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int p = tid; p < P; p += kSparseThreads) {   // pair p after the earlier pairs of its expert
+        const int e = min(max(tk_idx[p], 0), E - 1);
+        int r = 0;
+#pragma unroll 4
+        for (int q = 0; q < p; ++q) r += min(max(tk_idx[q], 0), E - 1) == e ? 1 : 0;
+        const int pos = eoff[e] + r;
+        s_perm[pos] = p;
+        s_perm_tok[pos] = p / k;
+        s_perm_w[pos] = tk_w[p];
     }
     __syncthreads();
     if (tr && tid == 0) tr[47] = global_ns();
     if (blockIdx.x == 0) {   // the workspace copy for statistics and debug calls
         const int n_t = *s_ntouched;
+#pragma unroll 1
         for (int p = tid; p < P; p += kSparseThreads) {
             a.ws.topk_idx[p] = tk_idx[p];
             a.ws.topk_w[p] = tk_w[p];
@@ -473,7 +516,9 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
             a.ws.perm_tok[p] = s_perm_tok[p];
             a.ws.perm_w[p] = s_perm_w[p];
         }
-        for (int e = tid; e < E; e += kSparseThreads) plan->offsets[e] = ecur[e] - ecnt[e];
+#pragma unroll 1
+        for (int e = tid; e < E; e += kSparseThreads) plan->offsets[e] = eoff[e];
+#pragma unroll 1
         for (int i = tid; i <= n_t; i += kSparseThreads) {
             if (i < n_t) plan->touched[i] = s_expert[i];
             plan->item_prefix[i] = s_prefix[i];
@@ -484,7 +529,7 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
             plan->n_routed_items = n_t * a.n_blk;
         }
     }
-    // the gate ring is written by the copy engine from here on
+    // the gate ring and gather buffers are written by the copy engine from here on
     fence_proxy_async_smem();
     __syncthreads();
 }
@@ -551,7 +596,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             mbar_init(&tfree[b], 4);
         }
         for (int b = 0; b < NU; ++b) {
-            mbar_init(&full_u[b], 32);   // one cp.async arrival per gather lane
+            mbar_init(&full_u[b], 1);   // the gather lane's expect_tx
             mbar_init(&empty_u[b], 1);
         }
         mbar_init(xfull, 1);
@@ -588,7 +633,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     volatile int *s_ntouched = reinterpret_cast<volatile int *>(smem + L.ctr_off + 56);
     int n_touched, n_routed_items;
     if (a.fused) {
-        route_in_kernel(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched);
+        route_in_kernel(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched,
+                        xfull);   // the token-tile barrier, unused in resident mode
         n_touched = *s_ntouched;
         n_routed_items = n_touched * a.n_blk;
     } else {
@@ -624,7 +670,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                        a.fused ? s_perm : a.ws.perm, a.fused ? s_perm_tok : a.ws.perm_tok,
                        a.fused ? s_perm_w : a.ws.perm_w};
 
-    const int n_items = a.n_shared_items + n_routed_items;
+    const int n_items = (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts;
     // static ranges (token-tile mode): contiguous items per CTA
     const int G = gridDim.x, b = blockIdx.x;
     const int per = n_items / G, rem = n_items % G;
@@ -651,15 +697,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     };
 
     // The gather: once an item's mask is final, its union-active records into
-    // the gather buffers, batch by batch, as 16-byte cp.async copies spread
-    // over a warp's 32 lanes (they take the load/store path and so do not
-    // queue behind the gate stream's bulk copies in the SM's TMA unit).  A
-    // warp's batch is handed over with cp.async.mbarrier.arrive, which in
-    // practice holds the warp's next copies back until its earlier ones have
-    // landed; so `owners` warps take turns, batch ub belonging to warp
-    // ub % owners, and that many batches are in flight.
+    // the gather buffers, batch by batch, one bulk copy per record (measured
+    // a little faster than 16-byte cp.async copies spread over the warps).
+    // `owners` gather warps may take turns, batch ub belonging to warp
+    // ub % owners; one warp is used.
     auto gather_loop = [&](int owner, int owners) {
-            const int rec_ck = (4 * d) / 16;   // 16-byte chunks per [up | down] record (4d bytes)
             uint32_t ub = 0, idle = 0;
             for (int ui = 0;;) {
                 int go = 0;
@@ -694,18 +736,24 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                         if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
                         ++nbatch;
                         uint8_t *dst = ud + (size_t)bi * L.ud_buf_bytes;
-                        for (int qq = 0; qq < nb; ++qq) {
-                            const size_t j = min(j0 + M.uni[s][b0 + qq], (size_t)a.f - 1);
-                            const uint16_t *src = M.wud + j * 2 * d;
-                            uint8_t *row = dst + (size_t)qq * L.gpitch;
-                            for (int cc = lane; cc < rec_ck; cc += 32) cp_async16(row + 16 * cc, src + 8 * cc, 16u);
+                        // one bulk copy of 4d bytes per record (both ends 16-byte aligned)
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&full_u[bi], (uint32_t)(nb * 4 * d));
+                            for (int qq = 0; qq < nb; ++qq) {
+                                const size_t j = min(j0 + M.uni[s][b0 + qq], (size_t)a.f - 1);
+                                bulk_g2s(dst + (size_t)qq * L.gpitch, M.wud + j * 2 * d, (uint32_t)(4 * d), &full_u[bi]);
+                            }
                         }
-                        cp_async_arrive_noinc(&full_u[bi]);   // one of the 32 expected arrivals
+                        __syncwarp();
                     }
                 }
                 ++ui;
             }
-            cp_async_wait_all();
+            // the last batch issued into each buffer has landed before the CTA may exit
+            if (lane == 0)
+                for (uint32_t b = ub > (uint32_t)NU ? ub - NU : 0; b < ub; ++b)
+                    if ((int)(b % (uint32_t)owners) == owner) mbar_drain(&full_u[b % NU], (b / NU) & 1);
+            __syncwarp();
     };
 
     if (warp == kWarpTma) {
@@ -755,10 +803,17 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 __threadfence_block();
                 *pub_items = i + 1;
                 if (id < 0) break;
-                const uint16_t *src = gate_src(locate_item(a, pc, id));
+                const uint16_t *src = gate_src(locate_item(a, pc, split_item(a, id)));
+                int s_lo, s_hi;
+                part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
                 bool ok = true;
-                for (int s = 0; s < spi; ++s, ++g) {
+                for (int s = s_lo; s < s_hi; ++s, ++g) {
                     const int slot = (int)(g % NS);
+                    // let the record gathers, the projections' critical path, use the
+                    // SM's memory bandwidth first while many records are pending
+                    for (uint32_t spin = 0; a.gate_yield > 0 && *rec_masked - *rec_done > a.gate_yield && spin < (1u << 14);
+                         ++spin)
+                        __nanosleep(128);
                     if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
                     if (tr && g < 4) tr[40 + g] = global_ns();
                     uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
@@ -795,8 +850,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int i = 0; ok; ++i) {
                 const int id = get_item(i);
                 if (id < 0) break;
-                const ItemPos p = locate_item(a, pc, id);
+                const ItemPos p = locate_item(a, pc, split_item(a, id));
                 const long long key = item_key(p);
+                int s_lo, s_hi;
+                part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
                 if (!a.resident && (i == 0 || key != prev_key)) {
                     ++q;
                     ok = mbar_wait(xfull, q & 1, err, 31);
@@ -805,7 +862,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 ok = ok && mbar_wait(&tfree[bsel], ((i / kAcc) & 1) ^ 1, err, 32);
                 tc_fence_after();
                 const uint32_t dt = tmem + 16 * bsel;
-                for (int s = 0; s < spi && ok; ++s, ++g) {
+                for (int s = s_lo; s < s_hi && ok; ++s, ++g) {
                     const int slot = (int)(g % NS);
                     ok = mbar_wait(&full_g[slot], (g / NS) & 1, err, 33);
                     tc_fence_after();
@@ -817,7 +874,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_bf16(dt, smem_desc_k_sw128(A + kb * kGateTile + 32 * kk),
-                                      smem_desc_k_sw128(B + kb * L.xt_kb + 32 * kk), idesc, (s | kb | kk) != 0 ? 1u : 0u);
+                                      smem_desc_k_sw128(B + kb * L.xt_kb + 32 * kk), idesc,
+                                      ((s - s_lo) | kb | kk) != 0 ? 1u : 0u);
                     umma_commit(&empty_g[slot]);   // the stage is free once these MMAs have read it
                 }
                 umma_commit(&gdone[bsel]);
@@ -854,7 +912,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         if (a.resident) {
             // the token operand streams with the gate tiles: this warp is the
             // second gather warp
-            if (!score_mode) gather_loop(1, 2);
+            // (the token operand streams with the gate stages: nothing to load here)
         } else {
             int q = -1;
             long long prev_key = 0;
@@ -878,7 +936,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         __syncwarp();
     } else if (warp == kWarpGather) {
         // ---------------------------------------------------------- gather warp
-        if (!score_mode) gather_loop(0, a.resident ? 2 : 1);
+        if (!score_mode) gather_loop(0, 1);
         __syncwarp();
     } else if (warp < 4) {
         // ------------------------------------------------ up warps: mask and up
@@ -895,7 +953,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         auto do_mask = [&](int i, int id) {
             ItemMeta &M = meta[i & 1];
-            const ItemPos p = locate_item(a, pc, id);
+            const int item = split_item(a, id), part = split_part(a, id);
+            const ItemPos p = locate_item(a, pc, item);
             int base;
             const int m = tile_tokens(a, pc, p, base);
             if (ct < m) {
@@ -912,14 +971,33 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 M.key = item_key(p);
                 M.m = m;
                 M.blk = p.blk;
-                M.masked = p.slot < 0 ? 0 : a.use_mask;
-                M.nsub = (m + MT - 1) / MT;
+                M.masked = part > 0 ? 0 : p.slot < 0 ? (a.use_mask && a.tau_shared > 0.f ? 1 : 0) : a.use_mask;
+                M.sidx = p.slot < 0 ? -1 - p.slot : -1;
+                M.part = part;
+                M.nsub = part > 0 ? 0 : (m + MT - 1) / MT;   // a non-owner part has no up/down work
                 M.wud = p.slot < 0 ? a.w.wsud + (size_t)(-1 - p.slot) * 2 * a.f * d
                                    : a.w.wud + (size_t)pc.expert[p.slot] * 2 * a.f * d;
             }
             consumer_sync(kUpThreads);
             unsigned long long *ti = (tr && i < 3) ? tr + 2 + 10 * i : nullptr;   // per-item stamps
             if (ti && ct == 0) ti[0] = global_ns();
+            // gate split: the item's partial sums, [part - 1][neuron][token]
+            float *gp = a.n_parts > 1 ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
+                                                          kSplitCols
+                                      : nullptr;
+            if (gp && part == 0) {   // the owner waits until the other parts have published theirs
+                if (ct == 0) {
+                    const int *cnt = a.ws.gcnt + min(item, a.ws.gcnt_n - 1);
+                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < a.n_parts - 1; ++spin) {
+                        if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                            atomicCAS(err, 0, 56);
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
+                consumer_sync(kUpThreads);
+            }
             if (warp < 4) {
                 const int bsel = i % kAcc;
                 mbar_wait(&gdone[bsel], (i / kAcc) & 1, err, 40);
@@ -930,24 +1008,39 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const int j = M.blk * kBlk + jl;
                 const bool jv = j < a.f;
                 const bool masked = M.masked != 0;
+                const float th = M.sidx >= 0 ? a.tau_shared : a.tau;
                 // a rolled loop over the tile's tokens: short code, one TMEM
                 // column each (the token's own column in resident mode)
 #pragma unroll 1
                 for (int t = 0; t < m; ++t) {
                     const int col = a.resident ? M.tok[t] : t;
-                    const float av = silu_f(tmem_ld1(taddr + col));
-                    const bool on = jv && (!masked || fabsf(av) >= a.tau);
+                    float g = tmem_ld1(taddr + col);
+                    if (gp) {
+                        const int c = min(col, kSplitCols - 1);
+                        if (part > 0) {   // publish this part's sum; no mask
+                            gp[((part - 1) * kBlk + jl) * kSplitCols + c] = g;
+                            continue;
+                        }
+                        for (int r = 1; r < a.n_parts; ++r) g += __ldcg(&gp[((r - 1) * kBlk + jl) * kSplitCols + c]);
+                    }
+                    const float av = silu_f(g);
+                    const bool on = jv && (!masked || fabsf(av) >= th);
                     const unsigned word = __ballot_sync(kFull, on);
                     M.a[t][jl] = f2bf_bits(av);
                     if (lane == 0) M.word[t][warp] = word;
-                    if (score_mode && jv) a.score_out[(size_t)M.pair[t] * a.f + j] = fabsf(av);
+                    if (score_mode && jv) {
+                        const size_t row = M.sidx >= 0 ? (size_t)M.tok[t] * a.S + M.sidx : (size_t)M.pair[t];
+                        a.score_out[row * a.f + j] = fabsf(av);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tfree[bsel]);   // the MMA may overwrite this accumulator
                 if (ti && ct == 0) ti[2] = ti[3] = global_ns();
             }
+            if (gp && part > 0) __threadfence();   // this thread's partial sums before the count
             consumer_sync(kUpThreads);
+            if (gp && part > 0 && ct == 0) atomicAdd(a.ws.gcnt + min(item, a.ws.gcnt_n - 1), 1);
             if (ti && ct == 0) ti[4] = global_ns();
             if (warp < M.nsub) {
                 // union of the pass's tokens, compacted in ascending neuron order
@@ -977,7 +1070,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             }
             // the pairs' mask words for statistics and the debug lists: written
             // after the publication, off the gather's critical path
-            if (M.masked && ct < m * 4) {
+            if (M.masked && M.sidx < 0 && ct < m * 4) {   // routed pairs only
                 const int t = ct >> 2, qw = ct & 3, chunk = M.blk * 4 + qw;
                 if (chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = M.word[t][qw];
             }
@@ -1017,7 +1110,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     if (tu && ct == 0 && s == 0 && b0 == 0) tu[6] = global_ns();
                     const uint8_t *buf = ud + (size_t)bi * L.ud_buf_bytes;
                     float *pw = part + (size_t)((hb * 4 + warp) * kMaxGB) * MT;
-                    if (L.gb <= 2)   // rows per reduction matched to the batch: no empty rows reduced
+                    // batches of at most two records (d_model >= 4096): rows per reduction
+                    // matched to the batch, no empty rows reduced
+                    if (NP >= 4 && L.gb <= 2)
                         group_rows<2, MT, NP>(buf, L.gpitch, nb, xf, d8, ct, lane, pw, 0);
                     else
                         for (int g0 = 0; g0 < nb; g0 += kRows)
@@ -1124,7 +1219,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 bool cont = false;
                 if (nsub == 1) {
                     const int nid = get_item(ii + 1);
-                    cont = nid >= 0 && item_key(locate_item(a, pc, nid)) == M.key;
+                    // (a non-owner part has no up/down work: stop accumulating there)
+                    cont = nid >= 0 && split_part(a, nid) == 0 &&
+                           item_key(locate_item(a, pc, split_item(a, nid))) == M.key;
                 }
                 if (!cont) {
 #pragma unroll
@@ -1173,7 +1270,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
 bool fused_possible(const Dims &dm, int T)
 {
     const SparseTiling t = sparse_tiling(T, dm.d);
-    return T <= t.nt && T * dm.k <= kMaxFusedPairs && T * dm.E <= kMaxFusedLogits && dm.d >= 64;
+    return T <= t.nt && T * dm.k <= kMaxFusedPairs && T * dm.E <= kMaxFusedLogits && dm.E <= kMaxFusedExperts &&
+           dm.d >= 64;
 }
 
 SparseTiling sparse_tiling(int T, int d)
@@ -1248,9 +1346,11 @@ static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_
 // sticky word and its own word cleared, so a later forward is not cut short.
 // With n4 = 0 it only does that.
 __global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4,
-                                               int *route_count, int *next_item, int *error_word, int *error_sticky)
+                                               int *route_count, int *next_item, int *error_word, int *error_sticky,
+                                               int *gcnt, int gcnt_n)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; gcnt && i < gcnt_n; i += gridDim.x * blockDim.x) gcnt[i] = 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *route_count = 0;
         *next_item = 0;
@@ -1286,7 +1386,7 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_y_out, y_acc, out, n4, ws.route_count, &ws.plan->next_item,
-                                       ws.error_word, ws.error_sticky);
+                                       ws.error_word, ws.error_sticky, ws.gcnt, ws.gcnt_n);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1316,7 +1416,7 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out, int inject, bool fused)
+                                 float *score_out, int inject, bool fused, float tau_shared, bool score_shared)
 {
     SparseArgs a;
     a.x = x;
@@ -1335,21 +1435,41 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.nt = til.nt;
     a.resident = T <= til.nt ? 1 : 0;
     a.tau = tau;
+    a.tau_shared = tau_shared;
+    a.score_shared = (score_out && score_shared) ? 1 : 0;
     a.use_mask = use_mask ? 1 : 0;
     a.score_out = score_out;
     a.inject = inject;
+    {   // MOE_GATE_YIELD=<records>: pause the gate stream while that many records await projection
+        const char *gy = std::getenv("MOE_GATE_YIELD");
+        a.gate_yield = gy ? (int)std::strtol(gy, nullptr, 10) : 0;
+    }
     a.fused = (fused && !score_out && fused_possible(dm, T)) ? 1 : 0;
     a.wr = w.wr;
     a.E = dm.E;
     a.max_pairs = a.fused ? T * dm.k : 0;
     if (a.fused && !encode(&a.xmap, x, dm.d, T, 2ull * dm.d, til.nt, true)) return cudaErrorInvalidValue;
     a.n_tok_tiles = (T + til.nt - 1) / til.nt;
-    a.n_shared_items = score_out ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
+    a.n_shared_items = (score_out && !a.score_shared) ? 0 : dm.S * a.n_tok_tiles * dm.n_blk;
     const int pairs = T * dm.k;
     a.max_touched = pairs < dm.E ? pairs : dm.E;
     if (!make_layout(dm.d, dm.dp, til, a.resident != 0, a.max_touched, a.max_pairs, a.L)) return cudaErrorInvalidValue;
     const int np = (dm.d / 8 + 127) / 128;
-    const long long bound = a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk;
+    // gate split: one- and two-token batches whose items are fewer than the SMs
+    // stream each item's gate on 2 or 4 CTAs (MOE_SPLIT=0 turns it off)
+    a.n_parts = 1;
+    {
+        const char *sp = std::getenv("MOE_SPLIT");
+        const long long base_max = a.n_shared_items + (long long)a.max_touched * dm.n_blk;
+        if (a.resident && !score_out && T <= kSplitCols && ws.gpart && ws.gcnt && base_max <= ws.gcnt_n &&
+            !(sp && std::strcmp(sp, "0") == 0))
+            for (int r = kMaxParts; r >= 2; r >>= 1)
+                if (base_max * r <= grid_cap && dm.n_kb / 2 >= r) {
+                    a.n_parts = r;
+                    break;
+                }
+    }
+    const long long bound = (a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk) * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
     if (grid < 1) grid = 1;
     cudaError_t e;

@@ -31,6 +31,8 @@ constexpr int kMaxExperts = 1024;
 constexpr int kChunk = 32;           // neurons per mask word
 constexpr int kBlk = 128;            // neurons per sparse work item (the gate MMA's M)
 constexpr int kDenseTileM = 128;     // tokens per dense GEMM tile
+constexpr int kSplitCols = 2;        // gate split: batches of at most this many tokens
+constexpr int kMaxParts = 4;         // gate split: parts per item
 
 // Routing plan written by the router's last CTA.
 struct Plan {
@@ -110,6 +112,15 @@ struct Workspace {
     // the plan's work-item counter it is zero when a forward starts (the
     // conversion kernel that ends every forward resets both)
     int *route_count;
+    int *cursor;        // [kMaxExperts] per-expert slots of the large-batch scatter
+    // gate split over several CTAs (batches of one or two tokens): partial gate
+    // sums of an item's non-owner parts [item][part - 1][128 neurons][2 tokens]
+    // and per item the count of parts published (zeroed by the conversion
+    // kernel that ends every forward); null when the layer's shape does not
+    // allow the split
+    float *gpart;
+    int *gcnt;
+    int gcnt_n;
     Plan *plan;
     // dense path
     uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts
@@ -162,7 +173,8 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out = nullptr, int inject = 0, bool fused = false);
+                                 float *score_out = nullptr, int inject = 0, bool fused = false,
+                                 float tau_shared = 0.f, bool score_shared = false);
 // Whether a sparse forward of T tokens can route inside the expert kernel.
 bool fused_possible(const Dims &dm, int T);
 // dst[b][c][col_off + r] = src[b][r][c] with row stride ld (elements).
@@ -191,7 +203,8 @@ bool encode(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, ui
 
 bool dense_supported(const Dims &dm);
 bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st);
+// tau_shared: the shared experts' threshold on a masked forward (<= 0: dense).
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
-                         float tau, bool use_mask, uint16_t *out, cudaStream_t s);
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared = 0.f);
 
 }  // namespace moe

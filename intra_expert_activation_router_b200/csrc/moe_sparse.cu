@@ -1,5 +1,6 @@
 // moe_sparse.cu -- the C ABI (include/moe_sparse.h): argument checking,
 // weight repacking, workspace ownership and path dispatch.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdlib>
@@ -55,6 +56,7 @@ struct moe_sparse_s {
     unsigned *hist;      // 256 bins, inside the workspace
     int inject_next;     // test-only fault for the next sparse forward (moe_debug_inject)
     int fused_router;    // route decode batches inside the expert kernel (moe_set_fused_router)
+    float tau_shared;    // the shared experts' threshold on masked forwards (moe_set_shared_tau)
     int last_fused;      // the last forward routed inside the expert kernel
 };
 
@@ -150,14 +152,20 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     const size_t wsbytes = 4 * T * E + 4 * P + 4 * P + 4 * P + 8 * P + 4 * P * (d_ff / 32) + 4 * T * d_model +
                            4 * T + 4 * ((T + 7) / 8) + 64 + sizeof(moe::Plan) + 2 * (P + T) * d_model +
                            2 * (P + n_shared * T) * d_ff + 2 * 2 * T * d_model + 32 * (size_t)dm.dp + 64 + 1024 +
-                           64 + 40 * 256;
+                           64 + 4 * moe::kMaxExperts + 40 * 256;
+    // gate split workspace (batches of one or two tokens): items of such a batch
+    // number at most (min(2k, E) + S) x blocks
+    const long long split_items = (long long)((2 * top_k < E ? 2 * top_k : E) + n_shared) * dm.n_blk;
+    const bool split_ok = split_items <= 4096;
+    const size_t part_floats = (size_t)(moe::kMaxParts - 1) * moe::kBlk * moe::kSplitCols;   // per item
+    const size_t split_bytes = split_ok ? (size_t)split_items * (part_floats * sizeof(float) + sizeof(int)) + 2 * 256 : 0;
     if (inject_alloc_fail("weights") || cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) {
         cudaGetLastError();
         h->weight_mem = nullptr;
         free_handle(h);
         return MOE_ENOMEM;
     }
-    if (inject_alloc_fail("workspace") || cudaMalloc(&h->ws_mem, wsbytes) != cudaSuccess) {
+    if (inject_alloc_fail("workspace") || cudaMalloc(&h->ws_mem, wsbytes + split_bytes) != cudaSuccess) {
         cudaGetLastError();
         h->ws_mem = nullptr;
         free_handle(h);
@@ -183,7 +191,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     }
     h->w = {wr, wg, wud, wsg, wsud, wdt, wsdt};
 
-    Block sb{(char *)h->ws_mem, 0, wsbytes};
+    Block sb{(char *)h->ws_mem, 0, wsbytes + split_bytes};
     moe::Workspace &ws = h->ws;
     ws.logits = (float *)sb.take(4 * T * E);
     ws.topk_idx = (int *)sb.take(4 * P);
@@ -199,6 +207,13 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.error_word = (int *)sb.take(4);
     ws.error_sticky = (int *)sb.take(4);
     ws.route_count = (int *)sb.take(4);
+    ws.cursor = (int *)sb.take(4 * moe::kMaxExperts);
+    if (split_ok) {
+        ws.gpart = (float *)sb.take((size_t)split_items * part_floats * sizeof(float));
+        ws.gcnt = (int *)sb.take((size_t)split_items * sizeof(int));
+        ws.gcnt_n = ws.gpart && ws.gcnt ? (int)split_items : 0;
+        if (!ws.gcnt_n) ws.gpart = nullptr, ws.gcnt = nullptr;
+    }
     ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
     ws.x_perm = (uint16_t *)sb.take(2 * (P + T) * d_model);
     ws.h_perm = (uint16_t *)sb.take(2 * (P + n_shared * T) * d_ff);
@@ -207,13 +222,13 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count) {
+    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count || !ws.cursor) {
         free_handle(h);
         return MOE_ENOMEM;
     }
 
     cudaStream_t st = nullptr;
-    bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes, st) == cudaSuccess;
+    bool ok = cudaMemsetAsync(h->ws_mem, 0, wsbytes + split_bytes, st) == cudaSuccess;
     ok = ok && cudaMemcpyAsync(wr, w->w_router, 2 * (size_t)E * d_model, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
     const int d = d_model;
     ok = ok && moe::launch_repack_gate_tiles((const uint16_t *)w->w_gate, wg, E, dm, st) == cudaSuccess;
@@ -294,13 +309,13 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
             e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
-                                          h->inject_next, fused);
+                                          h->inject_next, fused, h->tau_shared);
         h->inject_next = 0;
     } else {
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
-            e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st);
+            e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st, h->tau_shared);
     }
     if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[2], st, ev_flags);
     h->last_T = T;
@@ -355,6 +370,70 @@ extern "C" int moe_set_t_star(moe_handle h, int t_star)
     return MOE_OK;
 }
 
+extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau, int *t_star_out, void *stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!x || !t_star_out || T_max < 1 || T_max > h->dm.max_tokens || std::isnan(tau)) return MOE_EINVAL;
+    if (!aligned16(x)) return MOE_EALIGN;
+    if (!h->dense.ok) {   // no dense branch: AUTO always takes the sparse one
+        h->t_star = INT_MAX;
+        *t_star_out = INT_MAX;
+        return MOE_OK;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    int l2 = 0;
+    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, h->device) != cudaSuccess) return MOE_ECUDA;
+    const size_t flush_bytes = 2 * (size_t)(l2 > 0 ? l2 : (64 << 20));
+    void *flush = nullptr;
+    if (cudaMalloc(&flush, flush_bytes) != cudaSuccess) { cudaGetLastError(); return MOE_ENOMEM; }
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+        if (e0) cudaEventDestroy(e0);
+        cudaFree(flush);
+        return MOE_ECUDA;
+    }
+    const int saved_ev = h->n_ev;
+    h->n_ev = 0;   // the caller's launch events stay out of the tuning runs
+    // the median of five device-timed forwards of the first T rows of x, L2 flushed before each
+    auto time_path = [&](int T, int path, float *us) -> int {
+        float t[5];
+        for (int r = -1; r < 5; ++r) {   // one untimed run first
+            if (cudaMemsetAsync(flush, r & 0xff, flush_bytes, st) != cudaSuccess) return MOE_ECUDA;
+            if (cudaEventRecord(e0, st) != cudaSuccess) return MOE_ECUDA;
+            const int frc = run_forward(h, x, T, tau, true, h->ws.out_stage, stream, path);
+            if (frc) return frc;
+            if (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess) return MOE_ECUDA;
+            if (r >= 0 && cudaEventElapsedTime(&t[r], e0, e1) != cudaSuccess) return MOE_ECUDA;
+        }
+        std::sort(t, t + 5);
+        *us = 1000.f * t[2];
+        return MOE_OK;
+    };
+    // batch sizes 1, 2, 3, 4, 6, 8, 12, 16, 24, ... (steps of about 1.5x) up to T_max
+    int best = 0;
+    rc = MOE_OK;
+    for (int T = 1, last = 0; T <= T_max && rc == MOE_OK;) {
+        float us_s = 0.f, us_d = 0.f;
+        rc = time_path(T, MOE_PATH_SPARSE, &us_s);
+        if (rc == MOE_OK) rc = time_path(T, MOE_PATH_DENSE, &us_d);
+        if (rc != MOE_OK) break;
+        if (us_s > us_d) break;   // the dense branch is faster from here on
+        best = T;
+        last = T;
+        T = T < 4 ? T + 1 : (T % 3 == 0 ? T * 4 / 3 : T * 3 / 2);
+        if (T > T_max && last < T_max) T = T_max;
+    }
+    h->n_ev = saved_ev;
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    cudaFree(flush);
+    if (rc != MOE_OK) return rc;
+    h->t_star = best;
+    *t_star_out = best;
+    return MOE_OK;
+}
+
 extern "C" int moe_debug_router(moe_handle h, const void *x, int T, int *idx_out, float *w_out, void *stream)
 {
     int rc = check_handle(h);
@@ -383,20 +462,22 @@ extern "C" int moe_debug_active(moe_handle h, const void *x, int T, float tau, u
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
-extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
-                                 void *stream)
+// The floor(q N)-th smallest score of a population: the routed pairs' (N = T k
+// d_ff) or the shared experts' neurons (N = T S d_ff).
+static int calibrate(moe_handle h, const void *x, int T, double sparsity, float *tau_out, void *stream, bool shared)
 {
     int rc = check_handle(h);
     if (rc) return rc;
     if (!x || !tau_out || T < 1 || T > h->dm.max_tokens || std::isnan(sparsity)) return MOE_EINVAL;
+    if (shared && h->dm.S == 0) return MOE_EINVAL;
     if (!aligned16(x)) return MOE_EALIGN;
     const moe::Dims &dm = h->dm;
-    const size_t n = (size_t)T * dm.k * dm.f;
+    const size_t n = (size_t)T * (shared ? dm.S : dm.k) * dm.f;
     if (sparsity <= 0.0) { *tau_out = 0.0f; return MOE_OK; }
     const double kq = std::floor(sparsity * (double)n);
     if (kq >= (double)n) { *tau_out = INFINITY; return MOE_OK; }
     if (!h->scores) {
-        const size_t cap = (size_t)dm.max_tokens * dm.k * dm.f * sizeof(float);
+        const size_t cap = (size_t)dm.max_tokens * (dm.k > dm.S ? dm.k : dm.S) * dm.f * sizeof(float);
         if (inject_alloc_fail("scores") || cudaMalloc(&h->scores, cap) != cudaSuccess) {
             cudaGetLastError();
             h->scores = nullptr;
@@ -409,7 +490,7 @@ extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double spar
     cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, til.nt, st);
     if (e == cudaSuccess)
         e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, til, h->n_sm, st,
-                                      h->scores);
+                                      h->scores, 0, false, 0.0f, shared);
     // exact selection of the kq-th smallest, 8 bits per pass, most significant first
     unsigned long long want = (unsigned long long)kq;
     uint32_t prefix = 0, pmask = 0;
@@ -434,6 +515,26 @@ extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double spar
     float tau;
     std::memcpy(&tau, &prefix, sizeof tau);
     *tau_out = tau;
+    return MOE_OK;
+}
+
+extern "C" int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
+                                 void *stream)
+{
+    return calibrate(h, x, T, sparsity, tau_out, stream, false);
+}
+
+extern "C" int moe_calibrate_tau_shared(moe_handle h, const void *x, int T, double sparsity, float *tau_out,
+                                        void *stream)
+{
+    return calibrate(h, x, T, sparsity, tau_out, stream, true);
+}
+
+extern "C" int moe_set_shared_tau(moe_handle h, float tau_shared)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (std::isnan(tau_shared)) return MOE_EINVAL;
+    h->tau_shared = tau_shared;
     return MOE_OK;
 }
 

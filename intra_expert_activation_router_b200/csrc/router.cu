@@ -54,12 +54,12 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
     for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
     if (staged)
         for (int p = tid; p < P; p += blockDim.x) {
-            s_idx[p] = __ldcg(&a.ws.topk_idx[p]);
+            s_idx[p] = min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1);
             s_w[p] = __ldcg(&a.ws.topk_w[p]);
         }
     __syncthreads();
     for (int p = tid; p < P; p += blockDim.x)
-        atomicAdd(&s_cnt[staged ? s_idx[p] : __ldcg(&a.ws.topk_idx[p])], 1);
+        atomicAdd(&s_cnt[staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)], 1);
     __syncthreads();
     if (warp == 0) {
         // exclusive scans over experts: positions, touched slots, work items, dense tiles
@@ -107,10 +107,16 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
             plan->next_item = 0;
         }
         __syncwarp();
+        // large batches: the scatter is a kernel of its own (k_plan_scatter),
+        // one pair per thread through per-expert cursors, zeroed here
+        if (!staged) {
+            for (int e = lane; e < E; e += 32) a.ws.cursor[e] = 0;
+            return;
+        }
         // stable scatter, 32 pairs at a time in pair order
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
-            const int e = p < P ? (staged ? s_idx[p] : __ldcg(&a.ws.topk_idx[p])) : -1 - lane;
+            const int e = p < P ? (staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)) : -1 - lane;
             const unsigned same = __match_any_sync(kFull, e);
             const int rank = __popc(same & ((1u << lane) - 1));
             int pos = 0;
@@ -252,7 +258,14 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
         if (a.E <= kRankTopk) {
             // rank of each logit = number of logits ranked before it (larger, or
             // equal with a lower index); the ones with rank < k are the top-k,
-            // written straight to their rank -- no serial selection rounds
+            // written straight to their rank -- no serial selection rounds.
+            // Valid defaults first: only non-finite logits could leave a rank
+            // unwritten.
+            for (int r = lane; r < a.k; r += 32) {
+                a.ws.topk_idx[(size_t)t * a.k + r] = 0;
+                a.ws.topk_w[(size_t)t * a.k + r] = 0.f;
+            }
+            __syncwarp();
             for (int j = lane; j < a.E; j += 32) {
                 const float v = row[j];
                 int rank = 0;
@@ -311,6 +324,22 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     if (tr && threadIdx.x == 0) tr[5] = global_ns();
 }
 
+// The permutation of a large batch's pairs (more than kStagePairs): pair p goes
+// to its expert's first position plus a slot taken from the expert's cursor.
+// The order of an expert's pairs is then arbitrary, which changes neither
+// branch's result (rows are independent; the combine is a sum).
+__global__ void __launch_bounds__(256) k_plan_scatter(Workspace ws, int P, int k, int E)
+{
+    const Plan *plan = ws.plan;
+    for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
+        const int e = min(max(__ldcg(&ws.topk_idx[p]), 0), E - 1);
+        const int pos = min(__ldcg(&plan->offsets[e]) + atomicAdd(&ws.cursor[e], 1), P - 1);
+        ws.perm[pos] = p;
+        ws.perm_tok[pos] = p / k;
+        ws.perm_w[pos] = __ldcg(&ws.topk_w[p]);
+    }
+}
+
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                           const uint16_t *x, int T, int tile_tokens, cudaStream_t st)
 {
@@ -334,6 +363,12 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     if (plan_smem > smem) smem = plan_smem;
     // at most max(32 KB, 2*1024*4 + 8*4096 = 40 KB): inside the default 48 KB window
     k_router<<<grid, 256, smem, st>>>(a);
+    if ((long long)T * dm.k > kStagePairs) {
+        const int P = T * dm.k;
+        int blocks = (P + 255) / 256;
+        if (blocks > 148 * 8) blocks = 148 * 8;
+        k_plan_scatter<<<blocks, 256, 0, st>>>(ws, P, dm.k, dm.E);
+    }
     return cudaGetLastError();
 }
 

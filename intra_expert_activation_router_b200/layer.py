@@ -69,6 +69,20 @@ class MoESparseLayer:
     def set_t_star(self, t_star: int):
         B.moe_set_t_star(self.h, t_star)
 
+    def tune_t_star(self, x, tau: float, stream=None) -> int:
+        """Measure both branches on batches of x's first rows (up to all of x) and set T*."""
+        self._check_x(x)
+        return B.moe_tune_t_star(self.h, x, x.shape[0], float(tau), stream)
+
+    def set_shared_tau(self, tau_shared: float):
+        """The shared experts' own threshold on later masked forwards (<= 0: dense)."""
+        B.moe_set_shared_tau(self.h, float(tau_shared))
+
+    def calibrate_tau_shared(self, x, sparsity: float, stream=None) -> float:
+        """tau_shared keeping about 1 - sparsity of the shared experts' neurons of this batch."""
+        self._check_x(x)
+        return B.moe_calibrate_tau_shared(self.h, x, x.shape[0], sparsity, stream)
+
     def set_fused_router(self, enable: bool):
         B.moe_set_fused_router(self.h, 1 if enable else 0)
 

@@ -87,7 +87,7 @@ def check_active(ref, tau, idx_lists, cnt, tie):
     return flipped, int(band.sum()), gpu
 
 
-def expected_under_gpu_mask(o, inputs, top_k, tau, ref, gpu_mask, flipped, tie, nthreads=0):
+def expected_under_gpu_mask(o, inputs, top_k, tau, ref, gpu_mask, flipped, tie, nthreads=0, tau_shared=0.0):
     """The oracle's output per token, where a token whose band neuron the GPU
     decided the other way is evaluated under the GPU's mask instead."""
     y = ref.y.copy()
@@ -96,14 +96,14 @@ def expected_under_gpu_mask(o, inputs, top_k, tau, ref, gpu_mask, flipped, tie, 
         sub = dict(inputs)
         sub["x"] = inputs["x"][rows]
         r2 = o.forward(**sub, top_k=top_k, tau=tau, active=gpu_mask[rows], want_scores=True,
-                       nthreads=nthreads)
+                       nthreads=nthreads, tau_shared=tau_shared)
         assert np.array_equal(r2.topk_idx, ref.topk_idx[rows])
         y[rows] = r2.y
     return y
 
 
 def check_output_any_band_decision(o, inputs, top_k, tau, ref, out_gpu, tie, band_rel, max_band=8,
-                                   nthreads=0):
+                                   nthreads=0, tau_shared=0.0):
     """Output check for a path whose mask is not exported: a token with n
     neurons within band_rel*tau of tau must match the oracle under one of the
     2**n decisions of those neurons (all other neurons as the oracle decides).
@@ -128,7 +128,7 @@ def check_output_any_band_decision(o, inputs, top_k, tau, ref, out_gpu, tie, ban
             for b, (r, j) in enumerate(pos):
                 mask[0, r, j] = bool((combo >> b) & 1)
             yc = o.forward(**sub, top_k=top_k, tau=tau, active=mask, want_scores=False,
-                           nthreads=nthreads).y[0]
+                           nthreads=nthreads, tau_shared=tau_shared).y[0]
             nr = np.linalg.norm(yc)
             rel = np.linalg.norm(y[t] - yc) / nr if nr > 0 else (0.0 if not np.any(y[t]) else math.inf)
             best = min(best, rel)
@@ -160,3 +160,18 @@ def gpu_layer(shape, device="cuda", max_tokens=4096, weights=None):
     W = weights if weights is not None else mi.make_weights(shape, device=device)
     layer = MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max_tokens)
     return layer, W
+
+
+def threshold_off_scores(scores, q, eps=1e-4):
+    """A threshold near the q-quantile of `scores` that no score lies within
+    eps (relative) of: halfway between two neighbouring scores, so that fp32
+    and fp64 scores decide every neuron alike."""
+    s = np.sort(np.asarray(scores, dtype=np.float64).reshape(-1))
+    m = int(math.floor(q * s.size))
+    for delta in range(s.size):
+        for mm in (m + delta, m - delta):
+            if 1 <= mm < s.size:
+                tau = float(np.float32(0.5 * (s[mm - 1] + s[mm])))
+                if tau > 0 and not np.any(np.abs(s - tau) <= eps * tau):
+                    return tau
+    raise AssertionError("no threshold clear of the scores")

@@ -132,6 +132,27 @@ def test_auto_switch_picks_by_batch(o):
     layer.set_t_star(16)
 
 
+@pytest.mark.parametrize("name,q", [("olmoe", 0.9), ("dsv2lite", 0.9), ("large", 0.98)])
+def test_tuned_switch_point_selects_by_batch(o, name, q):
+    """moe_tune_t_star measures both branches on the device; AUTO then takes the
+    sparse branch up to the measured T* and the dense branch above it."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, 64, device="cuda")
+    tau = layer.calibrate_tau(x, q)
+    t_star = layer.tune_t_star(x, tau)
+    try:
+        assert 1 <= t_star <= 64, t_star
+        assert layer.stats()["t_star"] == t_star
+        for T in sorted({1, t_star, min(t_star + 1, 64), 64}):
+            layer.forward(x[:T].contiguous(), tau)
+            want = m.MOE_PATH_SPARSE if T <= t_star else m.MOE_PATH_DENSE
+            assert layer.stats()["path"] == want, (T, t_star)
+    finally:
+        layer.set_t_star(16)
+
+
 def test_dense_unsupported_shape_rejected():
     import intra_expert_activation_router_b200 as m
     sh = mi.custom_shape(264, 4, 32, 4, 0)   # d not a multiple of 256: no dense branch

@@ -186,6 +186,73 @@ def test_calibrate_tau_matches_oracle(o, name, T, qs):
     assert math.isinf(layer.calibrate_tau(x, 1.0))
 
 
+@pytest.mark.parametrize("name,T,q,q_s", [("dsv2lite", 8, 0.9, 0.5), ("dsv2lite", 32, 0.9, 0.8),
+                                          ("tiny", 16, 0.9, 0.5), ("large", 1, 0.98, 0.9)])
+def test_shared_threshold(o, name, T, q, q_s):
+    """The shared experts' own threshold (looser than the routed one): the
+    sparse branch (in-kernel routing at 8 and 16 tokens, token tiles at 32)
+    and the dense branch against the oracle with the same two thresholds."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    tau = pu.calibrate(o, inputs, sh.top_k, q, NTHREADS)
+    r0 = o.forward(**inputs, top_k=sh.top_k, tau=math.inf, nthreads=NTHREADS)
+    tau_s = pu.threshold_off_scores(r0.score_shared, q_s)
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=tau, tau_shared=tau_s, nthreads=NTHREADS)
+    kept = float(np.mean(r0.score_shared >= tau_s))
+    assert 0.0 < kept < 1.0
+    layer.set_shared_tau(tau_s)
+    try:
+        layer.set_path(m.MOE_PATH_SPARSE)
+        out = layer.forward(x, tau)
+        out_dbg = torch.empty_like(x)
+        lists, cnt = layer.active_lists(x, tau, out=out_dbg)
+        idx, w = layer.router(x)
+        torch.cuda.synchronize()
+        tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
+        flipped, _, gmask = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
+        y_expect = pu.expected_under_gpu_mask(o, inputs, sh.top_k, tau, ref, gmask, flipped, tie, NTHREADS, tau_s)
+        pu.check_output(y_expect, out, tie)
+        pu.check_output(y_expect, out_dbg, tie)
+        # the unmasked shared experts would give another layer: the threshold is applied
+        ref_dense_shared = o.forward(**inputs, top_k=sh.top_k, tau=tau, nthreads=NTHREADS, want_scores=False)
+        assert np.linalg.norm(ref_dense_shared.y - ref.y) > 0.05 * np.linalg.norm(ref.y)
+        layer.set_path(m.MOE_PATH_DENSE)
+        out_d = layer.forward(x, tau)
+        torch.cuda.synchronize()
+        pu.check_output_any_band_decision(o, inputs, sh.top_k, tau, ref, out_d, tie, 1e-5, nthreads=NTHREADS,
+                                          tau_shared=tau_s)
+    finally:
+        layer.set_shared_tau(0.0)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
+@pytest.mark.parametrize("name,T,qs", [("tiny", 16, (0.5, 0.9)), ("dsv2lite", 8, (0.5, 0.8, 0.95)),
+                                       ("large", 1, (0.5, 0.9))])
+def test_calibrate_tau_shared_matches_oracle(o, name, T, qs):
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    ref = o.forward(**inputs, top_k=sh.top_k, tau=math.inf, nthreads=NTHREADS)
+    s = np.sort(ref.score_shared.reshape(-1))
+    N = s.size
+    eps = 1e-4
+    for q in qs:
+        tau_g = layer.calibrate_tau_shared(x, q)
+        mq = int(math.floor(q * N))
+        lo, hi = tau_g * (1 - eps), tau_g * (1 + eps)
+        assert np.sum(s < lo) <= mq < np.sum(s <= hi), (q, tau_g, s[mq])
+        band = int(np.sum((s >= lo) & (s <= hi)))
+        assert abs(int(np.sum(s >= tau_g)) - (N - mq)) <= 1 + band
+    assert layer.calibrate_tau_shared(x, 0.0) == 0.0
+    assert math.isinf(layer.calibrate_tau_shared(x, 1.0))
+
+
 def test_gate_values_beyond_fp16_range(o):
     """|g| up to ~1e6, far above the fp16 range: the sparse path keeps silu(g)
     finite and matches the oracle (routed and shared experts)."""
