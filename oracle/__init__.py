@@ -70,6 +70,9 @@ class Oracle:
         c = self._lib.oracle_calibrate_tau
         c.restype = ctypes.c_double
         c.argtypes = [_P, ctypes.c_long, ctypes.c_double]
+        rm = self._lib.oracle_rank_mask
+        rm.restype = ctypes.c_int
+        rm.argtypes = [_P, ctypes.c_long, ctypes.c_int, ctypes.c_int, _P]
 
     @staticmethod
     def _ptr(a):
@@ -115,6 +118,34 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle_moe_forward failed ({rc})")
         return OracleResult(y, idx, w, lg, sc, ac, ssh)
+
+    def rank_mask(self, scores: np.ndarray, budget: int) -> np.ndarray:
+        """Per pair (the last axis holds one pair's f scores), 1 for the
+        ``budget`` largest scores compared in float, ties to the lower index,
+        NaN never kept; see ``oracle_rank_mask``."""
+        s = np.ascontiguousarray(scores, dtype=np.float64)
+        f = s.shape[-1]
+        out = np.zeros(s.shape, np.uint8)
+        rc = self._lib.oracle_rank_mask(self._ptr(s), s.size // f, f, int(budget), self._ptr(out))
+        if rc != 0:
+            raise RuntimeError(f"oracle_rank_mask failed ({rc})")
+        return out
+
+    def forward_budget(self, x, w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None,
+                       ws_down=None, *, top_k: int, budget: int, nthreads: int = 0,
+                       tau_shared: float = 0.0) -> OracleResult:
+        """The layer with a rank budget in place of the routed threshold: each
+        selected pair keeps its ``budget`` highest-scoring neurons
+        (``rank_mask`` of its scores); the shared experts keep their
+        ``tau_shared`` rule.  Composition of three oracle calls: the scores
+        (forward at tau = 0), the rank mask, the layer under that mask."""
+        args = (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+        first = self.forward(*args, top_k=top_k, tau=0.0, nthreads=nthreads, tau_shared=tau_shared)
+        mask = self.rank_mask(first.score, budget)
+        res = self.forward(*args, top_k=top_k, tau=0.0, nthreads=nthreads, active=mask,
+                           tau_shared=tau_shared)
+        res.score = first.score
+        return res
 
     def calibrate_tau(self, scores: np.ndarray, sparsity: float) -> float:
         """tau = the floor(q*N)-th smallest of the routed pairs' scores s = |silu(g)|.

@@ -217,3 +217,53 @@ double oracle_calibrate_tau(const double *s, long n, double q)
     free(c);
     return tau;
 }
+
+/* Rank budget per pair (technical summary, Methodology item 1: the
+ * lowest-scoring neurons of an expert are zeroed progressively, as an
+ * alternative to one threshold): of each pair's f scores keep the r largest.
+ * The scores are compared rounded to float, the precision the threshold is
+ * decided in; equal scores go to the lower neuron index; a NaN score is never
+ * kept (it ranks below every number), so a pair keeps min(r, its non-NaN
+ * scores) neurons.  The definition is written as a sort of the pair's
+ * (score, index) entries by score descending, index ascending, the first r
+ * entries being kept.
+ *   s     [n_pairs][f] scores (e.g. the `score` output above)
+ *   mask  [n_pairs][f] out: 1 kept, 0 not
+ * Returns 0, or -1 on bad sizes / allocation failure. */
+typedef struct {
+    double v;
+    int j;
+} rank_entry;
+
+static int cmp_rank(const void *pa, const void *pb)
+{
+    const rank_entry *a = (const rank_entry *)pa, *b = (const rank_entry *)pb;
+    const float va = (float)a->v, vb = (float)b->v;
+    if (va > vb) return -1;
+    if (va < vb) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+int oracle_rank_mask(const double *s, long n_pairs, int f, int r, uint8_t *mask)
+{
+    if (n_pairs < 0 || f < 1 || !s || !mask) return -1;
+    rank_entry *e = (rank_entry *)malloc(sizeof(rank_entry) * (size_t)f);
+    if (!e) return -1;
+    for (long p = 0; p < n_pairs; ++p) {
+        const double *sp = s + p * (long)f;
+        uint8_t *mp = mask + p * (long)f;
+        int n = 0;
+        for (int j = 0; j < f; ++j) {
+            mp[j] = 0;
+            if (sp[j] == sp[j]) {   /* not NaN */
+                e[n].v = sp[j];
+                e[n].j = j;
+                ++n;
+            }
+        }
+        qsort(e, (size_t)n, sizeof(rank_entry), cmp_rank);
+        for (int q = 0; q < n && q < r; ++q) mp[e[q].j] = 1;
+    }
+    free(e);
+    return 0;
+}

@@ -363,9 +363,118 @@ def pin_calibration(o):
     assert math.isinf(o._lib.oracle_calibrate_tau(o._ptr(s), s.size, 1.0))
 
 
+def _rank_brute(row, r):
+    """Scalar-Python rank rule: neuron j is kept iff fewer than r non-NaN
+    scores beat it, a score beating j when it is larger in float32, or equal
+    with a lower index; NaN is never kept and beats nobody."""
+    v = [np.float32(z) for z in row]
+    keep = []
+    for j, vj in enumerate(v):
+        if vj != vj:
+            keep.append(0)
+            continue
+        above = sum(1 for i, vi in enumerate(v) if vi == vi and (vi > vj or (vi == vj and i < j)))
+        keep.append(1 if above < r else 0)
+    return keep
+
+
+def pin_rank_bruteforce(o):
+    """The per-pair rank budget against a scalar enumeration of its rule, on
+    scores with exact ties, NaN, zeros, +inf and a pair that is distinct in
+    double but tied in float; the kept count is min(r, non-NaN) and budgets
+    nest."""
+    rng = np.random.default_rng(81)
+    f = 12
+    rows = [np.abs(rng.standard_normal(f)),
+            np.round(np.abs(rng.standard_normal(f)) * 2) / 2,     # many exact ties
+            np.zeros(f),                                        # all tied: lowest indices
+            np.array([1.0, math.nan, 0.5, 1.0, math.inf, 0.0, math.nan, 0.5, 2.0, 1.0, 0.25, 0.0]),
+            np.array([0.5] * 10 + [1.0, 1.0 + 1e-12])]           # float tie, double order reversed
+    s = np.array(rows)
+    prev = None
+    for r in range(0, f + 2):
+        m = o.rank_mask(s, r)
+        want = np.array([_rank_brute(row, r) for row in rows], np.uint8)
+        assert np.array_equal(m, want), ("rank mask", r, m.tolist(), want.tolist())
+        n_valid = (~np.isnan(s)).sum(axis=1)
+        assert np.array_equal(m.sum(axis=1), np.minimum(r, n_valid)), ("count", r)
+        if prev is not None:
+            assert np.all(prev <= m), ("nesting", r)
+        prev = m
+    assert o.rank_mask(s[4:5], 1)[0, 10] == 1   # 1.0 and 1.0+1e-12 tie in float: index 10 wins
+
+
+def pin_rank_layer(o):
+    """The layer under a rank budget: budget 0 is the shared-only layer (tau =
+    +inf), budget >= f the unmasked one (tau = 0); one pair with distinct
+    float scores equals the threshold layer at its r-th largest score; a zero
+    token keeps its r lowest neurons; a scalar-Python enumeration of the whole
+    layer at r = 3."""
+    d, E, f, k, S, T = 16, 4, 8, 2, 1, 3
+    x, W = _rand_layer(83, d, E, f, k, S, T, scale_x=1.0)
+    args = {n: _bits(t) for n, t in W.items()}
+    xb = _bits(x)
+    inf_ = _call(o, x, W, k, math.inf)
+    zero = _call(o, x, W, k, 0.0)
+    assert _rel(o.forward_budget(xb, **args, top_k=k, budget=0).y, inf_.y) < 1e-15
+    assert _rel(o.forward_budget(xb, **args, top_k=k, budget=f).y, zero.y) < 1e-15
+    assert _rel(o.forward_budget(xb, **args, top_k=k, budget=f + 5).y, zero.y) < 1e-15
+    # one token, one expert: the budget is the threshold at the r-th largest score
+    x1, W1 = _rand_layer(84, d, 4, 16, 1, 0, 1, scale_x=1.0)
+    a1 = {n: _bits(t) for n, t in W1.items()}
+    sc = _call(o, x1, W1, 1, 0.0).score.reshape(-1).astype(np.float32)
+    assert len(set(sc.tolist())) == sc.size
+    for r in (1, 5, 11):
+        tau = float(np.sort(sc)[::-1][r - 1])
+        rb = o.forward_budget(_bits(x1), **a1, top_k=1, budget=r)
+        rt = _call(o, x1, W1, 1, tau)
+        assert np.array_equal(rb.active, rt.active) and int(rb.active.sum()) == r, ("threshold", r)
+        assert _rel(rb.y, rt.y) < 1e-15
+    # a zero token: every score is 0, a tie broken toward the lower index
+    x0 = x.clone()
+    x0[1] = 0
+    r0 = o.forward_budget(_bits(x0), **args, top_k=k, budget=3)
+    assert np.array_equal(r0.active[1], np.array([[1, 1, 1, 0, 0, 0, 0, 0]] * k, np.uint8))
+    # scalar enumeration of the layer at r = 3
+    X = x.float().double().tolist()
+    Wr = W["w_router"].double().tolist()
+    Wg, Wu, Wd = (W["w_gate"].double().tolist(), W["w_up"].double().tolist(),
+                  W["w_down"].double().tolist())
+    Sg, Su, Sd = (W["ws_gate"].double().tolist(), W["ws_up"].double().tolist(),
+                  W["ws_down"].double().tolist())
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+
+    r = 3
+    y = [[0.0] * d for _ in range(T)]
+    for t in range(T):
+        lg = [sum(X[t][i] * Wr[e][i] for i in range(d)) for e in range(E)]
+        mx = max(lg)
+        ex = [math.exp(v - mx) for v in lg]
+        p = [v / sum(ex) for v in ex]
+        for e in sorted(range(E), key=lambda e: (-p[e], e))[:k]:
+            gs = [sum(X[t][i] * Wg[e][i][j] for i in range(d)) for j in range(f)]
+            keep = _rank_brute([abs(silu(g)) for g in gs], r)
+            for j in range(f):
+                if keep[j]:
+                    u = sum(X[t][i] * Wu[e][i][j] for i in range(d))
+                    for i in range(d):
+                        y[t][i] += p[e] * silu(gs[j]) * u * Wd[e][j][i]
+        for s_ in range(S):
+            for j in range(f):
+                g = sum(X[t][i] * Sg[s_][i][j] for i in range(d))
+                u = sum(X[t][i] * Su[s_][i][j] for i in range(d))
+                for i in range(d):
+                    y[t][i] += silu(g) * u * Sd[s_][j][i]
+    rb = o.forward_budget(xb, **args, top_k=k, budget=r)
+    assert _rel(rb.y, np.array(y)) < 1e-12, ("layer", _rel(rb.y, np.array(y)))
+    assert np.all(rb.active.sum(axis=2) == r)
+
+
 ALL_PINS = [pin_handworked, pin_tau0_is_dense, pin_tauinf_is_shared_only, pin_bruteforce,
             pin_mask_override, pin_shared_threshold, pin_nested_masks, pin_threshold_decomposition,
-            pin_router_ranking, pin_calibration]
+            pin_router_ranking, pin_calibration, pin_rank_bruteforce, pin_rank_layer]
 
 
 def run_all(o):

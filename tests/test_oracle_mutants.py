@@ -41,6 +41,13 @@ MUTANTS = [
     ("shared_mask_strict", "if (!((float)ss >= tau_shared)) continue;", "if (!((float)ss > tau_shared)) continue;"),
     ("shared_weighted", "for (int i = 0; i < d; ++i) yt[i] += h * bf16_to_double(down[(size_t)j * d + i]);",
      "for (int i = 0; i < d; ++i) yt[i] += 0.5 * h * bf16_to_double(down[(size_t)j * d + i]);"),
+    ("rank_tie_to_higher_index", "return (a->j > b->j) - (a->j < b->j);", "return (a->j < b->j) - (a->j > b->j);"),
+    ("rank_ascending", "if (va > vb) return -1;\n    if (va < vb) return 1;",
+     "if (va > vb) return 1;\n    if (va < vb) return -1;"),
+    ("rank_keeps_one_more", "for (int q = 0; q < n && q < r; ++q) mp[e[q].j] = 1;",
+     "for (int q = 0; q < n && q <= r; ++q) mp[e[q].j] = 1;"),
+    ("rank_keeps_nan", "if (sp[j] == sp[j]) {   /* not NaN */", "if (1) {"),
+    ("rank_in_double", "const float va = (float)a->v, vb = (float)b->v;", "const double va = a->v, vb = b->v;"),
 ]
 
 
