@@ -198,6 +198,24 @@ int moe_calibrate_tau(moe_handle h, const void *x, int T, double sparsity, float
  * count the shared experts in full. */
 int moe_set_shared_tau(moe_handle h, float tau_shared);
 
+/* A per-pair rank budget in place of the routed threshold ("Uncovering
+ * Intra-expert Activation Sparsity...", technical summary, Methodology item
+ * 1: the lowest-scoring neurons of an expert are zeroed progressively).  With
+ * r >= 0, later masked forwards (moe_sparse_forward, moe_debug_active) keep,
+ * for every routed (token, expert) pair, the r neurons with the largest
+ * s = |silu(g)| (fp32); equal scores go to the lower neuron index, a NaN score
+ * is never kept, so a pair keeps min(r, its non-NaN scores) neurons; `tau`
+ * is then unused for the routed experts, and the shared experts keep their
+ * moe_set_shared_tau rule.  r < 0 returns to the threshold (the default).
+ * The selection is exact and sort-free (a radix select of each pair's f
+ * scores).  The budget runs on the sparse path at every batch size: a forward
+ * forced onto the dense path (moe_set_path) returns MOE_ENOTSUP.  It costs
+ * two sparse passes (the routed gates, then the masked up/down reading the
+ * gates back) and one small selection kernel in between.  The first call with
+ * r >= 0 allocates max_tokens * top_k * (d_ff + 2) floats (MOE_ENOMEM if that
+ * fails, the setting unchanged); moe_sparse_destroy frees them. */
+int moe_set_rank_budget(moe_handle h, int r);
+
 /* As moe_calibrate_tau, over the N = T*n_shared*d_ff scores of the shared
  * experts' neurons: the floor(q*N)-th smallest |silu(x Ws_g)| (0-based, exact
  * selection); q <= 0 gives 0 and floor(q*N) >= N gives +inf.  MOE_EINVAL when
@@ -263,7 +281,13 @@ int moe_query_stats(moe_handle h, moe_stats *st);
  * Separately, when the environment variable MOE_INJECT_ALLOC_FAIL is
  * "weights" or "workspace", moe_sparse_create treats that device allocation
  * as failed (MOE_ENOMEM, nothing leaked); "scores" does the same for the
- * first moe_calibrate_tau's score buffer. */
+ * first moe_calibrate_tau's score buffer, "rank" for the first
+ * moe_set_rank_budget's buffers.
+ * Device error codes of the sparse kernel: 30-36 (copy, MMA and token-tile
+ * waits), 40-45 (the consumers' waits on accumulators, gathered records and
+ * the hand-off of h), 50-54 (waits for work items, slots and claims), 55
+ * (in-kernel routing: the other CTAs' logits), 56 (gate split: the other
+ * parts' sums), 57 (the combine at the end: the other CTAs' flushes). */
 #define MOE_INJECT_NONE 0
 #define MOE_INJECT_WITHHOLD_ITEMS 1
 int moe_debug_inject(moe_handle h, int kind);

@@ -134,12 +134,21 @@ struct SparseArgs {
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f] (or [token][S][f]), no up/down
     int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
-    int gate_yield;       // resident mode: pause the gate stream while more records than this await projection (0: never)
     int n_parts;          // gate split: parts per item (1: none); part 0, claimed last, owns the item
     int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
     const uint16_t *wr;   // fused: router weights [E][d]
     int E;
     int max_pairs;        // fused: T * k (permutation arrays kept in shared memory)
+    // rank budget, second pass: the routed pairs' silu(g) [pair][f] from the
+    // first pass (score mode, signed) and each pair's cut (v, J) -- neuron j
+    // is kept iff |silu(g_j)| > v, or == v and j <= J; routed items then
+    // stream no gate (the shared experts' items still do)
+    const float *a_in;
+    const float *rank_v;
+    const int *rank_j;
+    int score_signed;     // score mode: write silu(g) itself instead of |silu(g)|
+    int tail;             // combine here: y_acc -> bf16 `out` after a grid-wide arrival count
+    long long n_out4;     // float4 groups of y_acc converted (0 in score mode)
     SparseLayout L;
 };
 
@@ -534,6 +543,72 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
     __syncthreads();
 }
 
+// The combine, at the end of the kernel: every CTA has flushed its down sums
+// into y_acc (fp32 vector atomics, performed in L2) when the arrival count
+// reaches the grid; each CTA then converts its slice of y_acc to bf16 (round
+// to nearest even) into `out` and re-zeroes it.  The last CTA out resets the
+// forward's counters and moves the forward's error code into the sticky
+// word.  All CTAs of the grid are resident at once (one per SM, at most one
+// per SM), so the count completes; the wait is bounded all the same (code 57,
+// and that CTA's slice is left unconverted).
+__device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_flag)
+{
+    int *tail = a.ws.tail;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        atomicAdd(&tail[0], 1);
+        int ok = 1;
+        for (uint32_t spin = 0; ld_acquire_gpu(&tail[0]) < (int)gridDim.x; ++spin) {
+            if (spin > kSpinLimit) {
+                atomicCAS(a.ws.error_word, 0, 57);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        *s_flag = ok;
+    }
+    __syncthreads();
+    if (*s_flag) {
+        const float4 *src = reinterpret_cast<const float4 *>(a.ws.y_acc);
+        float4 *zero = reinterpret_cast<float4 *>(a.ws.y_acc);
+        uint2 *dst = reinterpret_cast<uint2 *>(a.out);
+#pragma unroll 1
+        for (long long i = (long long)blockIdx.x * kSparseThreads + tid; i < a.n_out4;
+             i += (long long)gridDim.x * kSparseThreads) {
+            const float4 v = __ldcg(src + i);
+            uint2 p;
+            p.x = (uint32_t)f2bf_bits(v.x) | ((uint32_t)f2bf_bits(v.y) << 16);
+            p.y = (uint32_t)f2bf_bits(v.z) | ((uint32_t)f2bf_bits(v.w) << 16);
+            dst[i] = p;
+            __stcg(zero + i, make_float4(0.f, 0.f, 0.f, 0.f));
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        *s_flag = atomicAdd(&tail[1], 1) == (int)gridDim.x - 1;
+        __threadfence();
+    }
+    __syncthreads();
+    if (*s_flag) {   // last CTA out: every CTA is past every use of the counters
+#pragma unroll 1
+        for (int i = tid; a.ws.gcnt && i < a.ws.gcnt_n; i += kSparseThreads) a.ws.gcnt[i] = 0;
+        if (tid == 0) {
+            *a.ws.route_count = 0;
+            a.ws.plan->next_item = 0;
+            const int e0 = *reinterpret_cast<volatile int *>(a.ws.error_word);
+            if (e0 != 0) {
+                atomicCAS(a.ws.error_sticky, 0, e0);
+                *a.ws.error_word = 0;
+            }
+            tail[0] = 0;
+            tail[1] = 0;
+        }
+    }
+}
+
 template <int MT, int NP>
 __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
 {
@@ -562,6 +637,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     volatile int *rec_masked = reinterpret_cast<volatile int *>(smem + L.ctr_off + 36);
     volatile int *rec_done = reinterpret_cast<volatile int *>(smem + L.ctr_off + 40);
     volatile int *s_items = reinterpret_cast<volatile int *>(smem + L.ctr_off + 64);   // [kIdRing]
+    int *s_tail_flag = reinterpret_cast<int *>(smem + L.ctr_off + 20);
     int *s_prefix = reinterpret_cast<int *>(smem + L.plan_off);
     int *s_expert = s_prefix + a.max_touched + 1;
     int *s_off = s_expert + a.max_touched;
@@ -803,17 +879,14 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 __threadfence_block();
                 *pub_items = i + 1;
                 if (id < 0) break;
-                const uint16_t *src = gate_src(locate_item(a, pc, split_item(a, id)));
+                const ItemPos ip = locate_item(a, pc, split_item(a, id));
+                const uint16_t *src = gate_src(ip);
                 int s_lo, s_hi;
                 part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
+                if (a.a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
                 for (int s = s_lo; s < s_hi; ++s, ++g) {
                     const int slot = (int)(g % NS);
-                    // let the record gathers, the projections' critical path, use the
-                    // SM's memory bandwidth first while many records are pending
-                    for (uint32_t spin = 0; a.gate_yield > 0 && *rec_masked - *rec_done > a.gate_yield && spin < (1u << 14);
-                         ++spin)
-                        __nanosleep(128);
                     if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
                     if (tr && g < 4) tr[40 + g] = global_ns();
                     uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
@@ -854,6 +927,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const long long key = item_key(p);
                 int s_lo, s_hi;
                 part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
+                const bool skip = a.a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
+                if (skip) s_hi = s_lo;
                 if (!a.resident && (i == 0 || key != prev_key)) {
                     ++q;
                     ok = mbar_wait(xfull, q & 1, err, 31);
@@ -878,7 +953,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                                       ((s - s_lo) | kb | kk) != 0 ? 1u : 0u);
                     umma_commit(&empty_g[slot]);   // the stage is free once these MMAs have read it
                 }
-                umma_commit(&gdone[bsel]);
+                if (skip)
+                    mbar_arrive(&gdone[bsel]);
+                else
+                    umma_commit(&gdone[bsel]);
                 if (tr && i == 0) tr[57] = global_ns();
                 if (!a.resident) {   // static ranges: the next id is first + i + 1
                     const bool last_of_tile =
@@ -1009,28 +1087,40 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const bool jv = j < a.f;
                 const bool masked = M.masked != 0;
                 const float th = M.sidx >= 0 ? a.tau_shared : a.tau;
+                const bool from_a = a.a_in && M.sidx < 0;   // rank pass: silu(g) and the cut from global
                 // a rolled loop over the tile's tokens: short code, one TMEM
                 // column each (the token's own column in resident mode)
 #pragma unroll 1
                 for (int t = 0; t < m; ++t) {
-                    const int col = a.resident ? M.tok[t] : t;
-                    float g = tmem_ld1(taddr + col);
-                    if (gp) {
-                        const int c = min(col, kSplitCols - 1);
-                        if (part > 0) {   // publish this part's sum; no mask
-                            gp[((part - 1) * kBlk + jl) * kSplitCols + c] = g;
-                            continue;
+                    float av;
+                    bool keep;
+                    if (from_a) {
+                        const int pr = M.pair[t];
+                        av = jv ? __ldcg(&a.a_in[(size_t)pr * a.f + j]) : 0.f;
+                        const float sv = fabsf(av), cv = __ldcg(&a.rank_v[pr]);
+                        keep = sv > cv || (sv == cv && j <= __ldcg(&a.rank_j[pr]));
+                    } else {
+                        const int col = a.resident ? M.tok[t] : t;
+                        float g = tmem_ld1(taddr + col);
+                        if (gp) {
+                            const int c = min(col, kSplitCols - 1);
+                            if (part > 0) {   // publish this part's sum; no mask
+                                gp[((part - 1) * kBlk + jl) * kSplitCols + c] = g;
+                                continue;
+                            }
+                            for (int r = 1; r < a.n_parts; ++r)
+                                g += __ldcg(&gp[((r - 1) * kBlk + jl) * kSplitCols + c]);
                         }
-                        for (int r = 1; r < a.n_parts; ++r) g += __ldcg(&gp[((r - 1) * kBlk + jl) * kSplitCols + c]);
+                        av = silu_f(g);
+                        keep = fabsf(av) >= th;
                     }
-                    const float av = silu_f(g);
-                    const bool on = jv && (!masked || fabsf(av) >= th);
+                    const bool on = jv && (!masked || keep);
                     const unsigned word = __ballot_sync(kFull, on);
                     M.a[t][jl] = f2bf_bits(av);
                     if (lane == 0) M.word[t][warp] = word;
                     if (score_mode && jv) {
                         const size_t row = M.sidx >= 0 ? (size_t)M.tok[t] * a.S + M.sidx : (size_t)M.pair[t];
-                        a.score_out[row * a.f + j] = fabsf(av);
+                        a.score_out[row * a.f + j] = a.score_signed ? av : fabsf(av);
                     }
                 }
                 tc_fence_before();
@@ -1262,6 +1352,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         tmem_dealloc(tmem, kTmemCols);
     }
     if (tr && tid == 0) tr[62] = global_ns();
+    if (a.tail) combine_tail(a, tid, s_tail_flag);
 }
 
 // Routing inside the expert kernel needs: the batch as one token tile
@@ -1416,8 +1507,10 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
-                                 float *score_out, int inject, bool fused, float tau_shared, bool score_shared)
+                                 float *score_out, int inject, bool fused, float tau_shared, bool score_shared,
+                                 const RankPass *rank)
 {
+    if (rank && !rank->second) score_out = rank->a;   // first pass: signed silu(g) of the routed pairs
     SparseArgs a;
     a.x = x;
     a.out = out;
@@ -1440,11 +1533,12 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.use_mask = use_mask ? 1 : 0;
     a.score_out = score_out;
     a.inject = inject;
-    {   // MOE_GATE_YIELD=<records>: pause the gate stream while that many records await projection
-        const char *gy = std::getenv("MOE_GATE_YIELD");
-        a.gate_yield = gy ? (int)std::strtol(gy, nullptr, 10) : 0;
-    }
-    a.fused = (fused && !score_out && fused_possible(dm, T)) ? 1 : 0;
+    a.score_signed = (rank && !rank->second) ? 1 : 0;
+    a.a_in = (rank && rank->second) ? rank->a : nullptr;
+    a.rank_v = a.a_in ? rank->v : nullptr;
+    a.rank_j = a.a_in ? rank->j : nullptr;
+    // the rank passes use the router's plan (the second pass must see the first one's pairs)
+    a.fused = (fused && !score_out && !rank && fused_possible(dm, T)) ? 1 : 0;
     a.wr = w.wr;
     a.E = dm.E;
     a.max_pairs = a.fused ? T * dm.k : 0;
@@ -1461,7 +1555,7 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     {
         const char *sp = std::getenv("MOE_SPLIT");
         const long long base_max = a.n_shared_items + (long long)a.max_touched * dm.n_blk;
-        if (a.resident && !score_out && T <= kSplitCols && ws.gpart && ws.gcnt && base_max <= ws.gcnt_n &&
+        if (a.resident && !score_out && !a.a_in && T <= kSplitCols && ws.gpart && ws.gcnt && base_max <= ws.gcnt_n &&
             !(sp && std::strcmp(sp, "0") == 0))
             for (int r = kMaxParts; r >= 2; r >>= 1)
                 if (base_max * r <= grid_cap && dm.n_kb / 2 >= r) {
@@ -1471,6 +1565,12 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     }
     const long long bound = (a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk) * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
+    // the combine at the end of the kernel (MOE_TAIL=0: a separate conversion kernel)
+    {
+        const char *tv = std::getenv("MOE_TAIL");
+        a.tail = (tv && std::strcmp(tv, "0") == 0) ? 0 : 1;
+        a.n_out4 = score_out ? 0 : (long long)T * dm.d / 4;
+    }
     if (grid < 1) grid = 1;
     cudaError_t e;
     switch (np * 8 + til.mt) {
@@ -1485,6 +1585,7 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
+    if (a.tail) return cudaSuccess;
     // score mode writes no output: only the counters are reset
     return launch_y_out(ws.y_acc, out, score_out ? 0 : (size_t)T * dm.d / 4, grid_cap, ws, st);
 }

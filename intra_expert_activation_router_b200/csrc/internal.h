@@ -112,6 +112,10 @@ struct Workspace {
     // the plan's work-item counter it is zero when a forward starts (the
     // conversion kernel that ends every forward resets both)
     int *route_count;
+    // the sparse kernel's combine: [0] CTAs whose down flushes have landed,
+    // [1] CTAs done converting; the last CTA out resets both (and the
+    // counters above), so they are zero when a forward starts
+    int *tail;
     int *cursor;        // [kMaxExperts] per-expert slots of the large-batch scatter
     // gate split over several CTAs (batches of one or two tokens): partial gate
     // sums of an item's non-owner parts [item][part - 1][128 neurons][2 tokens]
@@ -170,11 +174,24 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
 // no work item, so the consumers' bounded waits run out), 0 otherwise.
 // fused: the kernel routes the batch itself (no router launch before it);
 // only when fused_possible() holds.  *fused_used reports whether it did.
+// The rank budget's two sparse passes: the first (score mode, signed) writes
+// silu(g) of every routed pair into `a`; the second reads it back with each
+// pair's cut instead of recomputing the routed gates.
+struct RankPass {
+    float *a;          // [pairs][f] silu(g)
+    const float *v;    // [pairs] cut value (second pass)
+    const int *j;      // [pairs] last tied index kept (second pass)
+    bool second;
+};
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
                                  float *score_out = nullptr, int inject = 0, bool fused = false,
-                                 float tau_shared = 0.f, bool score_shared = false);
+                                 float tau_shared = 0.f, bool score_shared = false, const RankPass *rank = nullptr);
+// Per pair of a [pairs][f] silu(g) buffer, the cut (v, J) keeping its r
+// highest |silu(g)| (ties to the lower index, NaN never): neuron j is kept iff
+// |silu(g_j)| > v, or == v and j <= J.
+cudaError_t launch_rank_select(const float *a, int pairs, int f, int r, float *v_out, int *j_out, cudaStream_t st);
 // Whether a sparse forward of T tokens can route inside the expert kernel.
 bool fused_possible(const Dims &dm, int T);
 // dst[b][c][col_off + r] = src[b][r][c] with row stride ld (elements).

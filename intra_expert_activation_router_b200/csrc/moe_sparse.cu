@@ -58,12 +58,18 @@ struct moe_sparse_s {
     int fused_router;    // route decode batches inside the expert kernel (moe_set_fused_router)
     float tau_shared;    // the shared experts' threshold on masked forwards (moe_set_shared_tau)
     int last_fused;      // the last forward routed inside the expert kernel
+    // rank budget (moe_set_rank_budget): < 0 off; else each routed pair keeps
+    // its rank_r highest-scoring neurons on masked forwards
+    int rank_r;
+    float *rank_a;       // [max_tokens * k][f] silu(g) of the first pass
+    float *rank_v;       // [max_tokens * k] cut values
+    int *rank_j;         // [max_tokens * k] last tied index kept
 };
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Host-side fault injection for tests: MOE_INJECT_ALLOC_FAIL=<what> makes the
-// named device allocation ("weights", "workspace" or "scores") report failure
+// named device allocation ("weights", "workspace", "scores" or "rank") report failure
 // without being attempted, so the error paths can be exercised on a live GPU.
 static bool inject_alloc_fail(const char *what)
 {
@@ -102,6 +108,7 @@ static void free_handle(moe_handle h)
     if (h->weight_mem) cudaFree(h->weight_mem);
     if (h->ws_mem) cudaFree(h->ws_mem);
     if (h->scores) cudaFree(h->scores);
+    if (h->rank_a) cudaFree(h->rank_a);
     h->magic = 0;
     delete h;
 }
@@ -207,6 +214,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.error_word = (int *)sb.take(4);
     ws.error_sticky = (int *)sb.take(4);
     ws.route_count = (int *)sb.take(4);
+    ws.tail = (int *)sb.take(8);
     ws.cursor = (int *)sb.take(4 * moe::kMaxExperts);
     if (split_ok) {
         ws.gpart = (float *)sb.take((size_t)split_items * part_floats * sizeof(float));
@@ -222,7 +230,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count || !ws.cursor) {
+    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count || !ws.tail || !ws.cursor) {
         free_handle(h);
         return MOE_ENOMEM;
     }
@@ -255,6 +263,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
         return MOE_ECUDA;
     }
     h->fused_router = 1;
+    h->rank_r = -1;
     h->last_T = 0;
     h->last_path = MOE_PATH_SPARSE;
     h->last_masked = 1;
@@ -286,6 +295,12 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     int path = forced_path;
     if (path == MOE_PATH_AUTO) path = h->path;
     if (path == MOE_PATH_AUTO) path = (T <= h->t_star) ? MOE_PATH_SPARSE : MOE_PATH_DENSE;
+    const bool rank = masked && h->rank_r >= 0;
+    if (rank) {   // the rank budget is built on the sparse path only
+        if (forced_path == MOE_PATH_DENSE || (forced_path == MOE_PATH_AUTO && h->path == MOE_PATH_DENSE))
+            return MOE_ENOTSUP;
+        path = MOE_PATH_SPARSE;
+    }
     if (path == MOE_PATH_DENSE && !h->dense.ok) {
         if (forced_path == MOE_PATH_DENSE || h->path == MOE_PATH_DENSE) return MOE_ENOTSUP;
         path = MOE_PATH_SPARSE;   // AUTO on a shape the dense branch does not cover
@@ -304,12 +319,24 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     if (path == MOE_PATH_SPARSE) {
         const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
         // decode batches route inside the expert kernel: no router launch
-        fused = h->fused_router && moe::fused_possible(h->dm, T);
+        fused = !rank && h->fused_router && moe::fused_possible(h->dm, T);
         if (e == cudaSuccess && !fused) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
-        if (e == cudaSuccess)
+        if (rank) {   // silu(g) of the routed pairs, each pair's cut, then the masked layer
+            moe::RankPass r1{h->rank_a, nullptr, nullptr, false};
+            moe::RankPass r2{h->rank_a, h->rank_v, h->rank_j, true};
+            if (e == cudaSuccess)
+                e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
+                                              0, false, h->tau_shared, false, &r1);
+            if (e == cudaSuccess)
+                e = moe::launch_rank_select(h->rank_a, T * h->dm.k, h->dm.f, h->rank_r, h->rank_v, h->rank_j, st);
+            if (e == cudaSuccess)
+                e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
+                                              h->inject_next, false, h->tau_shared, false, &r2);
+        } else if (e == cudaSuccess) {
             e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
                                           h->inject_next, fused, h->tau_shared);
+        }
         h->inject_next = 0;
     } else {
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
@@ -535,6 +562,26 @@ extern "C" int moe_set_shared_tau(moe_handle h, float tau_shared)
     if (!is_live(h)) return MOE_EHANDLE;
     if (std::isnan(tau_shared)) return MOE_EINVAL;
     h->tau_shared = tau_shared;
+    return MOE_OK;
+}
+
+extern "C" int moe_set_rank_budget(moe_handle h, int r)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (r >= 0 && !h->rank_a) {
+        const size_t pairs = (size_t)h->dm.max_tokens * h->dm.k;
+        const size_t bytes = pairs * h->dm.f * sizeof(float) + 2 * ((pairs * 4 + 255) & ~size_t(255));
+        void *mem = nullptr;
+        if (inject_alloc_fail("rank") || cudaMalloc(&mem, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ENOMEM;
+        }
+        h->rank_a = (float *)mem;
+        uint8_t *tail = (uint8_t *)mem + pairs * h->dm.f * sizeof(float);
+        h->rank_v = (float *)tail;
+        h->rank_j = (int *)(tail + ((pairs * 4 + 255) & ~size_t(255)));
+    }
+    h->rank_r = r < 0 ? -1 : r;
     return MOE_OK;
 }
 

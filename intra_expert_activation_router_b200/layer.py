@@ -78,6 +78,11 @@ class MoESparseLayer:
         """The shared experts' own threshold on later masked forwards (<= 0: dense)."""
         B.moe_set_shared_tau(self.h, float(tau_shared))
 
+    def set_rank_budget(self, r: int):
+        """Keep each routed pair's r highest-scoring neurons on later masked
+        forwards instead of thresholding at tau (r < 0: back to the threshold)."""
+        B.moe_set_rank_budget(self.h, int(r))
+
     def calibrate_tau_shared(self, x, sparsity: float, stream=None) -> float:
         """tau_shared keeping about 1 - sparsity of the shared experts' neurons of this batch."""
         self._check_x(x)

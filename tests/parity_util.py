@@ -87,6 +87,44 @@ def check_active(ref, tau, idx_lists, cnt, tie):
     return flipped, int(band.sum()), gpu
 
 
+def gpu_mask_from_lists(idx_lists, cnt, f):
+    """[T][k][f] bool from the ascending active lists (first cnt valid)."""
+    T, k = cnt.shape
+    gpu = np.zeros((T, k, f), bool)
+    for t in range(T):
+        for r in range(k):
+            c = int(cnt[t, r])
+            lst = idx_lists[t, r, :c].astype(np.int64)
+            assert np.all(np.diff(lst) > 0), f"list not ascending at ({t},{r})"
+            gpu[t, r, lst] = True
+    return gpu
+
+
+def check_rank_mask(o, scores, budget, gpu_mask, tie, band_rel=BAND_REL):
+    """The CUDA path's per-pair rank selection against the oracle's scores.
+
+    Exact: every pair keeps min(budget, f) neurons (the inputs hold no NaN).
+    Valid: no kept neuron scores (oracle, rounded to float) below a dropped one
+    by more than band_rel of the larger; the GPU's fp32 g may order two
+    neurons that close the other way.  Returns (tokens whose selection differs
+    from the oracle's rank mask, the oracle's rank mask)."""
+    T, k, f = scores.shape
+    want = o.rank_mask(scores, budget).astype(bool)
+    cnt = gpu_mask.sum(axis=2)
+    assert np.all(cnt[~tie] == min(budget, f)), f"kept counts {np.unique(cnt[~tie])}, want {min(budget, f)}"
+    s = scores.astype(np.float32).astype(np.float64)
+    for t in range(T):
+        if tie[t]:
+            continue
+        for r in range(k):
+            kept, dropped = s[t, r][gpu_mask[t, r]], s[t, r][~gpu_mask[t, r]]
+            if kept.size and dropped.size:
+                lo, hi = kept.min(), dropped.max()
+                assert lo >= hi - band_rel * max(abs(hi), 1e-30), (t, r, lo, hi)
+    differ = np.any(gpu_mask != want, axis=(1, 2)) & ~tie
+    return differ, want
+
+
 def expected_under_gpu_mask(o, inputs, top_k, tau, ref, gpu_mask, flipped, tie, nthreads=0, tau_shared=0.0):
     """The oracle's output per token, where a token whose band neuron the GPU
     decided the other way is evaluated under the GPU's mask instead."""

@@ -104,6 +104,10 @@ def test_allocation_failure_injection(o, monkeypatch):
         with pytest.raises(m.MoeError) as ei:
             layer.calibrate_tau(x, 0.9)
         assert ei.value.code == m.MOE_ENOMEM
+        monkeypatch.setenv("MOE_INJECT_ALLOC_FAIL", "rank")
+        with pytest.raises(m.MoeError) as ei:   # the rank budget's buffers: the threshold stays in force
+            layer.set_rank_budget(50)
+        assert ei.value.code == m.MOE_ENOMEM
         monkeypatch.delenv("MOE_INJECT_ALLOC_FAIL")
         tau = layer.calibrate_tau(x, 0.9)   # the handle is still usable
         out = layer.forward(x, tau)

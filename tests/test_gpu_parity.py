@@ -413,3 +413,126 @@ def test_argument_errors_live_handle():
     with pytest.raises(m.MoeError) as ei:
         m.moe_sparse_forward(h, x, 4, 1.0, out)
     assert ei.value.code == m.MOE_EHANDLE
+
+
+def _rank_case(o, layer, inputs, x, top_k, budget, tau_s=0.0):
+    """One rank-budget forward (and its debug lists) against the oracle."""
+    out = layer.forward(x, 0.5)   # tau is unused for the routed experts under a budget
+    out_dbg = torch.empty_like(x)
+    lists, cnt = layer.active_lists(x, 0.5, out=out_dbg)
+    idx, w = layer.router(x)
+    torch.cuda.synchronize()
+    ref = o.forward_budget(**inputs, top_k=top_k, budget=budget, nthreads=NTHREADS, tau_shared=tau_s)
+    tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), top_k)
+    f = ref.score.shape[2]
+    gmask = pu.gpu_mask_from_lists(lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), f)
+    differ, want = pu.check_rank_mask(o, ref.score, budget, gmask, tie)
+    assert np.array_equal(ref.active.astype(bool)[~tie], want[~tie])
+    y = ref.y.copy()
+    rows = np.where(differ)[0]
+    if rows.size:   # a near-equal pair of scores ordered the other way: the layer under the GPU's choice
+        sub = dict(inputs)
+        sub["x"] = inputs["x"][rows]
+        y[rows] = o.forward(**sub, top_k=top_k, tau=0.0, active=gmask[rows], nthreads=NTHREADS,
+                            tau_shared=tau_s).y
+    pu.check_output(y, out, tie)
+    pu.check_output(y, out_dbg, tie)
+    return gmask, ref
+
+
+@pytest.mark.parametrize("name,T,frac", [("tiny", 16, 0.1), ("olmoe", 1, 0.1), ("olmoe", 4, 0.1),
+                                         ("olmoe", 16, 0.1), ("olmoe", 40, 0.05), ("dsv2lite", 8, 0.1),
+                                         ("large", 1, 0.02)])
+def test_rank_budget(o, name, T, frac):
+    """Per-pair rank budget (each routed pair keeps its r highest scores):
+    exact counts, a valid selection under the oracle's scores, and the layer
+    output against the oracle under that selection; in-kernel-routing sizes,
+    a token-tile size (40) and shapes with shared experts."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    budget = max(1, int(round(frac * sh.d_ff)))
+    layer.set_rank_budget(budget)
+    try:
+        _rank_case(o, layer, inputs, x, sh.top_k, budget)
+        st = layer.stats()
+        assert st["path"] == m.MOE_PATH_SPARSE and st["device_error"] == 0
+    finally:
+        layer.set_rank_budget(-1)
+
+
+def test_rank_budget_edges_and_shared_threshold(o):
+    """Budget 0 (the shared experts alone), budget = d_ff and above (the
+    unmasked layer), a looser shared threshold beside the budget, the dense
+    path refused, and the threshold restored afterwards."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["dsv2lite"]
+    layer, W, host = layer_for("dsv2lite")
+    T = 8
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    try:
+        for budget in (0, sh.d_ff, sh.d_ff + 100):
+            layer.set_rank_budget(budget)
+            gmask, ref = _rank_case(o, layer, inputs, x, sh.top_k, budget)
+            assert int(gmask.sum()) == T * sh.top_k * min(budget, sh.d_ff)
+        r_inf = o.forward(**inputs, top_k=sh.top_k, tau=math.inf, nthreads=NTHREADS, want_scores=False)
+        layer.set_rank_budget(0)
+        pu.check_output(r_inf.y, layer.forward(x, 0.5))
+        r0 = o.forward(**inputs, top_k=sh.top_k, tau=math.inf, nthreads=NTHREADS)
+        tau_s = pu.threshold_off_scores(r0.score_shared, 0.5)
+        layer.set_shared_tau(tau_s)
+        layer.set_rank_budget(141)
+        _rank_case(o, layer, inputs, x, sh.top_k, 141, tau_s)
+        layer.set_path(m.MOE_PATH_DENSE)
+        with pytest.raises(m.MoeError):
+            layer.forward(x, 0.5)
+        layer.set_path(m.MOE_PATH_AUTO)
+        layer.set_rank_budget(-1)
+        layer.set_shared_tau(0.0)
+        tau = pu.calibrate(o, inputs, sh.top_k, 0.9, NTHREADS)
+        ref = o.forward(**inputs, top_k=sh.top_k, tau=tau, nthreads=NTHREADS)
+        out = layer.forward(x, tau)
+        lists, cnt = layer.active_lists(x, tau)
+        torch.cuda.synchronize()
+        tie = np.zeros(T, bool)
+        flipped, _, gm = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), tie)
+        pu.check_output(pu.expected_under_gpu_mask(o, inputs, sh.top_k, tau, ref, gm, flipped, tie, NTHREADS), out)
+    finally:
+        layer.set_rank_budget(-1)
+        layer.set_shared_tau(0.0)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
+def test_rank_budget_exact_ties():
+    """Exact ties: gate columns repeated four times give four identical scores
+    per neuron group, and a zero token scores 0 everywhere; the selection must
+    keep the lower indices of a tied group first (checked on the GPU's own
+    mask, no tolerance), and the zero token keeps neurons 0..r-1."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["tiny"]
+    W = mi.make_weights(sh, device="cuda")
+    q = sh.d_ff // 4
+    W.w_gate.copy_(W.w_gate[:, :, :q].repeat(1, 1, 4))
+    layer = m.MoESparseLayer.from_weights(W, sh.top_k, max_tokens=64)
+    try:
+        for T in (16, 40):
+            x = mi.make_x(sh, T, device="cuda")
+            x[1] = 0
+            for budget in (1, 6, 50, 130):   # 6, 50, 130 cut inside a group of four
+                layer.set_rank_budget(budget)
+                layer.forward(x, 0.5)
+                lists, cnt = layer.active_lists(x, 0.5)
+                torch.cuda.synchronize()
+                g = pu.gpu_mask_from_lists(lists.cpu().numpy().view(np.uint16), cnt.cpu().numpy(), sh.d_ff)
+                assert np.all(g.sum(axis=2) == budget)
+                grp = g.reshape(T, sh.top_k, 4, q)   # [.., member, j]: member m is neuron m*q + j
+                assert np.all(grp[:, :, 1:, :] <= grp[:, :, :-1, :]), "a tied group kept a higher index first"
+                assert np.all(g[1, :, :budget]) and not np.any(g[1, :, budget:])
+                assert layer.stats()["device_error"] == 0
+    finally:
+        layer.close()
