@@ -70,8 +70,9 @@ def parse():
     p.add_argument("--T", type=int, default=16)
     p.add_argument("--sparsity", type=float, default=0.9)
     p.add_argument("--path", choices=["auto", "sparse", "dense"], default="auto")
-    p.add_argument("--router", choices=["fused", "kernel"], default="fused",
-                   help="decode batches: route inside the expert kernel (default) or with the router kernel")
+    p.add_argument("--router", choices=["fused", "one_launch", "kernel"], default="fused",
+                   help="decode batches: route inside the expert kernel (default), also combine there "
+                        "(one launch), or route with the router kernel")
     p.add_argument("--sweep", choices=["full", "quick", "none"], default="full")
     p.add_argument("--no-sweep", action="store_true", help="same as --sweep none")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -302,49 +303,64 @@ def l2_flush(buf):
 def time_steps(layer, x, tau, out, flush, steps, graph=True):
     """Per-step CUDA-event timing with an L2 flush before each step (outside the events).
 
-    graph=True (the default): the K steps -- flush, start event, forward (whose
-    kernels record the launch events), end event -- are captured into one CUDA
-    graph and replayed once, so the host's enqueue cost cannot leave the GPU
-    idle inside a step; the device does exactly the same work.  graph=False
-    enqueues the steps one by one from Python (eager)."""
+    graph=True (the default): the K steps -- flush, start event, forward, end
+    event -- are captured into one CUDA graph and replayed once, so the host's
+    enqueue cost cannot leave the GPU idle inside a step; the device does
+    exactly the same work.  A second graph of the same K steps also records
+    the library's launch events (before the first kernel, before the expert
+    kernel, after the last kernel) for the per-kernel split; each event node
+    adds about a microsecond of its own, so the step times come from the first
+    graph, which has only the two events per step.  graph=False enqueues the
+    steps one by one from Python (eager), with the launch events.
+
+    Returns (step_ms, router_ms, expert_ms) per step."""
     import torch
     from intra_expert_activation_router_b200 import moe_set_launch_events
 
     def ev():
         return torch.cuda.Event(enable_timing=True, external=True)
 
-    starts = [ev() for _ in range(steps)]
-    ends = [ev() for _ in range(steps)]
-    kev = [[ev() for _ in range(3)] for _ in range(steps)]
     st = torch.cuda.current_stream()
-    for trio in kev:   # create the CUDA events before the library records them
-        for e in trio:
-            e.record(st)
-    torch.cuda.synchronize()
 
-    def body():
-        for i in range(steps):
-            l2_flush(flush)
-            starts[i].record()
-            moe_set_launch_events(layer.h, kev[i])
-            layer.forward(x, tau, out=out)
-            ends[i].record()
-        moe_set_launch_events(layer.h, None)
+    def run(with_kernel_events):
+        starts = [ev() for _ in range(steps)]
+        ends = [ev() for _ in range(steps)]
+        kev = [[ev() for _ in range(3)] for _ in range(steps)] if with_kernel_events else None
+        for e in starts + ends + [e for trio in (kev or []) for e in trio]:
+            e.record(st)   # create the CUDA events before the graph (or the library) records them
+        torch.cuda.synchronize()
 
-    if graph:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        def body():
+            for i in range(steps):
+                l2_flush(flush)
+                starts[i].record()
+                if kev:
+                    moe_set_launch_events(layer.h, kev[i])
+                layer.forward(x, tau, out=out)
+                ends[i].record()
+            if kev:
+                moe_set_launch_events(layer.h, None)
+
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                body()
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            del g
+        else:
             body()
-        torch.cuda.synchronize()
-        g.replay()
-        torch.cuda.synchronize()
-        del g
-    else:
-        body()
-        torch.cuda.synchronize()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    router_ms = [t[0].elapsed_time(t[1]) for t in kev]
-    expert_ms = [t[1].elapsed_time(t[2]) for t in kev]
+            torch.cuda.synchronize()
+        step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        if not kev:
+            return step_ms, None, None
+        return step_ms, [t[0].elapsed_time(t[1]) for t in kev], [t[1].elapsed_time(t[2]) for t in kev]
+
+    if not graph:
+        return run(True)
+    step_ms, _, _ = run(False)
+    _, router_ms, expert_ms = run(True)
     return step_ms, router_ms, expert_ms
 
 
@@ -421,6 +437,40 @@ def sweep_rows(dev, kind, peak, flush, steps=20):
     return rows
 
 
+def launch_mode_rows(dev, flush, steps=20):
+    """Decode batches of the OLMoE-shaped layer in the three launch
+    structures: router kernel + expert kernel + conversion (3 launches),
+    routing inside the expert kernel (2), routing and combine inside (1)."""
+    import torch
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    shape = mi.SHAPES["olmoe"]
+    W = mi.make_weights(shape, device=dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=16)
+    del W
+    layer.set_path(m.MOE_PATH_SPARSE)
+    rows = []
+    for T in (1, 4, 16):
+        x = mi.make_x(shape, T, device=dev)
+        out = torch.empty_like(x)
+        tau = layer.calibrate_tau(x, 0.9)
+        row = {"workload": "olmoe", "T": T, "sparsity": 0.9}
+        for name, fused, one in (("launches3_us", False, False), ("launches2_us", True, False),
+                                 ("launches1_us", True, True)):
+            layer.set_fused_router(fused, one_launch=one)
+            for _ in range(3):
+                layer.forward(x, tau, out=out)
+            sm_, _, _ = time_steps(layer, x, tau, out, flush, steps)
+            row[name] = 1000 * statistics.mean(sm_)
+            if layer.stats()["device_error"]:
+                row[name + "_device_error"] = True
+        rows.append(row)
+        log(json.dumps({k: (round(v, 2) if isinstance(v, float) else v) for k, v in row.items()}))
+    layer.close()
+    torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -442,7 +492,7 @@ def run_ours(args):
     layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=max(T, 64))
     if args.path != "auto":
         layer.set_path({"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
-    layer.set_fused_router(args.router == "fused")
+    layer.set_fused_router(args.router != "kernel", one_launch=args.router == "one_launch")
     out = torch.empty_like(x)
     tau = layer.calibrate_tau(x, args.sparsity)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -494,6 +544,7 @@ def run_ours(args):
     layer.close()
 
     sweep = sweep_rows(dev, sweep_kind, peak, flush) if rank == 0 and sweep_kind != "none" else []
+    modes = launch_mode_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -533,12 +584,13 @@ def run_ours(args):
                     "d2h_bytes_per_step": T * shape.d_model * 2},
             # sparse: router (unless routed in the expert kernel), expert kernel, y conversion;
             # dense: router, gather, GEMM1 and GEMM2 per routed/shared group, convert
-            "gpu_launches": ((2 if st["fused_router"] else 3) if path == "sparse"
+            "gpu_launches": ({0: 3, 1: 2, 2: 1}[st["fused_router"]] if path == "sparse"
                              else 5 + 2 * shape.n_shared) * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"]},
             "stats": {"n_touched": st["n_touched"], "n_active": st["n_active"], "n_union": st["n_union"]},
             "sweep": sweep,
+            "launch_modes": modes,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

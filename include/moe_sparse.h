@@ -92,8 +92,9 @@ typedef struct {
     double dense_bytes;    /* the same for the dense path (all neurons)          */
     int device_error;      /* first device error code since the previous
                               moe_query_stats (0: none)                          */
-    int fused_router;      /* 1 if the last forward routed the batch inside the
-                              expert kernel (no separate router launch)          */
+    int fused_router;      /* the last forward's moe_set_fused_router mode if it
+                              routed the batch inside the expert kernel (1: no
+                              router launch, 2: one launch), else 0              */
 } moe_stats;
 
 /* Create a layer.  Copies and repacks the weights into library-owned device
@@ -155,13 +156,19 @@ int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau, int *t_st
  * T * E <= 8192, d_model >= 64) normally route inside the expert kernel: each
  * CTA computes some experts' logits, all CTAs then select the top-k and build
  * the plan themselves, so no router kernel and no plan hand-off precede the
- * gate stream.  enable = 0 uses the separate router kernel instead (same
+ * gate stream.  mode = 0 uses the separate router kernel instead (same
  * results up to the order of fp32 sums in the logits); 1 restores the
- * default.  This assumes every CTA of the expert kernel (at most one per SM)
- * can be resident at once, which holds unless the context is restricted to
- * fewer SMs than the device has; otherwise the routing wait runs out and
- * reports error code 55. */
-int moe_set_fused_router(moe_handle h, int enable);
+ * default (two launches: the expert kernel, then a small kernel converting
+ * the fp32 accumulator to the bf16 output); 2 also does that conversion at
+ * the end of the expert kernel, after a grid-wide count of the CTAs whose
+ * sums have landed, so such a forward is one launch (router, gate, mask,
+ * gather, up/down and combine; measured about 2 us slower than mode 1 at
+ * 1 and 16 tokens on B200, which is why it is not the default).  Modes 1
+ * and 2 assume every CTA of the expert kernel (at most one per SM) can be
+ * resident at once, which holds unless the context is restricted to fewer
+ * SMs than the device has; otherwise the routing wait runs out and reports
+ * error code 55 (57 for the combine's count).  Other modes: MOE_EINVAL. */
+int moe_set_fused_router(moe_handle h, int mode);
 
 /* Router only: idx_out [T][top_k] int32 and w_out [T][top_k] fp32, both
  * DEVICE pointers, in rank order.  Asynchronous. */
@@ -244,9 +251,11 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
  * of the CTA's first three items i, at 2 + 10*i: metadata ready, gate
  * accumulator ready, mask read out (twice), mask step synchronised, mask and
  * lists published, first gathered batch in (up warps), first h in (down
- * warps), up projection done, down projection and flush done; [32 + 4u] for
- * the gather of item u < 2: mask seen, then the issue times of its first
- * three batches; [40 + g] issue of gate stage g < 4; [44]..[47] routing
+ * warps), up projection done, down projection and flush done; the gate
+ * lane's totals: [32] ns waiting to claim an item, [33] ns waiting for a free
+ * ring stage, [34] stages issued, [35] issue time of the last stage; the up
+ * warps' totals: [36] ns in mask steps, [37] ns waiting for the next item's
+ * id and metadata slot; [40 + g] issue of gate stage g < 4; [44]..[47] routing
  * inside the kernel: start, own logits computed, logits staged, plan built;
  * [48 + q] token rows of
  * tile q < 4 ready (batches of more than 16 tokens; smaller batches stream

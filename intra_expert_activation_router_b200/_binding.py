@@ -247,8 +247,8 @@ def moe_tune_t_star(h, x, T_max: int, tau: float, stream=None) -> int:
     return t.value
 
 
-def moe_set_fused_router(h, enable: int):
-    _check(_lib.moe_set_fused_router(h, int(enable)), "moe_set_fused_router")
+def moe_set_fused_router(h, mode: int):
+    _check(_lib.moe_set_fused_router(h, int(mode)), "moe_set_fused_router")
 
 
 def moe_debug_inject(h, kind: int):

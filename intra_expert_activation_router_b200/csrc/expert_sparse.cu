@@ -840,6 +840,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         if (lane == 0 && a.inject != 1) {
             const uint64_t pol = policy_evict_first();
             uint32_t g = 0;
+            unsigned long long t_claim = 0, t_ring = 0, t_last = 0;   // trace only
             int next = a.resident ? atomicAdd(&plan->next_item, 1) : 0;
             for (int i = 0;; ++i) {
                 int id;
@@ -847,6 +848,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     if (i > 0 && next < n_items) {
                         // item i - 1 masked and the up/down backlog short: claim the
                         // next item (its gate streams while the backlog drains)
+                        const unsigned long long tc0 = tr ? global_ns() : 0;
                         bool ok = true;
                         for (uint32_t spin = 0;; ++spin) {
                             if (*mask_done >= i) {
@@ -861,6 +863,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                             __nanosleep(128);
                         }
                         next = ok ? atomicAdd(&plan->next_item, 1) : n_items;
+                        if (tr) t_claim += global_ns() - tc0;
                     }
                     id = next < n_items ? next : -1;
                 } else {
@@ -887,8 +890,13 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 bool ok = true;
                 for (int s = s_lo; s < s_hi; ++s, ++g) {
                     const int slot = (int)(g % NS);
+                    const unsigned long long tr0 = tr ? global_ns() : 0;
                     if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
-                    if (tr && g < 4) tr[40 + g] = global_ns();
+                    if (tr) {
+                        t_last = global_ns();
+                        t_ring += t_last - tr0;
+                        if (g < 4) tr[40 + g] = t_last;
+                    }
                     uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
                     mbar_arrive_expect_tx(&full_g[slot], kStageBytes + L.xs_bytes);
                     if (a.fused) {   // the token operand's blocks 2s, 2s+1 straight from x (L2-resident)
@@ -910,6 +918,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             }
             // every copy issued has landed before the CTA may exit
             for (int s = 0; s < NS && (uint32_t)s < g; ++s) mbar_drain(&full_g[s], (((g - s + NS - 1) / NS) - 1) & 1);
+            if (tr) {
+                tr[32] = t_claim;
+                tr[33] = t_ring;
+                tr[34] = g;
+                tr[35] = t_last;
+            }
         }
         __syncwarp();
     } else if (warp == kWarpMma) {
@@ -1165,7 +1179,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = M.word[t][qw];
             }
         };
+        unsigned long long t_item = 0, t_mask = 0;   // trace only
         for (;; ++ii) {
+            const unsigned long long ti0 = tr ? global_ns() : 0;
             const int id = get_item(ii);
             if (id < 0) {
                 if (ct == 0) *items_end = ii;   // every item of this CTA has been masked
@@ -1179,7 +1195,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 }
                 __nanosleep(64);
             }
+            const unsigned long long ti1 = tr ? global_ns() : 0;
             do_mask(ii, id);
+            if (tr) {
+                t_item += ti1 - ti0;
+                t_mask += global_ns() - ti1;
+            }
             if (score_mode) continue;
             const ItemMeta &M = meta[ii & 1];
             const int m = M.m, nsub = min(M.nsub, kMaxSub);
@@ -1229,6 +1250,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             if (tu && ct == 0) tu[8] = global_ns();
         }
         if (tr && ct == 0) {
+            tr[36] = t_mask;
+            tr[37] = t_item;
             tr[52] = t_wait;
             tr[53] = t_work;
             tr[61] = (unsigned long long)n_rec;
@@ -1508,7 +1531,7 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
                                  float *score_out, int inject, bool fused, float tau_shared, bool score_shared,
-                                 const RankPass *rank)
+                                 const RankPass *rank, bool combine_here)
 {
     if (rank && !rank->second) score_out = rank->a;   // first pass: signed silu(g) of the routed pairs
     SparseArgs a;
@@ -1565,12 +1588,10 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     }
     const long long bound = (a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk) * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
-    // the combine at the end of the kernel (MOE_TAIL=0: a separate conversion kernel)
-    {
-        const char *tv = std::getenv("MOE_TAIL");
-        a.tail = (tv && std::strcmp(tv, "0") == 0) ? 0 : 1;
-        a.n_out4 = score_out ? 0 : (long long)T * dm.d / 4;
-    }
+    // the combine at the end of this kernel (one launch per forward), else a
+    // separate conversion kernel
+    a.tail = combine_here ? 1 : 0;
+    a.n_out4 = score_out ? 0 : (long long)T * dm.d / 4;
     if (grid < 1) grid = 1;
     cudaError_t e;
     switch (np * 8 + til.mt) {

@@ -187,7 +187,8 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
                                  const uint16_t *x, int T, float tau, bool use_mask,
                                  uint16_t *out, SparseTiling til, int grid_cap, cudaStream_t st,
                                  float *score_out = nullptr, int inject = 0, bool fused = false,
-                                 float tau_shared = 0.f, bool score_shared = false, const RankPass *rank = nullptr);
+                                 float tau_shared = 0.f, bool score_shared = false, const RankPass *rank = nullptr,
+                                 bool combine_here = false);
 // Per pair of a [pairs][f] silu(g) buffer, the cut (v, J) keeping its r
 // highest |silu(g)| (ties to the lower index, NaN never): neuron j is kept iff
 // |silu(g_j)| > v, or == v and j <= J.

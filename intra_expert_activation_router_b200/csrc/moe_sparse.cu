@@ -335,7 +335,8 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
                                               h->inject_next, false, h->tau_shared, false, &r2);
         } else if (e == cudaSuccess) {
             e = moe::launch_expert_sparse(h->dm, h->w, h->ws, xb, T, tau, masked, ob, til, h->n_sm, st, nullptr,
-                                          h->inject_next, fused, h->tau_shared);
+                                          h->inject_next, fused, h->tau_shared, false, nullptr,
+                                          fused && h->fused_router == 2);
         }
         h->inject_next = 0;
     } else {
@@ -348,7 +349,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     h->last_T = T;
     h->last_path = path;
     h->last_masked = masked;
-    h->last_fused = fused ? 1 : 0;
+    h->last_fused = fused ? h->fused_router : 0;
     h->last_stream = st;
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -655,11 +656,11 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
     return err ? MOE_EDEVICE : MOE_OK;
 }
 
-extern "C" int moe_set_fused_router(moe_handle h, int enable)
+extern "C" int moe_set_fused_router(moe_handle h, int mode)
 {
     if (!is_live(h)) return MOE_EHANDLE;
-    if (enable != 0 && enable != 1) return MOE_EINVAL;
-    h->fused_router = enable;
+    if (mode < 0 || mode > 2) return MOE_EINVAL;
+    h->fused_router = mode;
     return MOE_OK;
 }
 

@@ -88,8 +88,10 @@ class MoESparseLayer:
         self._check_x(x)
         return B.moe_calibrate_tau_shared(self.h, x, x.shape[0], sparsity, stream)
 
-    def set_fused_router(self, enable: bool):
-        B.moe_set_fused_router(self.h, 1 if enable else 0)
+    def set_fused_router(self, enable, one_launch: bool = False):
+        """Route decode batches inside the expert kernel (the default); with
+        one_launch also combine there, so a forward is a single launch."""
+        B.moe_set_fused_router(self.h, (2 if one_launch else 1) if enable else 0)
 
     def router(self, x, stream=None):
         self._check_x(x)

@@ -117,6 +117,22 @@ def test_router_kernel_path(o, name, T, q):
         layer.set_fused_router(True)
 
 
+@pytest.mark.parametrize("name,T,q", [("olmoe", 1, 0.9), ("olmoe", 2, 0.9), ("olmoe", 16, 0.9), ("tiny", 16, 0.9),
+                                      ("dsv2lite", 8, 0.9), ("large", 1, 0.98), ("olmoe", 40, 0.9)])
+def test_one_launch_forward(o, name, T, q):
+    """Routing and the combine inside the expert kernel (one launch per
+    forward) against the oracle; 40 tokens exceed one token tile, so that
+    forward falls back to the router kernel and the conversion kernel."""
+    layer, W, host = layer_for(name)
+    layer.set_fused_router(True, one_launch=True)
+    try:
+        for _ in range(2):   # counters left for the next forward must be reset by the kernel itself
+            run_case(o, name, T, q)
+        assert layer.stats()["fused_router"] == (2 if T <= 16 else 0)
+    finally:
+        layer.set_fused_router(True)
+
+
 def test_in_kernel_routing_is_used_for_decode_batches(o):
     sh = mi.SHAPES["olmoe"]
     layer, W, host = layer_for("olmoe")
