@@ -14,12 +14,14 @@
 //            D[128 x 256] = H_tile . WdT rows^T; epilogue y_acc[token] +=
 //            w * D with fp32 vector atomics
 //   convert  out = bf16(y_acc), y_acc re-zeroed
-// Shared experts run as extra GEMM1/GEMM2 grids over all T tokens with the
-// mask off and weight 1.  Each GEMM CTA computes one tile: warp 0 issues the
-// TMA loads into a 4-stage ring, warp 1 issues the MMAs from one thread, all
-// four warps read the accumulator back for the epilogue.  Operands are K-major
-// with the 128-byte swizzle; the gate weights are stored in HBM as exactly
-// these tiles (gate_tile_off), so each is one plain 16 KB bulk copy.
+// Shared experts run as extra GEMM1/GEMM2 grids over all T tokens with their
+// own threshold (none by default) and weight 1.  The GEMM kernel is
+// persistent (one CTA per SM walking its tiles): warp 0 issues the TMA loads
+// into a 4-stage ring, warp 1 issues the MMAs from one thread into two TMEM
+// accumulators in turn, and four epilogue warps read one accumulator back
+// while the MMAs fill the other.  Operands are K-major with the 128-byte
+// swizzle; the gate weights are stored in HBM as exactly these tiles
+// (gate_tile_off), so each is one plain 16 KB bulk copy.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -31,7 +33,8 @@ namespace moe {
 constexpr int kBM = 128;            // token rows per tile
 constexpr int kBK = 64;             // K per stage (128 bytes of bf16)
 constexpr int kDStages = 4;
-constexpr int kDenseThreads = 128;
+constexpr int kDenseThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kAccCols = 256;        // one accumulator: 128 lanes x 256 fp32 columns
 constexpr int kATileBytes = kBM * kBK * 2;    // 16 KB
 constexpr int kBTileBytes = 256 * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -101,6 +104,62 @@ __global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict_
 
 namespace moe {
 
+// One output tile of a launch: A rows [row0, row0 + valid), weight rows
+// wrow0 + n0 .. of expert (or shared expert) ex.  Tiles are numbered with
+// the output block fastest, so that the tiles in flight at once cover a few
+// token tiles completely: a token tile's activations are read by its output
+// blocks from L2, an expert's weights by its token tiles at about the same
+// time.
+struct DenseTile {
+    int row0, valid, wrow0, ex, n0, bx;
+};
+
+__device__ __forceinline__ int dense_out_blocks(const DenseArgs &a)
+{
+    return a.mode == kGateUp ? a.wrows / 128 : a.wrows / 256;
+}
+
+__device__ __forceinline__ int dense_n_tiles(const DenseArgs &a)
+{
+    const int m_tiles = a.shared ? (a.T + kBM - 1) / kBM : a.plan->n_dense_tiles;
+    return m_tiles * dense_out_blocks(a);
+}
+
+__device__ __forceinline__ DenseTile dense_tile(const DenseArgs &a, int t)
+{
+    const int n_out = dense_out_blocks(a);
+    DenseTile d;
+    d.bx = t % n_out;
+    const int by = t / n_out;
+    if (!a.shared) {
+        const Plan *plan = a.plan;
+        int lo = 0, hi = plan->n_touched - 1;   // last slot with tile_prefix <= by
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (plan->tile_prefix[mid] <= by) lo = mid; else hi = mid - 1;
+        }
+        const int e = plan->touched[lo];
+        const int local = by - plan->tile_prefix[lo];
+        const int off = plan->offsets[e], cnt = plan->offsets[e + 1] - off;
+        d.row0 = off + kBM * local;
+        d.valid = min(kBM, cnt - kBM * local);
+        d.wrow0 = e * a.wrows;
+        d.ex = e;
+    } else {
+        d.row0 = kBM * by;
+        d.valid = min(kBM, a.T - d.row0);
+        d.wrow0 = a.sidx * a.wrows;
+        d.ex = a.sidx;
+    }
+    d.n0 = d.bx * (a.mode == kGateUp ? 128 : 256);
+    return d;
+}
+
+// Persistent: one CTA per SM walks the launch's tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ...  Warp 0 streams every tile's K blocks into a
+// 4-stage ring without pausing between tiles, warp 1 issues the MMAs into one
+// of two 256-column TMEM accumulators, and warps 2-5 (one TMEM lane quarter
+// each) run the epilogue of tile i while the MMAs of tile i + 1 proceed.
 __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_constant__ DenseMaps maps, DenseArgs a)
 {
     extern __shared__ uint8_t dsmem_raw[];
@@ -108,152 +167,162 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDStages * kStageBytes);
     uint64_t *empty = full + kDStages;
-    uint64_t *done = empty + kDStages;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(done + 1);
+    uint64_t *accf = empty + kDStages;   // [2] accumulator ready (MMA commit)
+    uint64_t *acce = accf + 2;           // [2] accumulator read out (4 epilogue warps)
+    uint64_t *mdrain = acce + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mdrain + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    // ---- the tile: expert rows [row0, row0 + valid) of A, weight rows wrow0 + n0 ..
-    // The grid is flat with the output block fastest, so that the CTAs of one
-    // wave cover a few token tiles completely: a tile's activations are read by
-    // its output blocks from L2, an expert's weights by its token tiles at about
-    // the same time.
-    const int n_out = a.mode == kGateUp ? a.wrows / 128 : a.wrows / 256;   // output blocks
-    const int bx = (int)(blockIdx.x % (unsigned)n_out), by = (int)(blockIdx.x / (unsigned)n_out);
-    int row0, valid, wrow0, ex;
-    if (!a.shared) {
-        const Plan *plan = a.plan;
-        const int n_tiles = plan->n_dense_tiles;
-        if (by >= n_tiles) return;
-        const int mt = by;
-        int lo = 0, hi = plan->n_touched - 1;   // last slot with tile_prefix <= mt
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (plan->tile_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
-        }
-        const int e = plan->touched[lo];
-        const int local = mt - plan->tile_prefix[lo];
-        const int off = plan->offsets[e], cnt = plan->offsets[e + 1] - off;
-        row0 = off + kBM * local;
-        valid = min(kBM, cnt - kBM * local);
-        wrow0 = e * a.wrows;
-        ex = e;
-    } else {
-        row0 = kBM * by;
-        valid = min(kBM, a.T - row0);
-        if (valid <= 0) return;
-        wrow0 = a.sidx * a.wrows;
-        ex = a.sidx;
-    }
-    const int ntile = a.mode == kGateUp ? 128 : 256;
-    const int n0 = bx * ntile;
 
     if (tid == 0) {
         for (int s = 0; s < kDStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+        }
+        mbar_init(mdrain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&maps.a);
         if (a.mode == kGateUp) tma_prefetch_desc(&maps.b1);
         else tma_prefetch_desc(&maps.b0);
     }
-    if (warp == 0) {
-        tmem_alloc(s_tmem, 256);
+    if (warp == 1) {
+        tmem_alloc(s_tmem, 2 * kAccCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    const int n_tiles = dense_n_tiles(a);
 
-    if (warp == 0 && lane == 0) {
-        // ---- TMA producer
-        const uint32_t bytes = kATileBytes + (a.mode == kGateUp ? 2 * (kBTileBytes / 2) : kBTileBytes);
-        for (int kb = 0; kb < a.kb; ++kb) {
-            const int s = kb % kDStages;
-            mbar_wait(&empty[s], ((kb / kDStages) & 1) ^ 1, a.err, 31);
-            uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
-            mbar_arrive_expect_tx(&full[s], bytes);
-            tma_load_2d(A, &maps.a, kb * kBK, a.a_base + row0, &full[s]);
-            if (a.mode == kGateUp) {
-                const uint16_t *gt = a.gate + (((size_t)ex * a.n_blk + bx) * a.n_kb + kb) * (kBM * kBK);
-                bulk_g2s(B, gt, kBTileBytes / 2, &full[s]);
-                tma_load_2d(B + kBTileBytes / 2, &maps.b1, kb * kBK, wrow0 + n0, &full[s]);
-            } else {
-                tma_load_2d(B, &maps.b0, kb * kBK, wrow0 + n0, &full[s]);
-            }
-        }
-    } else if (warp == 1 && lane == 0) {
-        // ---- MMA issuer: M = 128, N = 256, K = 16 per instruction
-        const uint32_t idesc = idesc_bf16_f32(kBM, 256);
-        for (int kb = 0; kb < a.kb; ++kb) {
-            const int s = kb % kDStages;
-            mbar_wait(&full[s], (kb / kDStages) & 1, a.err, 32);
-            tc_fence_after();
-            const uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-                umma_bf16(tmem, smem_desc_k_sw128(A + 32 * kk), smem_desc_k_sw128(B + 32 * kk), idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
-            umma_commit(&empty[s]);   // the stage is free once these MMAs have read it
-        }
-        umma_commit(done);
-    }
-    __syncwarp();
-
-    // ---- epilogue: thread = accumulator row (TMEM lane 32*warp + lane)
-    mbar_wait(done, 0, a.err, 33);
-    tc_fence_after();
-    const int row = warp * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    if (a.mode == kGateUp) {
-        uint16_t *hrow = a.h + (size_t)(a.h_base + row0 + row) * a.h_ld + n0;
-        for (int c = 0; c < 128; c += 16) {
-            float g[16], u[16];
-            tmem_ld16(tl + c, g);
-            tmem_ld16(tl + 128 + c, u);
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float hv[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const float av = silu_f(g[2 * i + j]);
-                    const bool on = !a.use_mask || fabsf(av) >= a.tau;
-                    hv[j] = on ? av * u[2 * i + j] : 0.f;
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer
+            const uint32_t bytes = kATileBytes + (a.mode == kGateUp ? 2 * (kBTileBytes / 2) : kBTileBytes);
+            uint32_t st = 0;   // stages issued
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const DenseTile dt = dense_tile(a, t);
+                for (int kb = 0; kb < a.kb; ++kb, ++st) {
+                    const int s = (int)(st % kDStages);
+                    if (!mbar_wait(&empty[s], ((st / kDStages) & 1) ^ 1, a.err, 31)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    tma_load_2d(A, &maps.a, kb * kBK, a.a_base + dt.row0, &full[s]);
+                    if (a.mode == kGateUp) {
+                        const uint16_t *gt =
+                            a.gate + (((size_t)dt.ex * a.n_blk + dt.bx) * a.n_kb + kb) * (kBM * kBK);
+                        bulk_g2s(B, gt, kBTileBytes / 2, &full[s]);
+                        tma_load_2d(B + kBTileBytes / 2, &maps.b1, kb * kBK, dt.wrow0 + dt.n0, &full[s]);
+                    } else {
+                        tma_load_2d(B, &maps.b0, kb * kBK, dt.wrow0 + dt.n0, &full[s]);
+                    }
                 }
-                pk[i] = (uint32_t)f2bf_bits(hv[0]) | ((uint32_t)f2bf_bits(hv[1]) << 16);
             }
-            if (row < valid) {
-                reinterpret_cast<uint4 *>(hrow + c)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                reinterpret_cast<uint4 *>(hrow + c)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
+            // every copy issued has landed before the CTA may exit
+            for (int s = 0; s < kDStages && (uint32_t)s < st; ++s)
+                mbar_drain(&full[s], (((st - s + kDStages - 1) / kDStages) - 1) & 1);
         }
-    } else {
-        int tok = 0;
-        float w = 1.f;
-        if (row < valid) {
-            tok = a.shared ? row0 + row : a.perm_tok[row0 + row];
-            w = a.shared ? 1.f : a.perm_w[row0 + row];
-        }
-        float *yrow = a.y_acc + (size_t)tok * a.d + n0;
-        for (int c = 0; c < 256; c += 16) {
-            float y[16];
-            tmem_ld16(tl + c, y);
-            if (row < valid) {
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer: M = 128, N = 256, K = 16 per instruction
+            const uint32_t idesc = idesc_bf16_f32(kBM, 256);
+            uint32_t st = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                ok = mbar_wait(&acce[acc], ((lt >> 1) & 1) ^ 1, a.err, 34);   // the epilogue read it out
+                tc_fence_after();
+                const uint32_t dt = tmem + acc * kAccCols;
+                for (int kb = 0; kb < a.kb && ok; ++kb, ++st) {
+                    const int s = (int)(st % kDStages);
+                    ok = mbar_wait(&full[s], (st / kDStages) & 1, a.err, 32);
+                    tc_fence_after();
+                    const uint8_t *A = smem + s * kStageBytes, *B = A + kATileBytes;
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    atomicAdd(reinterpret_cast<float4 *>(yrow + c + i),
-                              make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]));
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16(dt, smem_desc_k_sw128(A + 32 * kk), smem_desc_k_sw128(B + 32 * kk), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+                    umma_commit(&empty[s]);   // the stage is free once these MMAs have read it
+                }
+                if (ok) umma_commit(&accf[acc]);
             }
+            umma_commit(mdrain);   // all MMAs complete before the accumulators are freed
+            mbar_drain(mdrain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: thread = accumulator row (TMEM lane 32 * (warp % 4) + lane)
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int lt = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            const bool ok = mbar_wait(&accf[acc], (lt >> 1) & 1, a.err, 33);
+            tc_fence_after();
+            if (!ok) break;
+            const DenseTile dt = dense_tile(a, t);
+            const uint32_t tl = tmem + acc * kAccCols + ((uint32_t)(q * 32) << 16);
+            if (a.mode == kGateUp) {
+                uint16_t *hrow = a.h + (size_t)(a.h_base + dt.row0 + row) * a.h_ld + dt.n0;
+                for (int c = 0; c < 128; c += 16) {
+                    float g[16], u[16];
+                    tmem_ld16(tl + c, g);
+                    tmem_ld16(tl + 128 + c, u);
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float hv[2];
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const float av = silu_f(g[2 * i + j]);
+                            const bool on = !a.use_mask || fabsf(av) >= a.tau;
+                            hv[j] = on ? av * u[2 * i + j] : 0.f;
+                        }
+                        pk[i] = (uint32_t)f2bf_bits(hv[0]) | ((uint32_t)f2bf_bits(hv[1]) << 16);
+                    }
+                    if (row < dt.valid) {
+                        reinterpret_cast<uint4 *>(hrow + c)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        reinterpret_cast<uint4 *>(hrow + c)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+                }
+            } else {
+                int tok = 0;
+                float w = 1.f;
+                if (row < dt.valid) {
+                    tok = a.shared ? dt.row0 + row : a.perm_tok[dt.row0 + row];
+                    w = a.shared ? 1.f : a.perm_w[dt.row0 + row];
+                }
+                float *yrow = a.y_acc + (size_t)tok * a.d + dt.n0;
+                for (int c = 0; c < 256; c += 16) {
+                    float y[16];
+                    tmem_ld16(tl + c, y);
+                    if (row < dt.valid) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            atomicAdd(reinterpret_cast<float4 *>(yrow + c + i),
+                                      make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[acc]);   // the MMA may overwrite this accumulator
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 2 * kAccCols);
     }
 }
 
@@ -334,8 +403,10 @@ bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, De
 }
 
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
-                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared)
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared, int n_sm)
 {
+    // persistent grids: at most one CTA per SM, never more than the launch's tiles
+    auto grid = [n_sm](long long tiles) { return (unsigned)(tiles < n_sm ? (tiles > 0 ? tiles : 1) : n_sm); };
     if (!st.ok) return cudaErrorNotSupported;
     static int smem_set[kMaxDevices] = {};
     cudaError_t e = ensure_dynamic_smem(k_dense_gemm, kDenseSmem, smem_set);
@@ -374,7 +445,7 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     a.shared = 0;
     a.a_base = 0;
     a.h_base = 0;
-    k_dense_gemm<<<(unsigned)(dm.f / 128) * mbound, kDenseThreads, kDenseSmem, s>>>(st.g1r, a);
+    k_dense_gemm<<<grid((long long)(dm.f / 128) * mbound), kDenseThreads, kDenseSmem, s>>>(st.g1r, a);
     if (dm.S > 0) {
         a.shared = 1;
         a.a_base = Pm;
@@ -385,7 +456,7 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
             DenseArgs az = a;
             az.sidx = z;
             az.h_base = Pm + z * Tm;   // shared expert z's H rows
-            k_dense_gemm<<<(unsigned)(dm.f / 128) * mshared, kDenseThreads, kDenseSmem, s>>>(st.g1s, az);
+            k_dense_gemm<<<grid((long long)(dm.f / 128) * mshared), kDenseThreads, kDenseSmem, s>>>(st.g1s, az);
         }
     }
     // GEMM2: down with the routing-weight epilogue
@@ -397,13 +468,13 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     a.shared = 0;
     a.a_base = 0;
     a.use_mask = use_mask ? 1 : 0;
-    k_dense_gemm<<<(unsigned)(dm.d / 256) * mbound, kDenseThreads, kDenseSmem, s>>>(st.g2r, a);
+    k_dense_gemm<<<grid((long long)(dm.d / 256) * mbound), kDenseThreads, kDenseSmem, s>>>(st.g2r, a);
     for (int z = 0; z < dm.S; ++z) {
         DenseArgs az = a;
         az.shared = 1;
         az.sidx = z;
         az.a_base = Pm + z * Tm;
-        k_dense_gemm<<<(unsigned)(dm.d / 256) * mshared, kDenseThreads, kDenseSmem, s>>>(st.g2s, az);
+        k_dense_gemm<<<grid((long long)(dm.d / 256) * mshared), kDenseThreads, kDenseSmem, s>>>(st.g2s, az);
     }
     // convert
     {

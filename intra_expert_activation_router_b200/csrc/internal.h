@@ -223,6 +223,6 @@ bool dense_supported(const Dims &dm);
 bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, DenseState *st);
 // tau_shared: the shared experts' threshold on a masked forward (<= 0: dense).
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
-                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared = 0.f);
+                         float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared, int n_sm);
 
 }  // namespace moe

@@ -343,7 +343,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
-            e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st, h->tau_shared);
+            e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st, h->tau_shared, h->n_sm);
     }
     if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[2], st, ev_flags);
     h->last_T = T;

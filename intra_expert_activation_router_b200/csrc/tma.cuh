@@ -94,6 +94,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, err, code);
 }
 
+// A bounded wait that does not give up early on another agent's error: used
+// only to drain copies before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return;
+}
+
 // Contiguous global -> shared copy completed on `bar` (bytes % 16 == 0, both
 // addresses 16-byte aligned).  A CTA is its own cluster of one here.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
