@@ -73,6 +73,9 @@ def parse():
     p.add_argument("--router", choices=["fused", "one_launch", "kernel"], default="fused",
                    help="decode batches: route inside the expert kernel (default), also combine there "
                         "(one launch), or route with the router kernel")
+    p.add_argument("--budget", type=int, default=-1,
+                   help="per-pair rank budget for the timed layer (keep each routed pair's r best neurons); "
+                        "-1: the threshold at --sparsity")
     p.add_argument("--sweep", choices=["full", "quick", "none"], default="full")
     p.add_argument("--no-sweep", action="store_true", help="same as --sweep none")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -213,9 +216,12 @@ def cpu_cores():
 
 def bench_config(args, world):
     """The workload description both arms print (identical dicts)."""
-    return {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": args.T,
-            "sparsity": args.sparsity, "parallelism": f"replicas{world}",
-            "l2": "flushed before every timed step (2x L2 written, then read back, outside the step events)"}
+    cfg = {"workload": WORKLOAD_TEXT.get(args.workload, args.workload), "T": args.T,
+           "sparsity": args.sparsity, "parallelism": f"replicas{world}",
+           "l2": "flushed before every timed step (2x L2 written, then read back, outside the step events)"}
+    if args.budget >= 0:
+        cfg["rank_budget"] = args.budget   # each routed pair keeps its `budget` best neurons; no threshold
+    return cfg
 
 
 def draw_inputs(shape, T, device):
@@ -226,20 +232,29 @@ def draw_inputs(shape, T, device):
     return mi.make_weights(shape, device=device), mi.make_x(shape, T, device=device)
 
 
-def oracle_time_sample(shape, W_host, x_host, tau, target_s, nthreads):
-    """The CPU oracle at threshold tau on repeats of the batch for about
-    target_s seconds (rank 0, N = 1).  Returns (tokens/s, repeats, seconds)."""
+def oracle_step(o, inputs, shape, tau, budget, nthreads):
+    """One forward of the CPU oracle: the threshold tau, or the per-pair rank
+    budget when budget >= 0."""
+    if budget >= 0:
+        return o.forward_budget(**inputs, top_k=shape.top_k, budget=budget, nthreads=nthreads)
+    return o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=nthreads)
+
+
+def oracle_time_sample(shape, W_host, x_host, tau, target_s, nthreads, budget=-1):
+    """The CPU oracle at threshold tau (or the rank budget) on repeats of the
+    batch for about target_s seconds (rank 0, N = 1).  Returns (tokens/s,
+    repeats, seconds)."""
     import oracle
     o = oracle.Oracle()
     inputs = oracle.layer_inputs(W_host, x_host)
     T = x_host.shape[0]
     t0 = time.perf_counter()
-    o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=nthreads)
+    oracle_step(o, inputs, shape, tau, budget, nthreads)
     one = time.perf_counter() - t0
     reps = max(1, min(500, int(math.ceil(target_s / max(one, 1e-6)))))
     t0 = time.perf_counter()
     for _ in range(reps):
-        o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=nthreads)
+        oracle_step(o, inputs, shape, tau, budget, nthreads)
     el = time.perf_counter() - t0
     return reps * T / el, reps, el
 
@@ -262,7 +277,7 @@ def run_reference(args):
     r = o.forward(**inputs, top_k=shape.top_k, tau=math.inf, nthreads=cores)
     tau = o.calibrate_tau(r.score, args.sparsity)
     t0 = time.perf_counter()
-    o.forward(**inputs, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+    oracle_step(o, inputs, shape, tau, args.budget, cores)
     full = time.perf_counter() - t0
     budget = 150.0
     n_tok = args.T
@@ -271,11 +286,11 @@ def run_reference(args):
     sub = dict(inputs)
     sub["x"] = inputs["x"][:n_tok]
     for _ in range(args.warmup):
-        o.forward(**sub, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+        oracle_step(o, sub, shape, tau, args.budget, cores)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        o.forward(**sub, top_k=shape.top_k, tau=tau, want_scores=False, nthreads=cores)
+        oracle_step(o, sub, shape, tau, args.budget, cores)
         times.append(time.perf_counter() - t0)
     ms = 1000 * statistics.mean(times)
     value = n_tok / (ms / 1000)
@@ -471,6 +486,45 @@ def launch_mode_rows(dev, flush, steps=20):
     return rows
 
 
+def rank_budget_rows(dev, flush, steps=20):
+    """The per-pair rank budget (each routed pair keeps its r = 10 % of d_ff
+    highest-scoring neurons) beside the threshold at 90 % sparsity, on the
+    OLMoE-shaped layer's decode batches.  The budget runs two sparse passes
+    (the routed gates, then the masked up/down) around a per-pair selection."""
+    import torch
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    shape = mi.SHAPES["olmoe"]
+    W = mi.make_weights(shape, device=dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=16)
+    del W
+    layer.set_path(m.MOE_PATH_SPARSE)
+    r = shape.d_ff // 10
+    rows = []
+    for T in (1, 4, 16):
+        x = mi.make_x(shape, T, device=dev)
+        out = torch.empty_like(x)
+        tau = layer.calibrate_tau(x, 0.9)
+        row = {"workload": "olmoe", "T": T, "budget": r, "tau": tau}
+        for name, budget in (("threshold", -1), ("budget", r)):
+            layer.set_rank_budget(budget)
+            for _ in range(3):
+                layer.forward(x, tau, out=out)
+            sm_, _, _ = time_steps(layer, x, tau, out, flush, steps)
+            st = layer.stats()
+            row[name + "_us"] = 1000 * statistics.mean(sm_)
+            row[name + "_alg_bytes"] = st["alg_bytes"]
+            row[name + "_n_active"] = st["n_active"]
+            if st["device_error"]:
+                row[name + "_device_error"] = st["device_error"]
+        layer.set_rank_budget(-1)
+        rows.append(row)
+        log(json.dumps({k: (round(v, 2) if isinstance(v, float) else v) for k, v in row.items()}))
+    layer.close()
+    torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -493,6 +547,8 @@ def run_ours(args):
     if args.path != "auto":
         layer.set_path({"sparse": m.MOE_PATH_SPARSE, "dense": m.MOE_PATH_DENSE}[args.path])
     layer.set_fused_router(args.router != "kernel", one_launch=args.router == "one_launch")
+    if args.budget >= 0:
+        layer.set_rank_budget(args.budget)
     out = torch.empty_like(x)
     tau = layer.calibrate_tau(x, args.sparsity)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -545,13 +601,14 @@ def run_ours(args):
 
     sweep = sweep_rows(dev, sweep_kind, peak, flush) if rank == 0 and sweep_kind != "none" else []
     modes = launch_mode_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
+    budget_rows = rank_budget_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = cpu_cores()
         W_host, x_host = W.to("cpu"), x.cpu()
-        tps, reps, el = oracle_time_sample(shape, W_host, x_host, tau, args.cpu_seconds, cores)
-        tps1, reps1, el1 = oracle_time_sample(shape, W_host, x_host[:4], tau, args.cpu_seconds / 2, 1)
+        tps, reps, el = oracle_time_sample(shape, W_host, x_host, tau, args.cpu_seconds, cores, args.budget)
+        tps1, reps1, el1 = oracle_time_sample(shape, W_host, x_host[:4], tau, args.cpu_seconds / 2, 1, args.budget)
         cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{reps} repeats of the {T}-token batch ({el:.1f} s, fp64 oracle at the bench's "
                          f"tau, OpenMP over tokens on {cores} threads)",
@@ -591,6 +648,7 @@ def run_ours(args):
             "stats": {"n_touched": st["n_touched"], "n_active": st["n_active"], "n_union": st["n_union"]},
             "sweep": sweep,
             "launch_modes": modes,
+            "rank_budget": budget_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

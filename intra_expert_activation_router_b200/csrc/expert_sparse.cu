@@ -148,7 +148,6 @@ struct SparseArgs {
     const int *rank_j;
     int score_signed;     // score mode: write silu(g) itself instead of |silu(g)|
     int tail;             // combine here: y_acc -> bf16 `out` after a grid-wide arrival count
-    int claim_ahead;      // resident mode: items a CTA may claim beyond its last masked one
     long long n_out4;     // float4 groups of y_acc converted (0 in score mode)
     SparseLayout L;
 };
@@ -844,7 +843,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                         const unsigned long long tc0 = tr ? global_ns() : 0;
                         bool ok = true;
                         for (uint32_t spin = 0;; ++spin) {
-                            if (*mask_done >= i - a.claim_ahead) {
+                            if (*mask_done >= i) {
                                 __threadfence_block();
                                 if (score_mode || *rec_masked - *rec_done <= kClaimBacklog) break;
                             }
@@ -1584,10 +1583,6 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     // the combine at the end of this kernel (one launch per forward), else a
     // separate conversion kernel
     a.tail = combine_here ? 1 : 0;
-    {
-        const char *ca = std::getenv("MOE_CLAIM_AHEAD");
-        a.claim_ahead = ca ? (int)std::strtol(ca, nullptr, 10) : 0;
-    }
     a.n_out4 = score_out ? 0 : (long long)T * dm.d / 4;
     if (grid < 1) grid = 1;
     cudaError_t e;
