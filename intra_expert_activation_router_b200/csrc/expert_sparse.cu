@@ -359,20 +359,27 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
     // 1. this CTA's experts' logits (fp32 accumulation of bf16 products); the
     //    batch's rows arrive by one bulk copy (x is [T][d], contiguous)
     int mine = 0;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 w0 = z, w1 = z;
     if ((int)blockIdx.x < E) {
         if (tid == 0) {
             mbar_arrive_expect_tx(xbar, (uint32_t)(T * d * 2));
             bulk_g2s(xs, a.x, (uint32_t)(T * d * 2), xbar);
         }
-        mbar_wait(xbar, 0, a.ws.error_word, 57);
+        // the first expert's router row is in flight while x arrives
+        const uint16_t *wrow = a.wr + (size_t)blockIdx.x * d;
+        if (tid < d8) w0 = ld_cached(wrow + 8 * tid);
+        if (tid + kSparseThreads < d8) w1 = ld_cached(wrow + 8 * (tid + kSparseThreads));
+        mbar_wait(xbar, 0, a.ws.error_word, 55);
     }
     __syncthreads();
 #pragma unroll 1
     for (int e = blockIdx.x; e < E; e += gridDim.x, ++mine) {
-        const uint16_t *wrow = a.wr + (size_t)e * d;
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        const uint4 w0 = tid < d8 ? ld_cached(wrow + 8 * tid) : z;
-        const uint4 w1 = tid + kSparseThreads < d8 ? ld_cached(wrow + 8 * (tid + kSparseThreads)) : z;
+        if (e != (int)blockIdx.x) {
+            const uint16_t *wrow = a.wr + (size_t)e * d;
+            w0 = tid < d8 ? ld_cached(wrow + 8 * tid) : z;
+            w1 = tid + kSparseThreads < d8 ? ld_cached(wrow + 8 * (tid + kSparseThreads)) : z;
+        }
 #pragma unroll 1
         for (int t0 = 0; t0 < T; t0 += 4) {   // four tokens per transposed warp reduction
             float acc[4];
@@ -833,7 +840,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             const uint64_t pol = policy_evict_first();
             uint32_t g = 0;
             unsigned long long t_claim = 0, t_ring = 0, t_last = 0;   // trace only
-            int next = a.resident ? atomicAdd(&plan->next_item, 1) : 0;
+            // resident mode: CTA b's first item is item b (all CTAs start at once,
+            // so no counter round trip); later ones come from the counter, past
+            // the grid's first items
+            int next = a.resident ? (int)blockIdx.x : 0;
             for (int i = 0;; ++i) {
                 int id;
                 if (a.resident) {
@@ -854,7 +864,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                             }
                             __nanosleep(128);
                         }
-                        next = ok ? atomicAdd(&plan->next_item, 1) : n_items;
+                        next = ok ? atomicAdd(&plan->next_item, 1) + (int)gridDim.x : n_items;
                         if (tr) t_claim += global_ns() - tc0;
                     }
                     id = next < n_items ? next : -1;
