@@ -140,7 +140,9 @@ int moe_set_t_star(moe_handle h, int t_star);
  * for batch sizes 1, 2, 3, 4, 6, 8, 12, 16, 24, ... up to T_max, the first T
  * rows of x (DEVICE [T_max][d_model] bf16, a representative batch) run through
  * both branches at threshold tau (the sparse branch's cost depends on it),
- * each timed on the device (median of five, L2 flushed before every run);
+ * each captured into a CUDA graph on a private stream and timed on the
+ * device as one graph launch (median of five, L2 flushed before every run),
+ * so neither branch is charged for host gaps between its kernels;
  * T* becomes the largest measured T at which the sparse branch was not
  * slower, and is stored in the handle and in *t_star_out (HOST pointer).
  * ("Uncovering Intra-expert Activation Sparsity...", technical summary,

@@ -409,31 +409,52 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
         *t_star_out = INT_MAX;
         return MOE_OK;
     }
-    cudaStream_t st = (cudaStream_t)stream;
+    // the caller's earlier work (x) is complete, then everything runs on a
+    // private stream, where each forward can be captured into a graph
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ECUDA;
     int l2 = 0;
     if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, h->device) != cudaSuccess) return MOE_ECUDA;
     const size_t flush_bytes = 2 * (size_t)(l2 > 0 ? l2 : (64 << 20));
     void *flush = nullptr;
     if (cudaMalloc(&flush, flush_bytes) != cudaSuccess) { cudaGetLastError(); return MOE_ENOMEM; }
+    cudaStream_t st = nullptr;
     cudaEvent_t e0 = nullptr, e1 = nullptr;
-    if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess || cudaEventCreate(&e0) != cudaSuccess ||
+        cudaEventCreate(&e1) != cudaSuccess) {
         if (e0) cudaEventDestroy(e0);
+        if (st) cudaStreamDestroy(st);
         cudaFree(flush);
+        cudaGetLastError();
         return MOE_ECUDA;
     }
     const int saved_ev = h->n_ev;
     h->n_ev = 0;   // the caller's launch events stay out of the tuning runs
-    // the median of five device-timed forwards of the first T rows of x, L2 flushed before each
+    // the median of five device-timed forwards of the first T rows of x, L2
+    // flushed before each; the forward is captured into a graph and launched
+    // whole, so neither branch pays for host-side gaps between its launches
     auto time_path = [&](int T, int path, float *us) -> int {
-        float t[5];
-        for (int r = -1; r < 5; ++r) {   // one untimed run first
-            if (cudaMemsetAsync(flush, r & 0xff, flush_bytes, st) != cudaSuccess) return MOE_ECUDA;
-            if (cudaEventRecord(e0, st) != cudaSuccess) return MOE_ECUDA;
-            const int frc = run_forward(h, x, T, tau, true, h->ws.out_stage, stream, path);
-            if (frc) return frc;
-            if (cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess) return MOE_ECUDA;
-            if (r >= 0 && cudaEventElapsedTime(&t[r], e0, e1) != cudaSuccess) return MOE_ECUDA;
+        cudaGraph_t g = nullptr;
+        cudaGraphExec_t ge = nullptr;
+        if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ECUDA;
+        const int frc = run_forward(h, x, T, tau, true, h->ws.out_stage, st, path);
+        const cudaError_t ce = cudaStreamEndCapture(st, &g);
+        if (frc || ce != cudaSuccess || cudaGraphInstantiate(&ge, g, 0) != cudaSuccess) {
+            if (g) cudaGraphDestroy(g);
+            cudaGetLastError();
+            return frc ? frc : MOE_ECUDA;
         }
+        float t[5];
+        int rc2 = MOE_OK;
+        for (int r = -1; r < 5 && rc2 == MOE_OK; ++r) {   // one untimed run first
+            if (cudaMemsetAsync(flush, r & 0xff, flush_bytes, st) != cudaSuccess ||
+                cudaEventRecord(e0, st) != cudaSuccess || cudaGraphLaunch(ge, st) != cudaSuccess ||
+                cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+                (r >= 0 && cudaEventElapsedTime(&t[r], e0, e1) != cudaSuccess))
+                rc2 = MOE_ECUDA;
+        }
+        cudaGraphExecDestroy(ge);
+        cudaGraphDestroy(g);
+        if (rc2 != MOE_OK) return rc2;
         std::sort(t, t + 5);
         *us = 1000.f * t[2];
         return MOE_OK;
@@ -455,6 +476,7 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
     h->n_ev = saved_ev;
     cudaEventDestroy(e0);
     cudaEventDestroy(e1);
+    cudaStreamDestroy(st);
     cudaFree(flush);
     if (rc != MOE_OK) return rc;
     h->t_star = best;
