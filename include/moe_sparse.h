@@ -273,6 +273,7 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
 int moe_set_trace(moe_handle h, void *buf, long long bytes);
 
 /* Statistics of the last forward.  Synchronises the stream of that forward
+ * (which must still exist; after moe_tune_t_star, the stream passed to it)
  * and reads device counters back; not for timed loops.
  * Device errors: forward calls do not synchronise, so they cannot report
  * what their kernels find (a bounded wait that ran out, error codes >= 30).

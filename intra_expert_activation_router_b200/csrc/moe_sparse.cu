@@ -474,6 +474,11 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
         if (T > T_max && last < T_max) T = T_max;
     }
     h->n_ev = saved_ev;
+    // the timing forwards ran on the private stream, which is about to go:
+    // moe_query_stats (which describes the last of them) synchronises the
+    // caller's stream instead; all of that work is complete already
+    if (cudaStreamSynchronize(st) != cudaSuccess && rc == MOE_OK) rc = MOE_ECUDA;
+    h->last_stream = (cudaStream_t)stream;
     cudaEventDestroy(e0);
     cudaEventDestroy(e1);
     cudaStreamDestroy(st);
