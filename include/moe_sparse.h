@@ -141,10 +141,12 @@ int moe_set_t_star(moe_handle h, int t_star);
  * rows of x (DEVICE [T_max][d_model] bf16, a representative batch) run through
  * both branches at threshold tau (the sparse branch's cost depends on it),
  * each captured into a CUDA graph on a private stream and timed on the
- * device as one graph launch (median of five, L2 flushed before every run),
- * so neither branch is charged for host gaps between its kernels;
- * T* becomes the largest measured T at which the sparse branch was not
- * slower, and is stored in the handle and in *t_star_out (HOST pointer).
+ * device as one graph launch (median of five; before every run a 2 x L2
+ * buffer is written and read back, so L2 holds no useful and no dirty line),
+ * so neither branch is charged for host gaps between its kernels; the
+ * search stops at the first T whose sparse time exceeds 98 % of the dense
+ * one, and T* becomes the last T before it; it is stored in the handle and
+ * in *t_star_out (HOST pointer).
  * ("Uncovering Intra-expert Activation Sparsity...", technical summary,
  * Methodology item 3, "Dynamic switching": sparse for small batches, dense
  * for large.)  Allocates and frees a 2 x L2-sized flush buffer; synchronises

@@ -148,11 +148,6 @@ struct SparseArgs {
     const int *rank_j;
     int score_signed;     // score mode: write silu(g) itself instead of |silu(g)|
     int tail;             // combine here: y_acc -> bf16 `out` after a grid-wide arrival count
-    // L2 prefetch while the batch is routed (the weights do not depend on the
-    // routing): the first pf_routed bytes of every routed expert's 128-neuron
-    // gate blocks (when most experts will be touched), pf_shared of every
-    // shared expert's (always touched); 0 = none
-    int pf_routed, pf_shared;
     long long n_out4;     // float4 groups of y_acc converted (0 in score mode)
     SparseLayout L;
 };
@@ -702,21 +697,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    // gate weights into L2 while the batch is routed (here, or by the router
-    // grid this launch overlaps): they do not depend on the routing
-    if (tid == kWarpTma * 32 && (a.pf_routed > 0 || a.pf_shared > 0)) {
-        const long long blk_bytes = (long long)a.n_kb * kGateTile;
-        const int n_sh = a.S * a.n_blk, n_all = n_sh + a.E * a.n_blk;
-#pragma unroll 1
-        for (int q = blockIdx.x; q < n_all; q += gridDim.x) {
-            const bool sh = q < n_sh;
-            const int nb = sh ? a.pf_shared : a.pf_routed;
-            const uint8_t *base = reinterpret_cast<const uint8_t *>(sh ? a.w.wsg_t : a.w.wg_t) +
-                                  (long long)(sh ? q : q - n_sh) * blk_bytes;
-#pragma unroll 1
-            for (int o = 0; o < nb; o += kStageBytes) prefetch_l2_bulk(base + o, (uint32_t)min(kStageBytes, nb - o));
-        }
-    }
     // everything above overlaps the router's tail (programmatic dependent
     // launch); the routing plan is read only after the router grid is done
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1613,23 +1593,6 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     // the combine at the end of this kernel (one launch per forward), else a
     // separate conversion kernel
     a.tail = combine_here ? 1 : 0;
-    // L2 prefetch during routing: the shared experts' gates always (up to
-    // 32 MB); the routed experts' first quarter of every block when the batch
-    // is expected to touch at least half the experts, within 64 MB in all
-    a.pf_routed = a.pf_shared = 0;
-    const char *pfe = std::getenv("MOE_PREFETCH_L2");
-    if (!score_out && a.resident && !a.a_in && !inject && !(pfe && std::strcmp(pfe, "0") == 0)) {
-        const long long blk_bytes = (long long)dm.n_kb * kGateTile;
-        const long long sh_total = (long long)dm.S * dm.n_blk * blk_bytes;
-        if (dm.S > 0 && sh_total <= (32ll << 20)) a.pf_shared = (int)blk_bytes;
-        const double untouched = std::pow(1.0 - (double)dm.k / dm.E, (double)T);
-        if (1.0 - untouched >= 0.5) {
-            const long long budget = (64ll << 20) - (a.pf_shared ? sh_total : 0);
-            long long per = std::min(blk_bytes / 4, budget / ((long long)dm.E * dm.n_blk));
-            per = per / kStageBytes * kStageBytes;
-            if (per > 0) a.pf_routed = (int)per;
-        }
-    }
     a.n_out4 = score_out ? 0 : (long long)T * dm.d / 4;
     if (grid < 1) grid = 1;
     cudaError_t e;

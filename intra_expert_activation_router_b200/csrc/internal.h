@@ -209,6 +209,8 @@ cudaError_t launch_mask_compact(const Workspace &ws, int n_pairs, int f, uint16_
 cudaError_t launch_stats(const Dims &dm, const Workspace &ws, int T, unsigned long long *out3,
                          cudaStream_t st);
 
+// Read `bytes` (a multiple of 16) of a device buffer once, discarding the values.
+cudaError_t launch_read_all(const void *buf, size_t bytes, unsigned *sink, int n_sm, cudaStream_t st);
 cudaError_t launch_radix_hist(const uint32_t *v, size_t n, uint32_t prefix, uint32_t prefix_mask,
                               int shift, unsigned *hist, int n_sm, cudaStream_t st);
 

@@ -447,6 +447,7 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
         int rc2 = MOE_OK;
         for (int r = -1; r < 5 && rc2 == MOE_OK; ++r) {   // one untimed run first
             if (cudaMemsetAsync(flush, r & 0xff, flush_bytes, st) != cudaSuccess ||
+                moe::launch_read_all(flush, flush_bytes, h->hist, h->n_sm, st) != cudaSuccess ||
                 cudaEventRecord(e0, st) != cudaSuccess || cudaGraphLaunch(ge, st) != cudaSuccess ||
                 cudaEventRecord(e1, st) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
                 (r >= 0 && cudaEventElapsedTime(&t[r], e0, e1) != cudaSuccess))
@@ -467,7 +468,10 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
         rc = time_path(T, MOE_PATH_SPARSE, &us_s);
         if (rc == MOE_OK) rc = time_path(T, MOE_PATH_DENSE, &us_d);
         if (rc != MOE_OK) break;
-        if (us_s > us_d) break;   // the dense branch is faster from here on
+        // the dense branch is faster from here on (a sparse time within 2 % of
+        // the dense one counts as slower: near the crossover either choice is
+        // within that margin, and the dense branch's cost grows more slowly)
+        if (us_s > 0.98f * us_d) break;
         best = T;
         last = T;
         T = T < 4 ? T + 1 : (T % 3 == 0 ? T * 4 / 3 : T * 3 / 2);
