@@ -13,6 +13,7 @@ the pairs the router selected), which is stated in ``calibrate_tau``.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 import tempfile
@@ -73,6 +74,9 @@ class Oracle:
         rm = self._lib.oracle_rank_mask
         rm.restype = ctypes.c_int
         rm.argtypes = [_P, ctypes.c_long, ctypes.c_int, ctypes.c_int, _P]
+        ck = self._lib.oracle_capacity_keep
+        ck.restype = ctypes.c_int
+        ck.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P]
 
     @staticmethod
     def _ptr(a):
@@ -144,6 +148,45 @@ class Oracle:
         mask = self.rank_mask(first.score, budget)
         res = self.forward(*args, top_k=top_k, tau=0.0, nthreads=nthreads, active=mask,
                            tau_shared=tau_shared)
+        res.score = first.score
+        return res
+
+    @staticmethod
+    def capacity(gamma: float, T: int, top_k: int, E: int) -> int:
+        """The per-expert capacity C = ceil(gamma * N), N = T * top_k / E the
+        mean number of pairs per expert; gamma <= 0: no capacity (-1)."""
+        if not gamma > 0:
+            return -1
+        return int(math.ceil(gamma * (T * top_k) / E))
+
+    def capacity_keep(self, topk_idx: np.ndarray, topk_w: np.ndarray, E: int, C: int) -> np.ndarray:
+        """[T][k] 1 for the pairs each expert keeps under capacity C (see
+        ``oracle_capacity_keep``)."""
+        idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+        w = np.ascontiguousarray(topk_w, dtype=np.float64)
+        T, k = idx.shape
+        keep = np.zeros((T, k), np.uint8)
+        rc = self._lib.oracle_capacity_keep(self._ptr(idx), self._ptr(w), T, k, int(E), int(C), self._ptr(keep))
+        if rc != 0:
+            raise RuntimeError(f"oracle_capacity_keep failed ({rc})")
+        return keep
+
+    def forward_capacity(self, x, w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None,
+                         ws_down=None, *, top_k: int, tau: float, gamma: float, nthreads: int = 0,
+                         tau_shared: float = 0.0) -> OracleResult:
+        """The layer with capacity-aware token drop at capacity factor gamma:
+        the routing, then each expert's kept pairs (``capacity_keep``), then
+        the layer with the dropped pairs' neurons all inactive (a dropped pair
+        contributes nothing).  ``active`` of the result is the threshold mask
+        with the dropped pairs cleared."""
+        args = (x, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+        first = self.forward(*args, top_k=top_k, tau=tau, nthreads=nthreads, tau_shared=tau_shared)
+        T = first.topk_idx.shape[0]
+        E = first.logits.shape[1]
+        C = self.capacity(gamma, T, top_k, E)
+        keep = self.capacity_keep(first.topk_idx, first.topk_w, E, C)
+        active = first.active * keep[:, :, None]
+        res = self.forward(*args, top_k=top_k, tau=tau, nthreads=nthreads, active=active, tau_shared=tau_shared)
         res.score = first.score
         return res
 

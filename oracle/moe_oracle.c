@@ -267,3 +267,38 @@ int oracle_rank_mask(const double *s, long n_pairs, int f, int r, uint8_t *mask)
     free(e);
     return 0;
 }
+
+/* Capacity-aware token drop ("Capacity-Aware Inference" page, section
+ * "Capacity-Aware Token Drop"): an expert holds at most C of the (token,
+ * expert) pairs routed to it.  When more are routed to it, it keeps the C
+ * pairs with the largest routing weight p (the post-softmax gate score),
+ * compared rounded to float as the CUDA path decides it, equal weights going
+ * to the lower token index; the other pairs are dropped and contribute
+ * nothing.  Kept pairs keep their weights (no renormalisation) and the
+ * token's other experts are unaffected.  Written as its definition: a pair is
+ * kept iff fewer than C pairs of the same expert beat it.
+ *   idx, w  [T][k] the router's selection and weights (rank order)
+ *   keep    [T][k] out: 1 kept, 0 dropped
+ * C < 0 keeps every pair.  Returns 0, or -1 on bad sizes. */
+int oracle_capacity_keep(const int *idx, const double *w, int T, int k, int E, int C, uint8_t *keep)
+{
+    if (T < 0 || k <= 0 || E <= 0 || !idx || !w || !keep) return -1;
+    const long P = (long)T * k;
+    for (long p = 0; p < P; ++p) {
+        if (C < 0) {
+            keep[p] = 1;
+            continue;
+        }
+        const int e = idx[p];
+        const float wp = (float)w[p];
+        const long tp = p / k;
+        long better = 0;
+        for (long q = 0; q < P; ++q) {
+            if (q == p || idx[q] != e) continue;
+            const float wq = (float)w[q];
+            if (wq > wp || (wq == wp && q / k < tp)) ++better;
+        }
+        keep[p] = (uint8_t)(better < C);
+    }
+    return 0;
+}

@@ -472,9 +472,87 @@ def pin_rank_layer(o):
     assert np.all(rb.active.sum(axis=2) == r)
 
 
+def _capacity_sorted(idx, w, E, C):
+    """Each expert's pairs sorted by (float32 weight descending, token
+    ascending); the first C are kept (C < 0: all)."""
+    T, k = idx.shape
+    keep = np.zeros((T, k), np.uint8)
+    for e in range(E):
+        pairs = [(t, r) for t in range(T) for r in range(k) if idx[t, r] == e]
+        pairs.sort(key=lambda tr: (-float(np.float32(w[tr])), tr[0]))
+        for t, r in (pairs if C < 0 else pairs[:C]):
+            keep[t, r] = 1
+    return keep
+
+
+def pin_capacity_bruteforce(o):
+    """Capacity-aware token drop against a per-expert sort: random routings
+    with exact weight ties, a pair tied in float but ordered in double, every
+    capacity from none to above T; kept count per expert = min(load, C);
+    capacities nest."""
+    rng = np.random.default_rng(91)
+    T, k, E = 12, 3, 5
+    idx = np.zeros((T, k), np.int32)
+    for t in range(T):
+        idx[t] = rng.choice(E, size=k, replace=False)
+    w = np.round(rng.random((T, k)) * 4) / 8 + 0.05        # many exact ties
+    w[2, 0], w[7, 0] = 0.3, 0.3 + 1e-12                    # equal in float: token 2 first
+    idx[2, 0] = idx[7, 0] = 1
+    prev = None
+    for C in range(-1, T + 2):
+        got = o.capacity_keep(idx, w, E, C)
+        want = _capacity_sorted(idx, w, E, C)
+        assert np.array_equal(got, want), ("capacity", C)
+        for e in range(E):
+            load = int((idx == e).sum())
+            assert int(got[idx == e].sum()) == (load if C < 0 else min(load, C)), ("count", C, e)
+        if prev is not None and C > 0:
+            assert np.all(prev <= got), ("nesting", C)
+        prev = got
+    assert o.capacity_keep(idx, w, E, -1).all() and not o.capacity_keep(idx, w, E, 0).any()
+    assert o.capacity(1.0, 16, 8, 64) == 2 and o.capacity(1.25, 16, 8, 64) == 3 and o.capacity(0.0, 16, 8, 64) == -1
+
+
+def pin_capacity_layer(o):
+    """The layer under capacity-aware token drop at tau = 0 against a torch
+    fp64 composition of the routed SwiGLU experts over the kept pairs only
+    (kept set from the per-expert sort), plus the shared expert; a capacity
+    of at least T equals the layer without it."""
+    d, E, f, k, S, T = 16, 4, 8, 2, 1, 7
+    x, W = _rand_layer(93, d, E, f, k, S, T, scale_x=1.0)
+    args = {n: _bits(t) for n, t in W.items()}
+    xb = _bits(x)
+    _, idx, p, _ = _torch_dense(x, W, k)
+    w = np.take_along_axis(p, idx, axis=1)
+    for gamma in (0.5, 0.8, 1.0):
+        C = o.capacity(gamma, T, k, E)
+        assert 0 < C < T
+        keep = _capacity_sorted(idx, w, E, C)
+        assert 0 < keep.sum() < T * k
+        xd = x.double()
+        y = torch.zeros_like(xd)
+        for t in range(T):
+            for r in range(k):
+                if keep[t, r]:
+                    e = int(idx[t, r])
+                    g = xd[t] @ W["w_gate"][e].double()
+                    u = xd[t] @ W["w_up"][e].double()
+                    y[t] += p[t, e] * ((F.silu(g) * u) @ W["w_down"][e].double())
+        for s_ in range(S):
+            g = xd @ W["ws_gate"][s_].double()
+            u = xd @ W["ws_up"][s_].double()
+            y += (F.silu(g) * u) @ W["ws_down"][s_].double()
+        r = o.forward_capacity(xb, **args, top_k=k, tau=0.0, gamma=gamma)
+        assert _rel(r.y, y.numpy()) < 1e-12, ("layer", gamma, _rel(r.y, y.numpy()))
+        assert np.array_equal(r.active.any(axis=2), keep.astype(bool))
+    big = o.forward_capacity(xb, **args, top_k=k, tau=0.0, gamma=100.0)
+    assert _rel(big.y, _call(o, x, W, k, 0.0).y) < 1e-15
+
+
 ALL_PINS = [pin_handworked, pin_tau0_is_dense, pin_tauinf_is_shared_only, pin_bruteforce,
             pin_mask_override, pin_shared_threshold, pin_nested_masks, pin_threshold_decomposition,
-            pin_router_ranking, pin_calibration, pin_rank_bruteforce, pin_rank_layer]
+            pin_router_ranking, pin_calibration, pin_rank_bruteforce, pin_rank_layer,
+            pin_capacity_bruteforce, pin_capacity_layer]
 
 
 def run_all(o):

@@ -48,6 +48,13 @@ MUTANTS = [
      "for (int q = 0; q < n && q <= r; ++q) mp[e[q].j] = 1;"),
     ("rank_keeps_nan", "if (sp[j] == sp[j]) {   /* not NaN */", "if (1) {"),
     ("rank_in_double", "const float va = (float)a->v, vb = (float)b->v;", "const double va = a->v, vb = b->v;"),
+    ("capacity_tie_to_higher_token", "if (wq > wp || (wq == wp && q / k < tp)) ++better;",
+     "if (wq > wp || (wq == wp && q / k > tp)) ++better;"),
+    ("capacity_keeps_lowest", "if (wq > wp || (wq == wp && q / k < tp)) ++better;",
+     "if (wq < wp || (wq == wp && q / k < tp)) ++better;"),
+    ("capacity_keeps_one_more", "keep[p] = (uint8_t)(better < C);", "keep[p] = (uint8_t)(better <= C);"),
+    ("capacity_across_experts", "if (q == p || idx[q] != e) continue;", "if (q == p) continue;"),
+    ("capacity_in_double", "const float wq = (float)w[q];", "const double wq = w[q];"),
 ]
 
 
