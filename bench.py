@@ -525,6 +525,44 @@ def rank_budget_rows(dev, flush, steps=20):
     return rows
 
 
+def capacity_rows(dev, flush, steps=20):
+    """Capacity-aware token drop (each expert keeps at most ceil(gamma T k / E)
+    pairs, the best by routing weight) beside the plain layer, on the
+    OLMoE-shaped layer at 90 % sparsity, both branches where each runs."""
+    import torch
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    shape = mi.SHAPES["olmoe"]
+    W = mi.make_weights(shape, device=dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=512)
+    del W
+    rows = []
+    for T, path in ((16, m.MOE_PATH_SPARSE), (64, m.MOE_PATH_DENSE), (512, m.MOE_PATH_DENSE)):
+        x = mi.make_x(shape, T, device=dev)
+        out = torch.empty_like(x)
+        tau = layer.calibrate_tau(x, 0.9)
+        layer.set_path(path)
+        row = {"workload": "olmoe", "T": T, "path": "sparse" if path == m.MOE_PATH_SPARSE else "dense"}
+        for name, gamma in (("plain", 0.0), ("gamma1", 1.0), ("gamma1_25", 1.25)):
+            layer.set_capacity(gamma)
+            for _ in range(3):
+                layer.forward(x, tau, out=out)
+            sm_, _, _ = time_steps(layer, x, tau, out, flush, steps)
+            st = layer.stats()
+            row[name + "_us"] = 1000 * statistics.mean(sm_)
+            row[name + "_capacity"] = st["capacity"]
+            row[name + "_alg_bytes"] = st["alg_bytes"] if row["path"] == "sparse" else st["dense_bytes"]
+            if st["device_error"]:
+                row[name + "_device_error"] = st["device_error"]
+        layer.set_capacity(0.0)
+        layer.set_path(m.MOE_PATH_AUTO)
+        rows.append(row)
+        log(json.dumps({k: (round(v, 2) if isinstance(v, float) else v) for k, v in row.items()}))
+    layer.close()
+    torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -602,6 +640,7 @@ def run_ours(args):
     sweep = sweep_rows(dev, sweep_kind, peak, flush) if rank == 0 and sweep_kind != "none" else []
     modes = launch_mode_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
     budget_rows = rank_budget_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
+    cap_rows = capacity_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -649,6 +688,7 @@ def run_ours(args):
             "sweep": sweep,
             "launch_modes": modes,
             "rank_budget": budget_rows,
+            "capacity_drop": cap_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -95,6 +95,8 @@ typedef struct {
     int fused_router;      /* the last forward's moe_set_fused_router mode if it
                               routed the batch inside the expert kernel (1: no
                               router launch, 2: one launch), else 0              */
+    int capacity;          /* pairs per expert the last forward kept at most
+                              (moe_set_capacity), -1 if it dropped none          */
 } moe_stats;
 
 /* Create a layer.  Copies and repacks the weights into library-owned device
@@ -226,6 +228,24 @@ int moe_set_shared_tau(moe_handle h, float tau_shared);
  * r >= 0 allocates max_tokens * top_k * (d_ff + 2) floats (MOE_ENOMEM if that
  * fails, the setting unchanged); moe_sparse_destroy frees them. */
 int moe_set_rank_budget(moe_handle h, int r);
+
+/* Capacity-aware token drop ("Capacity-Aware Inference" page, section
+ * "Capacity-Aware Token Drop"): with gamma > 0, on later forwards every
+ * routed expert holds at most C = ceil(gamma * T * top_k / E) of the batch's
+ * (token, expert) pairs (the mean load times the capacity factor, rounded
+ * up).  An expert routed more pairs keeps the C with the largest routing
+ * weight (softmax probability, fp32), equal weights going to the lower token
+ * index; the dropped pairs contribute nothing (their mask lists are empty),
+ * the kept ones keep their weights (no renormalisation), and the shared
+ * experts are unaffected.  moe_debug_router still reports the router's
+ * selection before the drop; moe_query_stats' counts are after it.  The drop
+ * is applied in the router kernel's bucketing, so such forwards do not route
+ * inside the expert kernel; a batch of more than 4096 pairs whose capacity is
+ * below T returns MOE_ENOTSUP (C >= T drops nothing and is always allowed).
+ * gamma <= 0 (the default) turns it off; NaN is MOE_EINVAL.  The dropping
+ * makes pairs' work depend on the rest of the batch, which is the method's
+ * intent; outputs then differ from the plain layer. */
+int moe_set_capacity(moe_handle h, float gamma);
 
 /* As moe_calibrate_tau, over the N = T*n_shared*d_ff scores of the shared
  * experts' neurons: the floor(q*N)-th smallest |silu(x Ws_g)| (0-based, exact

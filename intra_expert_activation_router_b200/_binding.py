@@ -51,7 +51,8 @@ class moe_stats(ctypes.Structure):
                 ("t_star", ctypes.c_int), ("n_active", ctypes.c_longlong),
                 ("n_union", ctypes.c_longlong), ("alg_bytes", ctypes.c_double),
                 ("dense_bytes", ctypes.c_double), ("device_error", ctypes.c_int),
-                ("fused_router", ctypes.c_int)]
+                ("fused_router", ctypes.c_int),
+                ("capacity", ctypes.c_int)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -82,6 +83,7 @@ def _load():
         "moe_set_fused_router": (I, [P, I]),
         "moe_set_shared_tau": (I, [P, F]),
         "moe_set_rank_budget": (I, [P, I]),
+        "moe_set_capacity": (I, [P, F]),
         "moe_calibrate_tau_shared": (I, [P, P, I, ctypes.c_double, ctypes.POINTER(F), P]),
         "moe_tune_t_star": (I, [P, P, I, F, ctypes.POINTER(I), P]),
         "moe_strerror": (ctypes.c_char_p, [I]),
@@ -99,7 +101,7 @@ EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
             "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
             "moe_debug_inject", "moe_set_fused_router", "moe_set_shared_tau", "moe_calibrate_tau_shared",
-            "moe_tune_t_star", "moe_set_rank_budget")
+            "moe_tune_t_star", "moe_set_rank_budget", "moe_set_capacity")
 
 
 def _addr(t):
@@ -226,6 +228,10 @@ def moe_router_topk_noalloc(x, T: int, w_router, E: int, d_model: int, top_k: in
 
 def moe_set_shared_tau(h, tau_shared: float):
     _check(_lib.moe_set_shared_tau(h, float(tau_shared)), "moe_set_shared_tau")
+
+
+def moe_set_capacity(h, gamma: float):
+    _check(_lib.moe_set_capacity(h, float(gamma)), "moe_set_capacity")
 
 
 def moe_set_rank_budget(h, r: int):

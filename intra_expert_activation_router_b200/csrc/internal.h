@@ -168,8 +168,10 @@ __device__ __forceinline__ unsigned long long global_ns()
 // Launchers (return cudaGetLastError()).
 // Routing plan with sparse work items of (expert, tile of `tile_tokens`
 // tokens, 128-neuron block).
+// cap >= 0: capacity-aware token drop, each expert keeps at most cap pairs
+// (batches of up to 4096 pairs; cudaErrorNotSupported above).
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st);
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap = -1);
 // inject: test-only fault (MOE_INJECT_WITHHOLD_ITEMS: the gate lane publishes
 // no work item, so the consumers' bounded waits run out), 0 otherwise.
 // fused: the kernel routes the batch itself (no router launch before it);

@@ -64,6 +64,8 @@ struct moe_sparse_s {
     float *rank_a;       // [max_tokens * k][f] silu(g) of the first pass
     float *rank_v;       // [max_tokens * k] cut values
     int *rank_j;         // [max_tokens * k] last tied index kept
+    float cap_gamma;     // capacity factor of the token drop (moe_set_capacity); <= 0: none
+    int last_cap;        // the capacity the last forward applied (-1: none)
 };
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -264,6 +266,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     }
     h->fused_router = 1;
     h->rank_r = -1;
+    h->last_cap = -1;
     h->last_T = 0;
     h->last_path = MOE_PATH_SPARSE;
     h->last_masked = 1;
@@ -296,6 +299,16 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     if (path == MOE_PATH_AUTO) path = h->path;
     if (path == MOE_PATH_AUTO) path = (T <= h->t_star) ? MOE_PATH_SPARSE : MOE_PATH_DENSE;
     const bool rank = masked && h->rank_r >= 0;
+    // capacity-aware token drop: C = ceil(gamma * T * k / E) pairs per expert;
+    // an expert holds at most T pairs, so C >= T drops nothing
+    int cap = -1;
+    if (h->cap_gamma > 0.f) {
+        const double c = std::ceil((double)h->cap_gamma * ((double)T * h->dm.k) / h->dm.E);
+        if (c < (double)T) {
+            if ((long long)T * h->dm.k > 4096) return MOE_ENOTSUP;
+            cap = (int)c;
+        }
+    }
     if (rank) {   // the rank budget is built on the sparse path only
         if (forced_path == MOE_PATH_DENSE || (forced_path == MOE_PATH_AUTO && h->path == MOE_PATH_DENSE))
             return MOE_ENOTSUP;
@@ -311,16 +324,17 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     cudaError_t e = cudaSuccess;
     // inside a stream capture the launch events must be external nodes, so that
     // every replay records them; outside a capture a plain record
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (h->n_ev && cudaStreamIsCapturing(st, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusNone;
-    const unsigned ev_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    cudaStreamCaptureStatus capst = cudaStreamCaptureStatusNone;
+    if (h->n_ev && cudaStreamIsCapturing(st, &capst) != cudaSuccess) capst = cudaStreamCaptureStatusNone;
+    const unsigned ev_flags =
+        capst == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
     if (h->n_ev) e = cudaEventRecordWithFlags(h->ev[0], st, ev_flags);
     bool fused = false;
     if (path == MOE_PATH_SPARSE) {
         const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
         // decode batches route inside the expert kernel: no router launch
-        fused = !rank && h->fused_router && moe::fused_possible(h->dm, T);
-        if (e == cudaSuccess && !fused) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st);
+        fused = !rank && cap < 0 && h->fused_router && moe::fused_possible(h->dm, T);
+        if (e == cudaSuccess && !fused) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st, cap);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (rank) {   // silu(g) of the routed pairs, each pair's cut, then the masked layer
             moe::RankPass r1{h->rank_a, nullptr, nullptr, false};
@@ -340,7 +354,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         }
         h->inject_next = 0;
     } else {
-        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st);
+        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st, cap);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
             e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st, h->tau_shared, h->n_sm);
@@ -350,6 +364,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     h->last_path = path;
     h->last_masked = masked;
     h->last_fused = fused ? h->fused_router : 0;
+    h->last_cap = cap;
     h->last_stream = st;
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -617,6 +632,14 @@ extern "C" int moe_set_rank_budget(moe_handle h, int r)
     return MOE_OK;
 }
 
+extern "C" int moe_set_capacity(moe_handle h, float gamma)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (std::isnan(gamma)) return MOE_EINVAL;
+    h->cap_gamma = gamma > 0.f ? gamma : 0.f;
+    return MOE_OK;
+}
+
 extern "C" int moe_set_launch_events(moe_handle h, void *const *events, int n)
 {
     if (!is_live(h)) return MOE_EHANDLE;
@@ -656,6 +679,7 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
     st->n_tokens = h->last_T;
     st->t_star = h->t_star;
     st->fused_router = h->last_fused;
+    st->capacity = h->last_cap;
     if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
     // the first error code since the previous call: an earlier forward's (kept
     // in the sticky word by the router of the next forward), else the last

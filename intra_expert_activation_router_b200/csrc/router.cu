@@ -36,6 +36,8 @@ struct RouterArgs {
     int mt, n_chunks;   // sparse work items per expert: ceil(tokens / mt) * n_chunks
     int dp;             // d rounded up to 128
     int xtile;          // T <= xtile <= 16: also write x into ws.x_tiles with xtile rows; else 0
+    int cap;            // capacity-aware token drop: pairs an expert keeps (-1: no capacity)
+    int mask_words;     // 32-neuron mask words per pair (cleared for dropped pairs)
     Workspace ws;
 };
 
@@ -61,6 +63,35 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
     for (int p = tid; p < P; p += blockDim.x)
         atomicAdd(&s_cnt[staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)], 1);
     __syncthreads();
+    if (staged && a.cap >= 0) {
+        // Capacity-aware token drop ("Capacity-Aware Inference", "Capacity-
+        // Aware Token Drop"): an expert routed more than cap pairs keeps the
+        // cap with the largest routing weight, ties to the lower token.  A pair
+        // is dropped when at least cap pairs of its expert beat it; it then
+        // belongs to no expert's list and its mask words read as empty.
+        uint32_t drop = 0;   // bit i: pair tid + i * blockDim.x (P <= kStagePairs = 16 * 256)
+        for (int p = tid, i = 0; p < P; p += blockDim.x, ++i) {
+            const int e = s_idx[p];
+            if (s_cnt[e] <= a.cap) continue;
+            const float wp = s_w[p];
+            const int tp = p / a.k;
+            int better = 0;
+            for (int q = 0; q < P; ++q) {
+                if (q == p || s_idx[q] != e) continue;
+                const float wq = s_w[q];
+                better += (wq > wp || (wq == wp && q / a.k < tp)) ? 1 : 0;
+            }
+            if (better >= a.cap) drop |= 1u << i;
+        }
+        __syncthreads();
+        for (int p = tid, i = 0; p < P; p += blockDim.x, ++i)
+            if ((drop >> i) & 1u) {
+                atomicSub(&s_cnt[s_idx[p]], 1);
+                s_idx[p] = E;
+                for (int c = 0; c < a.mask_words; ++c) a.ws.mask[(size_t)p * a.mask_words + c] = 0u;
+            }
+        __syncthreads();
+    }
     if (warp == 0) {
         // exclusive scans over experts: positions, touched slots, work items, dense tiles
         const int per = (E + 31) / 32;
@@ -116,14 +147,17 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
         // stable scatter, 32 pairs at a time in pair order
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
-            const int e = p < P ? (staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)) : -1 - lane;
+            // a dropped pair (expert E) takes no position
+            const int ep = p < P ? (staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)) : E;
+            const bool live = ep < E;
+            const int e = live ? ep : -1 - lane;
             const unsigned same = __match_any_sync(kFull, e);
             const int rank = __popc(same & ((1u << lane) - 1));
             int pos = 0;
-            if (p < P) pos = s_cur[e] + rank;
+            if (live) pos = s_cur[e] + rank;
             __syncwarp();
-            if (p < P && rank == 0) s_cur[e] += __popc(same);
-            if (p < P) {
+            if (live && rank == 0) s_cur[e] += __popc(same);
+            if (live) {
                 a.ws.perm[pos] = p;
                 a.ws.perm_tok[pos] = p / a.k;
                 a.ws.perm_w[pos] = staged ? s_w[p] : __ldcg(&a.ws.topk_w[p]);
@@ -341,8 +375,9 @@ __global__ void __launch_bounds__(256) k_plan_scatter(Workspace ws, int P, int k
 }
 
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st)
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap)
 {
+    if (cap >= 0 && (long long)T * dm.k > kStagePairs) return cudaErrorNotSupported;
     RouterArgs a;
     a.x = x;
     a.wr = w.wr;
@@ -354,6 +389,8 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     a.n_chunks = dm.n_blk;
     a.dp = dm.dp;
     a.xtile = (T <= tile_tokens && tile_tokens <= 16) ? tile_tokens : 0;
+    a.cap = cap;
+    a.mask_words = dm.f / kChunk;
     a.ws = ws;
     dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
     const size_t P = (size_t)T * dm.k;

@@ -83,6 +83,12 @@ class MoESparseLayer:
         forwards instead of thresholding at tau (r < 0: back to the threshold)."""
         B.moe_set_rank_budget(self.h, int(r))
 
+    def set_capacity(self, gamma: float):
+        """Capacity-aware token drop on later forwards: each expert keeps at most
+        ceil(gamma * T * top_k / E) pairs, the ones with the largest routing
+        weight (gamma <= 0: off)."""
+        B.moe_set_capacity(self.h, float(gamma))
+
     def calibrate_tau_shared(self, x, sparsity: float, stream=None) -> float:
         """tau_shared keeping about 1 - sparsity of the shared experts' neurons of this batch."""
         self._check_x(x)

@@ -552,3 +552,92 @@ def test_rank_budget_exact_ties():
                 assert layer.stats()["device_error"] == 0
     finally:
         layer.close()
+
+
+@pytest.mark.parametrize("name,T,gamma,path", [("tiny", 16, 1.0, "sparse"), ("olmoe", 16, 1.0, "sparse"),
+                                               ("olmoe", 16, 1.5, "sparse"), ("olmoe", 40, 1.0, "sparse"),
+                                               ("olmoe", 256, 1.25, "dense"), ("dsv2lite", 32, 1.0, "sparse"),
+                                               ("dsv2lite", 32, 1.0, "dense")])
+def test_capacity_drop(o, name, T, gamma, path):
+    """Capacity-aware token drop: each expert keeps at most ceil(gamma T k / E)
+    pairs, the ones with the largest routing weight.  The kept pairs are
+    compared with the oracle's exactly, except experts whose cut falls between
+    weights within 1e-6 of each other (fp32 softmax against the oracle's
+    rounding); the output against the oracle under the GPU's kept set and mask."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    g32 = float(np.float32(gamma))
+    C = oracle.Oracle.capacity(g32, T, sh.top_k, sh.n_experts)
+    assert 0 < C < T
+    tau = pu.calibrate(o, inputs, sh.top_k, 0.9, NTHREADS)
+    ref = o.forward_capacity(**inputs, top_k=sh.top_k, tau=tau, gamma=g32, nthreads=NTHREADS)
+    layer.set_capacity(gamma)
+    try:
+        layer.set_path(m.MOE_PATH_SPARSE if path == "sparse" else m.MOE_PATH_DENSE)
+        out = layer.forward(x, tau)
+        st = layer.stats()
+        assert st["capacity"] == C and st["device_error"] == 0
+        idx, w = layer.router(x)
+        torch.cuda.synchronize()
+        tie = pu.check_router(ref, idx.cpu().numpy(), w.cpu().numpy(), sh.top_k)
+        keep_ref = ref.active.any(axis=2)
+        # experts whose C-th and (C+1)-th weights are within 1e-6: either order is right
+        wr = ref.topk_w.astype(np.float32)
+        amb_e = set()
+        for e in np.unique(ref.topk_idx):
+            ws_ = np.sort(wr[ref.topk_idx == e])[::-1]
+            if ws_.size > C and ws_[C - 1] - ws_[C] <= 1e-6 * ws_[C - 1]:
+                amb_e.add(int(e))
+        assert len(amb_e) <= 2, amb_e
+        amb = np.isin(ref.topk_idx, list(amb_e))
+        if path == "sparse":
+            lists, cnt = layer.active_lists(x, tau)
+            torch.cuda.synchronize()
+            cnt = cnt.cpu().numpy()
+            keep_gpu = cnt > 0
+            ok = ~amb & ~tie[:, None]
+            assert np.array_equal(keep_gpu[ok], keep_ref[ok]), "kept pairs differ"
+            flipped, _, gm = pu.check_active(ref, tau, lists.cpu().numpy().view(np.uint16), cnt, tie | amb.any(axis=1))
+            y = pu.expected_under_gpu_mask(o, inputs, sh.top_k, tau, ref, gm, flipped, tie, NTHREADS)
+            pu.check_output(y, out, tie | amb.any(axis=1))
+        else:
+            import dataclasses
+            sc = ref.score.copy()
+            sc[~keep_ref] = -1.0   # a dropped pair's neurons are never near the threshold
+            pu.check_output_any_band_decision(o, inputs, sh.top_k, tau, dataclasses.replace(ref, score=sc), out,
+                                              tie | amb.any(axis=1), 1e-5, nthreads=NTHREADS)
+        # a large factor drops nothing: the plain layer
+        layer.set_capacity(1000.0)
+        out2 = layer.forward(x, tau)
+        assert layer.stats()["capacity"] == -1
+        ref2 = o.forward(**inputs, top_k=sh.top_k, tau=tau, nthreads=NTHREADS)
+        if path == "dense":
+            pu.check_output_any_band_decision(o, inputs, sh.top_k, tau, ref2, out2, tie, 1e-5, nthreads=NTHREADS)
+    finally:
+        layer.set_capacity(0.0)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
+def test_capacity_limits(o):
+    """A capacity below T on more than 4096 pairs is refused; gamma <= 0 turns
+    the drop off; NaN is rejected."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    x = mi.make_x(sh, 1024, device="cuda")
+    layer.set_capacity(1.0)
+    try:
+        with pytest.raises(m.MoeError) as ei:
+            layer.forward(x, 1.0)
+        assert ei.value.code == m.MOE_ENOTSUP
+        layer.set_capacity(-1.0)
+        layer.forward(x[:8], 1.0)
+        assert layer.stats()["capacity"] == -1
+        with pytest.raises(m.MoeError):
+            layer.set_capacity(float("nan"))
+    finally:
+        layer.set_capacity(0.0)
