@@ -47,7 +47,7 @@ __device__ __forceinline__ bool better(float v1, int i1, float v0, int i0)
 }
 
 // Build the routing plan from topk_idx; executed by one whole CTA.
-__device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_idx, float *s_w)
+__device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_idx, float *s_w, int *s_seg)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, P = a.T * a.k;
@@ -66,26 +66,55 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
     if (staged && a.cap >= 0) {
         // Capacity-aware token drop ("Capacity-Aware Inference", "Capacity-
         // Aware Token Drop"): an expert routed more than cap pairs keeps the
-        // cap with the largest routing weight, ties to the lower token.  A pair
-        // is dropped when at least cap pairs of its expert beat it; it then
-        // belongs to no expert's list and its mask words read as empty.
-        uint32_t drop = 0;   // bit i: pair tid + i * blockDim.x (P <= kStagePairs = 16 * 256)
-        for (int p = tid, i = 0; p < P; p += blockDim.x, ++i) {
-            const int e = s_idx[p];
-            if (s_cnt[e] <= a.cap) continue;
-            const float wp = s_w[p];
-            const int tp = p / a.k;
-            int better = 0;
-            for (int q = 0; q < P; ++q) {
-                if (q == p || s_idx[q] != e) continue;
-                const float wq = s_w[q];
-                better += (wq > wp || (wq == wp && q / a.k < tp)) ? 1 : 0;
+        // cap with the largest routing weight, ties to the lower token.  The
+        // pairs are first grouped by expert in token order (s_seg); a pair of
+        // an over-capacity expert is dropped when at least cap pairs of its
+        // group beat it.  A dropped pair then belongs to no expert's list
+        // (sentinel E) and its mask words read as empty.
+        if (warp == 0) {
+            int run = 0;
+            for (int e0 = 0; e0 < E; e0 += 32) {
+                const int e = e0 + lane, c = e < E ? s_cnt[e] : 0;
+                int inc = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(kFull, inc, o);
+                    if (lane >= o) inc += u;
+                }
+                if (e < E) s_cur[e] = run + inc - c;
+                run += __shfl_sync(kFull, inc, 31);
             }
-            if (better >= a.cap) drop |= 1u << i;
+            __syncwarp();
+            for (int base = 0; base < P; base += 32) {   // stable: 32 pairs at a time, in pair order
+                const int p = base + lane;
+                const int e = p < P ? s_idx[p] : -1 - lane;
+                const unsigned same = __match_any_sync(kFull, e);
+                const int rank = __popc(same & ((1u << lane) - 1));
+                const int pos = p < P ? s_cur[e] + rank : 0;
+                __syncwarp();
+                if (p < P && rank == 0) s_cur[e] += __popc(same);
+                if (p < P) s_seg[pos] = p;
+                __syncwarp();
+            }
+        }
+        __syncthreads();   // s_cur[e] now ends expert e's group
+        uint32_t drop = 0;   // bit i: the pair at group position tid + i * blockDim.x
+        for (int i = tid, bit = 0; i < P; i += blockDim.x, ++bit) {
+            const int p = s_seg[i], e = s_idx[p];
+            if (s_cnt[e] <= a.cap) continue;
+            const int g1 = s_cur[e], g0 = g1 - s_cnt[e];
+            const float wp = s_w[p];
+            int better = 0;
+            for (int j = g0; j < g1; ++j) {   // earlier positions hold lower tokens
+                const float wq = s_w[s_seg[j]];
+                better += (wq > wp || (wq == wp && j < i)) ? 1 : 0;
+            }
+            if (better >= a.cap) drop |= 1u << bit;
         }
         __syncthreads();
-        for (int p = tid, i = 0; p < P; p += blockDim.x, ++i)
-            if ((drop >> i) & 1u) {
+        for (int i = tid, bit = 0; i < P; i += blockDim.x, ++bit)
+            if ((drop >> bit) & 1u) {
+                const int p = s_seg[i];
                 atomicSub(&s_cnt[s_idx[p]], 1);
                 s_idx[p] = E;
                 for (int c = 0; c < a.mask_words; ++c) a.ws.mask[(size_t)p * a.mask_words + c] = 0u;
@@ -353,7 +382,8 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     const bool staged = P <= kStagePairs;
     if (tr && threadIdx.x == 0) tr[4] = global_ns();
     build_plan(a, s_int, s_int + a.E, staged ? s_int + 2 * a.E : nullptr,
-               staged ? reinterpret_cast<float *>(s_int + 2 * a.E + P) : nullptr);
+               staged ? reinterpret_cast<float *>(s_int + 2 * a.E + P) : nullptr,
+               staged && a.cap >= 0 ? s_int + 2 * a.E + 2 * P : nullptr);
     __syncthreads();
     if (tr && threadIdx.x == 0) tr[5] = global_ns();
 }
@@ -396,9 +426,15 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     const size_t P = (size_t)T * dm.k;
     size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // softmax rows
     if (smem < 16 * (size_t)kRtTok * 256) smem = 16 * (size_t)kRtTok * 256;   // x chunk
-    size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (P <= kStagePairs ? 8 * P : 0);
+    size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (P <= kStagePairs ? (cap >= 0 ? 12 : 8) * P : 0);
     if (plan_smem > smem) smem = plan_smem;
-    // at most max(32 KB, 2*1024*4 + 8*4096 = 40 KB): inside the default 48 KB window
+    // at most max(32 KB, 2*1024*4 + 12*4096 = 56 KB): above the default 48 KB
+    // window only with a capacity
+    static int smem_set[kMaxDevices] = {};
+    if (smem > 48 * 1024) {
+        const cudaError_t e = ensure_dynamic_smem(k_router, (int)smem, smem_set);
+        if (e != cudaSuccess) return e;
+    }
     k_router<<<grid, 256, smem, st>>>(a);
     if ((long long)T * dm.k > kStagePairs) {
         const int P = T * dm.k;
