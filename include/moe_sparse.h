@@ -146,8 +146,9 @@ int moe_set_t_star(moe_handle h, int t_star);
  * device as one graph launch (median of five; before every run a 2 x L2
  * buffer is written and read back, so L2 holds no useful and no dirty line),
  * so neither branch is charged for host gaps between its kernels; the
- * search stops at the first T whose sparse time exceeds 98 % of the dense
- * one, and T* becomes the last T before it; it is stored in the handle and
+ * search stops at the first T whose sparse time exceeds 90 % of the dense
+ * one (the sparse branch's cost varies with how a batch routes), and T*
+ * becomes the last T before it; it is stored in the handle and
  * in *t_star_out (HOST pointer).
  * ("Uncovering Intra-expert Activation Sparsity...", technical summary,
  * Methodology item 3, "Dynamic switching": sparse for small batches, dense

@@ -483,10 +483,12 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
         rc = time_path(T, MOE_PATH_SPARSE, &us_s);
         if (rc == MOE_OK) rc = time_path(T, MOE_PATH_DENSE, &us_d);
         if (rc != MOE_OK) break;
-        // the dense branch is faster from here on (a sparse time within 2 % of
-        // the dense one counts as slower: near the crossover either choice is
-        // within that margin, and the dense branch's cost grows more slowly)
-        if (us_s > 0.98f * us_d) break;
+        // the dense branch is faster from here on.  A sparse time within 10 %
+        // of the dense one counts as slower: the sparse branch's cost depends
+        // on how the batch routes (its load balance over the experts), which
+        // the representative batch only samples, while the dense branch's cost
+        // is nearly the same for every batch of a size
+        if (us_s > 0.9f * us_d) break;
         best = T;
         last = T;
         T = T < 4 ? T + 1 : (T % 3 == 0 ? T * 4 / 3 : T * 3 / 2);
