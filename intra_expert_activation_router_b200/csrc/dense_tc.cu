@@ -18,7 +18,7 @@
 // own threshold (none by default) and weight 1.  The GEMM kernel is
 // persistent (one CTA per SM walking its tiles): warp 0 issues the TMA loads
 // into a 4-stage ring, warp 1 issues the MMAs from one thread into two TMEM
-// accumulators in turn, and four epilogue warps read one accumulator back
+// accumulators in turn, and eight epilogue warps read one accumulator back
 // while the MMAs fill the other.  Operands are K-major with the 128-byte
 // swizzle; the gate weights are stored in HBM as exactly these tiles
 // (gate_tile_off), so each is one plain 16 KB bulk copy.
@@ -33,7 +33,8 @@ namespace moe {
 constexpr int kBM = 128;            // token rows per tile
 constexpr int kBK = 64;             // K per stage (128 bytes of bf16)
 constexpr int kDStages = 4;
-constexpr int kDenseThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kDenseThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each half of the columns
 constexpr int kAccCols = 256;        // one accumulator: 128 lanes x 256 fp32 columns
 constexpr int kATileBytes = kBM * kBK * 2;    // 16 KB
 constexpr int kBTileBytes = 256 * kBK * 2;    // 32 KB
@@ -158,8 +159,9 @@ __device__ __forceinline__ DenseTile dense_tile(const DenseArgs &a, int t)
 // Persistent: one CTA per SM walks the launch's tiles t = blockIdx.x,
 // blockIdx.x + gridDim.x, ...  Warp 0 streams every tile's K blocks into a
 // 4-stage ring without pausing between tiles, warp 1 issues the MMAs into one
-// of two 256-column TMEM accumulators, and warps 2-5 (one TMEM lane quarter
-// each) run the epilogue of tile i while the MMAs of tile i + 1 proceed.
+// of two 256-column TMEM accumulators, and warps 2-9 (two per TMEM lane
+// quarter, each half of the columns) run the epilogue of tile i while the
+// MMAs of tile i + 1 proceed.
 __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_constant__ DenseMaps maps, DenseArgs a)
 {
     extern __shared__ uint8_t dsmem_raw[];
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDStages * kStageBytes);
     uint64_t *empty = full + kDStages;
     uint64_t *accf = empty + kDStages;   // [2] accumulator ready (MMA commit)
-    uint64_t *acce = accf + 2;           // [2] accumulator read out (4 epilogue warps)
+    uint64_t *acce = accf + 2;           // [2] accumulator read out (the epilogue warps)
     uint64_t *mdrain = acce + 2;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mdrain + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 4);
+            mbar_init(&acce[b], kEpiWarps);
         }
         mbar_init(mdrain, 1);
         fence_mbar_init();
@@ -260,8 +262,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
         }
         __syncwarp();
     } else {
-        // ---- epilogue: thread = accumulator row (TMEM lane 32 * (warp % 4) + lane)
-        const int q = warp & 3;
+        // ---- epilogue: thread = accumulator row (TMEM lane 32 * (warp % 4) + lane);
+        // warps 2-5 take the first half of the tile's columns, warps 6-9 the second
+        const int q = warp & 3, half = (warp - 2) >> 2;
         const int row = q * 32 + lane;
         int lt = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
             const uint32_t tl = tmem + acc * kAccCols + ((uint32_t)(q * 32) << 16);
             if (a.mode == kGateUp) {
                 uint16_t *hrow = a.h + (size_t)(a.h_base + dt.row0 + row) * a.h_ld + dt.n0;
-                for (int c = 0; c < 128; c += 16) {
+                for (int c = 64 * half; c < 64 * half + 64; c += 16) {
                     float g[16], u[16];
                     tmem_ld16(tl + c, g);
                     tmem_ld16(tl + 128 + c, u);
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
                     w = a.shared ? 1.f : a.perm_w[dt.row0 + row];
                 }
                 float *yrow = a.y_acc + (size_t)tok * a.d + dt.n0;
-                for (int c = 0; c < 256; c += 16) {
+                for (int c = 128 * half; c < 128 * half + 128; c += 16) {
                     float y[16];
                     tmem_ld16(tl + c, y);
                     if (row < dt.valid) {

@@ -117,6 +117,8 @@ struct Workspace {
     // counters above), so they are zero when a forward starts
     int *tail;
     int *cursor;        // [kMaxExperts] per-expert slots of the large-batch scatter
+    int *ecount;        // [kMaxExperts] pairs per expert, counted by the router's token tiles
+                        // (zeroed again by the plan builder, so zero between calls)
     // gate split over several CTAs (batches of one or two tokens): partial gate
     // sums of an item's non-owner parts [item][part - 1][128 neurons][2 tokens]
     // and per item the count of parts published (zeroed by the conversion

@@ -218,6 +218,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.route_count = (int *)sb.take(4);
     ws.tail = (int *)sb.take(8);
     ws.cursor = (int *)sb.take(4 * moe::kMaxExperts);
+    ws.ecount = (int *)sb.take(4 * moe::kMaxExperts);
     if (split_ok) {
         ws.gpart = (float *)sb.take((size_t)split_items * part_floats * sizeof(float));
         ws.gcnt = (int *)sb.take((size_t)split_items * sizeof(int));
@@ -232,7 +233,7 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     ws.x_tiles = (uint16_t *)sb.take(32 * (size_t)dm.dp);
     h->stats_dev = (unsigned long long *)sb.take(64);
     h->hist = (unsigned *)sb.take(256 * sizeof(unsigned));
-    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count || !ws.tail || !ws.cursor) {
+    if (!h->stats_dev || !h->hist || !ws.x_tiles || !ws.error_sticky || !ws.route_count || !ws.tail || !ws.cursor || !ws.ecount) {
         free_handle(h);
         return MOE_ENOMEM;
     }

@@ -53,15 +53,22 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
     const int E = a.E, P = a.T * a.k;
     const bool staged = s_idx != nullptr;   // top-k of all pairs held in shared memory
     Plan *plan = a.ws.plan;
-    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
-    if (staged)
+    // large batches: the token tiles counted their pairs per expert (ecount);
+    // staged ones count here, from exactly the indices the scatter places.
+    // Either way ecount is left zero for the next call.
+    for (int e = tid; e < E; e += blockDim.x) {
+        s_cnt[e] = staged ? 0 : __ldcg(&a.ws.ecount[e]);
+        a.ws.ecount[e] = 0;
+    }
+    if (staged) {
+#pragma unroll 4
         for (int p = tid; p < P; p += blockDim.x) {
             s_idx[p] = min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1);
             s_w[p] = __ldcg(&a.ws.topk_w[p]);
         }
-    __syncthreads();
-    for (int p = tid; p < P; p += blockDim.x)
-        atomicAdd(&s_cnt[staged ? s_idx[p] : min(max(__ldcg(&a.ws.topk_idx[p]), 0), E - 1)], 1);
+        __syncthreads();
+        for (int p = tid; p < P; p += blockDim.x) atomicAdd(&s_cnt[s_idx[p]], 1);
+    }
     __syncthreads();
     if (staged && a.cap >= 0) {
         // Capacity-aware token drop ("Capacity-Aware Inference", "Capacity-
@@ -237,10 +244,19 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
             const int v = quarter * 64 + lane + 32 * q;
             wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
         }
+        // the tile's rows of this chunk: every load issued before the first store
+        // (nt * cv <= 8 * 256, at most one 16-byte vector per row and thread)
+        uint4 xv[kRtTok];
+#pragma unroll
+        for (int j = 0; j < kRtTok; ++j) {
+            const int i = threadIdx.x + j * 256;
+            if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + c0 + (i % cv) * 8);
+        }
         __syncthreads();   // the previous chunk's x is no longer read
-        for (int i = threadIdx.x; i < nt * cv; i += blockDim.x) {
-            const int r = i / cv, v = i % cv;
-            xs[r * 256 + v] = ld_cached(a.x + (size_t)(t0 + r) * a.d + c0 + v * 8);
+#pragma unroll
+        for (int j = 0; j < kRtTok; ++j) {
+            const int i = threadIdx.x + j * 256;
+            if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
         }
         __syncthreads();
         if (a.xtile > 0 && blockIdx.x == 0) {   // the tile's rows of the swizzled token operand
@@ -336,6 +352,7 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
                 if (rank < a.k) {
                     a.ws.topk_idx[(size_t)t * a.k + rank] = j;
                     a.ws.topk_w[(size_t)t * a.k + rank] = expf(v - m) / s;
+                    atomicAdd(&a.ws.ecount[j], 1);
                 }
             }
         } else {
@@ -358,6 +375,7 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
                 if (lane == 0) {
                     a.ws.topk_idx[(size_t)t * a.k + r] = bi;
                     a.ws.topk_w[(size_t)t * a.k + r] = expf(bv - m) / s;
+                    atomicAdd(&a.ws.ecount[min(max(bi, 0), a.E - 1)], 1);
                 }
             }
         }
