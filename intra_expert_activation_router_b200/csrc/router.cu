@@ -36,6 +36,7 @@ struct RouterArgs {
     int mt, n_chunks;   // sparse work items per expert: ceil(tokens / mt) * n_chunks
     int dp;             // d rounded up to 128
     int xtile;          // T <= xtile <= 16: also write x into ws.x_tiles with xtile rows; else 0
+    int epc;            // experts per CTA (even): gridDim.x = ceil(E / epc)
     int cap;            // capacity-aware token drop: pairs an expert keeps (-1: no capacity)
     int mask_words;     // 32-neuron mask words per pair (cleared for dropped pairs)
     Workspace ws;
@@ -227,60 +228,98 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     if (tr && threadIdx.x == 0) tr[0] = global_ns();
 
     // 1. logits: the tile's x rows in shared memory (chunks of 2048); warp w
-    //    takes expert blockIdx.x*2 + w/4 and a quarter of each chunk, so the
-    //    router spreads over E/2 CTAs per token tile; the four quarter sums
-    //    meet in shared memory
-    const int e = blockIdx.x * kRtExp + (warp >> 2);
+    //    takes expert 2p + w/4 of the CTA's pass p and a quarter of each chunk,
+    //    the four quarter sums meeting in shared memory.  A CTA covers `epc`
+    //    experts of its token tile in epc/2 passes: 2 for small batches (the
+    //    router spread over E/2 CTAs per tile), more for large ones, whose
+    //    tiles are many -- then the tile's rows are staged once for all its
+    //    passes (d <= 2048: a single chunk) and each pass's router rows are
+    //    loaded during the previous pass.
     const int quarter = warp & 3;
-    float acc[kRtTok];
-#pragma unroll
-    for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
-    uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);   // [kRtTok][256] 16-byte vectors
-    for (int c0 = 0; c0 < a.d; c0 += 2048) {
-        const int cv = min(2048, a.d - c0) / 8;
-        uint4 wv[2];
+    uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);                       // [kRtTok][256] 16-byte vectors
+    float *qsum = s_dyn + kRtTok * 256 * 4;                              // [8 warps][kRtTok], after x
+    const int e_first = blockIdx.x * a.epc;
+    const int passes = a.epc / kRtExp;
+    const bool one_chunk = a.d <= 2048;
+    auto load_w = [&](int e, int c0, int cv, uint4 (&wv)[2]) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             const int v = quarter * 64 + lane + 32 * q;
             wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
         }
-        // the tile's rows of this chunk: every load issued before the first store
-        // (nt * cv <= 8 * 256, at most one 16-byte vector per row and thread)
-        uint4 xv[kRtTok];
+    };
+    uint4 wnext[2];
+    load_w(e_first + (warp >> 2), 0, min(2048, a.d) / 8, wnext);
+#pragma unroll 1
+    for (int pass = 0; pass < passes; ++pass) {
+        const int e = e_first + pass * kRtExp + (warp >> 2);
+        float acc[kRtTok];
 #pragma unroll
-        for (int j = 0; j < kRtTok; ++j) {
-            const int i = threadIdx.x + j * 256;
-            if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + c0 + (i % cv) * 8);
-        }
-        __syncthreads();   // the previous chunk's x is no longer read
+        for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
+        for (int c0 = 0; c0 < a.d; c0 += 2048) {
+            const int cv = min(2048, a.d - c0) / 8;
+            uint4 wv[2];
+            if (one_chunk) {
+                wv[0] = wnext[0];
+                wv[1] = wnext[1];
+                if (pass + 1 < passes) load_w(e + kRtExp, 0, cv, wnext);   // the next pass's rows, in flight now
+            } else {
+                load_w(e, c0, cv, wv);
+            }
+            if (pass == 0 || !one_chunk) {
+                // the tile's rows of this chunk: every load issued before the first
+                // store (nt * cv <= 8 * 256, at most one 16-byte vector per row and thread)
+                uint4 xv[kRtTok];
 #pragma unroll
-        for (int j = 0; j < kRtTok; ++j) {
-            const int i = threadIdx.x + j * 256;
-            if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
+                for (int j = 0; j < kRtTok; ++j) {
+                    const int i = threadIdx.x + j * 256;
+                    if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + c0 + (i % cv) * 8);
+                }
+                __syncthreads();   // the previous chunk's x is no longer read
+#pragma unroll
+                for (int j = 0; j < kRtTok; ++j) {
+                    const int i = threadIdx.x + j * 256;
+                    if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
+                }
+                __syncthreads();
+                if (a.xtile > 0 && blockIdx.x == 0 && pass == 0) {   // the tile's rows of the swizzled token operand
+                    for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
+                        const int r = i / cv, v = i % cv, t = t0 + r;
+                        if (t < a.xtile) {
+                            const int cc = c0 / 8 + v;   // 16-byte block of the row
+                            *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
+                                                       (((cc & 7) ^ (t & 7)) << 3)) =
+                                r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+            }
+            if (e < a.E) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int v = quarter * 64 + lane + 32 * q;
+                    if (v < cv) {
+#pragma unroll
+                        for (int r = 0; r < kRtTok; ++r)
+                            if (r < nt) acc[r] = dot8(wv[q], xs[r * 256 + v], acc[r]);
+                    }
+                }
+            }
         }
+#pragma unroll
+        for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
+        if (lane == 0)
+            for (int r = 0; r < kRtTok; ++r) qsum[warp * kRtTok + r] = acc[r];
         __syncthreads();
-        if (a.xtile > 0 && blockIdx.x == 0) {   // the tile's rows of the swizzled token operand
-            for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
-                const int r = i / cv, v = i % cv, t = t0 + r;
-                if (t < a.xtile) {
-                    const int cc = c0 / 8 + v;   // 16-byte block of the row
-                    *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
-                                               (((cc & 7) ^ (t & 7)) << 3)) =
-                        r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
-                }
+        if (threadIdx.x < kRtExp * kRtTok) {
+            const int ee = threadIdx.x / kRtTok, r = threadIdx.x % kRtTok;
+            const int eg = e_first + pass * kRtExp + ee;
+            if (eg < a.E && r < nt) {
+                const float *q4 = qsum + (ee * 4) * kRtTok + r;
+                a.ws.logits[(size_t)(t0 + r) * a.E + eg] = q4[0] + q4[kRtTok] + q4[2 * kRtTok] + q4[3 * kRtTok];
             }
         }
-        if (e < a.E) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int v = quarter * 64 + lane + 32 * q;
-                if (v < cv) {
-#pragma unroll
-                    for (int r = 0; r < kRtTok; ++r)
-                        if (r < nt) acc[r] = dot8(wv[q], xs[r * 256 + v], acc[r]);
-                }
-            }
-        }
+        __syncthreads();   // qsum is rewritten by the next pass
     }
     if (a.xtile > 0 && blockIdx.x == 0) {   // inputs past d: zero
         const int npad = (a.dp - a.d) / 8;
@@ -289,21 +328,6 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
             if (t < a.xtile)
                 *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
                                            (((cc & 7) ^ (t & 7)) << 3)) = make_uint4(0, 0, 0, 0);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
-    __syncthreads();   // x no longer needed: reuse shared memory for the quarter sums
-    float *qsum = s_dyn;   // [8 warps][kRtTok]
-    if (lane == 0)
-        for (int r = 0; r < kRtTok; ++r) qsum[warp * kRtTok + r] = acc[r];
-    __syncthreads();
-    if (threadIdx.x < kRtExp * kRtTok) {
-        const int ee = threadIdx.x / kRtTok, r = threadIdx.x % kRtTok;
-        const int eg = blockIdx.x * kRtExp + ee;
-        if (eg < a.E && r < nt) {
-            const float* q4 = qsum + (ee * 4) * kRtTok + r;
-            a.ws.logits[(size_t)(t0 + r) * a.E + eg] = q4[0] + q4[kRtTok] + q4[2 * kRtTok] + q4[3 * kRtTok];
         }
     }
 
@@ -440,10 +464,23 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     a.cap = cap;
     a.mask_words = dm.f / kChunk;
     a.ws = ws;
-    dim3 grid((dm.E + kRtExp - 1) / kRtExp, (T + kRtTok - 1) / kRtTok);
+    // experts per CTA: 2 unless that makes more than about two CTAs per SM
+    // (large batches); then more, so a CTA stages its tile's rows once for
+    // several experts (single-chunk rows only, d <= 2048)
+    const long long tiles = (T + kRtTok - 1) / kRtTok;
+    int epc = kRtExp;
+    if (dm.d <= 2048) {
+        const long long want = 2 * 148;
+        const long long pairs_per_tile = (dm.E + kRtExp - 1) / kRtExp;
+        long long per = (pairs_per_tile * tiles + want - 1) / want;   // expert pairs per CTA
+        if (per > pairs_per_tile) per = pairs_per_tile;
+        if (per > 1) epc = (int)per * kRtExp;
+    }
+    a.epc = epc;
+    dim3 grid((dm.E + epc - 1) / epc, (unsigned)tiles);
     const size_t P = (size_t)T * dm.k;
     size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // softmax rows
-    if (smem < 16 * (size_t)kRtTok * 256) smem = 16 * (size_t)kRtTok * 256;   // x chunk
+    if (smem < 16 * (size_t)kRtTok * 256 + 4 * 8 * kRtTok) smem = 16 * (size_t)kRtTok * 256 + 4 * 8 * kRtTok;   // x chunk, quarter sums
     size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (P <= kStagePairs ? (cap >= 0 ? 12 : 8) * P : 0);
     if (plan_smem > smem) smem = plan_smem;
     // at most max(32 KB, 2*1024*4 + 12*4096 = 56 KB): above the default 48 KB
