@@ -227,70 +227,109 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     unsigned long long *tr = (a.ws.trace_router && cta < a.ws.trace_router_ctas) ? a.ws.trace_router + cta * 8 : nullptr;
     if (tr && threadIdx.x == 0) tr[0] = global_ns();
 
-    // 1. logits: the tile's x rows in shared memory (chunks of 2048); warp w
-    //    takes expert 2p + w/4 of the CTA's pass p and a quarter of each chunk,
-    //    the four quarter sums meeting in shared memory.  A CTA covers `epc`
-    //    experts of its token tile in epc/2 passes: 2 for small batches (the
-    //    router spread over E/2 CTAs per tile), more for large ones, whose
-    //    tiles are many -- then the tile's rows are staged once for all its
-    //    passes (d <= 2048: a single chunk) and each pass's router rows are
-    //    loaded during the previous pass.
+    // 1. logits of the CTA's `epc` experts for its token tile, the tile's x
+    //    rows in shared memory: 2 experts for small batches (the router spread
+    //    over E/2 CTAs per tile), more for large ones, whose tiles are many.
     const int quarter = warp & 3;
     uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);                       // [kRtTok][256] 16-byte vectors
     float *qsum = s_dyn + kRtTok * 256 * 4;                              // [8 warps][kRtTok], after x
     const int e_first = blockIdx.x * a.epc;
-    const int passes = a.epc / kRtExp;
-    const bool one_chunk = a.d <= 2048;
-    auto load_w = [&](int e, int c0, int cv, uint4 (&wv)[2]) {
+    if (a.epc > kRtExp) {
+        // large batches (d <= 2048): the tile's rows once, then one expert per
+        // warp at a time over the whole of d (lane: 16-byte vectors lane,
+        // lane + 32, ...), its router row loaded while the previous expert's
+        // dots run; no cross-warp sums
+        const int cv = a.d / 8;
+        {
+            uint4 xv[kRtTok];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int v = quarter * 64 + lane + 32 * q;
-            wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < kRtTok; ++j) {
+                const int i = threadIdx.x + j * 256;
+                if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + (i % cv) * 8);
+            }
+#pragma unroll
+            for (int j = 0; j < kRtTok; ++j) {
+                const int i = threadIdx.x + j * 256;
+                if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
+            }
         }
-    };
-    uint4 wnext[2];
-    load_w(e_first + (warp >> 2), 0, min(2048, a.d) / 8, wnext);
+        __syncthreads();
+        const int e_end = min(e_first + a.epc, a.E);
+        uint4 wn[8];
+        auto load_row = [&](int e) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int v = lane + 32 * q;
+                wn[q] = (e < e_end && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + v * 8) : make_uint4(0, 0, 0, 0);
+            }
+        };
+        load_row(e_first + warp);
 #pragma unroll 1
-    for (int pass = 0; pass < passes; ++pass) {
-        const int e = e_first + pass * kRtExp + (warp >> 2);
+        for (int e = e_first + warp; e < e_end; e += 8) {
+            uint4 wv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) wv[q] = wn[q];
+            load_row(e + 8);
+            float acc[kRtTok];
+#pragma unroll
+            for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int v = lane + 32 * q;
+                if (v < cv) {
+#pragma unroll
+                    for (int r = 0; r < kRtTok; ++r)
+                        if (r < nt) acc[r] = dot8(wv[q], xs[r * 256 + v], acc[r]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kRtTok; ++r) acc[r] = warp_sum(acc[r]);
+            if (lane < nt) {
+                float v = acc[0];
+#pragma unroll
+                for (int r = 1; r < kRtTok; ++r) v = lane == r ? acc[r] : v;
+                a.ws.logits[(size_t)(t0 + lane) * a.E + e] = v;
+            }
+        }
+    } else {
+        // small batches: expert 2 blockIdx.x + w/4 per warp, a quarter of each
+        // 2048-wide chunk of d per warp, the four quarter sums meeting in
+        // shared memory
+        const int e = e_first + (warp >> 2);
         float acc[kRtTok];
 #pragma unroll
         for (int r = 0; r < kRtTok; ++r) acc[r] = 0.f;
         for (int c0 = 0; c0 < a.d; c0 += 2048) {
             const int cv = min(2048, a.d - c0) / 8;
             uint4 wv[2];
-            if (one_chunk) {
-                wv[0] = wnext[0];
-                wv[1] = wnext[1];
-                if (pass + 1 < passes) load_w(e + kRtExp, 0, cv, wnext);   // the next pass's rows, in flight now
-            } else {
-                load_w(e, c0, cv, wv);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int v = quarter * 64 + lane + 32 * q;
+                wv[q] = (e < a.E && v < cv) ? ld_cached(a.wr + (size_t)e * a.d + c0 + v * 8) : make_uint4(0, 0, 0, 0);
             }
-            if (pass == 0 || !one_chunk) {
-                // the tile's rows of this chunk: every load issued before the first
-                // store (nt * cv <= 8 * 256, at most one 16-byte vector per row and thread)
-                uint4 xv[kRtTok];
+            // the tile's rows of this chunk: every load issued before the first
+            // store (nt * cv <= 8 * 256, at most one 16-byte vector per row and thread)
+            uint4 xv[kRtTok];
 #pragma unroll
-                for (int j = 0; j < kRtTok; ++j) {
-                    const int i = threadIdx.x + j * 256;
-                    if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + c0 + (i % cv) * 8);
-                }
-                __syncthreads();   // the previous chunk's x is no longer read
+            for (int j = 0; j < kRtTok; ++j) {
+                const int i = threadIdx.x + j * 256;
+                if (i < nt * cv) xv[j] = ld_cached(a.x + (size_t)(t0 + i / cv) * a.d + c0 + (i % cv) * 8);
+            }
+            __syncthreads();   // the previous chunk's x is no longer read
 #pragma unroll
-                for (int j = 0; j < kRtTok; ++j) {
-                    const int i = threadIdx.x + j * 256;
-                    if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
-                }
-                __syncthreads();
-                if (a.xtile > 0 && blockIdx.x == 0 && pass == 0) {   // the tile's rows of the swizzled token operand
-                    for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
-                        const int r = i / cv, v = i % cv, t = t0 + r;
-                        if (t < a.xtile) {
-                            const int cc = c0 / 8 + v;   // 16-byte block of the row
-                            *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
-                                                       (((cc & 7) ^ (t & 7)) << 3)) =
-                                r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
-                        }
+            for (int j = 0; j < kRtTok; ++j) {
+                const int i = threadIdx.x + j * 256;
+                if (i < nt * cv) xs[(i / cv) * 256 + i % cv] = xv[j];
+            }
+            __syncthreads();
+            if (a.xtile > 0 && blockIdx.x == 0) {   // the tile's rows of the swizzled token operand
+                for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
+                    const int r = i / cv, v = i % cv, t = t0 + r;
+                    if (t < a.xtile) {
+                        const int cc = c0 / 8 + v;   // 16-byte block of the row
+                        *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(cc >> 3) * a.xtile + t) * 64 +
+                                                   (((cc & 7) ^ (t & 7)) << 3)) =
+                            r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
                     }
                 }
             }
@@ -313,13 +352,12 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
         __syncthreads();
         if (threadIdx.x < kRtExp * kRtTok) {
             const int ee = threadIdx.x / kRtTok, r = threadIdx.x % kRtTok;
-            const int eg = e_first + pass * kRtExp + ee;
+            const int eg = e_first + ee;
             if (eg < a.E && r < nt) {
                 const float *q4 = qsum + (ee * 4) * kRtTok + r;
                 a.ws.logits[(size_t)(t0 + r) * a.E + eg] = q4[0] + q4[kRtTok] + q4[2 * kRtTok] + q4[3 * kRtTok];
             }
         }
-        __syncthreads();   // qsum is rewritten by the next pass
     }
     if (a.xtile > 0 && blockIdx.x == 0) {   // inputs past d: zero
         const int npad = (a.dp - a.d) / 8;
