@@ -254,6 +254,15 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
             }
         }
         __syncthreads();
+        if (a.xtile > 0 && blockIdx.x == 0) {   // the tile's rows of the swizzled token operand
+            for (int i = threadIdx.x; i < kRtTok * cv; i += blockDim.x) {
+                const int r = i / cv, v = i % cv, t = t0 + r;
+                if (t < a.xtile)
+                    *reinterpret_cast<uint4 *>(a.ws.x_tiles + ((size_t)(v >> 3) * a.xtile + t) * 64 +
+                                               (((v & 7) ^ (t & 7)) << 3)) =
+                        r < nt ? xs[r * 256 + v] : make_uint4(0, 0, 0, 0);
+            }
+        }
         const int e_end = min(e_first + a.epc, a.E);
         uint4 wn[8];
         auto load_row = [&](int e) {
