@@ -41,7 +41,7 @@ constexpr int kBTileBytes = 256 * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kDenseSmem = kDStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
 
-enum DenseMode { kGateUp = 0, kDown = 1 };
+enum DenseMode { kGateUp = 0, kDown = 1, kLogits = 2 };
 
 struct DenseArgs {
     int mode;
@@ -117,12 +117,12 @@ struct DenseTile {
 
 __device__ __forceinline__ int dense_out_blocks(const DenseArgs &a)
 {
-    return a.mode == kGateUp ? a.wrows / 128 : a.wrows / 256;
+    return a.mode == kGateUp ? a.wrows / 128 : (a.wrows + 255) / 256;
 }
 
 __device__ __forceinline__ int dense_n_tiles(const DenseArgs &a)
 {
-    const int m_tiles = a.shared ? (a.T + kBM - 1) / kBM : a.plan->n_dense_tiles;
+    const int m_tiles = (a.shared || a.mode == kLogits) ? (a.T + kBM - 1) / kBM : a.plan->n_dense_tiles;
     return m_tiles * dense_out_blocks(a);
 }
 
@@ -132,7 +132,12 @@ __device__ __forceinline__ DenseTile dense_tile(const DenseArgs &a, int t)
     DenseTile d;
     d.bx = t % n_out;
     const int by = t / n_out;
-    if (!a.shared) {
+    if (a.mode == kLogits) {   // the batch's own rows against all experts' router rows
+        d.row0 = kBM * by;
+        d.valid = min(kBM, a.T - d.row0);
+        d.wrow0 = 0;
+        d.ex = 0;
+    } else if (!a.shared) {
         const Plan *plan = a.plan;
         int lo = 0, hi = plan->n_touched - 1;   // last slot with tile_prefix <= by
         while (lo < hi) {
@@ -297,6 +302,17 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
                         reinterpret_cast<uint4 *>(hrow + c)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
                 }
+            } else if (a.mode == kLogits) {
+                // logits[token][expert] (fp32) for the experts inside the matrix
+                float *lrow = a.y_acc + (size_t)(dt.row0 + row) * a.d;
+                for (int c = 128 * half; c < 128 * half + 128; c += 16) {
+                    float y[16];
+                    tmem_ld16(tl + c, y);
+                    if (row < dt.valid)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (dt.n0 + c + i < a.wrows) lrow[dt.n0 + c + i] = y[i];
+                }
             } else {
                 int tok = 0;
                 float w = 1.f;
@@ -401,8 +417,34 @@ bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, De
         ok = ok && encode(&st->g2s.b0, w.wsdt, f, S * d, 2 * f, 256, true);
         st->g2s.b1 = st->g2s.b0;
     }
+    ok = ok && encode(&st->router_b, w.wr, d, E, 2 * d, 256, true);
     st->ok = ok;
     return ok;
+}
+
+cudaError_t launch_logits_tc(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
+                             int n_sm, cudaStream_t s)
+{
+    if (!st.ok) return cudaErrorNotSupported;
+    static int smem_set[kMaxDevices] = {};
+    cudaError_t e = ensure_dynamic_smem(k_dense_gemm, kDenseSmem, smem_set);
+    if (e != cudaSuccess) return e;
+    DenseMaps maps;
+    if (!encode(&maps.a, x, dm.d, T, 2ull * dm.d, kBM, true)) return cudaErrorInvalidValue;
+    maps.b0 = st.router_b;
+    maps.b1 = st.router_b;
+    DenseArgs a = {};
+    a.mode = kLogits;
+    a.T = T;
+    a.K = dm.d;
+    a.kb = dm.d / kBK;
+    a.wrows = dm.E;
+    a.y_acc = ws.logits;
+    a.d = dm.E;   // the logits' row length
+    a.err = ws.error_word;
+    const long long tiles = (long long)((T + kBM - 1) / kBM) * ((dm.E + 255) / 256);
+    k_dense_gemm<<<(unsigned)(tiles < n_sm ? tiles : n_sm), kDenseThreads, kDenseSmem, s>>>(maps, a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,

@@ -71,6 +71,7 @@ struct DenseState {
     bool ok;                           // shape supported and maps encoded
     DenseMaps g1r, g1s, g2r, g2s;      // GEMM1/GEMM2, routed/shared
     const uint16_t *gate_r, *gate_s;   // gate tiles, routed / shared experts
+    CUtensorMap router_b;              // the router rows Wr [E][d] (box 64 x 256) for the logits GEMM
 };
 
 // Element offset of gate weight (neuron j, input k) inside one expert's tiles.
@@ -173,7 +174,8 @@ __device__ __forceinline__ unsigned long long global_ns()
 // cap >= 0: capacity-aware token drop, each expert keeps at most cap pairs
 // (batches of up to 4096 pairs; cudaErrorNotSupported above).
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap = -1);
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap = -1,
+                          bool logits_ready = false);
 // inject: test-only fault (MOE_INJECT_WITHHOLD_ITEMS: the gate lane publishes
 // no work item, so the consumers' bounded waits run out), 0 otherwise.
 // fused: the kernel routes the batch itself (no router launch before it);
@@ -230,5 +232,10 @@ bool dense_setup(const Dims &dm, const DeviceWeights &w, const Workspace &ws, De
 // tau_shared: the shared experts' threshold on a masked forward (<= 0: dense).
 cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
                          float tau, bool use_mask, uint16_t *out, cudaStream_t s, float tau_shared, int n_sm);
+// The router's logits (ws.logits [T][E], fp32) as a tcgen05 GEMM of x [T][d]
+// and Wr [E][d] on the dense branch's kernel, for large batches; the router
+// kernel then runs with logits_ready.
+cudaError_t launch_logits_tc(const Dims &dm, const Workspace &ws, const DenseState &st, const uint16_t *x, int T,
+                             int n_sm, cudaStream_t s);
 
 }  // namespace moe

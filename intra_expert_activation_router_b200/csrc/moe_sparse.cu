@@ -286,6 +286,21 @@ extern "C" void moe_sparse_destroy(moe_handle h)
     free_handle(h);
 }
 
+// The router for a batch: from 64 tokens on (when the layer has the dense
+// branch) the logits are one tcgen05 GEMM and the router kernel only selects
+// and buckets; smaller batches keep the router kernel's own logits, which
+// are spread over more CTAs and cost one launch less.
+constexpr int kTcLogitsMinT = 64;
+static cudaError_t route(moe_handle h, const uint16_t *xb, int T, int tile_tokens, cudaStream_t st, int cap = -1)
+{
+    if (T >= kTcLogitsMinT && h->dense.ok) {
+        cudaError_t e = moe::launch_logits_tc(h->dm, h->ws, h->dense, xb, T, h->n_sm, st);
+        if (e != cudaSuccess) return e;
+        return moe::launch_router(h->dm, h->w, h->ws, xb, T, tile_tokens, st, cap, true);
+    }
+    return moe::launch_router(h->dm, h->w, h->ws, xb, T, tile_tokens, st, cap);
+}
+
 static int run_forward(moe_handle h, const void *x, int T, float tau, bool masked, void *out,
                        void *stream, int forced_path)
 {
@@ -335,7 +350,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
         // decode batches route inside the expert kernel: no router launch
         fused = !rank && cap < 0 && h->fused_router && moe::fused_possible(h->dm, T);
-        if (e == cudaSuccess && !fused) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, til.nt, st, cap);
+        if (e == cudaSuccess && !fused) e = route(h, xb, T, til.nt, st, cap);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (rank) {   // silu(g) of the routed pairs, each pair's cut, then the masked layer
             moe::RankPass r1{h->rank_a, nullptr, nullptr, false};
@@ -355,7 +370,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
         }
         h->inject_next = 0;
     } else {
-        if (e == cudaSuccess) e = moe::launch_router(h->dm, h->w, h->ws, xb, T, 8, st, cap);
+        if (e == cudaSuccess) e = route(h, xb, T, 8, st, cap);
         if (e == cudaSuccess && h->n_ev) e = cudaEventRecordWithFlags(h->ev[1], st, ev_flags);
         if (e == cudaSuccess)
             e = moe::launch_dense(h->dm, h->ws, h->dense, xb, T, tau, masked, ob, st, h->tau_shared, h->n_sm);
@@ -519,7 +534,7 @@ extern "C" int moe_debug_router(moe_handle h, const void *x, int T, int *idx_out
     if (!aligned16(x)) return MOE_EALIGN;
     cudaStream_t st = (cudaStream_t)stream;
     const size_t n = (size_t)T * h->dm.k;
-    cudaError_t e = moe::launch_router(h->dm, h->w, h->ws, (const uint16_t *)x, T, 1, st);
+    cudaError_t e = route(h, (const uint16_t *)x, T, 1, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(idx_out, h->ws.topk_idx, 4 * n, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(w_out, h->ws.topk_w, 4 * n, cudaMemcpyDeviceToDevice, st);
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
@@ -564,7 +579,7 @@ static int calibrate(moe_handle h, const void *x, int T, double sparsity, float 
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
     const moe::SparseTiling til = moe::sparse_tiling(T, dm.d);
-    cudaError_t e = moe::launch_router(dm, h->w, h->ws, xb, T, til.nt, st);
+    cudaError_t e = route(h, xb, T, til.nt, st);
     if (e == cudaSuccess)
         e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, til, h->n_sm, st,
                                       h->scores, 0, false, 0.0f, shared);

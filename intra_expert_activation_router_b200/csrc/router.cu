@@ -37,6 +37,7 @@ struct RouterArgs {
     int dp;             // d rounded up to 128
     int xtile;          // T <= xtile <= 16: also write x into ws.x_tiles with xtile rows; else 0
     int epc;            // experts per CTA (even): gridDim.x = ceil(E / epc)
+    int logits_ready;   // ws.logits already holds the batch's logits (a tensor-core GEMM): no phase 1
     int cap;            // capacity-aware token drop: pairs an expert keeps (-1: no capacity)
     int mask_words;     // 32-neuron mask words per pair (cleared for dropped pairs)
     Workspace ws;
@@ -234,7 +235,9 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     uint4 *xs = reinterpret_cast<uint4 *>(s_dyn);                       // [kRtTok][256] 16-byte vectors
     float *qsum = s_dyn + kRtTok * 256 * 4;                              // [8 warps][kRtTok], after x
     const int e_first = blockIdx.x * a.epc;
-    if (a.epc > kRtExp) {
+    if (a.logits_ready) {
+        // nothing to compute: the tile's logits are in place
+    } else if (a.epc > kRtExp) {
         // large batches (d <= 2048): the tile's rows once, then one expert per
         // warp at a time over the whole of d (lane: 16-byte vectors lane,
         // lane + 32, ...), its router row loaded while the previous expert's
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(256) k_plan_scatter(Workspace ws, int P, int k
 }
 
 cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
-                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap)
+                          const uint16_t *x, int T, int tile_tokens, cudaStream_t st, int cap, bool logits_ready)
 {
     if (cap >= 0 && (long long)T * dm.k > kStagePairs) return cudaErrorNotSupported;
     RouterArgs a;
@@ -523,6 +526,8 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
         if (per > pairs_per_tile) per = pairs_per_tile;
         if (per > 1) epc = (int)per * kRtExp;
     }
+    a.logits_ready = logits_ready ? 1 : 0;
+    if (logits_ready) epc = (dm.E + 1) & ~1;   // one CTA per token tile: softmax, top-k, plan
     a.epc = epc;
     dim3 grid((dm.E + epc - 1) / epc, (unsigned)tiles);
     const size_t P = (size_t)T * dm.k;
