@@ -286,11 +286,11 @@ extern "C" void moe_sparse_destroy(moe_handle h)
     free_handle(h);
 }
 
-// The router for a batch: from 64 tokens on (when the layer has the dense
+// The router for a batch: from 1024 tokens on (when the layer has the dense
 // branch) the logits are one tcgen05 GEMM and the router kernel only selects
 // and buckets; smaller batches keep the router kernel's own logits, which
 // are spread over more CTAs and cost one launch less.
-constexpr int kTcLogitsMinT = 64;
+constexpr int kTcLogitsMinT = 1024;
 static cudaError_t route(moe_handle h, const uint16_t *xb, int T, int tile_tokens, cudaStream_t st, int cap = -1)
 {
     if (T >= kTcLogitsMinT && h->dense.ok) {
