@@ -305,79 +305,6 @@ __device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nr
     if ((lane & ((1 << SH) - 1)) == 0 && q < nrows) part_w[(row_off + q) * MT + r] = val;
 }
 
-// ---- the up projection on the tensor cores (warp-level mma, bf16 in, fp32
-// accumulate).  A batch's gathered up rows are the A operand (16 rows, the
-// batch's records first; ldmatrix reads them straight from their
-// row-contiguous buffer), the pass's tokens the B operand (8 columns, the
-// tokens first), held in registers.  Up warp q takes the k-steps
-// [q KS_n, (q + 1) KS_n) of d's KS_n = ceil(d / 64) per warp, 16 inputs each;
-// inputs past d read as zero in B (their A values come from the record's
-// down half, finite weights, times zero).  The four warps' sums meet in
-// `part` as before.  For d >= 64 (the record, 4 d bytes, then holds every
-// A column read) and d <= 128 * 8 * NP, KS = 16 NP k-steps per warp at most.
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *smem_row)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"((uint32_t)__cvta_generic_to_shared(smem_row)));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                 "{%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// B fragments of the pass's tokens for up warp `quarter`: xb[ks][0|1] = the
-// bf16 pairs x[n][k + 2 t] and x[n][k + 8 + 2 t], k = 16 (quarter KS_n + ks),
-// n = lane / 4 (the token slot; zero past the pass's tokens), t = lane % 4.
-template <int KS>
-__device__ __forceinline__ void load_x_mma(const uint16_t *x, const int *tok, int ms, int d, int quarter, int lane,
-                                           uint32_t (&xb)[KS][2])
-{
-    const int n = lane >> 2, t = lane & 3, ks_n = (d + 63) / 64;
-    const uint32_t *row = (n < ms) ? reinterpret_cast<const uint32_t *>(x + (size_t)tok[n] * d) : nullptr;
-    const int k0 = 16 * quarter * ks_n + 2 * t;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-        const int k = k0 + 16 * ks;
-        const bool in = row && ks < ks_n;
-        xb[ks][0] = (in && k < d) ? __ldcg(row + k / 2) : 0u;
-        xb[ks][1] = (in && k + 8 < d) ? __ldcg(row + (k + 8) / 2) : 0u;
-    }
-}
-
-// This warp's share of u[q][r] for the batch's nb records (rows of `buf`,
-// `pitch` bytes apart, up half first) into part_w[q * MT + r].
-template <int MT, int KS>
-__device__ __forceinline__ void up_mma(const uint8_t *buf, int pitch, int nb, int d, int quarter, int lane,
-                                       const uint32_t (&xb)[KS][2], float *part_w)
-{
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int ks_n = (d + 63) / 64;
-    // ldmatrix: lane L addresses row (L & 7) | (L & 8) of the 16-row tile, columns (L >> 4) * 8
-    const int arow = (lane & 7) | (lane & 8);
-    const uint8_t *a_base = buf + (size_t)(arow < nb ? arow : 0) * pitch + (size_t)((lane >> 4) * 8) * 2 +
-                            (size_t)quarter * ks_n * 32;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-        if (ks < ks_n) {
-            uint32_t a[4];
-            ldmatrix_x4(a, a_base + 32 * ks);
-            mma_bf16_16816(acc, a, xb[ks][0], xb[ks][1]);
-        }
-    }
-    // acc[0], acc[1]: record lane / 4, tokens 2 (lane % 4) and 2 (lane % 4) + 1
-    const int q = lane >> 2, r = 2 * (lane & 3);
-    if (q < nb) {
-        if (r < MT) part_w[q * MT + r] = acc[0];
-        if (r + 1 < MT) part_w[q * MT + r + 1] = acc[1];
-    }
-}
-
 __device__ __forceinline__ int ld_acquire_gpu(const int *p)
 {
     int v;
@@ -1114,7 +1041,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         // reduction per 4 rows, the four warps' partials summed by warp 0 into
         // h = silu(g) u where the bit is set, handed to the down warps
         const int ct = tid;   // 0..127
-        const bool use_mma = d >= 64;   // the up dots on the tensor cores (d <= 2048: NP <= 2)
         const int d8 = d >> 3;
         uint32_t ub = 0;
         int n_rec = 0, ii = 0;
@@ -1283,19 +1209,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             unsigned long long *tu = (tr && ii < 3) ? tr + 2 + 10 * ii : nullptr;
             for (int s = 0; s < nsub; ++s) {
                 const int r0 = s * MT, ms = min(MT, m - r0);
-                // the pass's token rows (L2-resident): B fragments for the tensor-core
-                // up dots (d of 1025 .. 2048 always, 64 .. 1024 too), else packed
-                // fp32 slices for the CUDA-core ones
-                uint64_t xf[NP == 2 ? 1 : NP][NP == 2 ? 1 : MT][4];
-                uint32_t xb[NP <= 2 ? 16 * NP : 1][2];
-                if constexpr (NP == 2) {
-                    load_x_mma<32>(a.x, M.tok + r0, ms, d, warp, lane, xb);
-                } else if constexpr (NP == 1) {
-                    if (use_mma) load_x_mma<16>(a.x, M.tok + r0, ms, d, warp, lane, xb);
-                    else load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);
-                } else {
-                    load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);
-                }
+                uint64_t xf[NP][MT][4];
+                load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);   // the pass's token rows (L2-resident)
                 const int n_uni = min(max(M.n_uni[s], 0), kBlk);
                 n_rec += n_uni;
                 for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
@@ -1310,22 +1225,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     float *pw = part + (size_t)((hb * 4 + warp) * kMaxGB) * MT;
                     // batches of at most two records (d_model >= 4096): rows per reduction
                     // matched to the batch, no empty rows reduced
-                    if constexpr (NP == 2) {
-                        up_mma<MT, 32>(buf, L.gpitch, nb, d, warp, lane, xb, pw);
-                    } else if constexpr (NP == 1) {
-                        if (use_mma)
-                            up_mma<MT, 16>(buf, L.gpitch, nb, d, warp, lane, xb, pw);
-                        else
-                            for (int g0 = 0; g0 < nb; g0 += kRows)
-                                group_rows<kRows, MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0),
-                                                          xf, d8, ct, lane, pw, g0);
-                    } else if (L.gb <= 2) {
+                    if (NP >= 4 && L.gb <= 2)
                         group_rows<2, MT, NP>(buf, L.gpitch, nb, xf, d8, ct, lane, pw, 0);
-                    } else {
+                    else
                         for (int g0 = 0; g0 < nb; g0 += kRows)
                             group_rows<kRows, MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0), xf,
                                                       d8, ct, lane, pw, g0);
-                    }
                     consumer_sync(kUpThreads);   // the four warps' partials are in
                     if (warp == 0) {
                         mbar_wait(&hsfree[hb], ((ub >> 1) & 1) ^ 1, err, 44);   // the down warps read this slot out
