@@ -27,7 +27,15 @@ namespace moe {
 
 constexpr int kRtTok = 8;   // tokens per router CTA
 constexpr int kRtExp = 2;   // experts per router CTA (four warps each)
-constexpr int kStagePairs = 4096;   // plan built from shared memory up to this many pairs
+constexpr int kStagePairs = 4096;   // plan built from shared memory up to this many pairs ...
+constexpr int kSmallPlan = 256;     // ... when there are at most this many, or a capacity applies;
+                                    // else from the token tiles' counts and k_plan_scatter (one CTA
+                                    // placing pairs one warp-step at a time took 30 us at 2048 pairs)
+
+__host__ __device__ __forceinline__ bool plan_staged(long long P, int cap)
+{
+    return P <= kStagePairs && (cap >= 0 || P <= kSmallPlan);
+}
 constexpr int kRankTopk = 256;      // up to this many experts, top-k by ranking all logits
 
 struct RouterArgs {
@@ -471,7 +479,7 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     }
     int *s_int = reinterpret_cast<int *>(s_dyn);
     const int P = a.T * a.k;
-    const bool staged = P <= kStagePairs;
+    const bool staged = plan_staged(P, a.cap);
     if (tr && threadIdx.x == 0) tr[4] = global_ns();
     build_plan(a, s_int, s_int + a.E, staged ? s_int + 2 * a.E : nullptr,
                staged ? reinterpret_cast<float *>(s_int + 2 * a.E + P) : nullptr,
@@ -533,7 +541,7 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
     const size_t P = (size_t)T * dm.k;
     size_t smem = sizeof(float) * (size_t)kRtTok * dm.E;   // softmax rows
     if (smem < 16 * (size_t)kRtTok * 256 + 4 * 8 * kRtTok) smem = 16 * (size_t)kRtTok * 256 + 4 * 8 * kRtTok;   // x chunk, quarter sums
-    size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (P <= kStagePairs ? (cap >= 0 ? 12 : 8) * P : 0);
+    size_t plan_smem = sizeof(int) * 2 * (size_t)dm.E + (plan_staged((long long)P, cap) ? (cap >= 0 ? 12 : 8) * P : 0);
     if (plan_smem > smem) smem = plan_smem;
     // at most max(32 KB, 2*1024*4 + 12*4096 = 56 KB): above the default 48 KB
     // window only with a capacity
@@ -543,7 +551,7 @@ cudaError_t launch_router(const Dims &dm, const DeviceWeights &w, const Workspac
         if (e != cudaSuccess) return e;
     }
     k_router<<<grid, 256, smem, st>>>(a);
-    if ((long long)T * dm.k > kStagePairs) {
+    if (!plan_staged((long long)T * dm.k, cap)) {
         const int P = T * dm.k;
         int blocks = (P + 255) / 256;
         if (blocks > 148 * 8) blocks = 148 * 8;
