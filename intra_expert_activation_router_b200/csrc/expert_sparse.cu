@@ -264,7 +264,7 @@ __device__ __forceinline__ void load_x(const uint16_t *x, const int *tok, int m,
 // part_w[(row_off + q) * MT + r].
 template <int R, int MT, int NP>
 __device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nrows, const uint64_t (&xf)[NP][MT][4],
-                                           int d8, int t128, int lane, float *part_w, int row_off, int ms)
+                                           int d8, int t128, int lane, float *part_w, int row_off)
 {
     constexpr int NV = R * MT;
     constexpr int SH = 5 - Log2<NV>::value;
@@ -285,12 +285,10 @@ __device__ __forceinline__ void group_rows(const uint8_t *lo, int stride, int nr
                                         bf16x2_f2(wv[q].w)};
 #pragma unroll
                 for (int r = 0; r < MT; ++r) {
-                    if (r < ms) {   // token slots past the pass's tokens stay zero
-                        uint64_t a2 = acc2[q * MT + r];
+                    uint64_t a2 = acc2[q * MT + r];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) a2 = ffma2(w2[i], xf[p][r][i], a2);
-                        acc2[q * MT + r] = a2;
-                    }
+                    for (int i = 0; i < 4; ++i) a2 = ffma2(w2[i], xf[p][r][i], a2);
+                    acc2[q * MT + r] = a2;
                 }
             }
         }
@@ -1228,11 +1226,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     // batches of at most two records (d_model >= 4096): rows per reduction
                     // matched to the batch, no empty rows reduced
                     if (NP >= 4 && L.gb <= 2)
-                        group_rows<2, MT, NP>(buf, L.gpitch, nb, xf, d8, ct, lane, pw, 0, ms);
+                        group_rows<2, MT, NP>(buf, L.gpitch, nb, xf, d8, ct, lane, pw, 0);
                     else
                         for (int g0 = 0; g0 < nb; g0 += kRows)
                             group_rows<kRows, MT, NP>(buf + (size_t)g0 * L.gpitch, L.gpitch, min(kRows, nb - g0), xf,
-                                                      d8, ct, lane, pw, g0, ms);
+                                                      d8, ct, lane, pw, g0);
                     consumer_sync(kUpThreads);   // the four warps' partials are in
                     if (warp == 0) {
                         mbar_wait(&hsfree[hb], ((ub >> 1) & 1) ^ 1, err, 44);   // the down warps read this slot out
@@ -1314,12 +1312,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                                                         bf16x2_f2(wv.w)};
 #pragma unroll
                                 for (int r = 0; r < MT; ++r) {
-                                    if (r < ms) {   // h is zero past the pass's tokens
-                                        const float hv = hq[q * MT + r];
-                                        const uint64_t h2 = f2_pack(hv, hv);
+                                    const float hv = hq[q * MT + r];
+                                    const uint64_t h2 = f2_pack(hv, hv);
 #pragma unroll
-                                        for (int i = 0; i < 4; ++i) acc_y[p][i][r] = ffma2(w2[i], h2, acc_y[p][i][r]);
-                                    }
+                                    for (int i = 0; i < 4; ++i) acc_y[p][i][r] = ffma2(w2[i], h2, acc_y[p][i][r]);
                                 }
                             }
                         }
