@@ -563,6 +563,43 @@ def capacity_rows(dev, flush, steps=20):
     return rows
 
 
+def deterministic_rows(dev, flush, steps=20):
+    """The deterministic combine (each contribution in a row of its own,
+    summed in one fixed order) beside the default fp32-atomic one, on the
+    OLMoE-shaped layer at 90 % sparsity: decode batches on the sparse branch
+    and a larger one on the dense branch."""
+    import torch
+    import moe_inputs as mi
+    import intra_expert_activation_router_b200 as m
+    shape = mi.SHAPES["olmoe"]
+    W = mi.make_weights(shape, device=dev)
+    layer = m.MoESparseLayer.from_weights(W, shape.top_k, max_tokens=256)
+    del W
+    rows = []
+    for T, path in ((1, m.MOE_PATH_SPARSE), (16, m.MOE_PATH_SPARSE), (256, m.MOE_PATH_DENSE)):
+        x = mi.make_x(shape, T, device=dev)
+        out = torch.empty_like(x)
+        tau = layer.calibrate_tau(x, 0.9)
+        layer.set_path(path)
+        row = {"workload": "olmoe", "T": T, "path": "sparse" if path == m.MOE_PATH_SPARSE else "dense"}
+        for name, det in (("atomic", False), ("deterministic", True)):
+            layer.set_deterministic(det)
+            for _ in range(3):
+                layer.forward(x, tau, out=out)
+            sm_, _, _ = time_steps(layer, x, tau, out, flush, steps)
+            st = layer.stats()
+            row[name + "_us"] = 1000 * statistics.mean(sm_)
+            if st["device_error"]:
+                row[name + "_device_error"] = st["device_error"]
+        layer.set_deterministic(False)
+        layer.set_path(m.MOE_PATH_AUTO)
+        rows.append(row)
+        log(json.dumps({k: (round(v, 2) if isinstance(v, float) else v) for k, v in row.items()}))
+    layer.close()
+    torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -641,6 +678,7 @@ def run_ours(args):
     modes = launch_mode_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
     budget_rows = rank_budget_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
     cap_rows = capacity_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
+    det_rows = deterministic_rows(dev, flush) if rank == 0 and sweep_kind != "none" else []
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -689,6 +727,7 @@ def run_ours(args):
             "launch_modes": modes,
             "rank_budget": budget_rows,
             "capacity_drop": cap_rows,
+            "deterministic_combine": det_rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

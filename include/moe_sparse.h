@@ -97,6 +97,8 @@ typedef struct {
                               router launch, 2: one launch), else 0              */
     int capacity;          /* pairs per expert the last forward kept at most
                               (moe_set_capacity), -1 if it dropped none          */
+    int deterministic;     /* the last forward combined in a fixed order
+                              (moe_set_deterministic)                            */
 } moe_stats;
 
 /* Create a layer.  Copies and repacks the weights into library-owned device
@@ -146,9 +148,11 @@ int moe_set_t_star(moe_handle h, int t_star);
  * device as one graph launch (median of five; before every run a 2 x L2
  * buffer is written and read back, so L2 holds no useful and no dirty line),
  * so neither branch is charged for host gaps between its kernels; the
- * search stops at the first T whose sparse time exceeds 90 % of the dense
- * one (the sparse branch's cost varies with how a batch routes), and T*
- * becomes the last T before it; it is stored in the handle and
+ * sparse time is the mean over two disjoint batches of T rows (the first
+ * and the last T rows of x) where T_max >= 2T, since the sparse branch's
+ * cost varies with how a batch routes; the search stops at the first T whose
+ * sparse time exceeds 95 % of the dense one, and T* becomes the last T
+ * before it; it is stored in the handle and
  * in *t_star_out (HOST pointer).
  * ("Uncovering Intra-expert Activation Sparsity...", technical summary,
  * Methodology item 3, "Dynamic switching": sparse for small batches, dense
@@ -247,6 +251,26 @@ int moe_set_rank_budget(moe_handle h, int r);
  * makes pairs' work depend on the rest of the batch, which is the method's
  * intent; outputs then differ from the plain layer. */
 int moe_set_capacity(moe_handle h, float gamma);
+
+/* Deterministic combine ("Uncovering Intra-expert Activation Sparsity ...",
+ * technical summary, Methodology item 3: the routed experts' outputs are
+ * weighted and summed into the token's output, plus the shared experts').
+ * By default every contribution is added into an fp32 accumulator with
+ * atomics, so the rounding of that sum follows the order in which the
+ * hardware lands them and a repeated forward can differ in the last bf16
+ * bit.  With enable != 0, later forwards (both paths, every launch mode)
+ * write each contribution -- one per (token, routing slot or shared expert,
+ * 128-neuron block) on the sparse path, per (token, slot) on the dense one --
+ * to a row of its own with plain stores, and the conversion adds a token's
+ * rows in one fixed order: identical inputs then give bit-identical outputs,
+ * whatever the schedule.  The cost is the rows' traffic: the sparse path
+ * writes and reads back T * (top_k + n_shared) * ceil(d_ff / 128) * d_model
+ * floats (8 MiB at 16 tokens of a 64-expert top-8 layer with d_model 2048 and
+ * d_ff 1024).  The first call with enable != 0 allocates max_tokens *
+ * (top_k + n_shared) * ceil(d_ff / 128) * d_model floats (MOE_ENOMEM if that
+ * fails, the setting unchanged) and clears them; moe_sparse_destroy frees
+ * them.  Not stream-ordered: call it between forwards, with none in flight. */
+int moe_set_deterministic(moe_handle h, int enable);
 
 /* As moe_calibrate_tau, over the N = T*n_shared*d_ff scores of the shared
  * experts' neurons: the floor(q*N)-th smallest |silu(x Ws_g)| (0-based, exact

@@ -16,6 +16,7 @@ _BINDING_NAMES = {
     "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
     "moe_debug_inject", "MOE_INJECT_NONE", "MOE_INJECT_WITHHOLD_ITEMS", "moe_set_fused_router",
     "moe_set_shared_tau", "moe_calibrate_tau_shared", "moe_tune_t_star", "moe_set_rank_budget", "moe_set_capacity",
+    "moe_set_deterministic",
 }
 
 

@@ -52,7 +52,7 @@ class moe_stats(ctypes.Structure):
                 ("n_union", ctypes.c_longlong), ("alg_bytes", ctypes.c_double),
                 ("dense_bytes", ctypes.c_double), ("device_error", ctypes.c_int),
                 ("fused_router", ctypes.c_int),
-                ("capacity", ctypes.c_int)]
+                ("capacity", ctypes.c_int), ("deterministic", ctypes.c_int)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -84,6 +84,7 @@ def _load():
         "moe_set_shared_tau": (I, [P, F]),
         "moe_set_rank_budget": (I, [P, I]),
         "moe_set_capacity": (I, [P, F]),
+        "moe_set_deterministic": (I, [P, I]),
         "moe_calibrate_tau_shared": (I, [P, P, I, ctypes.c_double, ctypes.POINTER(F), P]),
         "moe_tune_t_star": (I, [P, P, I, F, ctypes.POINTER(I), P]),
         "moe_strerror": (ctypes.c_char_p, [I]),
@@ -101,7 +102,7 @@ EXPORTED = ("moe_sparse_create", "moe_sparse_forward", "moe_dense_forward",
             "moe_debug_router", "moe_debug_active", "moe_query_stats", "moe_strerror",
             "moe_calibrate_tau", "moe_set_launch_events", "moe_set_trace", "moe_router_topk_noalloc",
             "moe_debug_inject", "moe_set_fused_router", "moe_set_shared_tau", "moe_calibrate_tau_shared",
-            "moe_tune_t_star", "moe_set_rank_budget", "moe_set_capacity")
+            "moe_tune_t_star", "moe_set_rank_budget", "moe_set_capacity", "moe_set_deterministic")
 
 
 def _addr(t):
@@ -232,6 +233,10 @@ def moe_set_shared_tau(h, tau_shared: float):
 
 def moe_set_capacity(h, gamma: float):
     _check(_lib.moe_set_capacity(h, float(gamma)), "moe_set_capacity")
+
+
+def moe_set_deterministic(h, enable: bool):
+    _check(_lib.moe_set_deterministic(h, 1 if enable else 0), "moe_set_deterministic")
 
 
 def moe_set_rank_budget(h, r: int):

@@ -74,8 +74,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
             sys.stdout.write(log)
     objs = [o for o, _ in results]
     tmp = OUT + ".tmp"
-    r = subprocess.run([cc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lcuda"]
-                       if False else [cc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs],
+    r = subprocess.run([cc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs],
                        capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -141,4 +141,64 @@ __device__ __forceinline__ uint16_t f2bf_bits(float v)
     return *reinterpret_cast<uint16_t *>(&b);
 }
 
+// Deterministic combine: partials [T][rows][d] fp32, one row per
+// (routing slot, neuron block) of a token, each written by exactly one
+// producer with plain stores; out[t] = bf16(sum of the token's rows), the sum
+// taken in one fixed order whatever the schedule was (8 lanes per four
+// outputs: lane l adds rows l, l + 8, ... in turn, then a fixed butterfly
+// over the 8 lanes), and every row read is re-zeroed, so rows of pairs that
+// produced nothing (a dropped pair) read as zero next time.  warp0 / n_warps:
+// this warp's index and the warp count of the calling grid; every lane of a
+// warp runs the same iterations (the shuffles need all 32).
+__device__ __forceinline__ void det_combine(float *__restrict__ part, int rows, int d, uint16_t *__restrict__ out,
+                                            long long n_out4, long long warp0, long long n_warps, int lane)
+{
+    const int d4 = d >> 2, l8 = lane & 7;
+    float4 *src = reinterpret_cast<float4 *>(part);
+#pragma unroll 1
+    for (long long g0 = warp0 * 4; g0 < n_out4; g0 += n_warps * 4) {
+        const long long g = g0 + (lane >> 3);
+        const bool valid = g < n_out4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+            const long long t = g / d4, c4 = g % d4;
+            float4 *base = src + (size_t)t * rows * d4 + c4;
+            // eight rows per lane in flight at once: all loads, then the zero
+            // stores (issued after the loads, so no load waits behind a store
+            // it might alias), then the adds in row order
+#pragma unroll 1
+            for (int j0 = l8; j0 < rows; j0 += 64) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    v[u] = j0 + 8 * u < rows ? __ldcg(base + (size_t)(j0 + 8 * u) * d4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (j0 + 8 * u < rows) __stcg(base + (size_t)(j0 + 8 * u) * d4, make_float4(0.f, 0.f, 0.f, 0.f));
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (j0 + 8 * u < rows) {
+                        acc.x += v[u].x;
+                        acc.y += v[u].y;
+                        acc.z += v[u].z;
+                        acc.w += v[u].w;
+                    }
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+        }
+        if (valid && l8 == 0) {
+            uint2 p;
+            p.x = (uint32_t)f2bf_bits(acc.x) | ((uint32_t)f2bf_bits(acc.y) << 16);
+            p.y = (uint32_t)f2bf_bits(acc.z) | ((uint32_t)f2bf_bits(acc.w) << 16);
+            reinterpret_cast<uint2 *>(out)[g] = p;
+        }
+    }
+}
+
 }  // namespace moe

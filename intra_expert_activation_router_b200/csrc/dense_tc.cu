@@ -56,10 +56,12 @@ struct DenseArgs {
     float tau;
     int use_mask;
     const Plan *plan;
-    const int *perm_tok;
+    const int *perm, *perm_tok;
     const float *perm_w;
     uint16_t *h;       // GEMM1 output
     float *y_acc;      // GEMM2 output
+    float *ypart;      // GEMM2 output, deterministic mode: [T][k + S][d] rows
+    int k, kS;         // top-k, k + S
     int d;
     int *err;
 };
@@ -82,7 +84,7 @@ __global__ void k_dense_gather(const uint16_t *__restrict__ x, const int *__rest
 // of a dense forward: it also moves the forward's error code into the sticky
 // word and clears its own word (as the sparse path's conversion kernel does).
 __global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4, int *error_word,
-                                int *error_sticky)
+                                int *error_sticky, float *ypart, int rows, int d)
 {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         const int e0 = *error_word;
@@ -91,7 +93,11 @@ __global__ void k_dense_convert(float *__restrict__ y_acc, uint16_t *__restrict_
             *error_word = 0;
         }
     }
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    if (ypart)   // deterministic mode: each token's k + S rows, summed in order
+        det_combine(ypart, rows, d, out, (long long)n4, ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+                    ((long long)gridDim.x * blockDim.x) >> 5, threadIdx.x & 31);
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; !ypart && i < n4;
+         i += (size_t)gridDim.x * blockDim.x) {
         const float4 v = reinterpret_cast<const float4 *>(y_acc)[i];
         uint2 p;
         p.x = (uint32_t)f2bf_bits(v.x) | ((uint32_t)f2bf_bits(v.y) << 16);
@@ -321,14 +327,23 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
                     w = a.shared ? 1.f : a.perm_w[dt.row0 + row];
                 }
                 float *yrow = a.y_acc + (size_t)tok * a.d + dt.n0;
+                if (a.ypart) {   // deterministic mode: the pair's own row, each element written once
+                    const int slot = a.shared ? a.k + a.sidx
+                                              : (row < dt.valid ? a.perm[dt.row0 + row] % a.k : 0);
+                    yrow = a.ypart + ((size_t)tok * a.kS + slot) * a.d + dt.n0;
+                }
                 for (int c = 128 * half; c < 128 * half + 128; c += 16) {
                     float y[16];
                     tmem_ld16(tl + c, y);
                     if (row < dt.valid) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4)
-                            atomicAdd(reinterpret_cast<float4 *>(yrow + c + i),
-                                      make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]));
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 v = make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]);
+                            if (a.ypart)
+                                __stcg(reinterpret_cast<float4 *>(yrow + c + i), v);
+                            else
+                                atomicAdd(reinterpret_cast<float4 *>(yrow + c + i), v);
+                        }
                     }
                 }
             }
@@ -472,11 +487,15 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     a.tau = tau;
     a.use_mask = use_mask ? 1 : 0;
     a.plan = ws.plan;
+    a.perm = ws.perm;
     a.perm_tok = ws.perm_tok;
     a.perm_w = ws.perm_w;
     a.h = ws.h_perm;
     a.h_ld = dm.f;
     a.y_acc = ws.y_acc;
+    a.ypart = ws.ypart;
+    a.k = dm.k;
+    a.kS = dm.k + dm.S;
     a.d = dm.d;
     a.err = ws.error_word;
     // GEMM1: gate | up with the mask epilogue
@@ -524,9 +543,10 @@ cudaError_t launch_dense(const Dims &dm, const Workspace &ws, const DenseState &
     // convert
     {
         const size_t n4 = (size_t)T * dm.d / 4;
-        size_t blocks = (n4 + 255) / 256;
+        size_t blocks = ((ws.ypart ? 8 : 1) * n4 + 255) / 256;   // deterministic: 8 threads per four outputs
         if (blocks > 148 * 16) blocks = 148 * 16;
-        k_dense_convert<<<(unsigned)blocks, 256, 0, s>>>(ws.y_acc, out, n4, ws.error_word, ws.error_sticky);
+        k_dense_convert<<<(unsigned)blocks, 256, 0, s>>>(ws.y_acc, out, n4, ws.error_word, ws.error_sticky, ws.ypart,
+                                                         dm.k + dm.S, dm.d);
     }
     return cudaGetLastError();
 }

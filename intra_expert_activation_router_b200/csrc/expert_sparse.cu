@@ -569,7 +569,11 @@ __device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_f
         *s_flag = ok;
     }
     __syncthreads();
-    if (*s_flag) {
+    if (*s_flag && a.ws.ypart) {
+        const int warps = kSparseThreads / 32;
+        det_combine(a.ws.ypart, (a.k + a.S) * a.n_blk, a.d, a.out, a.n_out4, (long long)blockIdx.x * warps + (tid >> 5),
+                    (long long)gridDim.x * warps, tid & 31);
+    } else if (*s_flag) {
         const float4 *src = reinterpret_cast<const float4 *>(a.ws.y_acc);
         float4 *zero = reinterpret_cast<float4 *>(a.ws.y_acc);
         uint2 *dst = reinterpret_cast<uint2 *>(a.out);
@@ -1332,7 +1336,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 // same tokens (looked up only now: in resident mode the next item
                 // is claimed once this one's backlog has drained)
                 bool cont = false;
-                if (nsub == 1) {
+                if (nsub == 1 && !a.ws.ypart) {   // (deterministic mode: one row per block)
                     const int nid = get_item(ii + 1);
                     // (a non-owner part has no up/down work: stop accumulating there)
                     cont = nid >= 0 && split_part(a, nid) == 0 &&
@@ -1349,9 +1353,22 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                                 float y[8];
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) f2_unpack(acc_y[p][i][r], y[2 * i], y[2 * i + 1]);
-                                float4 *dst = reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
-                                atomicAdd(dst, make_float4(wt * y[0], wt * y[1], wt * y[2], wt * y[3]));
-                                atomicAdd(dst + 1, make_float4(wt * y[4], wt * y[5], wt * y[6], wt * y[7]));
+                                const float4 y0 = make_float4(wt * y[0], wt * y[1], wt * y[2], wt * y[3]);
+                                const float4 y1 = make_float4(wt * y[4], wt * y[5], wt * y[6], wt * y[7]);
+                                if (a.ws.ypart) {
+                                    // deterministic mode: this (routing slot, block)'s own row
+                                    // [token][k + S][n_blk][d], summed in order by the combine
+                                    const int t = M.tok[r0 + r], kS = a.k + a.S;
+                                    const int slot = M.sidx >= 0 ? a.k + M.sidx : M.pair[r0 + r] % a.k;
+                                    float4 *dst = reinterpret_cast<float4 *>(
+                                        a.ws.ypart + (((size_t)t * kS + slot) * a.n_blk + M.blk) * d + v * 8);
+                                    __stcg(dst, y0);
+                                    __stcg(dst + 1, y1);
+                                } else {
+                                    float4 *dst = reinterpret_cast<float4 *>(a.ws.y_acc + (size_t)M.tok[r0 + r] * d + v * 8);
+                                    atomicAdd(dst, y0);
+                                    atomicAdd(dst + 1, y1);
+                                }
                             }
 #pragma unroll
                             for (int i = 0; i < 4; ++i) acc_y[p][i][r] = 0ull;
@@ -1463,7 +1480,7 @@ static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_
 // With n4 = 0 it only does that.
 __global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16_t *__restrict__ out, size_t n4,
                                                int *route_count, int *next_item, int *error_word, int *error_sticky,
-                                               int *gcnt, int gcnt_n)
+                                               int *gcnt, int gcnt_n, float *ypart, int rows, int d)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; gcnt && i < gcnt_n; i += gridDim.x * blockDim.x) gcnt[i] = 0;
@@ -1476,7 +1493,11 @@ __global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16
             *error_word = 0;
         }
     }
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    if (ypart)   // deterministic mode: the rows of every token, summed in order
+        det_combine(ypart, rows, d, out, (long long)n4, ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+                    ((long long)gridDim.x * blockDim.x) >> 5, threadIdx.x & 31);
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; !ypart && i < n4;
+         i += (size_t)gridDim.x * blockDim.x) {
         const float4 v = __ldcg(reinterpret_cast<const float4 *>(y_acc) + i);
         uint2 p;
         p.x = (uint32_t)f2bf_bits(v.x) | ((uint32_t)f2bf_bits(v.y) << 16);
@@ -1486,11 +1507,13 @@ __global__ void __launch_bounds__(256) k_y_out(float *__restrict__ y_acc, uint16
     }
 }
 
-static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm, const Workspace &ws,
-                                cudaStream_t st)
+static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm, const Workspace &ws, int rows,
+                                int d, cudaStream_t st)
 {
-    size_t blocks = (n4 + 255) / 256;
-    if (blocks > (size_t)n_sm * 4) blocks = (size_t)n_sm * 4;
+    // deterministic mode: 8 threads per four outputs
+    const size_t threads = ws.ypart ? n4 * 8 : n4;
+    size_t blocks = (threads + 255) / 256;
+    if (blocks > (size_t)n_sm * (ws.ypart ? 8 : 4)) blocks = (size_t)n_sm * (ws.ypart ? 8 : 4);
     if (blocks < 1) blocks = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);
@@ -1502,7 +1525,7 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_y_out, y_acc, out, n4, ws.route_count, &ws.plan->next_item,
-                                       ws.error_word, ws.error_sticky, ws.gcnt, ws.gcnt_n);
+                                       ws.error_word, ws.error_sticky, ws.gcnt, ws.gcnt_n, ws.ypart, rows, d);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1610,7 +1633,8 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     if (e != cudaSuccess) return e;
     if (a.tail) return cudaSuccess;
     // score mode writes no output: only the counters are reset
-    return launch_y_out(ws.y_acc, out, score_out ? 0 : (size_t)T * dm.d / 4, grid_cap, ws, st);
+    return launch_y_out(ws.y_acc, out, score_out ? 0 : (size_t)T * dm.d / 4, grid_cap, ws, (dm.k + dm.S) * dm.n_blk,
+                        dm.d, st);
 }
 
 }  // namespace moe

@@ -98,6 +98,12 @@ struct Workspace {
     float *perm_w;      // [T*k] routing weight of perm[i]
     uint32_t *mask;
     float *y_acc;
+    // deterministic combine (moe_set_deterministic), null when off: one fp32
+    // row of d per (token, routing slot or shared expert, neuron block) --
+    // [T][k + S][n_blk][d] on the sparse path, [T][k + S][d] on the dense one
+    // -- each written once with plain stores, summed in a fixed order by the
+    // conversion and re-zeroed there (all-zero between calls)
+    float *ypart;
     int *tok_cnt;
     int *tile_ticket;   // one per router token tile, kept zero between calls
     int *done_ticket;   // one, kept zero between calls

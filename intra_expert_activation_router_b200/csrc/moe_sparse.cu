@@ -66,12 +66,16 @@ struct moe_sparse_s {
     int *rank_j;         // [max_tokens * k] last tied index kept
     float cap_gamma;     // capacity factor of the token drop (moe_set_capacity); <= 0: none
     int last_cap;        // the capacity the last forward applied (-1: none)
+    float *det_rows;     // deterministic combine's rows (moe_set_deterministic), allocated on first use
+    int det;             // later forwards combine in a fixed order (ws.ypart = det_rows)
+    int last_det;
 };
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Host-side fault injection for tests: MOE_INJECT_ALLOC_FAIL=<what> makes the
-// named device allocation ("weights", "workspace", "scores" or "rank") report failure
+// named device allocation ("weights", "workspace", "scores", "rank" or
+// "deterministic") report failure
 // without being attempted, so the error paths can be exercised on a live GPU.
 static bool inject_alloc_fail(const char *what)
 {
@@ -111,6 +115,7 @@ static void free_handle(moe_handle h)
     if (h->ws_mem) cudaFree(h->ws_mem);
     if (h->scores) cudaFree(h->scores);
     if (h->rank_a) cudaFree(h->rank_a);
+    if (h->det_rows) cudaFree(h->det_rows);
     h->magic = 0;
     delete h;
 }
@@ -381,6 +386,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     h->last_masked = masked;
     h->last_fused = fused ? h->fused_router : 0;
     h->last_cap = cap;
+    h->last_det = h->det;
     h->last_stream = st;
     return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
@@ -463,11 +469,12 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
     // the median of five device-timed forwards of the first T rows of x, L2
     // flushed before each; the forward is captured into a graph and launched
     // whole, so neither branch pays for host-side gaps between its launches
-    auto time_path = [&](int T, int path, float *us) -> int {
+    auto time_path = [&](int T, int path, int row0, float *us) -> int {
         cudaGraph_t g = nullptr;
         cudaGraphExec_t ge = nullptr;
+        const void *xs = (const uint16_t *)x + (size_t)row0 * h->dm.d;
         if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ECUDA;
-        const int frc = run_forward(h, x, T, tau, true, h->ws.out_stage, st, path);
+        const int frc = run_forward(h, xs, T, tau, true, h->ws.out_stage, st, path);
         const cudaError_t ce = cudaStreamEndCapture(st, &g);
         if (frc || ce != cudaSuccess || cudaGraphInstantiate(&ge, g, 0) != cudaSuccess) {
             if (g) cudaGraphDestroy(g);
@@ -495,16 +502,21 @@ extern "C" int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau
     int best = 0;
     rc = MOE_OK;
     for (int T = 1, last = 0; T <= T_max && rc == MOE_OK;) {
-        float us_s = 0.f, us_d = 0.f;
-        rc = time_path(T, MOE_PATH_SPARSE, &us_s);
-        if (rc == MOE_OK) rc = time_path(T, MOE_PATH_DENSE, &us_d);
+        float us_s = 0.f, us_d = 0.f, us_s2 = 0.f;
+        rc = time_path(T, MOE_PATH_SPARSE, 0, &us_s);
+        // the sparse branch's cost depends on how the batch routes (its load
+        // balance over the experts): where x holds them, a second, disjoint
+        // batch of the same size is timed too and the two averaged.  The
+        // dense branch's cost is nearly the same for every batch of a size.
+        if (rc == MOE_OK && 2 * T <= T_max) {
+            rc = time_path(T, MOE_PATH_SPARSE, T_max - T, &us_s2);
+            us_s = 0.5f * (us_s + us_s2);
+        }
+        if (rc == MOE_OK) rc = time_path(T, MOE_PATH_DENSE, 0, &us_d);
         if (rc != MOE_OK) break;
-        // the dense branch is faster from here on.  A sparse time within 10 %
-        // of the dense one counts as slower: the sparse branch's cost depends
-        // on how the batch routes (its load balance over the experts), which
-        // the representative batch only samples, while the dense branch's cost
-        // is nearly the same for every batch of a size
-        if (us_s > 0.9f * us_d) break;
+        // the dense branch is faster from here on; a sparse time within 5 %
+        // of the dense one counts as slower (the batches only sample routing)
+        if (us_s > 0.95f * us_d) break;
         best = T;
         last = T;
         T = T < 4 ? T + 1 : (T % 3 == 0 ? T * 4 / 3 : T * 3 / 2);
@@ -658,6 +670,30 @@ extern "C" int moe_set_capacity(moe_handle h, float gamma)
     return MOE_OK;
 }
 
+extern "C" int moe_set_deterministic(moe_handle h, int enable)
+{
+    if (!is_live(h)) return MOE_EHANDLE;
+    if (enable) {
+        const size_t bytes =
+            (size_t)h->dm.max_tokens * (h->dm.k + h->dm.S) * h->dm.n_blk * h->dm.d * sizeof(float);
+        if (!h->det_rows) {
+            void *mem = nullptr;
+            if (inject_alloc_fail("deterministic") || cudaMalloc(&mem, bytes) != cudaSuccess) {
+                cudaGetLastError();
+                return MOE_ENOMEM;
+            }
+            h->det_rows = (float *)mem;
+        }
+        // all-zero before the first forward that uses the rows (and again after
+        // any earlier forward that a device error cut short)
+        if (cudaMemset(h->det_rows, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+            return MOE_ECUDA;
+    }
+    h->det = enable ? 1 : 0;
+    h->ws.ypart = h->det ? h->det_rows : nullptr;
+    return MOE_OK;
+}
+
 extern "C" int moe_set_launch_events(moe_handle h, void *const *events, int n)
 {
     if (!is_live(h)) return MOE_EHANDLE;
@@ -698,6 +734,7 @@ extern "C" int moe_query_stats(moe_handle h, moe_stats *st)
     st->t_star = h->t_star;
     st->fused_router = h->last_fused;
     st->capacity = h->last_cap;
+    st->deterministic = h->last_det;
     if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ECUDA;
     // the first error code since the previous call: an earlier forward's (kept
     // in the sticky word by the router of the next forward), else the last

@@ -89,6 +89,11 @@ class MoESparseLayer:
         weight (gamma <= 0: off)."""
         B.moe_set_capacity(self.h, float(gamma))
 
+    def set_deterministic(self, enable: bool = True):
+        """Combine each token's contributions in one fixed order on later
+        forwards (bit-identical repeats), instead of fp32 atomics."""
+        B.moe_set_deterministic(self.h, bool(enable))
+
     def calibrate_tau_shared(self, x, sparsity: float, stream=None) -> float:
         """tau_shared keeping about 1 - sparsity of the shared experts' neurons of this batch."""
         self._check_x(x)

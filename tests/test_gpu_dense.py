@@ -102,6 +102,27 @@ def test_large_dense(o):
     run_dense(o, "large", 64, 0.98, sample=8)
 
 
+@pytest.mark.parametrize("name,T", [("olmoe", 64), ("olmoe", 1000), ("dsv2lite", 8), ("dsv2lite", 128)])
+def test_dense_deterministic_combine(o, name, T):
+    """moe_set_deterministic on the dense branch: each (token, slot) row of
+    the down GEMM's epilogue written once, the k + S rows of a token summed in
+    order: oracle parity as for the atomic combine, and repeats bit-identical."""
+    import intra_expert_activation_router_b200 as m
+    layer, W, host = layer_for(name)
+    layer.set_deterministic(True)
+    try:
+        layer, x, tau, out = run_dense(o, name, T, 0.9, sample=None if T <= 64 else 12)
+        assert layer.stats()["deterministic"] == 1
+        layer.set_path(m.MOE_PATH_DENSE)
+        reps = [layer.forward(x, tau).clone() for _ in range(3)]
+        torch.cuda.synchronize()
+        for u in reps:
+            assert torch.equal(u, out)
+    finally:
+        layer.set_deterministic(False)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
 def test_dense_matches_sparse(o):
     """Both branches of the same layer at the same tau agree (up to h's bf16 rounding)."""
     import intra_expert_activation_router_b200 as m

@@ -108,11 +108,15 @@ def test_allocation_failure_injection(o, monkeypatch):
         with pytest.raises(m.MoeError) as ei:   # the rank budget's buffers: the threshold stays in force
             layer.set_rank_budget(50)
         assert ei.value.code == m.MOE_ENOMEM
+        monkeypatch.setenv("MOE_INJECT_ALLOC_FAIL", "deterministic")
+        with pytest.raises(m.MoeError) as ei:   # the deterministic combine's rows: atomics stay in force
+            layer.set_deterministic(True)
+        assert ei.value.code == m.MOE_ENOMEM
         monkeypatch.delenv("MOE_INJECT_ALLOC_FAIL")
         tau = layer.calibrate_tau(x, 0.9)   # the handle is still usable
         out = layer.forward(x, tau)
         torch.cuda.synchronize()
-        assert layer.stats()["rc"] == m.MOE_OK
+        assert layer.stats()["rc"] == m.MOE_OK and layer.stats()["deterministic"] == 0
         _check_against_oracle(o, W, sh, x, tau, out)
     finally:
         layer.close()

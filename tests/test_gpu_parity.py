@@ -327,6 +327,62 @@ def test_repeat_and_interleave(o):
         assert bool((d <= tol).all())
 
 
+@pytest.mark.parametrize("name,T,mode", [("olmoe", 1, "fused"), ("olmoe", 16, "fused"), ("olmoe", 16, "one_launch"),
+                                         ("olmoe", 16, "kernel"), ("olmoe", 40, "kernel"), ("dsv2lite", 8, "fused"),
+                                         ("dsv2lite", 8, "one_launch"), ("tiny", 16, "kernel"), ("large", 1, "fused")])
+def test_deterministic_combine(o, name, T, mode):
+    """moe_set_deterministic: every (token, slot, neuron block) contribution in
+    a row of its own, a token's rows summed in one fixed order.  The output
+    against the oracle as everywhere else; repeated forwards, interleaved with
+    another batch, bit-identical; with the capacity drop on, dropped pairs'
+    rows (never written) read as zero, and the next forward without the drop
+    is the plain deterministic one again."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES[name]
+    q = 0.98 if name == "large" else 0.9
+    layer, W, host = layer_for(name)
+    layer.set_fused_router(mode != "kernel", one_launch=(mode == "one_launch"))
+    layer.set_deterministic(True)
+    try:
+        tau, worst, _ = run_case(o, name, T, q)
+        st = layer.stats()
+        assert st["deterministic"] == 1 and st["device_error"] == 0
+        assert st["fused_router"] == ({"kernel": 0, "fused": 1, "one_launch": 2}[mode] if T <= 16 else 0)
+        layer.set_path(m.MOE_PATH_SPARSE)
+        x = mi.make_x(sh, T, device="cuda")
+        xo = mi.make_x(sh, 7, device="cuda", seed=5)
+        outs = []
+        for _ in range(4):
+            outs.append(layer.forward(x, tau).clone())
+            layer.forward(xo, tau)
+        torch.cuda.synchronize()
+        for u in outs[1:]:
+            assert torch.equal(u, outs[0])
+        if name != "large":   # capacity drop: only where gamma = 1 drops pairs at this T
+            layer.set_capacity(1.0)
+            try:
+                layer.set_deterministic(False)
+                plain = layer.forward(x, tau).clone()
+                layer.set_deterministic(True)
+                c1 = layer.forward(x, tau).clone()
+                c2 = layer.forward(x, tau).clone()
+                torch.cuda.synchronize()
+                C = -(-T * sh.top_k // sh.n_experts)
+                assert layer.stats()["capacity"] == (C if C < T else -1)
+                assert torch.equal(c1, c2)
+                dd = (c1.float() - plain.float()).abs()
+                assert bool((dd <= plain.float().abs() * 2.0 ** -7 + 1e-6).all())
+            finally:
+                layer.set_capacity(0.0)
+            again = layer.forward(x, tau)
+            torch.cuda.synchronize()
+            assert torch.equal(again, outs[0])
+    finally:
+        layer.set_deterministic(False)
+        layer.set_fused_router(True)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
 def test_host_pointer_entry(o):
     from intra_expert_activation_router_b200 import moe_sparse_forward_host
     sh = mi.SHAPES["olmoe"]
