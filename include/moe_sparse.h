@@ -293,6 +293,9 @@ int moe_set_launch_events(moe_handle h, void *const *events, int n);
 
 /* Tracing hook: when buf (DEVICE, 8-byte aligned, `bytes` long) is set, later
  * forwards stamp the GPU global timer (ns) at phase boundaries of each CTA.
+ * The sparse path then runs a separately compiled, traced copy of its expert
+ * kernel (same results; the stamps cost 4-7 % of a decode step, which the
+ * untraced kernel does not pay).
  * The first half of the buffer holds 8 stamps per router CTA (CTA index
  * y*gridDim.x + x): start, logits done, top-k start, top-k done, plan start,
  * plan done (the last two only in the CTA that builds the plan).  The second
@@ -341,7 +344,8 @@ int moe_query_stats(moe_handle h, moe_stats *st);
  * "weights" or "workspace", moe_sparse_create treats that device allocation
  * as failed (MOE_ENOMEM, nothing leaked); "scores" does the same for the
  * first moe_calibrate_tau's score buffer, "rank" for the first
- * moe_set_rank_budget's buffers.
+ * moe_set_rank_budget's buffers, "deterministic" for the first enabling
+ * moe_set_deterministic's rows.
  * Device error codes of the sparse kernel: 30-36 (copy, MMA and token-tile
  * waits), 40-45 (the consumers' waits on accumulators, gathered records and
  * the hand-off of h), 50-54 (waits for work items, slots and claims), 55

@@ -334,7 +334,9 @@ __device__ __forceinline__ bool route_better(float v1, int i1, float v0, int i0)
 //      (expert, then token) -- in its own shared memory; CTA 0 also writes it
 //      to the workspace, where the statistics and debug calls read it.
 // `scratch` (the gate ring, idle until the plan exists) holds the
-// temporaries.  Called by every thread of the CTA.
+// temporaries.  Called by every thread of the CTA.  TR: the traced build
+// (phase stamps into the workspace's trace buffer).
+template <bool TR>
 __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scratch, int *s_prefix, int *s_expert,
                                              int *s_off, int *s_cnt, int *s_perm, int *s_perm_tok, float *s_perm_w,
                                              volatile int *s_ntouched, uint64_t *xbar)
@@ -352,7 +354,7 @@ __device__ __noinline__ void route_in_kernel(const SparseArgs &a, uint8_t *scrat
     int *ecnt = reinterpret_cast<int *>(tk_w + P);                    // [E] pairs per expert
     int *eoff = ecnt + E;                                             // [E] first position per expert
     Plan *plan = a.ws.plan;
-    unsigned long long *tr = (a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
+    unsigned long long *tr = (TR && a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
                                  ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
     if (tr && tid == 0) tr[44] = global_ns();
 
@@ -612,7 +614,10 @@ __device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_f
     }
 }
 
-template <int MT, int NP>
+// TR: the traced instantiation, launched only while moe_set_trace holds a
+// buffer; the stamps' clock reads and branches cost 4-7 % of a decode step,
+// so the untraced kernel has none of them.
+template <int MT, int NP, bool TR>
 __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
 {
     extern __shared__ uint8_t dsm_raw[];
@@ -661,7 +666,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     int *err = a.ws.error_word;
     const int d = a.d;
     const bool score_mode = a.score_out != nullptr;
-    unsigned long long *tr = (a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
+    unsigned long long *tr = (TR && a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
                                  ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
     if (tr && tid == 0) tr[0] = global_ns();
 
@@ -712,7 +717,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     volatile int *s_ntouched = reinterpret_cast<volatile int *>(smem + L.ctr_off + 56);
     int n_touched, n_routed_items;
     if (a.fused) {
-        route_in_kernel(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched,
+        route_in_kernel<TR>(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched,
                         xfull);   // the token-tile barrier, unused in resident mode
         n_touched = *s_ntouched;
         n_routed_items = n_touched * a.n_blk;
@@ -1530,10 +1535,10 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     return cudaGetLastError();
 }
 
-template <int MT, int NP>
-static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
+template <int MT, int NP, bool TR>
+static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    auto kern = k_expert_sparse<MT, NP>;
+    auto kern = k_expert_sparse<MT, NP, TR>;
     static int smem_set[kMaxDevices] = {};
     cudaError_t e = ensure_dynamic_smem(kern, a.L.total, smem_set);
     if (e != cudaSuccess) return e;
@@ -1550,6 +1555,12 @@ static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
     e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+template <int MT, int NP>
+static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
+{
+    return a.ws.trace_expert ? launch_mt_tr<MT, NP, true>(a, grid, st) : launch_mt_tr<MT, NP, false>(a, grid, st);
 }
 
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,

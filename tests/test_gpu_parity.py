@@ -383,6 +383,46 @@ def test_deterministic_combine(o, name, T, mode):
         layer.set_path(m.MOE_PATH_AUTO)
 
 
+@pytest.mark.parametrize("T,fused", [(1, True), (16, True), (16, False)])
+def test_traced_kernel(o, T, fused):
+    """moe_set_trace switches the sparse path to the traced instantiation of
+    the expert kernel: with the deterministic combine its output is bit-equal
+    to the untraced kernel's, every CTA that ran stamps a start and an end
+    (end >= start), the item counts add up to the forward's work items, and
+    turning tracing off goes back to the untraced kernel."""
+    import intra_expert_activation_router_b200 as m
+    sh = mi.SHAPES["olmoe"]
+    layer, W, host = layer_for("olmoe")
+    x = mi.make_x(sh, T, device="cuda")
+    layer.set_path(m.MOE_PATH_SPARSE)
+    layer.set_fused_router(fused)
+    layer.set_deterministic(True)
+    words = 2 * 148 * 64 + 1024
+    buf = torch.zeros(words, dtype=torch.int64, device="cuda")
+    try:
+        plain = layer.forward(x, 1.0).clone()
+        m.moe_set_trace(layer.h, buf, words * 8)
+        traced = layer.forward(x, 1.0).clone()
+        m.moe_set_trace(layer.h, None)
+        again = layer.forward(x, 1.0).clone()
+        torch.cuda.synchronize()
+        assert layer.stats()["device_error"] == 0
+        assert torch.equal(traced, plain) and torch.equal(again, plain)
+        b = buf.cpu().numpy()
+        router = words // 2
+        et = b[router:router + (words - router) // 64 * 64].reshape(-1, 64)
+        ran = et[:, 0] > 0
+        assert ran.sum() >= 8
+        assert (et[ran, 62] >= et[ran, 0]).all()
+        st = layer.stats()
+        assert int(et[ran, 63].sum()) >= st["n_touched"] * (sh.d_ff // 128)
+    finally:
+        m.moe_set_trace(layer.h, None)
+        layer.set_deterministic(False)
+        layer.set_fused_router(True)
+        layer.set_path(m.MOE_PATH_AUTO)
+
+
 def test_host_pointer_entry(o):
     from intra_expert_activation_router_b200 import moe_sparse_forward_host
     sh = mi.SHAPES["olmoe"]
