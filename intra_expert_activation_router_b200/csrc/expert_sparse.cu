@@ -787,6 +787,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     // ub % owners; one warp is used.
     auto gather_loop = [&](int owner, int owners) {
             uint32_t ub = 0, idle = 0;
+            int ubi = 0;        // ub % NU and (ub / NU) & 1, kept without a division (NU is not a constant)
+            uint32_t uph = 0;
             for (int ui = 0;;) {
                 int go = 0;
                 if (lane == 0)
@@ -812,11 +814,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const size_t j0 = (size_t)M.blk * kBlk;
                 for (int s = 0; s < nsub; ++s) {
                     const int n = min(max(M.n_uni[s], 0), kBlk);
-                    for (int b0 = 0; b0 < n; b0 += L.gb, ++ub) {
+                    for (int b0 = 0; b0 < n; b0 += L.gb, ++ub, ubi = ubi + 1 < NU ? ubi + 1 : 0, uph ^= ubi == 0) {
                         const int nb = min(L.gb, n - b0);
-                        const int bi = (int)(ub % NU);
+                        const int bi = ubi;
                         if ((int)(ub % (uint32_t)owners) != owner) continue;   // another gather warp's batch
-                        mbar_wait(&empty_u[bi], ((ub / NU) & 1) ^ 1, err, 36);
+                        mbar_wait(&empty_u[bi], uph ^ 1, err, 36);
                         if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
                         ++nbatch;
                         uint8_t *dst = ud + (size_t)bi * L.ud_buf_bytes;
@@ -848,6 +850,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         if (lane == 0 && a.inject != 1) {
             const uint64_t pol = policy_evict_first();
             uint32_t g = 0;
+            int gs = 0;         // g % NS and (g / NS) & 1, kept without a division
+            uint32_t gph = 0;
             unsigned long long t_claim = 0, t_ring = 0, t_last = 0;   // trace only
             // resident mode: CTA b's first item is item b (all CTAs start at once,
             // so no counter round trip); later ones come from the counter, past
@@ -899,10 +903,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
                 if (a.a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
-                for (int s = s_lo; s < s_hi; ++s, ++g) {
-                    const int slot = (int)(g % NS);
+                for (int s = s_lo; s < s_hi; ++s, ++g, gs = gs + 1 < NS ? gs + 1 : 0, gph ^= gs == 0) {
+                    const int slot = gs;
                     const unsigned long long tr0 = tr ? global_ns() : 0;
-                    if (!mbar_wait(&empty_g[slot], ((g / NS) & 1) ^ 1, err, 30)) { ok = false; break; }
+                    if (!mbar_wait(&empty_g[slot], gph ^ 1, err, 30)) { ok = false; break; }
                     if (tr) {
                         t_last = global_ns();
                         t_ring += t_last - tr0;
@@ -942,6 +946,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, 16);
             uint32_t g = 0;
+            int gs = 0;         // g % NS and (g / NS) & 1, kept without a division
+            uint32_t gph = 0;
             int q = -1;
             long long prev_key = 0;
             bool ok = true;
@@ -962,9 +968,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 ok = ok && mbar_wait(&tfree[bsel], ((i / kAcc) & 1) ^ 1, err, 32);
                 tc_fence_after();
                 const uint32_t dt = tmem + 16 * bsel;
-                for (int s = s_lo; s < s_hi && ok; ++s, ++g) {
-                    const int slot = (int)(g % NS);
-                    ok = mbar_wait(&full_g[slot], (g / NS) & 1, err, 33);
+                for (int s = s_lo; s < s_hi && ok; ++s, ++g, gs = gs + 1 < NS ? gs + 1 : 0, gph ^= gs == 0) {
+                    const int slot = gs;
+                    ok = mbar_wait(&full_g[slot], gph, err, 33);
                     tc_fence_after();
                     if (tr && i == 0 && s == 0) tr[56] = global_ns();
                     const uint8_t *A = ring + (size_t)slot * L.stage_pitch;
@@ -1052,6 +1058,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         const int ct = tid;   // 0..127
         const int d8 = d >> 3;
         uint32_t ub = 0;
+        int ubi = 0;        // ub % NU and (ub / NU) & 1, kept without a division
+        uint32_t uph = 0;
         int n_rec = 0, ii = 0;
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         auto do_mask = [&](int i, int id) {
@@ -1222,11 +1230,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 load_x<MT, NP>(a.x, M.tok + r0, ms, d, ct, xf);   // the pass's token rows (L2-resident)
                 const int n_uni = min(max(M.n_uni[s], 0), kBlk);
                 n_rec += n_uni;
-                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
+                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub, ubi = ubi + 1 < NU ? ubi + 1 : 0, uph ^= ubi == 0) {
                     const int nb = min(L.gb, n_uni - b0);
-                    const int bi = (int)(ub % NU), hb = (int)(ub & 1);
+                    const int bi = ubi, hb = (int)(ub & 1);
                     const unsigned long long tw0 = tr ? global_ns() : 0;
-                    mbar_wait(&full_u[bi], (ub / NU) & 1, err, 41);
+                    mbar_wait(&full_u[bi], uph, err, 41);
                     const unsigned long long tw1 = tr ? global_ns() : 0;
                     t_wait += tw1 - tw0;
                     if (tu && ct == 0 && s == 0 && b0 == 0) tu[6] = global_ns();
@@ -1284,6 +1292,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
 #pragma unroll
                 for (int r = 0; r < MT; ++r) acc_y[p][i][r] = 0ull;
         uint32_t ub = 0;
+        int ubi = 0;        // ub % NU, kept without a division
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         for (int ii = 0; !score_mode; ++ii) {
             bool have = false;
@@ -1300,9 +1309,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int s = 0; s < nsub; ++s) {
                 const int r0 = s * MT, ms = min(MT, m - r0);
                 const int n_uni = min(max(M.n_uni[s], 0), kBlk);
-                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub) {
+                for (int b0 = 0; b0 < n_uni; b0 += L.gb, ++ub, ubi = ubi + 1 < NU ? ubi + 1 : 0) {
                     const int nb = min(L.gb, n_uni - b0);
-                    const int bi = (int)(ub % NU), hb = (int)(ub & 1);
+                    const int bi = ubi, hb = (int)(ub & 1);
                     const unsigned long long tw0 = tr ? global_ns() : 0;
                     mbar_wait(&hsfull[hb], (ub >> 1) & 1, err, 45);
                     const unsigned long long tw1 = tr ? global_ns() : 0;
