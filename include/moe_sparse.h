@@ -350,7 +350,11 @@ int moe_query_stats(moe_handle h, moe_stats *st);
  * waits), 40-45 (the consumers' waits on accumulators, gathered records and
  * the hand-off of h), 50-54 (waits for work items, slots and claims), 55
  * (in-kernel routing: the other CTAs' logits), 56 (gate split: the other
- * parts' sums), 57 (the combine at the end: the other CTAs' flushes). */
+ * parts' sums), 57 (the combine at the end: the other CTAs' flushes), 58
+ * (gate split: the owner part's union list, which the other parts of the
+ * item wait for to project their share of its records; every part is claimed
+ * at kernel start, so this assumes all CTAs of the grid are resident, as the
+ * in-kernel routing does). */
 #define MOE_INJECT_NONE 0
 #define MOE_INJECT_WITHHOLD_ITEMS 1
 int moe_debug_inject(moe_handle h, int kind);

@@ -80,6 +80,7 @@ constexpr int kTmemCols = 16 * kAcc;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
+constexpr int kShareMinRecords = 32;   // gate split: shortest union list whose records the parts share
 constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
 constexpr int kMaxFusedPairs = 128;  // fused routing: (token, expert) pairs kept in shared memory
 constexpr int kMaxFusedLogits = 8192;   // fused routing: T * E logits staged in the gate ring
@@ -135,6 +136,8 @@ struct SparseArgs {
     float *score_out;     // score mode: write |silu(g)| [pair][f] (or [token][S][f]), no up/down
     int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
     int n_parts;          // gate split: parts per item (1: none); part 0, claimed last, owns the item
+    int share_records;    // gate split: the parts also share the item's records (part p projects the
+                          // p-th of n_parts ranges of the owner's union list)
     int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
     const uint16_t *wr;   // fused: router weights [E][d]
     int E;
@@ -616,8 +619,11 @@ __device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_f
 
 // TR: the traced instantiation, launched only while moe_set_trace holds a
 // buffer; the stamps' clock reads and branches cost 4-7 % of a decode step,
-// so the untraced kernel has none of them.
-template <int MT, int NP, bool TR>
+// so the untraced kernel has none of them.  SH: the gate split's parts also
+// share the item's records (one- and two-token batches only); a separate
+// instantiation too, since code the other kernels never run still slowed
+// them by about a microsecond.
+template <int MT, int NP, bool TR, bool SH>
 __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
 {
     extern __shared__ uint8_t dsm_raw[];
@@ -1082,10 +1088,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 M.key = item_key(p);
                 M.m = m;
                 M.blk = p.blk;
-                M.masked = part > 0 ? 0 : p.slot < 0 ? (a.use_mask && a.tau_shared > 0.f ? 1 : 0) : a.use_mask;
+                M.masked = part > 0 && !SH ? 0 : p.slot < 0 ? (a.use_mask && a.tau_shared > 0.f ? 1 : 0) : a.use_mask;
                 M.sidx = p.slot < 0 ? -1 - p.slot : -1;
                 M.part = part;
-                M.nsub = part > 0 ? 0 : (m + MT - 1) / MT;   // a non-owner part has no up/down work
+                // a non-owner part has up/down work only when the records are shared
+                M.nsub = part > 0 && !SH ? 0 : (m + MT - 1) / MT;
                 M.wud = p.slot < 0 ? a.w.wsud + (size_t)(-1 - p.slot) * 2 * a.f * d
                                    : a.w.wud + (size_t)pc.expert[p.slot] * 2 * a.f * d;
             }
@@ -1164,8 +1171,37 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             if (gp && part > 0) __threadfence();   // this thread's partial sums before the count
             consumer_sync(kUpThreads);
             if (gp && part > 0 && ct == 0) atomicAdd(a.ws.gcnt + min(item, a.ws.gcnt_n - 1), 1);
+            // records shared: the owner adds n_parts more to the count once its
+            // union list is published (below); another part waits for that and
+            // takes its range of the list.  Every part of an item is claimed in
+            // the kernel's first round (parts x items <= grid), so the owner is
+            // running; its own wait is only for the parts' sums, published above.
+            // (only batches of at most kSplitCols tokens split; the wider
+            // instantiations carry none of this code)
+            SplitShare *gsh = nullptr;
+            if constexpr (SH && MT <= kSplitCols)
+                if (gp) gsh = a.ws.gshare + min(item, a.ws.gcnt_n - 1);
+            if (gsh && part > 0) {
+                if (ct == 0) {
+                    const int *cnt = a.ws.gcnt + min(item, a.ws.gcnt_n - 1);
+                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < 2 * a.n_parts - 1; ++spin) {
+                        if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
+                            atomicCAS(err, 0, 58);
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
+                consumer_sync(kUpThreads);
+                const int n = min(max(__ldcg(&gsh->n), 0), kBlk);
+                const int lo = part * n / a.n_parts, hi = (part + 1) * n / a.n_parts;
+                if (ct < hi - lo) M.uni[0][ct] = __ldcg(&gsh->uni[lo + ct]);
+                for (int t = 0; t < min(m, kSplitCols); ++t) M.a[t][ct] = __ldcg(&gsh->a[t][ct]);
+                if (ct < min(m, kSplitCols) * 4) M.word[ct >> 2][ct & 3] = __ldcg(&gsh->word[ct >> 2][ct & 3]);
+                if (ct == 0) M.n_uni[0] = hi - lo;
+            }
             if (ti && ct == 0) ti[4] = global_ns();
-            if (warp < M.nsub) {
+            if (warp < M.nsub && !(gsh && part > 0)) {
                 // union of the pass's tokens, compacted in ascending neuron order
                 const int s = warp, t0 = s * MT, t1 = min(m, t0 + MT);
                 int n = 0;
@@ -1181,6 +1217,27 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (lane == 0) M.n_uni[s] = n;
             }
             consumer_sync(kUpThreads);
+            if (gsh && part == 0) {
+                // publish the union list and keep the first range, when the list
+                // is long enough for the other parts' extra hand-off and gather
+                // round trip to pay; else publish an empty list
+                const int n = min(max(M.n_uni[0], 0), kBlk);
+                const bool sh = n >= kShareMinRecords;
+                if (sh) {
+                    if (ct < n) gsh->uni[ct] = M.uni[0][ct];
+                    for (int t = 0; t < min(m, kSplitCols); ++t) gsh->a[t][ct] = M.a[t][ct];
+                    if (ct < min(m, kSplitCols) * 4) gsh->word[ct >> 2][ct & 3] = M.word[ct >> 2][ct & 3];
+                    __threadfence();
+                    consumer_sync(kUpThreads);
+                }
+                if (ct == 0) {
+                    gsh->n = sh ? n : 0;
+                    __threadfence();
+                    atomicAdd(a.ws.gcnt + min(item, a.ws.gcnt_n - 1), a.n_parts);
+                    if (sh) M.n_uni[0] = n / a.n_parts;
+                }
+                if (sh) consumer_sync(kUpThreads);
+            }
             if (ct == 0) {
                 if (!score_mode) {
                     int total = 0;
@@ -1193,7 +1250,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             }
             // the pairs' mask words for statistics and the debug lists: written
             // after the publication, off the gather's critical path
-            if (M.masked && M.sidx < 0 && ct < m * 4) {   // routed pairs only
+            if (M.masked && M.sidx < 0 && (!SH || M.part == 0) && ct < m * 4) {   // routed pairs only, by the owner
                 const int t = ct >> 2, qw = ct & 3, chunk = M.blk * 4 + qw;
                 if (chunk < a.n_chunks) a.ws.mask[(size_t)M.pair[t] * a.n_chunks + chunk] = M.word[t][qw];
             }
@@ -1544,10 +1601,10 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     return cudaGetLastError();
 }
 
-template <int MT, int NP, bool TR>
+template <int MT, int NP, bool TR, bool SH>
 static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    auto kern = k_expert_sparse<MT, NP, TR>;
+    auto kern = k_expert_sparse<MT, NP, TR, SH>;
     static int smem_set[kMaxDevices] = {};
     cudaError_t e = ensure_dynamic_smem(kern, a.L.total, smem_set);
     if (e != cudaSuccess) return e;
@@ -1569,7 +1626,12 @@ static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 template <int MT, int NP>
 static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    return a.ws.trace_expert ? launch_mt_tr<MT, NP, true>(a, grid, st) : launch_mt_tr<MT, NP, false>(a, grid, st);
+    if constexpr (MT <= kSplitCols)
+        if (a.share_records)
+            return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, true>(a, grid, st)
+                                     : launch_mt_tr<MT, NP, false, true>(a, grid, st);
+    return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, false>(a, grid, st)
+                             : launch_mt_tr<MT, NP, false, false>(a, grid, st);
 }
 
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
@@ -1631,6 +1693,13 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
                     break;
                 }
     }
+    // the parts also share the item's records where every item is one pass
+    // (nsub = 1), the combine takes any number of writers per row, and some
+    // items have long union lists: the shared experts' when no threshold
+    // applies to them (every neuron of a block active)
+    a.share_records =
+        (a.n_parts > 1 && til.mt >= T && !ws.ypart && ws.gshare && dm.S > 0 && (!use_mask || tau_shared <= 0.f)) ? 1
+                                                                                                              : 0;
     const long long bound = (a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk) * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
     // the combine at the end of this kernel (one launch per forward), else a

@@ -34,6 +34,17 @@ constexpr int kDenseTileM = 128;     // tokens per dense GEMM tile
 constexpr int kSplitCols = 2;        // gate split: batches of at most this many tokens
 constexpr int kMaxParts = 4;         // gate split: parts per item
 
+// Gate split, records shared: the owner part's union list and mask of an
+// item (kBlk = 128 neurons, at most kSplitCols tokens), published for the
+// other parts, which project their own share of the records.
+struct SplitShare {
+    int n;                                 // union-active neurons of the block
+    int pad[3];
+    uint8_t uni[128];                      // their positions in the block, ascending
+    uint32_t word[kSplitCols][4];          // per token: its active neurons, 32 per word
+    uint16_t a[kSplitCols][128];           // per token: silu(g) as bf16
+};
+
 // Routing plan written by the router's last CTA.
 struct Plan {
     int n_touched;                    // distinct experts selected
@@ -134,6 +145,7 @@ struct Workspace {
     float *gpart;
     int *gcnt;
     int gcnt_n;
+    SplitShare *gshare;   // [item]: the owner's union list, when the parts share the records
     Plan *plan;
     // dense path
     uint16_t *x_perm;   // [T*k + T][d] bf16: tokens in perm order, then x for the shared experts

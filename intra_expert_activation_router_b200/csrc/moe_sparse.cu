@@ -172,7 +172,9 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     const long long split_items = (long long)((2 * top_k < E ? 2 * top_k : E) + n_shared) * dm.n_blk;
     const bool split_ok = split_items <= 4096;
     const size_t part_floats = (size_t)(moe::kMaxParts - 1) * moe::kBlk * moe::kSplitCols;   // per item
-    const size_t split_bytes = split_ok ? (size_t)split_items * (part_floats * sizeof(float) + sizeof(int)) + 2 * 256 : 0;
+    const size_t split_bytes =
+        split_ok ? (size_t)split_items * (part_floats * sizeof(float) + sizeof(int) + sizeof(moe::SplitShare)) + 3 * 256
+                 : 0;
     if (inject_alloc_fail("weights") || cudaMalloc(&h->weight_mem, wbytes) != cudaSuccess) {
         cudaGetLastError();
         h->weight_mem = nullptr;
@@ -227,7 +229,8 @@ extern "C" int moe_sparse_create(const moe_weights *w, int E, int top_k, int d_m
     if (split_ok) {
         ws.gpart = (float *)sb.take((size_t)split_items * part_floats * sizeof(float));
         ws.gcnt = (int *)sb.take((size_t)split_items * sizeof(int));
-        ws.gcnt_n = ws.gpart && ws.gcnt ? (int)split_items : 0;
+        ws.gshare = (moe::SplitShare *)sb.take((size_t)split_items * sizeof(moe::SplitShare));
+        ws.gcnt_n = ws.gpart && ws.gcnt && ws.gshare ? (int)split_items : 0;
         if (!ws.gcnt_n) ws.gpart = nullptr, ws.gcnt = nullptr;
     }
     ws.plan = (moe::Plan *)sb.take(sizeof(moe::Plan));
