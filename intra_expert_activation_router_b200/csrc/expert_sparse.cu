@@ -135,7 +135,8 @@ struct SparseArgs {
     int max_touched;      // plan cache capacity
     float *score_out;     // score mode: write |silu(g)| [pair][f] (or [token][S][f]), no up/down
     int inject;           // test-only fault: 1 = publish no work item (consumers' waits run out)
-    int n_parts;          // gate split: parts per item (1: none); part 0, claimed last, owns the item
+    int n_parts;          // gate split: parts per routed item (1: none); part 0, claimed last, owns the item
+    int n_parts_s;        // the same for the shared experts' items
     int share_records;    // gate split: the parts also share the item's records (part p projects the
                           // p-th of n_parts ranges of the owner's union list)
     int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
@@ -204,12 +205,42 @@ __device__ __forceinline__ long long item_key(const ItemPos &p)
     return ((long long)(p.slot < 0 ? p.slot : p.slot + 1) << 32) | (unsigned)p.tile;
 }
 
-// Gate split: claim id -> (item, part).  An item's parts are claimed in the
-// order n_parts - 1, ..., 1, 0, so the owner (part 0), which waits for the
-// others' partial sums, is always claimed after them: every wait points to an
-// earlier claim, which its CTA publishes before it reaches any later wait.
-__device__ __forceinline__ int split_item(const SparseArgs &a, int id) { return id / a.n_parts; }
-__device__ __forceinline__ int split_part(const SparseArgs &a, int id) { return a.n_parts - 1 - id % a.n_parts; }
+// Gate split: claim id -> (item, part).  The shared experts' items come
+// first, n_parts_s claims each, then the routed items, n_parts each.  An
+// item's parts are claimed in the order P - 1, ..., 1, 0, so the owner (part
+// 0), which waits for the others' partial sums, is always claimed after them:
+// every such wait points to an earlier claim, which its CTA publishes before
+// it reaches any later wait.
+// PC: per-class part counts (the record-sharing instantiation); otherwise
+// every item has n_parts parts (n_parts_s == n_parts).
+template <bool PC>
+__device__ __forceinline__ int split_item(const SparseArgs &a, int id)
+{
+    if constexpr (PC) {
+        const int ns = a.n_shared_items * a.n_parts_s;
+        return id < ns ? id / a.n_parts_s : a.n_shared_items + (id - ns) / a.n_parts;
+    } else {
+        return id / a.n_parts;
+    }
+}
+template <bool PC>
+__device__ __forceinline__ int split_part(const SparseArgs &a, int id)
+{
+    if constexpr (PC) {
+        const int ns = a.n_shared_items * a.n_parts_s;
+        return id < ns ? a.n_parts_s - 1 - id % a.n_parts_s : a.n_parts - 1 - (id - ns) % a.n_parts;
+    } else {
+        return a.n_parts - 1 - id % a.n_parts;
+    }
+}
+template <bool PC>
+__device__ __forceinline__ int item_parts(const SparseArgs &a, int item)
+{
+    if constexpr (PC)
+        return item < a.n_shared_items ? a.n_parts_s : a.n_parts;
+    else
+        return a.n_parts;
+}
 
 // Stages [lo, hi) of the item's spi gate stages that a part streams.
 __device__ __forceinline__ void part_stages(int spi, int n_parts, int part, int &lo, int &hi)
@@ -760,7 +791,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                        a.fused ? s_perm : a.ws.perm, a.fused ? s_perm_tok : a.ws.perm_tok,
                        a.fused ? s_perm_w : a.ws.perm_w};
 
-    const int n_items = (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts;
+    const int n_items = SH ? a.n_shared_items * a.n_parts_s + (a.score_shared ? 0 : n_routed_items) * a.n_parts
+                           : (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts;
     // static ranges (token-tile mode): contiguous items per CTA
     const int G = gridDim.x, b = blockIdx.x;
     const int per = n_items / G, rem = n_items % G;
@@ -903,10 +935,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 __threadfence_block();
                 *pub_items = i + 1;
                 if (id < 0) break;
-                const ItemPos ip = locate_item(a, pc, split_item(a, id));
+                const ItemPos ip = locate_item(a, pc, split_item<SH>(a, id));
                 const uint16_t *src = gate_src(ip);
                 int s_lo, s_hi;
-                part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
+                part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
                 if (a.a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
                 for (int s = s_lo; s < s_hi; ++s, ++g, gs = gs + 1 < NS ? gs + 1 : 0, gph ^= gs == 0) {
@@ -960,10 +992,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int i = 0; ok; ++i) {
                 const int id = get_item(i);
                 if (id < 0) break;
-                const ItemPos p = locate_item(a, pc, split_item(a, id));
+                const ItemPos p = locate_item(a, pc, split_item<SH>(a, id));
                 const long long key = item_key(p);
                 int s_lo, s_hi;
-                part_stages(spi, a.n_parts, split_part(a, id), s_lo, s_hi);
+                part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
                 const bool skip = a.a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
                 if (skip) s_hi = s_lo;
                 if (!a.resident && (i == 0 || key != prev_key)) {
@@ -1070,7 +1102,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         auto do_mask = [&](int i, int id) {
             ItemMeta &M = meta[i & 1];
-            const int item = split_item(a, id), part = split_part(a, id);
+            const int item = split_item<SH>(a, id), part = split_part<SH>(a, id);
             const ItemPos p = locate_item(a, pc, item);
             int base;
             const int m = tile_tokens(a, pc, p, base);
@@ -1100,13 +1132,14 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             unsigned long long *ti = (tr && i < 3) ? tr + 2 + 10 * i : nullptr;   // per-item stamps
             if (ti && ct == 0) ti[0] = global_ns();
             // gate split: the item's partial sums, [part - 1][neuron][token]
-            float *gp = a.n_parts > 1 ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
+            const int np = item_parts<SH>(a, item);
+            float *gp = np > 1 ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
                                                           kSplitCols
                                       : nullptr;
             if (gp && part == 0) {   // the owner waits until the other parts have published theirs
                 if (ct == 0) {
                     const int *cnt = a.ws.gcnt + min(item, a.ws.gcnt_n - 1);
-                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < a.n_parts - 1; ++spin) {
+                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < np - 1; ++spin) {
                         if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
                             atomicCAS(err, 0, 56);
                             break;
@@ -1148,7 +1181,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                                 gp[((part - 1) * kBlk + jl) * kSplitCols + c] = g;
                                 continue;
                             }
-                            for (int r = 1; r < a.n_parts; ++r)
+                            for (int r = 1; r < np; ++r)
                                 g += __ldcg(&gp[((r - 1) * kBlk + jl) * kSplitCols + c]);
                         }
                         av = silu_f(g);
@@ -1184,7 +1217,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             if (gsh && part > 0) {
                 if (ct == 0) {
                     const int *cnt = a.ws.gcnt + min(item, a.ws.gcnt_n - 1);
-                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < 2 * a.n_parts - 1; ++spin) {
+                    for (uint32_t spin = 0; ld_acquire_gpu(cnt) < 2 * np - 1; ++spin) {
                         if (spin > kSpinLimit || (spin > 1024 && *reinterpret_cast<volatile int *>(err) != 0)) {
                             atomicCAS(err, 0, 58);
                             break;
@@ -1194,7 +1227,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 }
                 consumer_sync(kUpThreads);
                 const int n = min(max(__ldcg(&gsh->n), 0), kBlk);
-                const int lo = part * n / a.n_parts, hi = (part + 1) * n / a.n_parts;
+                const int lo = part * n / np, hi = (part + 1) * n / np;
                 if (ct < hi - lo) M.uni[0][ct] = __ldcg(&gsh->uni[lo + ct]);
                 for (int t = 0; t < min(m, kSplitCols); ++t) M.a[t][ct] = __ldcg(&gsh->a[t][ct]);
                 if (ct < min(m, kSplitCols) * 4) M.word[ct >> 2][ct & 3] = __ldcg(&gsh->word[ct >> 2][ct & 3]);
@@ -1233,8 +1266,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (ct == 0) {
                     gsh->n = sh ? n : 0;
                     __threadfence();
-                    atomicAdd(a.ws.gcnt + min(item, a.ws.gcnt_n - 1), a.n_parts);
-                    if (sh) M.n_uni[0] = n / a.n_parts;
+                    atomicAdd(a.ws.gcnt + min(item, a.ws.gcnt_n - 1), np);
+                    if (sh) M.n_uni[0] = n / np;
                 }
                 if (sh) consumer_sync(kUpThreads);
             }
@@ -1410,8 +1443,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (nsub == 1 && !a.ws.ypart) {   // (deterministic mode: one row per block)
                     const int nid = get_item(ii + 1);
                     // (a non-owner part has no up/down work: stop accumulating there)
-                    cont = nid >= 0 && split_part(a, nid) == 0 &&
-                           item_key(locate_item(a, pc, split_item(a, nid))) == M.key;
+                    cont = nid >= 0 && split_part<SH>(a, nid) == 0 &&
+                           item_key(locate_item(a, pc, split_item<SH>(a, nid))) == M.key;
                 }
                 if (!cont) {
 #pragma unroll
@@ -1681,26 +1714,40 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     const int np = (dm.d / 8 + 127) / 128;
     // gate split: one- and two-token batches whose items are fewer than the SMs
     // stream each item's gate on 2 or 4 CTAs (MOE_SPLIT=0 turns it off)
-    a.n_parts = 1;
+    a.n_parts = a.n_parts_s = 1;
+    // the shared experts' items are the heavy ones when no threshold applies
+    // to them (every neuron of a block active: 128 records each)
+    const bool dense_shared = a.n_shared_items > 0 && (!use_mask || tau_shared <= 0.f);
+    const long long routed_max = (long long)a.max_touched * dm.n_blk;
     {
         const char *sp = std::getenv("MOE_SPLIT");
-        const long long base_max = a.n_shared_items + (long long)a.max_touched * dm.n_blk;
+        const long long base_max = a.n_shared_items + routed_max;
         if (a.resident && !score_out && !a.a_in && T <= kSplitCols && ws.gpart && ws.gcnt && base_max <= ws.gcnt_n &&
-            !(sp && std::strcmp(sp, "0") == 0))
+            !(sp && std::strcmp(sp, "0") == 0)) {
             for (int r = kMaxParts; r >= 2; r >>= 1)
                 if (base_max * r <= grid_cap && dm.n_kb / 2 >= r) {
-                    a.n_parts = r;
+                    a.n_parts = a.n_parts_s = r;
                     break;
                 }
+            // then more parts for heavy shared items where the grid has room
+            // (the record-sharing kernel, below, is the one that maps per-class
+            // part counts)
+            if (dense_shared && til.mt >= T && !ws.ypart && ws.gshare)
+                for (int r = kMaxParts; r > a.n_parts_s; r >>= 1)
+                    if (a.n_shared_items * r + routed_max * a.n_parts <= grid_cap && dm.n_kb / 2 >= r) {
+                        a.n_parts_s = r;
+                        break;
+                    }
+        }
     }
     // the parts also share the item's records where every item is one pass
     // (nsub = 1), the combine takes any number of writers per row, and some
-    // items have long union lists: the shared experts' when no threshold
-    // applies to them (every neuron of a block active)
-    a.share_records =
-        (a.n_parts > 1 && til.mt >= T && !ws.ypart && ws.gshare && dm.S > 0 && (!use_mask || tau_shared <= 0.f)) ? 1
-                                                                                                              : 0;
-    const long long bound = (a.n_shared_items + (long long)(a.max_touched + pairs / til.nt) * dm.n_blk) * a.n_parts;
+    // items have long union lists (the dense shared experts')
+    a.share_records = ((a.n_parts > 1 || a.n_parts_s > 1) && til.mt >= T && !ws.ypart && ws.gshare && dense_shared)
+                          ? 1
+                          : 0;
+    const long long bound = (long long)a.n_shared_items * a.n_parts_s +
+                            (long long)(a.max_touched + pairs / til.nt) * dm.n_blk * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
     // the combine at the end of this kernel (one launch per forward), else a
     // separate conversion kernel
