@@ -81,6 +81,7 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
 constexpr int kShareMinRecords = 32;   // gate split: shortest union list whose records the parts share
+constexpr int kRecSplitParts = 2;      // record split of dense shared items: parts per item
 constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
 constexpr int kMaxFusedPairs = 128;  // fused routing: (token, expert) pairs kept in shared memory
 constexpr int kMaxFusedLogits = 8192;   // fused routing: T * E logits staged in the gate ring
@@ -138,7 +139,9 @@ struct SparseArgs {
     int n_parts;          // gate split: parts per routed item (1: none); part 0, claimed last, owns the item
     int n_parts_s;        // the same for the shared experts' items
     int share_records;    // gate split: the parts also share the item's records (part p projects the
-                          // p-th of n_parts ranges of the owner's union list)
+                          // p-th of n_parts ranges of the owner's union list); launches the SH kernel
+    int rec_split;        // instead of a gate split: each of a dense shared item's n_parts_s parts streams
+                          // the whole gate and projects the p-th range of its records (no hand-off)
     int fused;            // route the batch here (resident mode): logits, top-k and plan per CTA
     const uint16_t *wr;   // fused: router weights [E][d]
     int E;
@@ -938,7 +941,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const ItemPos ip = locate_item(a, pc, split_item<SH>(a, id));
                 const uint16_t *src = gate_src(ip);
                 int s_lo, s_hi;
-                part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                if (SH && a.rec_split) {   // every record-split part streams the whole gate
+                    s_lo = 0;
+                    s_hi = spi;
+                } else {
+                    part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                }
                 if (a.a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
                 for (int s = s_lo; s < s_hi; ++s, ++g, gs = gs + 1 < NS ? gs + 1 : 0, gph ^= gs == 0) {
@@ -995,7 +1003,12 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const ItemPos p = locate_item(a, pc, split_item<SH>(a, id));
                 const long long key = item_key(p);
                 int s_lo, s_hi;
-                part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                if (SH && a.rec_split) {   // every record-split part streams the whole gate
+                    s_lo = 0;
+                    s_hi = spi;
+                } else {
+                    part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                }
                 const bool skip = a.a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
                 if (skip) s_hi = s_lo;
                 if (!a.resident && (i == 0 || key != prev_key)) {
@@ -1133,7 +1146,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             if (ti && ct == 0) ti[0] = global_ns();
             // gate split: the item's partial sums, [part - 1][neuron][token]
             const int np = item_parts<SH>(a, item);
-            float *gp = np > 1 ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
+            float *gp = np > 1 && !(SH && a.rec_split) ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
                                                           kSplitCols
                                       : nullptr;
             if (gp && part == 0) {   // the owner waits until the other parts have published theirs
@@ -1246,6 +1259,21 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const unsigned bal = __ballot_sync(kFull, on);
                     if (on) M.uni[s][n + __popc(bal & ((1u << lane) - 1u))] = (uint8_t)(qw * 32 + lane);
                     n += __popc(bal);
+                }
+                if constexpr (SH) {
+                    if (a.rec_split && np > 1) {   // this part's range of the list, moved to its front
+                        const int lo = part * n / np, hi = (part + 1) * n / np;
+                        __syncwarp();
+                        uint8_t v[kBlk / 32];
+#pragma unroll
+                        for (int c = 0; c < kBlk / 32; ++c)
+                            v[c] = lane + 32 * c < hi - lo ? M.uni[s][lo + lane + 32 * c] : 0;
+                        __syncwarp();
+#pragma unroll
+                        for (int c = 0; c < kBlk / 32; ++c)
+                            if (lane + 32 * c < hi - lo) M.uni[s][lane + 32 * c] = v[c];
+                        n = hi - lo;
+                    }
                 }
                 if (lane == 0) M.n_uni[s] = n;
             }
@@ -1659,10 +1687,9 @@ static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 template <int MT, int NP>
 static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    if constexpr (MT <= kSplitCols)
-        if (a.share_records)
-            return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, true>(a, grid, st)
-                                     : launch_mt_tr<MT, NP, false, true>(a, grid, st);
+    if (a.share_records)
+        return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, true>(a, grid, st)
+                                 : launch_mt_tr<MT, NP, false, true>(a, grid, st);
     return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, false>(a, grid, st)
                              : launch_mt_tr<MT, NP, false, false>(a, grid, st);
 }
@@ -1746,6 +1773,15 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.share_records = ((a.n_parts > 1 || a.n_parts_s > 1) && til.mt >= T && !ws.ypart && ws.gshare && dense_shared)
                           ? 1
                           : 0;
+    // no gate split: a dense shared item (128 records per pass, the slowest
+    // item of the batch) is split by records instead, each part streaming
+    // the whole gate (its extra gate traffic buys a shorter critical path)
+    a.rec_split = 0;
+    if (a.n_parts == 1 && a.n_parts_s == 1 && dense_shared && a.resident && !score_out && !a.a_in && !ws.ypart) {
+        a.rec_split = 1;
+        a.n_parts_s = kRecSplitParts;
+        a.share_records = 1;
+    }
     const long long bound = (long long)a.n_shared_items * a.n_parts_s +
                             (long long)(a.max_touched + pairs / til.nt) * dm.n_blk * a.n_parts;
     int grid = bound < grid_cap ? (int)bound : grid_cap;
