@@ -81,7 +81,7 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxNU = 6;            // gather buffers
 constexpr int kIdRing = 16;          // published work-item ids
 constexpr int kShareMinRecords = 32;   // gate split: shortest union list whose records the parts share
-constexpr int kRecSplitParts = 2;      // record split of dense shared items: parts per item
+constexpr int kRecSplitMax = 4;        // record split of dense shared items: most parts per item
 constexpr int kClaimBacklog = 24;    // resident mode: records still to project when the next item is claimed
 constexpr int kMaxFusedPairs = 128;  // fused routing: (token, expert) pairs kept in shared memory
 constexpr int kMaxFusedLogits = 8192;   // fused routing: T * E logits staged in the gate ring
@@ -1776,10 +1776,12 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     // no gate split: a dense shared item (128 records per pass, the slowest
     // item of the batch) is split by records instead, each part streaming
     // the whole gate (its extra gate traffic buys a shorter critical path)
+    // (4 parts where every claim still has an SM of its own, else 2: beyond
+    // the grid the extra gate streams compete with the other items)
     a.rec_split = 0;
     if (a.n_parts == 1 && a.n_parts_s == 1 && dense_shared && a.resident && !score_out && !a.a_in && !ws.ypart) {
         a.rec_split = 1;
-        a.n_parts_s = kRecSplitParts;
+        a.n_parts_s = (long long)a.n_shared_items * kRecSplitMax + routed_max <= grid_cap ? kRecSplitMax : 2;
         a.share_records = 1;
     }
     const long long bound = (long long)a.n_shared_items * a.n_parts_s +
