@@ -84,8 +84,10 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
         // Capacity-aware token drop ("Capacity-Aware Inference", "Capacity-
         // Aware Token Drop"): an expert routed more than cap pairs keeps the
         // cap with the largest routing weight, ties to the lower token.  The
-        // pairs are first grouped by expert in token order (s_seg); a pair of
-        // an over-capacity expert is dropped when at least cap pairs of its
+        // pairs are first grouped by expert (s_seg; the order inside a group
+        // is whatever the atomics give, since the ranking breaks ties by the
+        // pair index, which orders an expert's pairs by token); a pair of an
+        // over-capacity expert is dropped when at least cap pairs of its
         // group beat it.  A dropped pair then belongs to no expert's list
         // (sentinel E) and its mask words read as empty.
         if (warp == 0) {
@@ -101,19 +103,9 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
                 if (e < E) s_cur[e] = run + inc - c;
                 run += __shfl_sync(kFull, inc, 31);
             }
-            __syncwarp();
-            for (int base = 0; base < P; base += 32) {   // stable: 32 pairs at a time, in pair order
-                const int p = base + lane;
-                const int e = p < P ? s_idx[p] : -1 - lane;
-                const unsigned same = __match_any_sync(kFull, e);
-                const int rank = __popc(same & ((1u << lane) - 1));
-                const int pos = p < P ? s_cur[e] + rank : 0;
-                __syncwarp();
-                if (p < P && rank == 0) s_cur[e] += __popc(same);
-                if (p < P) s_seg[pos] = p;
-                __syncwarp();
-            }
         }
+        __syncthreads();
+        for (int p = tid; p < P; p += blockDim.x) s_seg[atomicAdd(&s_cur[s_idx[p]], 1)] = p;
         __syncthreads();   // s_cur[e] now ends expert e's group
         uint32_t drop = 0;   // bit i: the pair at group position tid + i * blockDim.x
         for (int i = tid, bit = 0; i < P; i += blockDim.x, ++bit) {
@@ -122,9 +114,11 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
             const int g1 = s_cur[e], g0 = g1 - s_cnt[e];
             const float wp = s_w[p];
             int better = 0;
-            for (int j = g0; j < g1; ++j) {   // earlier positions hold lower tokens
-                const float wq = s_w[s_seg[j]];
-                better += (wq > wp || (wq == wp && j < i)) ? 1 : 0;
+#pragma unroll 8
+            for (int j = g0; j < g1; ++j) {
+                const int q = s_seg[j];
+                const float wq = s_w[q];
+                better += (wq > wp || (wq == wp && q < p)) ? 1 : 0;
             }
             if (better >= a.cap) drop |= 1u << bit;
         }
@@ -186,10 +180,27 @@ __device__ void build_plan(const RouterArgs &a, int *s_cnt, int *s_cur, int *s_i
         __syncwarp();
         // large batches: the scatter is a kernel of its own (k_plan_scatter),
         // one pair per thread through per-expert cursors, zeroed here
-        if (!staged) {
+        if (!staged)
             for (int e = lane; e < E; e += 32) a.ws.cursor[e] = 0;
-            return;
+    }
+    if (!staged) return;
+    __syncthreads();   // s_cur[e]: expert e's first position
+    if (P > kSmallPlan) {
+        // larger staged plans (the capacity drop's): one pair per thread
+        // through the shared-memory cursors; the order inside an expert is
+        // then arbitrary, which neither branch's result depends on
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int e = s_idx[p];
+            if (e < E) {   // a dropped pair (expert E) takes no position
+                const int pos = atomicAdd(&s_cur[e], 1);
+                a.ws.perm[pos] = p;
+                a.ws.perm_tok[pos] = p / a.k;
+                a.ws.perm_w[pos] = s_w[p];
+            }
         }
+        return;
+    }
+    if (warp == 0) {
         // stable scatter, 32 pairs at a time in pair order
         for (int base = 0; base < P; base += 32) {
             const int p = base + lane;
