@@ -174,6 +174,8 @@ struct PlanCache {      // the routing plan's per-slot arrays, copied to shared 
     const float *perm_w;
 };
 
+// DEC: the decode instantiation, always resident (see k_expert_sparse)
+template <bool DEC>
 __device__ __forceinline__ ItemPos locate_item(const SparseArgs &a, const PlanCache &pc, int item)
 {
     ItemPos p;
@@ -183,7 +185,7 @@ __device__ __forceinline__ ItemPos locate_item(const SparseArgs &a, const PlanCa
         const int r0 = item % per_s;
         p.tile = r0 / a.n_blk;
         p.blk = r0 % a.n_blk;
-    } else if (a.resident) {   // one tile per expert, slots heaviest first
+    } else if (DEC || a.resident) {   // one tile per expert, slots heaviest first
         const int ir = item - a.n_shared_items;
         p.slot = pc.order[min(ir / a.n_blk, pc.n_touched - 1)];
         p.tile = 0;
@@ -653,11 +655,15 @@ __device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_f
 
 // TR: the traced instantiation, launched only while moe_set_trace holds a
 // buffer; the stamps' clock reads and branches cost 4-7 % of a decode step,
-// so the untraced kernel has none of them.  SH: the gate split's parts also
-// share the item's records (one- and two-token batches only); a separate
-// instantiation too, since code the other kernels never run still slowed
-// them by about a microsecond.
-template <int MT, int NP, bool TR, bool SH>
+// so the untraced kernels have none of them.  DEC: the decode instantiation,
+// for batches resident as one token tile outside the rank budget's second
+// pass and fault injection: the token-tile mode, the rank pass and the
+// injection compiled out (5-7 % of a decode step).  SH (decode only): the
+// parts of a split item also share its records, per-class part counts, the
+// record split of dense shared items; a separate instantiation again, since
+// code the other kernels never run still slowed them by about a microsecond.
+// The traced kernel is the general one (not DEC, not SH).
+template <int MT, int NP, bool TR, bool SH, bool DEC>
 __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
 {
     extern __shared__ uint8_t dsm_raw[];
@@ -706,6 +712,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     int *err = a.ws.error_word;
     const int d = a.d;
     const bool score_mode = a.score_out != nullptr;
+    const bool resident = DEC || a.resident;        // compile-time true in the decode kernel
+    const float *const a_in = DEC ? nullptr : a.a_in;   // rank pass, second pass
+    const int inject = DEC ? 0 : a.inject;
     unsigned long long *tr = (TR && a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
                                  ? a.ws.trace_expert + blockIdx.x * 64 : nullptr;
     if (tr && tid == 0) tr[0] = global_ns();
@@ -775,7 +784,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         }
         __syncthreads();
     }
-    if (a.resident) {
+    if (resident) {
         // slots by decreasing token count (ties by slot): claimed in this order,
         // the most expensive items go first and the tail is made of cheap ones
         for (int i = tid; i < n_touched; i += blockDim.x) {
@@ -888,7 +897,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         // publishes the work-item ids (claimed from the plan's counter in
         // resident mode, else the CTA's static range), then streams each
         // item's gate tiles into the ring
-        if (lane == 0 && a.inject != 1) {
+        if (lane == 0 && inject != 1) {
             const uint64_t pol = policy_evict_first();
             uint32_t g = 0;
             int gs = 0;         // g % NS and (g / NS) & 1, kept without a division
@@ -897,10 +906,10 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             // resident mode: CTA b's first item is item b (all CTAs start at once,
             // so no counter round trip); later ones come from the counter, past
             // the grid's first items
-            int next = a.resident ? (int)blockIdx.x : 0;
+            int next = resident ? (int)blockIdx.x : 0;
             for (int i = 0;; ++i) {
                 int id;
-                if (a.resident) {
+                if (resident) {
                     if (i > 0 && next < n_items) {
                         // item i - 1 masked and the up/down backlog short: claim the
                         // next item (its gate streams while the backlog drains)
@@ -938,7 +947,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 __threadfence_block();
                 *pub_items = i + 1;
                 if (id < 0) break;
-                const ItemPos ip = locate_item(a, pc, split_item<SH>(a, id));
+                const ItemPos ip = locate_item<DEC>(a, pc, split_item<SH>(a, id));
                 const uint16_t *src = gate_src(ip);
                 int s_lo, s_hi;
                 if (SH && a.rec_split) {   // every record-split part streams the whole gate
@@ -947,7 +956,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 } else {
                     part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
                 }
-                if (a.a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
+                if (a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
                 for (int s = s_lo; s < s_hi; ++s, ++g, gs = gs + 1 < NS ? gs + 1 : 0, gph ^= gs == 0) {
                     const int slot = gs;
@@ -1000,7 +1009,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int i = 0; ok; ++i) {
                 const int id = get_item(i);
                 if (id < 0) break;
-                const ItemPos p = locate_item(a, pc, split_item<SH>(a, id));
+                const ItemPos p = locate_item<DEC>(a, pc, split_item<SH>(a, id));
                 const long long key = item_key(p);
                 int s_lo, s_hi;
                 if (SH && a.rec_split) {   // every record-split part streams the whole gate
@@ -1009,9 +1018,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 } else {
                     part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
                 }
-                const bool skip = a.a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
+                const bool skip = a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
                 if (skip) s_hi = s_lo;
-                if (!a.resident && (i == 0 || key != prev_key)) {
+                if (!resident && (i == 0 || key != prev_key)) {
                     ++q;
                     ok = mbar_wait(xfull, q & 1, err, 31);
                 }
@@ -1040,9 +1049,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 else
                     umma_commit(&gdone[bsel]);
                 if (tr && i == 0) tr[57] = global_ns();
-                if (!a.resident) {   // static ranges: the next id is first + i + 1
+                if (!resident) {   // static ranges: the next id is first + i + 1
                     const bool last_of_tile =
-                        i + 1 >= n_my || item_key(locate_item(a, pc, first + i + 1)) != key;
+                        i + 1 >= n_my || item_key(locate_item<DEC>(a, pc, first + i + 1)) != key;
                     if (last_of_tile) umma_commit(xfree);
                 }
                 prev_key = key;
@@ -1069,7 +1078,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             fence_proxy_async_smem();
             __syncwarp();
         };
-        if (a.resident) {
+        if (resident) {
             // the token operand streams with the gate tiles: this warp is the
             // second gather warp
             // (the token operand streams with the gate stages: nothing to load here)
@@ -1077,7 +1086,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             int q = -1;
             long long prev_key = 0;
             for (int i = 0; i < n_my; ++i) {
-                const ItemPos p = locate_item(a, pc, first + i);
+                const ItemPos p = locate_item<DEC>(a, pc, first + i);
                 const long long key = item_key(p);
                 if (i > 0 && key == prev_key) continue;
                 prev_key = key;
@@ -1116,7 +1125,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         auto do_mask = [&](int i, int id) {
             ItemMeta &M = meta[i & 1];
             const int item = split_item<SH>(a, id), part = split_part<SH>(a, id);
-            const ItemPos p = locate_item(a, pc, item);
+            const ItemPos p = locate_item<DEC>(a, pc, item);
             int base;
             const int m = tile_tokens(a, pc, p, base);
             if (ct < m) {
@@ -1173,7 +1182,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 const bool jv = j < a.f;
                 const bool masked = M.masked != 0;
                 const float th = M.sidx >= 0 ? a.tau_shared : a.tau;
-                const bool from_a = a.a_in && M.sidx < 0;   // rank pass: silu(g) and the cut from global
+                const bool from_a = a_in && M.sidx < 0;   // rank pass: silu(g) and the cut from global
                 // a rolled loop over the tile's tokens: short code, one TMEM
                 // column each (the token's own column in resident mode)
 #pragma unroll 1
@@ -1182,11 +1191,11 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     bool keep;
                     if (from_a) {
                         const int pr = M.pair[t];
-                        av = jv ? __ldcg(&a.a_in[(size_t)pr * a.f + j]) : 0.f;
+                        av = jv ? __ldcg(&a_in[(size_t)pr * a.f + j]) : 0.f;
                         const float sv = fabsf(av), cv = __ldcg(&a.rank_v[pr]);
                         keep = sv > cv || (sv == cv && j <= __ldcg(&a.rank_j[pr]));
                     } else {
-                        const int col = a.resident ? M.tok[t] : t;
+                        const int col = resident ? M.tok[t] : t;
                         float g = tmem_ld1(taddr + col);
                         if (gp) {
                             const int c = min(col, kSplitCols - 1);
@@ -1472,7 +1481,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     const int nid = get_item(ii + 1);
                     // (a non-owner part has no up/down work: stop accumulating there)
                     cont = nid >= 0 && split_part<SH>(a, nid) == 0 &&
-                           item_key(locate_item(a, pc, split_item<SH>(a, nid))) == M.key;
+                           item_key(locate_item<DEC>(a, pc, split_item<SH>(a, nid))) == M.key;
                 }
                 if (!cont) {
 #pragma unroll
@@ -1662,10 +1671,10 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     return cudaGetLastError();
 }
 
-template <int MT, int NP, bool TR, bool SH>
+template <int MT, int NP, bool TR, bool SH, bool DEC>
 static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    auto kern = k_expert_sparse<MT, NP, TR, SH>;
+    auto kern = k_expert_sparse<MT, NP, TR, SH, DEC>;
     static int smem_set[kMaxDevices] = {};
     cudaError_t e = ensure_dynamic_smem(kern, a.L.total, smem_set);
     if (e != cudaSuccess) return e;
@@ -1687,11 +1696,11 @@ static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 template <int MT, int NP>
 static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    if (a.share_records)
-        return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, true>(a, grid, st)
-                                 : launch_mt_tr<MT, NP, false, true>(a, grid, st);
-    return a.ws.trace_expert ? launch_mt_tr<MT, NP, true, false>(a, grid, st)
-                             : launch_mt_tr<MT, NP, false, false>(a, grid, st);
+    if (a.ws.trace_expert) return launch_mt_tr<MT, NP, true, false, false>(a, grid, st);
+    if (a.resident && !a.a_in && !a.inject)
+        return a.share_records ? launch_mt_tr<MT, NP, false, true, true>(a, grid, st)
+                               : launch_mt_tr<MT, NP, false, false, true>(a, grid, st);
+    return launch_mt_tr<MT, NP, false, false, false>(a, grid, st);
 }
 
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
@@ -1744,7 +1753,8 @@ cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const W
     a.n_parts = a.n_parts_s = 1;
     // the shared experts' items are the heavy ones when no threshold applies
     // to them (every neuron of a block active: 128 records each)
-    const bool dense_shared = a.n_shared_items > 0 && (!use_mask || tau_shared <= 0.f);
+    // (only the decode kernel has the per-class part counts and the sharing)
+    const bool dense_shared = a.n_shared_items > 0 && (!use_mask || tau_shared <= 0.f) && !ws.trace_expert && !inject;
     const long long routed_max = (long long)a.max_touched * dm.n_blk;
     {
         const char *sp = std::getenv("MOE_SPLIT");
