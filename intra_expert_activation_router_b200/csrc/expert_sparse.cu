@@ -656,14 +656,16 @@ __device__ __noinline__ void combine_tail(const SparseArgs &a, int tid, int *s_f
 // TR: the traced instantiation, launched only while moe_set_trace holds a
 // buffer; the stamps' clock reads and branches cost 4-7 % of a decode step,
 // so the untraced kernels have none of them.  DEC: the decode instantiation,
-// for batches resident as one token tile outside the rank budget's second
-// pass and fault injection: the token-tile mode, the rank pass and the
-// injection compiled out (5-7 % of a decode step).  SH (decode only): the
+// for batches resident as one token tile, outside the rank budget's passes,
+// the calibration's score mode and fault injection: the token-tile mode, the
+// rank pass, the score mode and the injection compiled out, and the routing
+// (inside the kernel, FU, or by the router kernel) fixed at compile time
+// (8-9 % of a decode step).  SH (decode only): the
 // parts of a split item also share its records, per-class part counts, the
 // record split of dense shared items; a separate instantiation again, since
 // code the other kernels never run still slowed them by about a microsecond.
 // The traced kernel is the general one (not DEC, not SH).
-template <int MT, int NP, bool TR, bool SH, bool DEC>
+template <int MT, int NP, bool TR, bool SH, bool DEC, bool FU>
 __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __grid_constant__ SparseArgs a)
 {
     extern __shared__ uint8_t dsm_raw[];
@@ -711,8 +713,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     Plan *plan = a.ws.plan;
     int *err = a.ws.error_word;
     const int d = a.d;
-    const bool score_mode = a.score_out != nullptr;
-    const bool resident = DEC || a.resident;        // compile-time true in the decode kernel
+    const bool score_mode = !DEC && a.score_out != nullptr;   // compile-time false in the decode kernel
+    const bool fused = DEC ? FU : a.fused != 0;               // compile-time in the decode kernels
+    const bool resident = DEC || a.resident;
     const float *const a_in = DEC ? nullptr : a.a_in;   // rank pass, second pass
     const int inject = DEC ? 0 : a.inject;
     unsigned long long *tr = (TR && a.ws.trace_expert && (int)blockIdx.x < a.ws.trace_expert_ctas)
@@ -765,7 +768,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     float *s_perm_w = reinterpret_cast<float *>(s_perm_tok + a.max_pairs);
     volatile int *s_ntouched = reinterpret_cast<volatile int *>(smem + L.ctr_off + 56);
     int n_touched, n_routed_items;
-    if (a.fused) {
+    if (fused) {
         route_in_kernel<TR>(a, ring, s_prefix, s_expert, s_off, s_cnt, s_perm, s_perm_tok, s_perm_w, s_ntouched,
                         xfull);   // the token-tile barrier, unused in resident mode
         n_touched = *s_ntouched;
@@ -800,8 +803,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     }
     if (tr && tid == 0) tr[1] = global_ns();
     const PlanCache pc{s_prefix, s_expert, s_off, s_cnt, s_order, n_touched,
-                       a.fused ? s_perm : a.ws.perm, a.fused ? s_perm_tok : a.ws.perm_tok,
-                       a.fused ? s_perm_w : a.ws.perm_w};
+                       fused ? s_perm : a.ws.perm, fused ? s_perm_tok : a.ws.perm_tok,
+                       fused ? s_perm_w : a.ws.perm_w};
 
     const int n_items = SH ? a.n_shared_items * a.n_parts_s + (a.score_shared ? 0 : n_routed_items) * a.n_parts
                            : (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts;
@@ -969,7 +972,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     }
                     uint8_t *stage = ring + (size_t)slot * L.stage_pitch;
                     mbar_arrive_expect_tx(&full_g[slot], kStageBytes + L.xs_bytes);
-                    if (a.fused) {   // the token operand's blocks 2s, 2s+1 straight from x (L2-resident)
+                    if (fused) {   // the token operand's blocks 2s, 2s+1 straight from x (L2-resident)
                         tma_load_2d(stage + kStageBytes, &a.xmap, 128 * s, 0, &full_g[slot]);
                         tma_load_2d(stage + kStageBytes + L.xt_kb, &a.xmap, 128 * s + 64, 0, &full_g[slot]);
                     } else if (L.xs_bytes) {   // the same, pre-swizzled by the router
@@ -1671,10 +1674,10 @@ static cudaError_t launch_y_out(float *y_acc, uint16_t *out, size_t n4, int n_sm
     return cudaGetLastError();
 }
 
-template <int MT, int NP, bool TR, bool SH, bool DEC>
+template <int MT, int NP, bool TR, bool SH, bool DEC, bool FU>
 static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    auto kern = k_expert_sparse<MT, NP, TR, SH, DEC>;
+    auto kern = k_expert_sparse<MT, NP, TR, SH, DEC, FU>;
     static int smem_set[kMaxDevices] = {};
     cudaError_t e = ensure_dynamic_smem(kern, a.L.total, smem_set);
     if (e != cudaSuccess) return e;
@@ -1696,11 +1699,15 @@ static cudaError_t launch_mt_tr(const SparseArgs &a, int grid, cudaStream_t st)
 template <int MT, int NP>
 static cudaError_t launch_mt(const SparseArgs &a, int grid, cudaStream_t st)
 {
-    if (a.ws.trace_expert) return launch_mt_tr<MT, NP, true, false, false>(a, grid, st);
-    if (a.resident && !a.a_in && !a.inject)
-        return a.share_records ? launch_mt_tr<MT, NP, false, true, true>(a, grid, st)
-                               : launch_mt_tr<MT, NP, false, false, true>(a, grid, st);
-    return launch_mt_tr<MT, NP, false, false, false>(a, grid, st);
+    if (a.ws.trace_expert) return launch_mt_tr<MT, NP, true, false, false, false>(a, grid, st);
+    if (a.resident && !a.a_in && !a.inject && !a.score_out) {
+        if (a.fused)
+            return a.share_records ? launch_mt_tr<MT, NP, false, true, true, true>(a, grid, st)
+                                   : launch_mt_tr<MT, NP, false, false, true, true>(a, grid, st);
+        return a.share_records ? launch_mt_tr<MT, NP, false, true, true, false>(a, grid, st)
+                               : launch_mt_tr<MT, NP, false, false, true, false>(a, grid, st);
+    }
+    return launch_mt_tr<MT, NP, false, false, false, false>(a, grid, st);
 }
 
 cudaError_t launch_expert_sparse(const Dims &dm, const DeviceWeights &w, const Workspace &ws,
