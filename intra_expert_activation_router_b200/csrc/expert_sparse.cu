@@ -1453,7 +1453,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     for (int p = 0; p < NP; ++p) {
                         const int v = ct + 128 * p;
                         if (v < d8) {
-                            for (int q = 0; q < nb; ++q) {
+#pragma unroll
+                            for (int q = 0; q < kRows; ++q) {   // nb <= gb <= kRows records
+                                if (q >= nb) break;
                                 const uint4 wv =
                                     *reinterpret_cast<const uint4 *>(buf + (size_t)q * L.gpitch + 2 * d + 16 * v);
                                 const uint64_t w2[4] = {bf16x2_f2(wv.x), bf16x2_f2(wv.y), bf16x2_f2(wv.z),
@@ -1589,7 +1591,7 @@ static bool make_layout(int d, int dp, SparseTiling til, bool resident, int max_
     // gather buffers of up to four records (rows per up reduction), at least
     // two of them; three gate stages when that leaves two buffers, else two
     int gb = 32768 / rec;
-    gb = gb < 1 ? 1 : gb > 4 ? 4 : gb;
+    gb = gb < 1 ? 1 : gb > kRows ? kRows : gb;
     int ns = 3;
     if ((kSmemLimit - fixed - ns * L.stage_pitch) / up(gb * L.gpitch) < 2) ns = 2;
     const int room = kSmemLimit - fixed - ns * L.stage_pitch;
