@@ -216,35 +216,42 @@ __device__ __forceinline__ long long item_key(const ItemPos &p)
 // 0), which waits for the others' partial sums, is always claimed after them:
 // every such wait points to an earlier claim, which its CTA publishes before
 // it reaches any later wait.
-// PC: per-class part counts (the record-sharing instantiation); otherwise
-// every item has n_parts parts (n_parts_s == n_parts).
-template <bool PC>
+// PM, the kernel's part mapping: 2 per-class part counts (the
+// record-sharing instantiation), 1 every item n_parts parts, 0 no split (the
+// kernels for more than kSplitCols tokens: every item one part, compile-time).
+template <int PM>
 __device__ __forceinline__ int split_item(const SparseArgs &a, int id)
 {
-    if constexpr (PC) {
+    if constexpr (PM == 2) {
         const int ns = a.n_shared_items * a.n_parts_s;
         return id < ns ? id / a.n_parts_s : a.n_shared_items + (id - ns) / a.n_parts;
-    } else {
+    } else if constexpr (PM == 1) {
         return id / a.n_parts;
+    } else {
+        return id;
     }
 }
-template <bool PC>
+template <int PM>
 __device__ __forceinline__ int split_part(const SparseArgs &a, int id)
 {
-    if constexpr (PC) {
+    if constexpr (PM == 2) {
         const int ns = a.n_shared_items * a.n_parts_s;
         return id < ns ? a.n_parts_s - 1 - id % a.n_parts_s : a.n_parts - 1 - (id - ns) % a.n_parts;
-    } else {
+    } else if constexpr (PM == 1) {
         return a.n_parts - 1 - id % a.n_parts;
+    } else {
+        return 0;
     }
 }
-template <bool PC>
+template <int PM>
 __device__ __forceinline__ int item_parts(const SparseArgs &a, int item)
 {
-    if constexpr (PC)
+    if constexpr (PM == 2)
         return item < a.n_shared_items ? a.n_parts_s : a.n_parts;
-    else
+    else if constexpr (PM == 1)
         return a.n_parts;
+    else
+        return 1;
 }
 
 // Stages [lo, hi) of the item's spi gate stages that a part streams.
@@ -713,6 +720,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     Plan *plan = a.ws.plan;
     int *err = a.ws.error_word;
     const int d = a.d;
+    constexpr int PM = SH ? 2 : (MT <= kSplitCols ? 1 : 0);   // the part mapping (split_item)
     const bool score_mode = !DEC && a.score_out != nullptr;   // compile-time false in the decode kernel
     const bool fused = DEC ? FU : a.fused != 0;               // compile-time in the decode kernels
     const bool resident = DEC || a.resident;
@@ -806,8 +814,9 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                        fused ? s_perm : a.ws.perm, fused ? s_perm_tok : a.ws.perm_tok,
                        fused ? s_perm_w : a.ws.perm_w};
 
-    const int n_items = SH ? a.n_shared_items * a.n_parts_s + (a.score_shared ? 0 : n_routed_items) * a.n_parts
-                           : (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts;
+    const int n_items = PM == 2   ? a.n_shared_items * a.n_parts_s + (a.score_shared ? 0 : n_routed_items) * a.n_parts
+                        : PM == 1 ? (a.n_shared_items + (a.score_shared ? 0 : n_routed_items)) * a.n_parts
+                                  : a.n_shared_items + (a.score_shared ? 0 : n_routed_items);
     // static ranges (token-tile mode): contiguous items per CTA
     const int G = gridDim.x, b = blockIdx.x;
     const int per = n_items / G, rem = n_items % G;
@@ -950,14 +959,14 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 __threadfence_block();
                 *pub_items = i + 1;
                 if (id < 0) break;
-                const ItemPos ip = locate_item<DEC>(a, pc, split_item<SH>(a, id));
+                const ItemPos ip = locate_item<DEC>(a, pc, split_item<PM>(a, id));
                 const uint16_t *src = gate_src(ip);
                 int s_lo, s_hi;
                 if (SH && a.rec_split) {   // every record-split part streams the whole gate
                     s_lo = 0;
                     s_hi = spi;
                 } else {
-                    part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                    part_stages(spi, item_parts<PM>(a, split_item<PM>(a, id)), split_part<PM>(a, id), s_lo, s_hi);
                 }
                 if (a_in && ip.slot >= 0) s_hi = s_lo;   // rank pass: this gate is computed already
                 bool ok = true;
@@ -1012,14 +1021,14 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             for (int i = 0; ok; ++i) {
                 const int id = get_item(i);
                 if (id < 0) break;
-                const ItemPos p = locate_item<DEC>(a, pc, split_item<SH>(a, id));
+                const ItemPos p = locate_item<DEC>(a, pc, split_item<PM>(a, id));
                 const long long key = item_key(p);
                 int s_lo, s_hi;
                 if (SH && a.rec_split) {   // every record-split part streams the whole gate
                     s_lo = 0;
                     s_hi = spi;
                 } else {
-                    part_stages(spi, item_parts<SH>(a, split_item<SH>(a, id)), split_part<SH>(a, id), s_lo, s_hi);
+                    part_stages(spi, item_parts<PM>(a, split_item<PM>(a, id)), split_part<PM>(a, id), s_lo, s_hi);
                 }
                 const bool skip = a_in && p.slot >= 0;   // rank pass: no MMA for a routed item
                 if (skip) s_hi = s_lo;
@@ -1127,7 +1136,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         unsigned long long t_wait = 0, t_work = 0;   // trace only
         auto do_mask = [&](int i, int id) {
             ItemMeta &M = meta[i & 1];
-            const int item = split_item<SH>(a, id), part = split_part<SH>(a, id);
+            const int item = split_item<PM>(a, id), part = split_part<PM>(a, id);
             const ItemPos p = locate_item<DEC>(a, pc, item);
             int base;
             const int m = tile_tokens(a, pc, p, base);
@@ -1157,7 +1166,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             unsigned long long *ti = (tr && i < 3) ? tr + 2 + 10 * i : nullptr;   // per-item stamps
             if (ti && ct == 0) ti[0] = global_ns();
             // gate split: the item's partial sums, [part - 1][neuron][token]
-            const int np = item_parts<SH>(a, item);
+            const int np = item_parts<PM>(a, item);
             float *gp = np > 1 && !(SH && a.rec_split) ? a.ws.gpart + (size_t)min(item, a.ws.gcnt_n - 1) * (kMaxParts - 1) * kBlk *
                                                           kSplitCols
                                       : nullptr;
@@ -1485,8 +1494,8 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 if (nsub == 1 && !a.ws.ypart) {   // (deterministic mode: one row per block)
                     const int nid = get_item(ii + 1);
                     // (a non-owner part has no up/down work: stop accumulating there)
-                    cont = nid >= 0 && split_part<SH>(a, nid) == 0 &&
-                           item_key(locate_item<DEC>(a, pc, split_item<SH>(a, nid))) == M.key;
+                    cont = nid >= 0 && split_part<PM>(a, nid) == 0 &&
+                           item_key(locate_item<DEC>(a, pc, split_item<PM>(a, nid))) == M.key;
                 }
                 if (!cont) {
 #pragma unroll
