@@ -39,7 +39,11 @@ constexpr int kAccCols = 256;        // one accumulator: 128 lanes x 256 fp32 co
 constexpr int kATileBytes = kBM * kBK * 2;    // 16 KB
 constexpr int kBTileBytes = 256 * kBK * 2;    // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kDenseSmem = kDStages * kStageBytes + 1024 /* alignment */ + 256 /* barriers */;
+// Down epilogue staging: per epilogue warp 32 rows x 16 columns of fp32,
+// rows padded to 20 floats (16-byte aligned, conflict-free quarter warps)
+constexpr int kStgPitch = 20;
+constexpr int kStgBytes = kEpiWarps * 32 * kStgPitch * 4;   // 20 KB
+constexpr int kDenseSmem = kDStages * kStageBytes + 256 /* barriers */ + kStgBytes + 1024 /* alignment */;
 
 enum DenseMode { kGateUp = 0, kDown = 1, kLogits = 2 };
 
@@ -184,6 +188,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
     uint64_t *acce = accf + 2;           // [2] accumulator read out (the epilogue warps)
     uint64_t *mdrain = acce + 2;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mdrain + 1);
+    float *stg_all = reinterpret_cast<float *>(smem + kDStages * kStageBytes + 256);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -331,19 +336,44 @@ __global__ void __launch_bounds__(kDenseThreads, 1) k_dense_gemm(const __grid_co
                     const int slot = a.shared ? a.k + a.sidx
                                               : (row < dt.valid ? a.perm[dt.row0 + row] % a.k : 0);
                     yrow = a.ypart + ((size_t)tok * a.kS + slot) * a.d + dt.n0;
-                }
-                for (int c = 128 * half; c < 128 * half + 128; c += 16) {
-                    float y[16];
-                    tmem_ld16(tl + c, y);
-                    if (row < dt.valid) {
+                    for (int c = 128 * half; c < 128 * half + 128; c += 16) {
+                        float y[16];
+                        tmem_ld16(tl + c, y);
+                        if (row < dt.valid)
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const float4 v = make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]);
-                            if (a.ypart)
-                                __stcg(reinterpret_cast<float4 *>(yrow + c + i), v);
-                            else
-                                atomicAdd(reinterpret_cast<float4 *>(yrow + c + i), v);
+                            for (int i = 0; i < 16; i += 4)
+                                __stcg(reinterpret_cast<float4 *>(yrow + c + i),
+                                       make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]));
+                    }
+                } else {
+                    // the warp's 32 rows, 16 columns at a time, through shared memory,
+                    // so that each vector reduction covers 64 contiguous bytes of 8
+                    // rows (whole 32-byte sectors) instead of 16 bytes of 32 rows
+                    float *stg = stg_all + (warp - 2) * 32 * kStgPitch;
+                    const int rr = lane >> 2, c4 = (lane & 3) * 4;
+                    int tok_r[4];
+                    bool ok_r[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        tok_r[j] = __shfl_sync(0xffffffffu, tok, 8 * j + rr);
+                        ok_r[j] = 32 * q + 8 * j + rr < dt.valid;
+                    }
+                    for (int c = 128 * half; c < 128 * half + 128; c += 16) {
+                        float y[16];
+                        tmem_ld16(tl + c, y);
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<float4 *>(stg + lane * kStgPitch + i) =
+                                make_float4(w * y[i], w * y[i + 1], w * y[i + 2], w * y[i + 3]);
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 v = *reinterpret_cast<const float4 *>(stg + (8 * j + rr) * kStgPitch + c4);
+                            if (ok_r[j])
+                                atomicAdd(reinterpret_cast<float4 *>(a.y_acc + (size_t)tok_r[j] * a.d + dt.n0 + c + c4),
+                                          v);
                         }
+                        __syncwarp();
                     }
                 }
             }
