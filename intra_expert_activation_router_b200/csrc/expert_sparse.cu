@@ -845,9 +845,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
     // The gather: once an item's mask is final, its union-active records into
     // the gather buffers, batch by batch, one bulk copy per record (measured
     // a little faster than 16-byte cp.async copies spread over the warps).
-    // `owners` gather warps may take turns, batch ub belonging to warp
-    // ub % owners; one warp is used.
-    auto gather_loop = [&](int owner, int owners) {
+    auto gather_loop = [&]() {
             uint32_t ub = 0, idle = 0;
             int ubi = 0;        // ub % NU and (ub / NU) & 1, kept without a division (NU is not a constant)
             uint32_t uph = 0;
@@ -869,7 +867,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                 idle = 0;
                 __threadfence_block();
                 const ItemMeta &M = meta[ui & 1];
-                unsigned long long *tg = (tr && ui < 2 && lane == 0 && owner == 0) ? tr + 32 + 4 * ui : nullptr;
+                unsigned long long *tg = (tr && ui < 2 && lane == 0) ? tr + 32 + 4 * ui : nullptr;
                 if (tg) tg[0] = global_ns();
                 int nbatch = 0;
                 const int nsub = min(max(M.nsub, 0), kMaxSub);
@@ -879,7 +877,6 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
                     for (int b0 = 0; b0 < n; b0 += L.gb, ++ub, ubi = ubi + 1 < NU ? ubi + 1 : 0, uph ^= ubi == 0) {
                         const int nb = min(L.gb, n - b0);
                         const int bi = ubi;
-                        if ((int)(ub % (uint32_t)owners) != owner) continue;   // another gather warp's batch
                         mbar_wait(&empty_u[bi], uph ^ 1, err, 36);
                         if (tg && nbatch < 3) tg[1 + nbatch] = global_ns();
                         ++nbatch;
@@ -900,7 +897,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             // the last batch issued into each buffer has landed before the CTA may exit
             if (lane == 0)
                 for (uint32_t b = ub > (uint32_t)NU ? ub - NU : 0; b < ub; ++b)
-                    if ((int)(b % (uint32_t)owners) == owner) mbar_drain(&full_u[b % NU], (b / NU) & 1);
+                    mbar_drain(&full_u[b % NU], (b / NU) & 1);
             __syncwarp();
     };
 
@@ -1091,9 +1088,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
             __syncwarp();
         };
         if (resident) {
-            // the token operand streams with the gate tiles: this warp is the
-            // second gather warp
-            // (the token operand streams with the gate stages: nothing to load here)
+            // the token operand streams with the gate stages: nothing to load here
         } else {
             int q = -1;
             long long prev_key = 0;
@@ -1117,7 +1112,7 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
         __syncwarp();
     } else if (warp == kWarpGather) {
         // ---------------------------------------------------------- gather warp
-        if (!score_mode) gather_loop(0, 1);
+        if (!score_mode) gather_loop();
         __syncwarp();
     } else if (warp < 4) {
         // ------------------------------------------------ up warps: mask and up

@@ -15,8 +15,9 @@
 //      E <= 256 every logit's rank is counted directly, above that k rounds of
 //      a warp arg-max select them.
 //   3. the last token tile builds the routing plan for the expert kernels:
-//      per-expert counts, offsets, a stable permutation of the pairs
-//      (t*k + rank) ordered by expert then token, the ascending list of
+//      per-expert counts, offsets, a permutation of the pairs (t*k + rank)
+//      ordered by expert (then by token up to kSmallPlan pairs; above that
+//      the order inside an expert is arbitrary), the ascending list of
 //      touched experts and the work-item prefix sums of both paths.
 // Tickets reset themselves, so the launch can be replayed (graphs) without
 // host-side clears.
@@ -499,7 +500,8 @@ __global__ void __launch_bounds__(256) k_router(RouterArgs a)
     if (tr && threadIdx.x == 0) tr[5] = global_ns();
 }
 
-// The permutation of a large batch's pairs (more than kStagePairs): pair p goes
+// The permutation of a larger batch's pairs (more than kSmallPlan, no
+// capacity): pair p goes
 // to its expert's first position plus a slot taken from the expert's cursor.
 // The order of an expert's pairs is then arbitrary, which changes neither
 // branch's result (rows are independent; the combine is a sum).
