@@ -20,9 +20,10 @@
 //
 // Work items are (expert, tile of up to NT of its tokens, block of 128
 // neurons).  With T <= NT ("resident" mode) the whole batch is the gate MMA's
-// token operand: the router writes it in the MMA's layout, and each ring
-// stage carries its two 64-input blocks (2 or 4 KB, re-read from L2 per
-// item) next to the 32 KB of gate tiles, which leaves the shared memory of a
+// token operand: the router writes it in the MMA's layout (or, when the batch
+// is routed inside this kernel, a TMA tensor map reads it straight from x),
+// and each ring stage carries its two 64-input blocks (2 or 4 KB, re-read
+// from L2 per item) next to the 32 KB of gate tiles, which leaves the shared memory of a
 // resident token tile to the gather buffers.  Items are claimed from a
 // counter in the plan, the experts with most tokens first.  A CTA claims its next item only
 // once its previous one is masked and at most kClaimBacklog of its gathered
