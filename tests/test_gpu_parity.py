@@ -423,6 +423,25 @@ def test_traced_kernel(o, T, fused):
         layer.set_path(m.MOE_PATH_AUTO)
 
 
+@pytest.mark.parametrize("name,T,mode", [("dsv2lite", 2, "fused"), ("dsv2lite", 4, "fused"), ("dsv2lite", 4, "kernel"),
+                                         ("tiny", 4, "fused"), ("tiny", 4, "one_launch"), ("large", 2, "fused"),
+                                         ("large", 4, "fused")])
+def test_dense_shared_items_split(o, name, T, mode):
+    """Layers whose shared experts run without a threshold split those heavy
+    items: by the gate's K stages with the records shared (one and two
+    tokens, where the grid allows) or by records, each part streaming the
+    whole gate (more tokens).  Both part counts (2, and 4 where every claim
+    has an SM) and both routing modes, against the oracle."""
+    layer, W, host = layer_for(name)
+    layer.set_fused_router(mode != "kernel", one_launch=(mode == "one_launch"))
+    try:
+        for _ in range(2):   # counters the split uses must be reset by the forward itself
+            run_case(o, name, T, 0.98 if name == "large" else 0.9)
+        assert layer.stats()["device_error"] == 0
+    finally:
+        layer.set_fused_router(True)
+
+
 def test_host_pointer_entry(o):
     from intra_expert_activation_router_b200 import moe_sparse_forward_host
     sh = mi.SHAPES["olmoe"]
