@@ -269,7 +269,10 @@ int moe_set_capacity(moe_handle h, float gamma);
  * d_ff 1024).  The first call with enable != 0 allocates max_tokens *
  * (top_k + n_shared) * ceil(d_ff / 128) * d_model floats (MOE_ENOMEM if that
  * fails, the setting unchanged) and clears them; moe_sparse_destroy frees
- * them.  Not stream-ordered: call it between forwards, with none in flight. */
+ * them.  With it on, no row has two writers, so an item is never split
+ * across CTAs by its records (on layers whose shared experts run without a
+ * threshold those items are then the slowest of a decode step).  Not
+ * stream-ordered: call it between forwards, with none in flight. */
 int moe_set_deterministic(moe_handle h, int enable);
 
 /* As moe_calibrate_tau, over the N = T*n_shared*d_ff scores of the shared
