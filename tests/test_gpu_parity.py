@@ -595,6 +595,31 @@ def test_rank_budget(o, name, T, frac):
         layer.set_rank_budget(-1)
 
 
+@pytest.mark.parametrize("name,T", [("olmoe", 16), ("dsv2lite", 8)])
+def test_rank_budget_deterministic(o, name, T):
+    """The rank budget's two passes (general kernel instantiation) with the
+    deterministic combine: oracle parity under the GPU's selection, and
+    repeats bit-identical."""
+    sh = mi.SHAPES[name]
+    layer, W, host = layer_for(name)
+    x = mi.make_x(sh, T, device="cuda")
+    inputs = dict(host)
+    inputs["x"] = mi.bf16_bits(x)
+    budget = max(1, int(round(0.1 * sh.d_ff)))
+    layer.set_rank_budget(budget)
+    layer.set_deterministic(True)
+    try:
+        _rank_case(o, layer, inputs, x, sh.top_k, budget)
+        reps = [layer.forward(x, 0.5).clone() for _ in range(3)]
+        torch.cuda.synchronize()
+        assert layer.stats()["deterministic"] == 1 and layer.stats()["device_error"] == 0
+        for u in reps[1:]:
+            assert torch.equal(u, reps[0])
+    finally:
+        layer.set_deterministic(False)
+        layer.set_rank_budget(-1)
+
+
 def test_rank_budget_edges_and_shared_threshold(o):
     """Budget 0 (the shared experts alone), budget = d_ff and above (the
     unmasked layer), a looser shared threshold beside the budget, the dense
