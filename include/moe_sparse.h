@@ -173,7 +173,7 @@ int moe_tune_t_star(moe_handle h, const void *x, int T_max, float tau, int *t_st
  * the fp32 accumulator to the bf16 output); 2 also does that conversion at
  * the end of the expert kernel, after a grid-wide count of the CTAs whose
  * sums have landed, so such a forward is one launch (router, gate, mask,
- * gather, up/down and combine; measured about 2 us slower than mode 1 at
+ * gather, up/down and combine; measured 2.5-3 us slower than mode 1 at
  * 1 and 16 tokens on B200, which is why it is not the default).  Modes 1
  * and 2 assume every CTA of the expert kernel (at most one per SM) can be
  * resident at once, which holds unless the context is restricted to fewer
