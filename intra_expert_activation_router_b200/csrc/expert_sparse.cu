@@ -1553,16 +1553,19 @@ __global__ void __launch_bounds__(kSparseThreads, 1) k_expert_sparse(const __gri
 // logits in the idle gate ring, and x at least one 64-input box wide.
 bool fused_possible(const Dims &dm, int T)
 {
-    const SparseTiling t = sparse_tiling(T, dm.d);
+    const SparseTiling t = sparse_tiling(T, dm.d, dm.S);
     return T <= t.nt && T * dm.k <= kMaxFusedPairs && T * dm.E <= kMaxFusedLogits && dm.E <= kMaxFusedExperts &&
            dm.d >= 64;
 }
 
-SparseTiling sparse_tiling(int T, int d)
+SparseTiling sparse_tiling(int T, int d, int n_shared)
 {
     SparseTiling t;
     const int np = (d / 8 + 127) / 128;   // 16-byte slices of d per up/down thread
-    t.mt = T <= 1 ? 1 : T <= 2 ? 2 : 4;
+    // passes of two tokens up to 8 tokens when no shared expert holds all of
+    // them (a routed item there mostly has one or two; measured 1-2 us
+    // faster), else of four (a shared item's every pass reads all its records)
+    t.mt = T <= 1 ? 1 : (T <= 2 || (n_shared == 0 && T <= 8)) ? 2 : 4;
     while (t.mt > 1 && t.mt * np > 8) t.mt >>= 1;
     const int dp = (d + 127) & ~127;
     // 16-token tiles when they fit in 64 KB and the batch needs them: a batch

@@ -98,7 +98,7 @@ __host__ __device__ __forceinline__ size_t gate_tile_off(int j, int k, int n_kb)
 struct SparseTiling {
     int nt, mt;
 };
-SparseTiling sparse_tiling(int T, int d);
+SparseTiling sparse_tiling(int T, int d, int n_shared);
 
 struct Workspace {
     float *logits;

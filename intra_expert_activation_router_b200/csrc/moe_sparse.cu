@@ -355,7 +355,7 @@ static int run_forward(moe_handle h, const void *x, int T, float tau, bool maske
     if (h->n_ev) e = cudaEventRecordWithFlags(h->ev[0], st, ev_flags);
     bool fused = false;
     if (path == MOE_PATH_SPARSE) {
-        const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d);
+        const moe::SparseTiling til = moe::sparse_tiling(T, h->dm.d, h->dm.S);
         // decode batches route inside the expert kernel: no router launch
         fused = !rank && cap < 0 && h->fused_router && moe::fused_possible(h->dm, T);
         if (e == cudaSuccess && !fused) e = route(h, xb, T, til.nt, st, cap);
@@ -593,7 +593,7 @@ static int calibrate(moe_handle h, const void *x, int T, double sparsity, float 
     }
     cudaStream_t st = (cudaStream_t)stream;
     const uint16_t *xb = (const uint16_t *)x;
-    const moe::SparseTiling til = moe::sparse_tiling(T, dm.d);
+    const moe::SparseTiling til = moe::sparse_tiling(T, dm.d, dm.S);
     cudaError_t e = route(h, xb, T, til.nt, st);
     if (e == cudaSuccess)
         e = moe::launch_expert_sparse(dm, h->w, h->ws, xb, T, 0.0f, false, h->ws.out_stage, til, h->n_sm, st,
